@@ -1,0 +1,127 @@
+"""Pins for the oracle's NVFP4 block quantizer."""
+
+import os
+
+import numpy as np
+import pytest
+
+from oracle import formats, nvfp4, philox
+
+
+def _golden_blocks(golden_dir):
+    cases = []
+    with open(os.path.join(golden_dir, "nvfp4_blocks.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            name, rounding, g, vals, us, scale, codes = (p.strip() for p in line.split("|"))
+            cases.append(dict(
+                name=name, rounding=rounding, g=float(g),
+                v=np.array([float(x) for x in vals.split()], dtype=np.float32),
+                u=None if us == "-" else np.array([float(x) for x in us.split()]),
+                scale=int(scale, 16), codes=[int(c, 16) for c in codes.split()]))
+    return cases
+
+
+def test_hand_worked_blocks(golden_dir):
+    cases = _golden_blocks(golden_dir)
+    assert len(cases) == 7
+    for c in cases:
+        u = None if c["u"] is None else c["u"][None, :]
+        codes, scales = nvfp4.quantize_blocks(c["v"][None, :], c["g"], c["rounding"], u)
+        assert int(scales[0, 0]) == c["scale"], c["name"]
+        assert [int(x) for x in codes[0]] == c["codes"], c["name"]
+
+
+def test_grid_values_are_lossless():
+    rng = np.random.default_rng(0)
+    mags = formats.E2M1_MAGNITUDES
+    for g in (1.0, 0.5, 2.0 ** -10):
+        idx = rng.integers(0, 8, size=(64, 32))
+        sign = rng.choice([-1.0, 1.0], size=idx.shape)
+        s = 2.0 ** rng.integers(-5, 5, size=(64, 2))
+        v = (mags[idx] * sign * np.repeat(s, 16, axis=1) * g).astype(np.float32)
+        v[:, 0] = 6.0 * s[:, 0] * g          # pin the block max so the scale is exact
+        v[:, 16] = 6.0 * s[:, 1] * g
+        codes, scales = nvfp4.quantize_blocks(v, g)
+        back = nvfp4.dequantize_blocks(codes, scales, g)
+        assert np.array_equal(back, v.astype(np.float64))
+
+
+def test_rn_error_is_at_most_half_a_grid_step():
+    rng = np.random.default_rng(1)
+    v = (rng.standard_normal((256, 64)) * np.exp(rng.uniform(-4, 4, size=(256, 1)))).astype(np.float32)
+    codes, scales = nvfp4.quantize_blocks(v)
+    back = nvfp4.dequantize_blocks(codes, scales)
+    d = np.repeat(formats.e4m3_decode(scales), 16, axis=1)
+    x = np.abs(v / d)
+    # local grid spacing of E2M1 around |x| (0.5 below 2, 1 below 4, 2 above)
+    step = np.where(x < 2, 0.5, np.where(x < 4, 1.0, 2.0))
+    bound = np.maximum(step / 2 * d, (np.abs(v) - 6 * d)) * (1 + 1e-6)
+    assert np.all(np.abs(back - v) <= bound + 1e-30)
+
+
+def test_zero_block_and_tiny_block():
+    v = np.zeros((1, 16), dtype=np.float32)
+    codes, scales = nvfp4.quantize_blocks(v)
+    assert scales[0, 0] == 0 and not codes.any()
+    v[0, 3] = 1e-30
+    codes, scales = nvfp4.quantize_blocks(v)
+    assert scales[0, 0] == 1                  # clamped to 2^-9
+
+
+def test_non_finite_is_rejected():
+    v = np.zeros((1, 16), dtype=np.float32)
+    v[0, 5] = np.nan
+    with pytest.raises(nvfp4.NonFiniteInput):
+        nvfp4.quantize_blocks(v)
+
+
+def test_sr_is_unbiased():
+    rng = np.random.default_rng(2)
+    v = rng.uniform(-5.9, 5.9, size=(1, 16)).astype(np.float32)
+    v[0, 0] = 6.0
+    acc = np.zeros(16)
+    n = 4096
+    for seed in range(n):
+        codes, scales = nvfp4.quantize_oriented(v, "row", rounding="sr", seed=seed, operand_id=0)
+        acc += nvfp4.dequantize_blocks(codes, scales)[0]
+    mean = acc / n
+    # each element is a two-point variable with spread <= 2 (grid step), sd <= 1
+    assert np.all(np.abs(mean - v[0]) <= 4.0 / np.sqrt(n) + 1e-6)
+
+
+def test_sr_rounds_to_a_neighbour():
+    rng = np.random.default_rng(3)
+    v = rng.standard_normal((32, 64)).astype(np.float32) * 3
+    c_rn, s_rn = nvfp4.quantize_blocks(v)
+    c_sr, s_sr = nvfp4.quantize_oriented(v, "row", rounding="sr", seed=5)
+    assert np.array_equal(s_rn, s_sr)
+    d = np.repeat(formats.e4m3_decode(s_rn), 16, axis=1)
+    x = v / d
+    mag_sr = formats.E2M1_MAGNITUDES[c_sr & 7]
+    lo = formats.E2M1_MAGNITUDES[np.clip(np.searchsorted(formats.E2M1_MAGNITUDES, np.abs(x), "right") - 1, 0, 7)]
+    hi = formats.E2M1_MAGNITUDES[np.clip(np.searchsorted(formats.E2M1_MAGNITUDES, np.abs(x), "right"), 0, 7)]
+    assert np.all((mag_sr == lo) | (mag_sr == hi))
+
+
+def test_orientation_and_packing():
+    rng = np.random.default_rng(4)
+    M = rng.standard_normal((48, 32)).astype(np.float32)
+    c_col, s_col = nvfp4.quantize_oriented(M, "col")
+    c_rowT, s_rowT = nvfp4.quantize_blocks(np.ascontiguousarray(M.T))
+    assert np.array_equal(c_col, c_rowT) and np.array_equal(s_col, s_rowT)
+    packed = nvfp4.pack_codes(c_col)
+    assert packed.shape == (32, 24)
+    assert np.array_equal(packed[:, 0] & 0xF, c_col[:, 0])
+    assert np.array_equal(packed[:, 0] >> 4, c_col[:, 1])
+    assert np.array_equal(nvfp4.unpack_codes(packed), c_col)
+
+
+def test_sr_uses_the_orientation_stream():
+    rng = np.random.default_rng(6)
+    M = rng.standard_normal((16, 16)).astype(np.float32)
+    u = philox.sr_uniforms(9, 2, philox.SR_SUB_COLWISE, 4, 256).reshape(16, 16)
+    want, _ = nvfp4.quantize_blocks(np.ascontiguousarray(M.T), 1.0, "sr", u)
+    got, _ = nvfp4.quantize_oriented(M, "col", rounding="sr", seed=9, operand_id=2, step=4)
+    assert np.array_equal(want, got)
