@@ -1,0 +1,230 @@
+/*
+ * libmetis -- the Metis spectral-domain W4A4G4 linear layer on NVIDIA B200.
+ *
+ * Method: "Metis: Training LLMs with FP4 Quantization" (ICLR 2026; papernotes.org
+ * notes).  Every matrix M of a GeMM (weight W, activation X, output gradient D)
+ * is split into a rank-k dominant part kept in high precision and a residual
+ * quantized to NVFP4 (key design 1):
+ *
+ *     M = U_k S_k V_k^T + M_R
+ *     Y = (Q(A_k) L_k Q(B_k^T) + Q(X_R)) (Q(U_k) S_k Q(V_k^T) + Q(W_R))
+ *
+ * with Q the NVFP4 block quantizer (E2M1 values, 16-element blocks, one E4M3
+ * scale per block; background section) and the singular values kept in fp32.
+ * The dominant subspace comes from l_k sampled rows and a Gaussian sketch of
+ * width k + s (key design 2) and is reused across steps (key design 3).
+ *
+ * Conventions for every call:
+ *   - All matrix pointers are DEVICE pointers owned by the caller; libmetis never
+ *     allocates or frees them.  The context owns only its workspace and a device
+ *     status word.
+ *   - Calls are asynchronous on the context's stream.  The returned status covers
+ *     host-side validation and launch only; numeric failures found on the device
+ *     latch bits of the status word (METIS_DEV_*), read by
+ *     metis_poll_device_status.  No kernel traps.
+ *   - Shapes: every matrix dimension is a multiple of 128 (and, where it is a GeMM
+ *     contraction length, of 256); 1 <= k <= 64; k + s <= 128; k + s <= l_k <= rows.
+ *   - Alignment: pointers 16-byte aligned; bf16 leading dimensions a multiple of 8
+ *     elements, fp32 ones a multiple of 4.
+ *   - Device: sm_100 (B200) only; anything else returns METIS_ERR_ARCH.
+ *   - On error nothing is launched and metis_last_error() describes the cause.
+ */
+#ifndef METIS_H
+#define METIS_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  METIS_OK = 0,
+  METIS_ERR_ARG = 1,        /* null pointer, bad enum or inconsistent descriptor */
+  METIS_ERR_SHAPE = 2,      /* a dimension outside the limits above */
+  METIS_ERR_ALIGN = 3,      /* pointer or leading-dimension alignment */
+  METIS_ERR_ARCH = 4,       /* device is not sm_100 */
+  METIS_ERR_CUDA = 5,       /* a CUDA runtime or driver call failed */
+  METIS_ERR_WORKSPACE = 6   /* the context could not grow its workspace */
+} metis_status;
+
+/* Bits of the device status word (latched; cleared by metis_poll_device_status). */
+#define METIS_DEV_NUMERIC   1u  /* a small dense factorization did not converge */
+#define METIS_DEV_NONFINITE 2u  /* NaN or Inf met in a quantizer or decomposition input */
+#define METIS_DEV_TIMEOUT   4u  /* a bounded wait inside a kernel ran out; its work was skipped */
+
+typedef struct metis_ctx metis_ctx;
+
+/* Creates a context on `device` issuing work on `stream` (a cudaStream_t, may be 0).
+ * Fails with METIS_ERR_ARCH unless the device is sm_100. */
+metis_status metis_create(int device, void* stream, metis_ctx** out);
+/* Frees the context's workspace and status word (synchronizes its stream). */
+void metis_destroy(metis_ctx* ctx);
+metis_status metis_set_stream(metis_ctx* ctx, void* stream);
+const char* metis_status_str(metis_status s);
+/* Message of the last failed call on this context; owned by the context. */
+const char* metis_last_error(const metis_ctx* ctx);
+/* Synchronizes the stream, returns the latched METIS_DEV_* bits, clears them if `clear`. */
+metis_status metis_poll_device_status(metis_ctx* ctx, uint32_t* bits, int clear);
+
+/* Dense bf16 device matrix, row-major with leading dimension `ld` (elements). */
+typedef struct {
+  const void* data;
+  int64_t rows, cols, ld;
+} metis_matrix;
+
+/*
+ * NVFP4 tensor in one orientation: logically outer x inner with 16-element blocks
+ * along inner (inner is the contraction dimension of the GeMM that reads it).
+ *   codes  : outer x inner/2 bytes, row-major; element 2t of a row sits in the low
+ *            nibble of byte t, element 2t+1 in the high nibble; code bit 3 = sign,
+ *            bits 0-2 index the E2M1 magnitudes {0,0.5,1,1.5,2,3,4,6}.
+ *   scales : E4M3 (OCP fn) block scales in 512-byte tiles, one tile per 128 rows x
+ *            64 inner elements; tile (ob, kb) starts at byte (ob*(inner/64)+kb)*512
+ *            and holds the scale of row o, block b at offset
+ *            (o%32)*16 + ((o%128)/32)*4 + (b%4)  -- the layout the tcgen05
+ *            block-scaled MMA reads from tensor memory.
+ *   tensor_scale : device pointer to one fp32 decode-side tensor scale g (a power
+ *            of two).  Decoded value = e2m1(code) * e4m3(scale) * g.
+ */
+typedef struct {
+  uint8_t* codes;
+  uint8_t* scales;
+  float* tensor_scale;
+  int64_t outer, inner;
+} metis_nvfp4;
+
+/* Bytes needed for the codes / scales of an outer x inner NVFP4 tensor. */
+int64_t metis_nvfp4_codes_bytes(int64_t outer, int64_t inner);
+int64_t metis_nvfp4_scales_bytes(int64_t outer, int64_t inner);
+
+/*
+ * Low-rank factors of one operand M (rows x cols):  U S V^T  (key design 1).
+ *   V  : cols x k fp32 row-major -- the reused subspace basis (key design 3).  Input
+ *        to every step, rotated in place within its span; overwritten on refresh.
+ *   U  : rows x k fp32 (output of every step), S : k fp32 descending (output).
+ *   Uq, Vq : NVFP4 of U^T and V^T (outer = 128, inner = rows / cols); rows >= k are
+ *        zero.  Blocks run along the long dimension; tensor scale is the smallest
+ *        power of two g with max|F| <= 6*448*g (set on the device).
+ *   sampled_rows (l_k int32) and omega (cols x (k+s) fp32): optional (nullable)
+ *        copies of the last refresh's row sample and Gaussian test matrix.
+ */
+typedef struct {
+  int64_t rows, cols;
+  int32_t k;
+  float* V;
+  float* U;
+  float* S;
+  metis_nvfp4 Uq;
+  metis_nvfp4 Vq;
+  int32_t* sampled_rows;
+  float* omega;
+} metis_factors;
+
+typedef struct {
+  int32_t k;             /* rank (training strategy: 1.5% of the hidden size) */
+  int32_t s;             /* sketch oversampling; sketch width k + s */
+  int32_t l_k;           /* sampled rows (key design 2); l_k == rows disables sampling */
+  uint64_t seed;         /* Philox4x32-10 key */
+  uint32_t operand_id;   /* separates the random streams of X, W, D */
+  int32_t rounding;      /* factor quantization: 0 round-to-nearest, 1 stochastic */
+} metis_decomp_params;
+
+/*
+ * Randomized decomposition of M (key designs 2 and 3).
+ * refresh != 0: sample l_k rows (Philox), draw Omega ~ N(0,1) (Philox + Box-Muller),
+ *   sketch Y = M_s Omega, CholQR(Y) = Q R, Bm = Q^T M_s, CholQR(Bm^T) = Q2 R2,
+ *   one-sided Jacobi SVD of R2^T, V = Q2 W'[:, :k].
+ * Every call: P = M V, CholQR(P) = Q_P R_P, Jacobi SVD R_P = U_r S_r V_r^T,
+ *   U = Q_P U_r, S = S_r, V <- V V_r (sign-fixed), then Uq and Vq.
+ * `step` enters the Philox counters (row sample, Omega, stochastic rounding).
+ * Errors: ERR_SHAPE for k/s/l_k outside the limits; device: METIS_DEV_NONFINITE,
+ * METIS_DEV_NUMERIC.
+ */
+metis_status metis_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_decomp_params* p,
+                             int refresh, uint32_t step, metis_factors* f);
+
+typedef struct {
+  int32_t rounding;      /* 0 round-to-nearest-even, 1 stochastic (training strategy) */
+  uint64_t seed;
+  uint32_t operand_id;
+  uint32_t step;
+  float tensor_scale;    /* decode-side tensor scale g of the residual (power of two, >0) */
+} metis_quant_params;
+
+/*
+ * Residual quantization (key design 1):  M_R = M - U diag(S) V^T  (factors f, fp32,
+ * unquantized; f == NULL or f->k == 0 quantizes M itself -- plain NVFP4), then NVFP4
+ * in one or both orientations:
+ *   rowwise (nullable): outer = rows, inner = cols  (blocks along columns)
+ *   colwise (nullable): outer = cols, inner = rows  (blocks along rows; M_R^T)
+ * Stochastic rounding uses the Philox SR stream (operand_id, sub 0 row-wise / 1
+ * column-wise, step).  Device: METIS_DEV_NONFINITE on NaN/Inf input.
+ */
+metis_status metis_residual_quantize_nvfp4(metis_ctx* ctx, const metis_matrix* M,
+                                           const metis_factors* f, const metis_quant_params* q,
+                                           metis_nvfp4* rowwise, metis_nvfp4* colwise);
+
+/*
+ * NVFP4 quantization of an fp32 device matrix R (rows x cols, leading dimension ld):
+ * the quantizer alone, bit-exact with the block rule (background section; training
+ * strategy for stochastic rounding).  Same outputs as above.
+ */
+metis_status metis_quantize_nvfp4_f32(metis_ctx* ctx, const float* R, int64_t rows, int64_t cols,
+                                      int64_t ld, const metis_quant_params* q,
+                                      metis_nvfp4* rowwise, metis_nvfp4* colwise);
+
+/* Output element types. */
+#define METIS_OUT_F32  0
+#define METIS_OUT_BF16 1
+
+/*
+ * Block-scaled FP4 GeMM with an optional bf16 rank-fold, the kernel behind the
+ * layer calls:
+ *   C[i][j] = alpha * col_scale[j] * ( sum_k A(i,k) B(j,k)  +  sum_t Fa[i][t] Fb[j][t] )
+ * A: outer = p (rows of C); B: outer >= q (q = n_cols, the columns of C);
+ * A.inner == B.inner = K, a multiple of 256.
+ * A and B codes are decoded WITHOUT their tensor scales; alpha = gA * gB is read
+ * from the devices' tensor_scale words.  Fa (p x fold_k) and Fb (q x fold_k) are
+ * bf16 row-major device matrices (both NULL with fold_k == 0); fold_k is a
+ * multiple of 64.  col_scale (q fp32) may be NULL (all ones).  C has leading
+ * dimension ldc and type c_dtype (METIS_OUT_*).
+ * q must be a multiple of 256, or one of 16, 32, 64 (thin GeMM; B.outer = 128 with
+ * rows >= q zero).  col_scale, when given, holds q values.
+ */
+metis_status metis_gemm_nvfp4(metis_ctx* ctx, const metis_nvfp4* A, const metis_nvfp4* B, int64_t n_cols,
+                              const void* Fa, const void* Fb, int32_t fold_k,
+                              const float* col_scale, void* C, int64_t ldc, int32_t c_dtype);
+
+/* One operand of the layer: residual in both orientations plus its factors
+ * (f may be NULL or have k == 0 for plain NVFP4). */
+typedef struct {
+  const metis_nvfp4* rowwise;
+  const metis_nvfp4* colwise;
+  const metis_factors* f;
+} metis_operand;
+
+/*
+ * Forward GeMM (key design 1 equation):  Y = X_hat W_hat  (l x n)
+ *   X_hat = Q(A) L Q(B)^T + Q(X_R)_rowwise,   W_hat = Q(U) S Q(V)^T + Q(W_R)_colwise.
+ * Evaluated as one FP4 GeMM Q(X_R) Q(W_R) plus the rank-fold of the low-rank terms
+ * into the same accumulator.  Y has leading dimension ldy and type y_dtype.
+ */
+metis_status metis_linear_fwd(metis_ctx* ctx, const metis_operand* X, const metis_operand* W,
+                              void* Y, int64_t ldy, int32_t y_dtype);
+
+/*
+ * Backward GeMMs (framework section: the split is embedded in every forward and
+ * backward GeMM):  dX = D_hat W_hat^T  (l x m, type dx_dtype),  dW = X_hat^T D_hat
+ * (m x n, fp32).  D uses its row-wise residual for dX and column-wise for dW; W its
+ * row-wise residual; X its column-wise residual.
+ */
+metis_status metis_linear_bwd(metis_ctx* ctx, const metis_operand* X, const metis_operand* W,
+                              const metis_operand* D, void* dX, int64_t lddx, int32_t dx_dtype,
+                              float* dW, int64_t lddw);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* METIS_H */

@@ -100,3 +100,14 @@ def sr_uniforms(seed, operand_id, sub, step, n):
     words = element_words(seed, tag(operand_id, PURPOSE_SR, sub), step, (n + 1) // 2)
     halves = np.stack([words & np.uint64(0xFFFF), words >> np.uint64(16)], axis=-1).reshape(-1)[:n]
     return halves.astype(np.float64) / 65536.0
+
+
+def sr_uniforms_at(seed, operand_id, sub, step, elements):
+    """The same uniforms as ``sr_uniforms`` for arbitrary element indices."""
+    e = np.asarray(elements, dtype=np.uint64)
+    q = e >> np.uint64(3)
+    uq, inv = np.unique(q, return_inverse=True)
+    words = stream_words(seed, tag(operand_id, PURPOSE_SR, sub), step, uq)
+    w = words[inv, ((e >> np.uint64(1)) & np.uint64(3)).astype(np.int64)]
+    half = np.where((e & np.uint64(1)) == 1, w >> np.uint64(16), w & np.uint64(0xFFFF))
+    return half.astype(np.float64) / 65536.0

@@ -1,0 +1,237 @@
+"""Python binding of libmetis, the B200 implementation of the Metis W4A4G4 linear layer.
+
+Method: "Metis: Training LLMs with FP4 Quantization" (ICLR 2026; papernotes.org
+notes).  Every call here marshals arguments into the C ABI declared in
+``include/metis.h`` and runs on the GPU inside ``libmetis.so``; PyTorch only
+provides device memory and the current CUDA stream.  There is no CPU path: if
+the library is missing, importing this package fails.
+
+Typical use (one operand):
+
+    ctx = Context()
+    st = ctx.new_factors(rows, cols, k)
+    ctx.decompose(M, k=k, s=s, l_k=l_k, seed=0, operand_id=0, refresh=True, step=0, factors=st)
+    row, col = ctx.new_nvfp4(rows, cols), ctx.new_nvfp4(cols, rows)
+    ctx.residual_quantize_nvfp4(M, st, rowwise=row, colwise=col, rounding=1, seed=0, operand_id=0, step=0)
+"""
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmetis.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing; build it with `python -m spectral_quantized_gemm_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+c_i32, c_i64, c_u32, c_u64, c_f32, c_p = (ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_uint64,
+                                           ctypes.c_float, ctypes.c_void_p)
+
+METIS_OK = 0
+STATUS_NAMES = {0: "OK", 1: "ERR_ARG", 2: "ERR_SHAPE", 3: "ERR_ALIGN", 4: "ERR_ARCH", 5: "ERR_CUDA",
+                6: "ERR_WORKSPACE"}
+DEV_NUMERIC, DEV_NONFINITE, DEV_TIMEOUT = 1, 2, 4
+OUT_F32, OUT_BF16 = 0, 1
+
+EXPORTED = ["metis_create", "metis_destroy", "metis_set_stream", "metis_status_str", "metis_last_error",
+            "metis_poll_device_status", "metis_nvfp4_codes_bytes", "metis_nvfp4_scales_bytes",
+            "metis_decompose", "metis_residual_quantize_nvfp4", "metis_quantize_nvfp4_f32", "metis_gemm_nvfp4",
+            "metis_linear_fwd", "metis_linear_bwd"]
+
+
+class Matrix(ctypes.Structure):
+    _fields_ = [("data", c_p), ("rows", c_i64), ("cols", c_i64), ("ld", c_i64)]
+
+
+class Nvfp4Struct(ctypes.Structure):
+    _fields_ = [("codes", c_p), ("scales", c_p), ("tensor_scale", c_p), ("outer", c_i64), ("inner", c_i64)]
+
+
+class FactorsStruct(ctypes.Structure):
+    _fields_ = [("rows", c_i64), ("cols", c_i64), ("k", c_i32), ("V", c_p), ("U", c_p), ("S", c_p),
+                ("Uq", Nvfp4Struct), ("Vq", Nvfp4Struct), ("sampled_rows", c_p), ("omega", c_p)]
+
+
+class DecompParams(ctypes.Structure):
+    _fields_ = [("k", c_i32), ("s", c_i32), ("l_k", c_i32), ("seed", c_u64), ("operand_id", c_u32),
+                ("rounding", c_i32)]
+
+
+class QuantParams(ctypes.Structure):
+    _fields_ = [("rounding", c_i32), ("seed", c_u64), ("operand_id", c_u32), ("step", c_u32),
+                ("tensor_scale", c_f32)]
+
+
+class OperandStruct(ctypes.Structure):
+    _fields_ = [("rowwise", ctypes.POINTER(Nvfp4Struct)), ("colwise", ctypes.POINTER(Nvfp4Struct)),
+                ("f", ctypes.POINTER(FactorsStruct))]
+
+
+def _sig(name, restype, *args):
+    fn = getattr(_lib, name)
+    fn.restype = restype
+    fn.argtypes = list(args)
+    return fn
+
+
+_create = _sig("metis_create", c_i32, ctypes.c_int, c_p, ctypes.POINTER(c_p))
+_destroy = _sig("metis_destroy", None, c_p)
+_set_stream = _sig("metis_set_stream", c_i32, c_p, c_p)
+_status_str = _sig("metis_status_str", ctypes.c_char_p, c_i32)
+_last_error = _sig("metis_last_error", ctypes.c_char_p, c_p)
+_poll = _sig("metis_poll_device_status", c_i32, c_p, ctypes.POINTER(c_u32), ctypes.c_int)
+_codes_bytes = _sig("metis_nvfp4_codes_bytes", c_i64, c_i64, c_i64)
+_scales_bytes = _sig("metis_nvfp4_scales_bytes", c_i64, c_i64, c_i64)
+_decompose = _sig("metis_decompose", c_i32, c_p, ctypes.POINTER(Matrix), ctypes.POINTER(DecompParams),
+                  ctypes.c_int, c_u32, ctypes.POINTER(FactorsStruct))
+_resq = _sig("metis_residual_quantize_nvfp4", c_i32, c_p, ctypes.POINTER(Matrix), ctypes.POINTER(FactorsStruct),
+             ctypes.POINTER(QuantParams), ctypes.POINTER(Nvfp4Struct), ctypes.POINTER(Nvfp4Struct))
+_quant_f32 = _sig("metis_quantize_nvfp4_f32", c_i32, c_p, c_p, c_i64, c_i64, c_i64, ctypes.POINTER(QuantParams),
+                  ctypes.POINTER(Nvfp4Struct), ctypes.POINTER(Nvfp4Struct))
+_gemm = _sig("metis_gemm_nvfp4", c_i32, c_p, ctypes.POINTER(Nvfp4Struct), ctypes.POINTER(Nvfp4Struct), c_i64, c_p,
+             c_p, c_i32, c_p, c_p, c_i64, c_i32)
+_fwd = _sig("metis_linear_fwd", c_i32, c_p, ctypes.POINTER(OperandStruct), ctypes.POINTER(OperandStruct), c_p,
+            c_i64, c_i32)
+_bwd = _sig("metis_linear_bwd", c_i32, c_p, ctypes.POINTER(OperandStruct), ctypes.POINTER(OperandStruct),
+            ctypes.POINTER(OperandStruct), c_p, c_i64, c_i32, c_p, c_i64)
+
+
+class MetisError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+def status_str(status):
+    return _status_str(status).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+class Nvfp4:
+    """Device buffers of one NVFP4 tensor (outer x inner, blocks along inner)."""
+
+    def __init__(self, outer, inner, device="cuda"):
+        self.outer, self.inner = int(outer), int(inner)
+        self.codes = torch.zeros(int(_codes_bytes(outer, inner)), dtype=torch.uint8, device=device)
+        self.scales = torch.zeros(int(_scales_bytes(outer, inner)), dtype=torch.uint8, device=device)
+        self.tensor_scale = torch.ones(4, dtype=torch.float32, device=device)
+        self.struct = Nvfp4Struct(self.codes.data_ptr(), self.scales.data_ptr(), self.tensor_scale.data_ptr(),
+                                  self.outer, self.inner)
+
+
+class Factors:
+    """Caller-owned factor state of one operand: V (basis), U, S and their NVFP4 copies."""
+
+    def __init__(self, rows, cols, k, s=0, l_k=0, device="cuda", keep_sketch=False):
+        self.rows, self.cols, self.k = int(rows), int(cols), int(k)
+        self.V = torch.zeros(cols, k, dtype=torch.float32, device=device)
+        self.U = torch.zeros(rows, k, dtype=torch.float32, device=device)
+        self.S = torch.zeros(max(k, 1), dtype=torch.float32, device=device)
+        self.Uq = Nvfp4(128, rows, device)
+        self.Vq = Nvfp4(128, cols, device)
+        self.sampled_rows = torch.zeros(max(l_k, 1), dtype=torch.int32, device=device) if keep_sketch else None
+        self.omega = torch.zeros(cols, max(k + s, 1), dtype=torch.float32, device=device) if keep_sketch else None
+        self.struct = FactorsStruct(self.rows, self.cols, self.k, self.V.data_ptr(), self.U.data_ptr(),
+                                    self.S.data_ptr(), self.Uq.struct, self.Vq.struct,
+                                    None if self.sampled_rows is None else self.sampled_rows.data_ptr(),
+                                    None if self.omega is None else self.omega.data_ptr())
+
+
+def _matrix(M):
+    if M.dtype != torch.bfloat16 or M.dim() != 2 or M.stride(1) != 1:
+        raise ValueError("expected a row-major 2-D bf16 CUDA tensor")
+    return Matrix(M.data_ptr(), M.shape[0], M.shape[1], M.stride(0))
+
+
+class Context:
+    """A libmetis context bound to one device; work goes to torch's current stream."""
+
+    def __init__(self, device=None):
+        if not torch.cuda.is_available():
+            raise RuntimeError("libmetis needs a CUDA device (sm_100)")
+        self.device = torch.device("cuda", torch.cuda.current_device() if device is None else device)
+        handle = c_p()
+        st = _create(self.device.index, c_p(torch.cuda.current_stream(self.device).cuda_stream),
+                     ctypes.byref(handle))
+        if st != METIS_OK:
+            raise MetisError(st, status_str(st))
+        self._h = handle
+
+    def close(self):
+        if getattr(self, "_h", None):
+            _destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _call(self, fn, *args):
+        _set_stream(self._h, c_p(torch.cuda.current_stream(self.device).cuda_stream))
+        st = fn(self._h, *args)
+        if st != METIS_OK:
+            raise MetisError(st, _last_error(self._h).decode())
+
+    # -- allocation helpers ------------------------------------------------
+    def new_nvfp4(self, outer, inner):
+        return Nvfp4(outer, inner, self.device)
+
+    def new_factors(self, rows, cols, k, s=0, l_k=0, keep_sketch=False):
+        return Factors(rows, cols, k, s, l_k, self.device, keep_sketch)
+
+    # -- the C ABI ---------------------------------------------------------
+    def poll_device_status(self, clear=True):
+        bits = c_u32(0)
+        self._call(_poll, ctypes.byref(bits), int(clear))
+        return bits.value
+
+    def decompose(self, M, k, s, l_k, seed, operand_id, refresh, step, factors, rounding=0):
+        p = DecompParams(k, s, l_k, seed, operand_id, rounding)
+        self._call(_decompose, ctypes.byref(_matrix(M)), ctypes.byref(p), int(bool(refresh)), step,
+                   ctypes.byref(factors.struct))
+
+    def residual_quantize_nvfp4(self, M, factors, rowwise=None, colwise=None, rounding=0, seed=0, operand_id=0,
+                                step=0, tensor_scale=1.0):
+        q = QuantParams(rounding, seed, operand_id, step, tensor_scale)
+        self._call(_resq, ctypes.byref(_matrix(M)), None if factors is None else ctypes.byref(factors.struct),
+                   ctypes.byref(q), None if rowwise is None else ctypes.byref(rowwise.struct),
+                   None if colwise is None else ctypes.byref(colwise.struct))
+
+    def quantize_nvfp4_f32(self, R, rowwise=None, colwise=None, rounding=0, seed=0, operand_id=0, step=0,
+                           tensor_scale=1.0):
+        if R.dtype != torch.float32 or R.dim() != 2 or R.stride(1) != 1:
+            raise ValueError("expected a row-major 2-D fp32 CUDA tensor")
+        q = QuantParams(rounding, seed, operand_id, step, tensor_scale)
+        self._call(_quant_f32, _ptr(R), R.shape[0], R.shape[1], R.stride(0), ctypes.byref(q),
+                   None if rowwise is None else ctypes.byref(rowwise.struct),
+                   None if colwise is None else ctypes.byref(colwise.struct))
+
+    def gemm_nvfp4(self, A, B, n_cols, C, Fa=None, Fb=None, col_scale=None):
+        fold_k = 0 if Fa is None else Fa.shape[1]
+        dtype = OUT_F32 if C.dtype == torch.float32 else OUT_BF16
+        self._call(_gemm, ctypes.byref(A.struct), ctypes.byref(B.struct), n_cols, _ptr(Fa), _ptr(Fb), fold_k,
+                   _ptr(col_scale), _ptr(C), C.stride(0), dtype)
+
+    @staticmethod
+    def operand(rowwise=None, colwise=None, factors=None):
+        return OperandStruct(None if rowwise is None else ctypes.pointer(rowwise.struct),
+                             None if colwise is None else ctypes.pointer(colwise.struct),
+                             None if factors is None else ctypes.pointer(factors.struct))
+
+    def linear_fwd(self, X, W, Y):
+        dtype = OUT_F32 if Y.dtype == torch.float32 else OUT_BF16
+        self._call(_fwd, ctypes.byref(X), ctypes.byref(W), _ptr(Y), Y.stride(0), dtype)
+
+    def linear_bwd(self, X, W, D, dX, dW):
+        dtype = OUT_F32 if dX.dtype == torch.float32 else OUT_BF16
+        self._call(_bwd, ctypes.byref(X), ctypes.byref(W), ctypes.byref(D), _ptr(dX), dX.stride(0), dtype,
+                   _ptr(dW), dW.stride(0))

@@ -1,0 +1,167 @@
+// Device helpers shared by the libmetis kernels: Philox4x32-10, the E2M1/E4M3
+// conversions of the NVFP4 block quantizer, and the device status word.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/metis.h"
+
+namespace metis {
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11).  Counter (c0..c3), key
+// (k0, k1); ten rounds, the key bumped by the Weyl constants between rounds.
+// ---------------------------------------------------------------------------
+struct Words4 {
+  uint32_t w[4];
+};
+
+__device__ __forceinline__ Words4 philox10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+                                           uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t lo0 = 0xD2511F53u * c0;
+    const uint32_t hi0 = __umulhi(0xD2511F53u, c0);
+    const uint32_t lo1 = 0xCD9E8D57u * c2;
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2);
+    const uint32_t n0 = hi1 ^ c1 ^ k0;
+    const uint32_t n2 = hi0 ^ c3 ^ k1;
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+  }
+  Words4 out;
+  out.w[0] = c0;
+  out.w[1] = c1;
+  out.w[2] = c2;
+  out.w[3] = c3;
+  return out;
+}
+
+// Stream layout: key = seed, counter = (q lo, q hi, tag, step),
+// tag = operand_id << 8 | purpose << 4 | sub.
+enum : uint32_t { kPurposeSample = 1, kPurposeOmega = 2, kPurposeSR = 3 };
+enum : uint32_t { kSrRowwise = 0, kSrColwise = 1, kSrLeft = 2, kSrRight = 3 };
+
+__host__ __device__ __forceinline__ uint32_t stream_tag(uint32_t operand_id, uint32_t purpose,
+                                                        uint32_t sub) {
+  return ((operand_id & 0xFFFFFFu) << 8) | ((purpose & 0xFu) << 4) | (sub & 0xFu);
+}
+
+__device__ __forceinline__ Words4 stream_call(uint64_t seed, uint32_t tag, uint32_t step, uint64_t q) {
+  return philox10((uint32_t)q, (uint32_t)(q >> 32), tag, step, (uint32_t)seed,
+                  (uint32_t)(seed >> 32));
+}
+
+// ---------------------------------------------------------------------------
+// Format conversions.  PTX cvt with .rn.satfinite: round to nearest even,
+// saturating to the largest finite value; the packed destination takes the
+// first source operand in its upper half.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e4m3_code_rn(float x) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
+  return (uint32_t)(r & 0xFFu);
+}
+
+// Exact fp32 value of a non-negative E4M3 code (OCP fn).
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+  const uint32_t e = (code >> 3) & 0xFu;
+  const uint32_t m = code & 7u;
+  if (e == 0) return (float)m * 0.001953125f;  // m * 2^-9
+  // (8 + m) * 2^(e - 10), built from the exponent bits
+  const float p2 = __uint_as_float((e - 10u + 127u) << 23);
+  return (float)(8u + m) * p2;
+}
+
+// Two fp32 values already on (or to be rounded to) the E2M1 grid -> one byte,
+// `lo` in bits 0-3 and `hi` in bits 4-7.
+__device__ __forceinline__ uint32_t e2m1x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+      : "=r"(r)
+      : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Stochastic rounding of a scaled value onto the E2M1 grid (sign kept):
+// magnitude a >= 6 gives 6; otherwise lo <= a < hi are grid neighbours and the
+// magnitude rounds up iff u < (a - lo) / (hi - lo).  All steps are exact.
+__device__ __forceinline__ float e2m1_sr_value(float x, float u) {
+  const float a = fabsf(x);
+  float q;
+  if (a >= 6.0f) {
+    q = 6.0f;
+  } else {
+    const float h = a < 2.0f ? 0.5f : (a < 4.0f ? 1.0f : 2.0f);
+    const float inv_h = a < 2.0f ? 2.0f : (a < 4.0f ? 1.0f : 0.5f);
+    const float t = a * inv_h;
+    const float fl = floorf(t);
+    const float p = t - fl;
+    q = (u < p ? fl + 1.0f : fl) * h;
+  }
+  return copysignf(q, x);
+}
+
+// Uniform of element e (16-bit half e&1 of word (e>>1)&3 of counter e>>3).
+__device__ __forceinline__ float sr_uniform_from_words(const Words4& w, uint32_t e_in_call) {
+  const uint32_t word = w.w[(e_in_call >> 1) & 3u];
+  const uint32_t half = (e_in_call & 1u) ? (word >> 16) : (word & 0xFFFFu);
+  return (float)half * (1.0f / 65536.0f);
+}
+
+// Byte offset of the scale of (row o, block b) inside the tiled scale array of
+// an NVFP4 tensor whose inner dimension has `kb_tiles` = inner/64 tiles.
+__host__ __device__ __forceinline__ int64_t scale_offset(int64_t o, int64_t b, int64_t kb_tiles) {
+  return ((o >> 7) * kb_tiles + (b >> 2)) * 512 + (o & 31) * 16 + ((o & 127) >> 5) * 4 + (b & 3);
+}
+
+// ---------------------------------------------------------------------------
+// NVFP4 block rule.  Given the block maximum and the tensor scale g, returns
+// the E4M3 scale code and the fp32 reciprocal of the decode scale d = s*g.
+// ---------------------------------------------------------------------------
+struct BlockScale {
+  uint32_t code;
+  float rcp;  // 1 / (s * g), IEEE round-to-nearest; 0 for an all-zero block
+};
+
+__device__ __forceinline__ BlockScale block_scale(float amax, float g) {
+  BlockScale bs;
+  const float target = __fdiv_rn(amax, __fmul_rn(6.0f, g));
+  uint32_t code = e4m3_code_rn(target);
+  if (amax > 0.0f && code == 0) code = 1;  // smallest E4M3 value 2^-9
+  bs.code = code;
+  bs.rcp = code ? __frcp_rn(__fmul_rn(e4m3_value(code), g)) : 0.0f;
+  return bs;
+}
+
+// Encodes 16 fp32 values of one block (already multiplied by the reciprocal
+// scale) into 8 bytes (two uint32).  rounding: 0 RN, 1 SR with uniforms u.
+__device__ __forceinline__ uint2 encode16(const float (&x)[16], int rounding, const float* u) {
+  uint32_t b[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float lo = x[2 * i], hi = x[2 * i + 1];
+    if (rounding) {
+      lo = e2m1_sr_value(lo, u[2 * i]);
+      hi = e2m1_sr_value(hi, u[2 * i + 1]);
+    }
+    b[i] = e2m1x2_rn(lo, hi);
+  }
+  uint2 r;
+  r.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+  r.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+  return r;
+}
+
+__device__ __forceinline__ void raise_status(uint32_t* status, uint32_t bits) {
+  if (status) atomicOr(status, bits);
+}
+
+}  // namespace metis

@@ -1,0 +1,388 @@
+// Block-scaled NVFP4 GeMM on the sm_100a tensor cores, with the Metis rank-fold.
+//
+// Method: "Metis: Training LLMs with FP4 Quantization" (papernotes.org notes),
+// key design 1.  Expanding the forward equation around the residual product,
+//   (L_A S_A R_A^T + A_R)(L_B S_B R_B^T + B_R)
+//     = A_R B_R + [L_A | T_B] [T_A ; R_B^T],
+//   T_A = S_A R_A^T (B_R + L_B S_B R_B^T),   T_B = A_R L_B S_B,
+// so every GeMM of the layer is one FP4 x FP4 product plus a rank-2k bf16
+// product.  This kernel runs both into the same fp32 tensor-memory accumulator:
+// the K loop streams NVFP4 stages (tcgen05 kind::mxf4nvf4, block16 UE4M3 scales)
+// and then the fold stages (kind::f16, bf16 operands) through one shared-memory
+// ring, and the epilogue scales by alpha (and an optional per-column factor).
+//
+// Structure (one CTA per SM, persistent over 128 x BN output tiles):
+//   warp 0      TMA producer: A/B tiles (128-byte swizzle), scale tiles (bulk copy)
+//   warp 1      tensor-memory owner and MMA issuer (one thread)
+//   warps 2..9  epilogue: tcgen05.ld of the accumulator, scale, store
+// Every mbarrier wait is bounded; on expiry the CTA raises METIS_DEV_TIMEOUT,
+// stops issuing work and exits after releasing its tensor memory.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "device_common.cuh"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace metis {
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kEpiWarps = 8;
+
+template <int BN>
+struct Cfg {
+  static constexpr int BM = 128;
+  static constexpr int A_BYTES = BM * 128;                // one 128-byte swizzle row per matrix row
+  static constexpr int B_BYTES = BN * 128;
+  static constexpr int SFB_ATOMS = BN > 128 ? 2 : 1;      // 128-row scale tiles of B
+  static constexpr int SFA_BYTES = 4 * 512;               // 4 k-tiles of 64 per 256-element stage
+  static constexpr int SFB_BYTES = SFB_ATOMS * 4 * 512;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int SF_STAGE_BYTES = SFA_BYTES + SFB_BYTES;
+  static constexpr int STAGES = BN > 128 ? 4 : 6;
+  static constexpr int ACC_COLS = BN;
+  static constexpr int SFA_COL = ACC_COLS;                // 4 columns per MMA k-step
+  static constexpr int SFB_COLS_PER_K = SFB_ATOMS * 4;
+  static constexpr int SFB_COL = SFA_COL + 16;
+  static constexpr int USED_COLS = SFB_COL + 4 * SFB_COLS_PER_K;
+  static constexpr int TMEM_COLS = USED_COLS <= 32 ? 32 : USED_COLS <= 64 ? 64 : USED_COLS <= 128 ? 128
+                                   : USED_COLS <= 256 ? 256 : 512;
+  static constexpr size_t SMEM = (size_t)STAGES * (STAGE_BYTES + SF_STAGE_BYTES) + 1024 + 256;
+  static_assert(USED_COLS <= 512, "tensor memory budget");
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+struct Params {
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  int64_t kb_tiles;  // K / 64: scale tiles per 128-row block
+  const float* ga;
+  const float* gb;
+  float alpha_extra;
+  const float* col_scale;
+  void* C;
+  int64_t ldc;
+  int c_dtype;
+  int m_tiles, n_tiles;
+  int k_stages, fold_stages;
+  uint32_t* status;
+};
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                      const __grid_constant__ CUtensorMap mapFa, const __grid_constant__ CUtensorMap mapFb,
+                      const Params p) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* tiles = smem;
+  uint8_t* sf = smem + C::STAGES * C::STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sf + C::STAGES * C::SF_STAGE_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + C::STAGES;
+  uint64_t* tmem_full = bars + 2 * C::STAGES;
+  uint64_t* tmem_empty = tmem_full + 1;
+  uint64_t* drain = tmem_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_full + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::mbar_init(tmem_full, 1);
+    tc::mbar_init(tmem_empty, kEpiWarps);
+    tc::mbar_init(drain, 1);
+    *abort_flag = 0;
+    tc::fence_barrier_init();
+    tc::prefetch_tensormap(&mapA);
+    tc::prefetch_tensormap(&mapB);
+    if (p.fold_stages) {
+      tc::prefetch_tensormap(&mapFa);
+      tc::prefetch_tensormap(&mapFb);
+    }
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int num_tiles = p.m_tiles * p.n_tiles;
+  const int total_stages = p.k_stages + p.fold_stages;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
+        const int mb = tile % p.m_tiles;
+        const int nb = tile / p.m_tiles;
+        for (int kk = 0; kk < total_stages; ++kk) {
+          if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+            *abort_flag = 1;
+            raise_status(p.status, METIS_DEV_TIMEOUT);
+            break;
+          }
+          uint8_t* sA = tiles + stage * C::STAGE_BYTES;
+          uint8_t* sB = sA + C::A_BYTES;
+          if (kk < p.k_stages) {
+            uint8_t* sSFA = sf + stage * C::SF_STAGE_BYTES;
+            uint8_t* sSFB = sSFA + C::SFA_BYTES;
+            tc::mbar_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES + C::SFA_BYTES + C::SFB_BYTES);
+            tc::tma_load_2d(sA, &mapA, &full[stage], kk * 128, mb * 128);
+            tc::tma_load_2d(sB, &mapB, &full[stage], kk * 128, nb * BN);
+            tc::bulk_load(sSFA, p.sfa + ((int64_t)mb * p.kb_tiles + kk * 4) * 512, C::SFA_BYTES, &full[stage]);
+            const int64_t nb128 = (int64_t)nb * BN / 128;
+#pragma unroll
+            for (int a = 0; a < C::SFB_ATOMS; ++a)
+              tc::bulk_load(sSFB + a * 2048, p.sfb + ((nb128 + a) * p.kb_tiles + kk * 4) * 512, 2048,
+                            &full[stage]);
+          } else {
+            const int f = kk - p.k_stages;
+            tc::mbar_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES);
+            tc::tma_load_2d(sA, &mapFa, &full[stage], f * 64, mb * 128);
+            tc::tma_load_2d(sB, &mapFb, &full[stage], f * 64, nb * BN);
+          }
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t acc_phase = 0;
+      const uint32_t id_fp4 = tc::idesc_nvf4(BN);
+      const uint32_t id_bf16 = tc::idesc_bf16(BN);
+      const uint32_t t_acc = tmem;
+      const uint32_t t_sfa = tmem + C::SFA_COL;
+      const uint32_t t_sfb = tmem + C::SFB_COL;
+      for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
+        if (!tc::mbar_wait(tmem_empty, acc_phase ^ 1u, abort_flag)) {
+          *abort_flag = 1;
+          raise_status(p.status, METIS_DEV_TIMEOUT);
+          break;
+        }
+        tc::tc_fence_after();
+        for (int kk = 0; kk < total_stages; ++kk) {
+          if (!tc::mbar_wait(&full[stage], phase, abort_flag)) {
+            *abort_flag = 1;
+            raise_status(p.status, METIS_DEV_TIMEOUT);
+            break;
+          }
+          tc::tc_fence_after();
+          const uint8_t* sA = tiles + stage * C::STAGE_BYTES;
+          const uint8_t* sB = sA + C::A_BYTES;
+          const uint64_t adesc = tc::sdesc_sw128(tc::smem_addr(sA));
+          const uint64_t bdesc = tc::sdesc_sw128(tc::smem_addr(sB));
+          if (kk < p.k_stages) {
+            const uint8_t* sSFA = sf + stage * C::SF_STAGE_BYTES;
+            const uint8_t* sSFB = sSFA + C::SFA_BYTES;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              tc::tc_copy_32x128b_x4(t_sfa + 4 * j, tc::sdesc_scales(tc::smem_addr(sSFA + 512 * j)));
+#pragma unroll
+              for (int a = 0; a < C::SFB_ATOMS; ++a)
+                tc::tc_copy_32x128b_x4(t_sfb + C::SFB_COLS_PER_K * j + 4 * a,
+                                       tc::sdesc_scales(tc::smem_addr(sSFB + 2048 * a + 512 * j)));
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              tc::mma_nvf4(t_acc, adesc + 2 * j, bdesc + 2 * j, id_fp4, t_sfa + 4 * j,
+                           t_sfb + C::SFB_COLS_PER_K * j, (kk | j) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              tc::mma_bf16(t_acc, adesc + 2 * j, bdesc + 2 * j, id_bf16, (kk | j) ? 1u : 0u);
+          }
+          tc::tc_commit(&empty[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (*abort_flag) break;
+        tc::tc_commit(tmem_full);
+        acc_phase ^= 1u;
+      }
+      // let every issued tensor-core operation finish before the memory is released
+      tc::tc_commit(drain);
+      tc::mbar_wait(drain, 0, nullptr);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                 // tensor-memory lane quarter of this warp
+    const int h = (warp - 2) >> 2;          // column half
+    constexpr int kColsPerWarp = BN >= 64 ? BN / 2 : BN;
+    const bool active = BN >= 64 || h == 0;
+    const float alpha = (*p.ga) * (*p.gb) * p.alpha_extra;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(tmem_full, acc_phase, abort_flag));
+      if (!ok) {
+        if (lane == 0) {
+          *abort_flag = 1;
+          raise_status(p.status, METIS_DEV_TIMEOUT);
+        }
+        break;
+      }
+      tc::tc_fence_after();
+      const int mb = tile % p.m_tiles;
+      const int nb = tile / p.m_tiles;
+      float v[kColsPerWarp];
+      const int col0 = active ? h * kColsPerWarp : 0;
+      if (active) {
+#pragma unroll
+        for (int c = 0; c < kColsPerWarp; c += 16) {
+          float t[16];
+          uint32_t r[16];
+          const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(col0 + c);
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+              "%13, %14, %15}, [%16];"
+              : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+                "=r"(r[15])
+              : "r"(taddr));
+#pragma unroll
+          for (int i = 0; i < 16; ++i) t[i] = __uint_as_float(r[i]);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[c + i] = t[i];
+        }
+        tc::tmem_load_wait();
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(tmem_empty);
+      if (active) {
+        const int64_t row = (int64_t)mb * 128 + q * 32 + lane;
+        const int64_t cbase = (int64_t)nb * BN + col0;
+        if (p.c_dtype == METIS_OUT_F32) {
+          float* dst = reinterpret_cast<float*>(p.C) + row * p.ldc + cbase;
+#pragma unroll
+          for (int c = 0; c < kColsPerWarp; c += 4) {
+            float4 o;
+            o.x = v[c] * alpha * (p.col_scale ? p.col_scale[cbase + c] : 1.0f);
+            o.y = v[c + 1] * alpha * (p.col_scale ? p.col_scale[cbase + c + 1] : 1.0f);
+            o.z = v[c + 2] * alpha * (p.col_scale ? p.col_scale[cbase + c + 2] : 1.0f);
+            o.w = v[c + 3] * alpha * (p.col_scale ? p.col_scale[cbase + c + 3] : 1.0f);
+            *reinterpret_cast<float4*>(dst + c) = o;
+          }
+        } else {
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.C) + row * p.ldc + cbase;
+#pragma unroll
+          for (int c = 0; c < kColsPerWarp; c += 8) {
+            uint4 o;
+            uint32_t* w = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float a = v[c + 2 * i] * alpha * (p.col_scale ? p.col_scale[cbase + c + 2 * i] : 1.0f);
+              const float b = v[c + 2 * i + 1] * alpha * (p.col_scale ? p.col_scale[cbase + c + 2 * i + 1] : 1.0f);
+              const __nv_bfloat162 pr = __floats2bfloat162_rn(a, b);
+              w[i] = *reinterpret_cast<const uint32_t*>(&pr);
+            }
+            *reinterpret_cast<uint4*>(dst + c) = o;
+          }
+        }
+      }
+      acc_phase ^= 1u;
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+bool make_map_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t inner, uint64_t outer,
+                 uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  return enc(map, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN>
+metis_status launch_bn(metis_ctx* ctx, const GemmArgs& a) {
+  using C = Cfg<BN>;
+  const int64_t p_rows = a.A->outer;
+  const int64_t K = a.A->inner;
+  const int64_t q_cols = a.q_cols;
+  CUtensorMap mA, mB, mFa, mFb;
+  if (!make_map_2d(&mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.A->codes, K / 2, p_rows, K / 2, 128, 128) ||
+      !make_map_2d(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.B->codes, K / 2, a.B->outer, K / 2, 128, BN))
+    return fail(ctx, METIS_ERR_CUDA, "cuTensorMapEncodeTiled failed for the NVFP4 operands");
+  if (a.fold_k > 0) {
+    if (!make_map_2d(&mFa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.Fa, a.fold_k, p_rows, (uint64_t)a.fold_k * 2, 64,
+                     128) ||
+        !make_map_2d(&mFb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.Fb, a.fold_k, a.B->outer, (uint64_t)a.fold_k * 2,
+                     64, BN))
+      return fail(ctx, METIS_ERR_CUDA, "cuTensorMapEncodeTiled failed for the fold operands");
+  } else {
+    mFa = mA;
+    mFb = mB;
+  }
+  Params prm;
+  prm.sfa = a.A->scales;
+  prm.sfb = a.B->scales;
+  prm.kb_tiles = K / 64;
+  prm.ga = a.A->tensor_scale;
+  prm.gb = a.B->tensor_scale;
+  prm.alpha_extra = a.alpha_extra;
+  prm.col_scale = a.col_scale;
+  prm.C = a.C;
+  prm.ldc = a.ldc;
+  prm.c_dtype = a.c_dtype;
+  prm.m_tiles = (int)(p_rows / 128);
+  prm.n_tiles = (int)(q_cols / BN);
+  prm.k_stages = (int)(K / 256);
+  prm.fold_stages = a.fold_k / 64;
+  prm.status = ctx->status;
+  auto kern = gemm_nvfp4_kernel<BN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  if (e != cudaSuccess) return check_cuda(ctx, e, "cudaFuncSetAttribute(gemm)");
+  const int tiles = prm.m_tiles * prm.n_tiles;
+  const int grid = std::min(tiles, ctx->sm_count);
+  kern<<<grid, kThreads, C::SMEM, ctx->stream>>>(mA, mB, mFa, mFb, prm);
+  return check_cuda(ctx, cudaGetLastError(), "gemm_nvfp4 launch");
+}
+
+}  // namespace
+
+metis_status launch_gemm_nvfp4(metis_ctx* ctx, const GemmArgs& a) {
+  if (a.q_cols % 256 == 0) return launch_bn<256>(ctx, a);
+  if (a.q_cols == 64) return launch_bn<64>(ctx, a);
+  if (a.q_cols == 32) return launch_bn<32>(ctx, a);
+  if (a.q_cols == 16) return launch_bn<16>(ctx, a);
+  return fail(ctx, METIS_ERR_SHAPE, "GeMM output columns must be a multiple of 256 or one of 16, 32, 64");
+}
+
+}  // namespace metis

@@ -1,0 +1,83 @@
+// Host-side internals of libmetis: the context, workspace and kernel launchers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <string>
+
+#include "../../include/metis.h"
+
+struct metis_ctx {
+  int device = 0;
+  cudaStream_t stream = nullptr;
+  int sm_count = 0;
+  uint32_t* status = nullptr;  // device status word (METIS_DEV_* bits)
+  char* ws = nullptr;          // device workspace, grown on demand
+  size_t ws_bytes = 0;
+  std::string last_error;
+};
+
+namespace metis {
+
+// Sub-allocator over the context workspace: hands out 256-byte aligned slices.
+struct Workspace {
+  char* base;
+  size_t cap;
+  size_t used = 0;
+  void* take(size_t bytes) {
+    size_t off = (used + 255) & ~size_t(255);
+    if (off + bytes > cap) return nullptr;
+    used = off + bytes;
+    return base + off;
+  }
+};
+
+metis_status ensure_workspace(metis_ctx* ctx, size_t bytes);
+metis_status fail(metis_ctx* ctx, metis_status s, const std::string& msg);
+metis_status check_cuda(metis_ctx* ctx, cudaError_t e, const char* what);
+
+// cuTensorMapEncodeTiled, fetched from the driver through the runtime.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled();
+
+// ---- quantize.cu ----
+cudaError_t launch_quantize_f32(const float* R, int64_t rows, int64_t cols, int64_t ld,
+                                const metis_quant_params& q, const metis_nvfp4* rowwise,
+                                const metis_nvfp4* colwise, uint32_t* status, cudaStream_t st);
+cudaError_t launch_residual_f32(const void* M_bf16, int64_t rows, int64_t cols, int64_t ld, const float* U,
+                                const float* S, const float* V, int32_t k, float* out, uint32_t* status,
+                                cudaStream_t st);
+cudaError_t launch_quantize_factor(const float* F, int64_t longdim, int32_t k, int32_t rounding, uint64_t seed,
+                                   uint32_t operand_id, uint32_t sub, uint32_t step, const metis_nvfp4* out,
+                                   float* amax_scratch, uint32_t* status, cudaStream_t st);
+
+// ---- gemm_fp4.cu ----
+struct GemmArgs {
+  const metis_nvfp4* A;
+  const metis_nvfp4* B;
+  const void* Fa;
+  const void* Fb;
+  int32_t fold_k;
+  const float* col_scale;
+  void* C;
+  int64_t ldc;
+  int32_t c_dtype;
+  float alpha_extra;  // multiplies alpha = gA * gB (1.0 normally)
+  int64_t q_cols;     // output columns: a multiple of 256, or 16 / 32 / 64 (thin)
+};
+metis_status launch_gemm_nvfp4(metis_ctx* ctx, const GemmArgs& a);
+
+// ---- decompose.cu ----
+metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_decomp_params* p, int refresh,
+                           uint32_t step, metis_factors* f);
+
+// ---- layer.cu ----
+metis_status run_linear(metis_ctx* ctx, const metis_operand* A, const metis_nvfp4* A_res, const metis_operand* B,
+                        const metis_nvfp4* B_res, bool a_transposed_factors, bool b_transposed_factors, void* C,
+                        int64_t ldc, int32_t c_dtype);
+
+}  // namespace metis

@@ -1,0 +1,279 @@
+// NVFP4 block quantization kernels.
+//
+// Method: "Metis: Training LLMs with FP4 Quantization" (papernotes.org notes),
+// background section (NVFP4: E2M1 values, 16-element blocks, one FP8 scale per
+// block from the block maximum) and training strategy (W4A4G4, stochastic
+// rounding on by default).  The block rule:
+//   s = E4M3_RN(amax / (6 g)) (2^-9 if that rounds to 0 for a non-zero block),
+//   x = v * RN(1 / (s g)),  code = E2M1_RN(x) or stochastic rounding of x.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "device_common.cuh"
+#include "internal.h"
+
+namespace metis {
+namespace {
+
+// One thread per 16-element block of the row-wise view (blocks along columns).
+__global__ void quantize_rowwise_f32_kernel(const float* __restrict__ R, int64_t rows, int64_t cols, int64_t ld,
+                                            float g, int rounding, uint64_t seed, uint32_t tag, uint32_t step,
+                                            uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                            float* tensor_scale, uint32_t* status) {
+  const int64_t nblk_row = cols / 16;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx == 0 && tensor_scale) *tensor_scale = g;
+  if (idx >= rows * nblk_row) return;
+  const int64_t o = idx / nblk_row;
+  const int64_t b = idx - o * nblk_row;
+  const float4* src = reinterpret_cast<const float4*>(R + o * ld + b * 16);
+  float v[16];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float4 t = src[i];
+    v[4 * i] = t.x;
+    v[4 * i + 1] = t.y;
+    v[4 * i + 2] = t.z;
+    v[4 * i + 3] = t.w;
+  }
+  float amax = 0.0f;
+  bool finite = true;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    finite &= isfinite(v[i]);
+    amax = fmaxf(amax, fabsf(v[i]));
+  }
+  if (!finite) raise_status(status, METIS_DEV_NONFINITE);
+  const BlockScale bs = block_scale(amax, g);
+  float x[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) x[i] = __fmul_rn(v[i], bs.rcp);
+  float u[16];
+  if (rounding) {
+    const uint64_t e0 = (uint64_t)o * (uint64_t)cols + (uint64_t)b * 16;
+    const Words4 w0 = stream_call(seed, tag, step, e0 >> 3);
+    const Words4 w1 = stream_call(seed, tag, step, (e0 >> 3) + 1);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      u[i] = sr_uniform_from_words(w0, i);
+      u[8 + i] = sr_uniform_from_words(w1, i);
+    }
+  }
+  uint2 packed = encode16(x, rounding, u);
+  if (bs.code == 0) packed = make_uint2(0, 0);
+  *reinterpret_cast<uint2*>(codes + o * (cols / 2) + b * 8) = packed;
+  scales[scale_offset(o, b, cols / 64)] = (uint8_t)bs.code;
+}
+
+// One thread per 16-row block of one column (column-wise view, blocks along rows).
+// Consecutive threads take consecutive columns so the loads coalesce.
+__global__ void quantize_colwise_f32_kernel(const float* __restrict__ R, int64_t rows, int64_t cols, int64_t ld,
+                                            float g, int rounding, uint64_t seed, uint32_t tag, uint32_t step,
+                                            uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                            float* tensor_scale, uint32_t* status) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx == 0 && tensor_scale) *tensor_scale = g;
+  const int64_t nblk = rows / 16;
+  if (idx >= nblk * cols) return;
+  const int64_t b = idx / cols;   // block along rows
+  const int64_t j = idx - b * cols;  // column = outer index of the transposed view
+  float v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = R[(b * 16 + i) * ld + j];
+  float amax = 0.0f;
+  bool finite = true;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    finite &= isfinite(v[i]);
+    amax = fmaxf(amax, fabsf(v[i]));
+  }
+  if (!finite) raise_status(status, METIS_DEV_NONFINITE);
+  const BlockScale bs = block_scale(amax, g);
+  float x[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) x[i] = __fmul_rn(v[i], bs.rcp);
+  float u[16];
+  if (rounding) {
+    const uint64_t e0 = (uint64_t)j * (uint64_t)rows + (uint64_t)b * 16;
+    const Words4 w0 = stream_call(seed, tag, step, e0 >> 3);
+    const Words4 w1 = stream_call(seed, tag, step, (e0 >> 3) + 1);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      u[i] = sr_uniform_from_words(w0, i);
+      u[8 + i] = sr_uniform_from_words(w1, i);
+    }
+  }
+  uint2 packed = encode16(x, rounding, u);
+  if (bs.code == 0) packed = make_uint2(0, 0);
+  *reinterpret_cast<uint2*>(codes + j * (rows / 2) + b * 8) = packed;
+  scales[scale_offset(j, b, rows / 64)] = (uint8_t)bs.code;
+}
+
+// out = fp32(M - (U diag(S)) V^T), a 64 x 64 tile per block, 4 x 4 per thread.
+__global__ void residual_f32_kernel(const __nv_bfloat16* __restrict__ M, int64_t rows, int64_t cols, int64_t ld,
+                                    const float* __restrict__ U, const float* __restrict__ S,
+                                    const float* __restrict__ V, int k, float* __restrict__ out) {
+  __shared__ float us[64][65];
+  __shared__ float vs[64][65];
+  const int64_t r0 = (int64_t)blockIdx.y * 64;
+  const int64_t c0 = (int64_t)blockIdx.x * 64;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4] = {};
+  for (int t0 = 0; t0 < k; t0 += 64) {
+    const int kt = min(64, k - t0);
+    for (int i = threadIdx.x; i < 64 * 64; i += blockDim.x) {
+      const int r = i / 64, t = i % 64;
+      us[r][t] = t < kt ? U[(r0 + r) * k + t0 + t] * S[t0 + t] : 0.0f;
+      vs[r][t] = t < kt ? V[(c0 + r) * k + t0 + t] : 0.0f;
+    }
+    __syncthreads();
+    for (int t = 0; t < kt; ++t) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        a[i] = us[ty * 4 + i][t];
+        b[i] = vs[tx * 4 + i][t];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t r = r0 + ty * 4 + i;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t c = c0 + tx * 4 + j;
+      out[r * cols + c] = __bfloat162float(M[r * ld + c]) - acc[i][j];
+    }
+  }
+}
+
+__global__ void absmax_kernel(const float* __restrict__ F, int64_t n, unsigned int* amax_bits, uint32_t* status) {
+  float m = 0.0f;
+  bool finite = true;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const float v = F[i];
+    finite &= isfinite(v);
+    m = fmaxf(m, fabsf(v));
+  }
+  if (!finite) raise_status(status, METIS_DEV_NONFINITE);
+#pragma unroll
+  for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if ((threadIdx.x & 31) == 0) atomicMax(amax_bits, __float_as_uint(m));
+}
+
+// Smallest power of two >= t (t >= 0 finite); 1 for t == 0.
+__device__ __forceinline__ float pow2_ceil(float t) {
+  if (!(t > 0.0f)) return 1.0f;
+  const uint32_t bits = __float_as_uint(t);
+  const uint32_t e = bits >> 23, m = bits & 0x7FFFFFu;
+  if (e == 0) {  // subnormal: t = m * 2^-149
+    const uint32_t top = 31u - __clz(m);
+    const uint32_t p = (m & (m - 1)) ? top + 1 : top;
+    return p >= 23 ? __uint_as_float(1u << 23) : __uint_as_float(1u << p);
+  }
+  if (m == 0) return t;
+  return __uint_as_float((e + 1) << 23);
+}
+
+// Factor F (long x k, fp32 row-major) -> NVFP4 of F^T (outer 128, inner long),
+// rows >= k written as zeros.  One thread per (row of F^T, 16-block).
+__global__ void quantize_factor_kernel(const float* __restrict__ F, int64_t longdim, int k, int rounding,
+                                       uint64_t seed, uint32_t tag, uint32_t step,
+                                       const unsigned int* __restrict__ amax_bits, uint8_t* __restrict__ codes,
+                                       uint8_t* __restrict__ scales, float* tensor_scale) {
+  const float amax_all = __uint_as_float(*amax_bits);
+  const float g = pow2_ceil(__fdiv_rn(amax_all, 2688.0f));
+  const int64_t nblk = longdim / 16;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx == 0) *tensor_scale = g;
+  if (idx >= 128 * nblk) return;
+  const int64_t j = idx / nblk;
+  const int64_t b = idx - j * nblk;
+  uint2 packed = make_uint2(0, 0);
+  uint32_t code = 0;
+  if (j < k) {
+    float v[16];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      v[i] = F[(b * 16 + i) * k + j];
+      amax = fmaxf(amax, fabsf(v[i]));
+    }
+    const BlockScale bs = block_scale(amax, g);
+    float x[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) x[i] = __fmul_rn(v[i], bs.rcp);
+    float u[16];
+    if (rounding) {
+      const uint64_t e0 = (uint64_t)j * (uint64_t)longdim + (uint64_t)b * 16;
+      const Words4 w0 = stream_call(seed, tag, step, e0 >> 3);
+      const Words4 w1 = stream_call(seed, tag, step, (e0 >> 3) + 1);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        u[i] = sr_uniform_from_words(w0, i);
+        u[8 + i] = sr_uniform_from_words(w1, i);
+      }
+    }
+    packed = encode16(x, rounding, u);
+    if (bs.code == 0) packed = make_uint2(0, 0);
+    code = bs.code;
+  }
+  *reinterpret_cast<uint2*>(codes + j * (longdim / 2) + b * 8) = packed;
+  scales[scale_offset(j, b, longdim / 64)] = (uint8_t)code;
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_f32(const float* R, int64_t rows, int64_t cols, int64_t ld,
+                                const metis_quant_params& q, const metis_nvfp4* rowwise,
+                                const metis_nvfp4* colwise, uint32_t* status, cudaStream_t st) {
+  const int threads = 256;
+  if (rowwise) {
+    const int64_t n = rows * (cols / 16);
+    quantize_rowwise_f32_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, st>>>(
+        R, rows, cols, ld, q.tensor_scale, q.rounding, q.seed, stream_tag(q.operand_id, kPurposeSR, kSrRowwise),
+        q.step, rowwise->codes, rowwise->scales, rowwise->tensor_scale, status);
+  }
+  if (colwise) {
+    const int64_t n = (rows / 16) * cols;
+    quantize_colwise_f32_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, st>>>(
+        R, rows, cols, ld, q.tensor_scale, q.rounding, q.seed, stream_tag(q.operand_id, kPurposeSR, kSrColwise),
+        q.step, colwise->codes, colwise->scales, colwise->tensor_scale, status);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_residual_f32(const void* M_bf16, int64_t rows, int64_t cols, int64_t ld, const float* U,
+                                const float* S, const float* V, int32_t k, float* out, uint32_t* status,
+                                cudaStream_t st) {
+  (void)status;
+  dim3 grid((unsigned)(cols / 64), (unsigned)(rows / 64));
+  residual_f32_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(M_bf16), rows, cols, ld, U, S,
+                                            V, k, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_factor(const float* F, int64_t longdim, int32_t k, int32_t rounding, uint64_t seed,
+                                   uint32_t operand_id, uint32_t sub, uint32_t step, const metis_nvfp4* out,
+                                   float* amax_scratch, uint32_t* status, cudaStream_t st) {
+  unsigned int* amax_bits = reinterpret_cast<unsigned int*>(amax_scratch);
+  cudaError_t e = cudaMemsetAsync(amax_bits, 0, sizeof(unsigned int), st);
+  if (e != cudaSuccess) return e;
+  const int64_t n = longdim * k;
+  const int blocks = (int)std::min<int64_t>((n + 255) / 256, 1024);
+  absmax_kernel<<<blocks, 256, 0, st>>>(F, n, amax_bits, status);
+  const int64_t nthreads = 128 * (longdim / 16);
+  quantize_factor_kernel<<<(unsigned)((nthreads + 255) / 256), 256, 0, st>>>(
+      F, longdim, k, rounding, seed, stream_tag(operand_id, kPurposeSR, sub), step, amax_bits, out->codes,
+      out->scales, out->tensor_scale);
+  return cudaGetLastError();
+}
+
+}  // namespace metis

@@ -1,0 +1,135 @@
+"""GPU randomized decomposition vs the oracle.
+
+Contract (the benchmark spec): identical sampled rows, the same Gaussian test matrix
+(within 1 fp32 ulp: both sides evaluate Box-Muller in fp64), and subspace
+cosines >= 0.999 for the recovered basis and factors.  Factor quantization is
+bit-exact given the GPU's own fp32 factors.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import decompose, linalg, metis, philox
+from tests.gpu_helpers import codes_unpacked
+from workloads import synth
+
+pytestmark = pytest.mark.gpu
+COS = 0.999
+
+
+def _gpu_decompose(ctx, M, k, s, l_k, seed, op, refresh=True, step=0, factors=None, rounding=0):
+    rows, cols = M.shape
+    f = factors or ctx.new_factors(rows, cols, k, s, l_k, keep_sketch=True)
+    ctx.decompose(M, k=k, s=s, l_k=l_k, seed=seed, operand_id=op, refresh=refresh, step=step, factors=f,
+                  rounding=rounding)
+    torch.cuda.synchronize()
+    return f
+
+
+def _compare(ctx, cfg, name, k, s, l_k, op, seed):
+    Mt = synth.operand_matrix(cfg, name)
+    M = Mt.double().numpy()
+    f = _gpu_decompose(ctx, Mt.cuda(), k, s, l_k, seed, op)
+    assert ctx.poll_device_status() == 0
+    ref = decompose.refresh_basis(M, k, s, l_k, seed, op, 0)
+    assert np.array_equal(f.sampled_rows.cpu().numpy()[:l_k], ref["rows"])
+    om = f.omega.cpu().numpy()
+    ulp = np.spacing(np.abs(ref["omega"]).astype(np.float32))
+    assert np.all(np.abs(om - ref["omega"]) <= ulp)
+    U, S, V = decompose.step_factors(M, ref["V"])
+    gV, gU, gS = f.V.cpu().double().numpy(), f.U.cpu().double().numpy(), f.S.cpu().double().numpy()[:k]
+    assert linalg.principal_cosines(gV, V).min() >= COS
+    assert linalg.principal_cosines(gU, U).min() >= COS
+    assert np.max(np.abs(gS - S) / S[0]) < 1e-3
+    assert np.all(np.diff(gS) <= 1e-6 * gS[0])
+    assert np.allclose(gV.T @ gV, np.eye(k), atol=1e-4)
+    assert np.allclose(gU.T @ gU, np.eye(k), atol=1e-3)
+    for j in range(k):                        # sign convention
+        assert gV[np.argmax(np.abs(gV[:, j])), j] > 0
+    # the split reproduces the projection of M onto the basis
+    low = (gU * gS) @ gV.T
+    proj = M @ gV @ gV.T
+    assert np.linalg.norm(low - proj) / np.linalg.norm(proj) < 1e-4
+    return f, M
+
+
+def test_tiny_workload(ctx, metis_lib):
+    cfg = synth.CONFIGS["tiny_fwd"]
+    _compare(ctx, cfg, "X", 4, 4, 32, 0, 0)
+    _compare(ctx, cfg, "W", 4, 4, 256, 1, 0)
+
+
+def test_gpt2_shapes(ctx, metis_lib):
+    cfg = synth.CONFIGS["gpt2_small_mlp_up"]
+    _compare(ctx, cfg, "X", 12, 8, 82, 0, 1)
+    _compare(ctx, cfg, "W", 12, 8, 768, 1, 1)
+
+
+def test_llama_x_and_wide_sketch(ctx, metis_lib):
+    cfg = synth.CONFIGS["llama3_8b_mlp_up"]
+    _compare(ctx, cfg, "X", 64, 8, 82, 0, 2)
+    # widest supported sketch (k + s = 128) on a smaller matrix
+    cfg2 = synth.scaled_config("llama3_8b_mlp_up", l=1024, m=1024, n=1024)
+    _compare(ctx, cfg2, "X", 64, 64, 256, 0, 2)
+
+
+def test_reuse_keeps_the_span(ctx, metis_lib):
+    cfg = synth.CONFIGS["gpt2_small_mlp_up"]
+    Mt = synth.operand_matrix(cfg, "X")
+    f = _gpu_decompose(ctx, Mt.cuda(), 12, 8, 82, 1, 0)
+    V0 = f.V.cpu().double().numpy()
+    M1 = synth.perturbed(dict(cfg, perturb=1e-2), "X", Mt, 1)
+    _gpu_decompose(ctx, M1.cuda(), 12, 8, 82, 1, 0, refresh=False, step=1, factors=f)
+    V1 = f.V.cpu().double().numpy()
+    assert linalg.principal_cosines(V0, V1).min() > 1 - 1e-6
+    U, S, V = decompose.step_factors(M1.double().numpy(), V0)
+    assert np.max(np.abs(f.S.cpu().double().numpy()[:12] - S) / S[0]) < 1e-3
+
+
+def test_factor_quantization_bit_exact(ctx, metis_lib):
+    cfg = synth.CONFIGS["gpt2_small_mlp_up"]
+    Mt = synth.operand_matrix(cfg, "X")
+    f = _gpu_decompose(ctx, Mt.cuda(), 12, 8, 82, 1, 0, rounding=1, step=5)
+    for fac, q, sub, n in ((f.U, f.Uq, philox.SR_SUB_LEFT, 8192), (f.V, f.Vq, philox.SR_SUB_RIGHT, 768)):
+        F = fac.cpu().numpy()
+        codes, scales, g = codes_unpacked(q)
+        wc, ws, wg = metis.quantize_factor(F, seed=1, operand_id=0, sub=sub, step=5, rounding="sr")
+        assert g == wg
+        assert np.array_equal(codes[:12], wc) and np.array_equal(scales[:12], ws)
+        assert not codes[12:].any() and not scales[12:].any()
+
+
+def test_planted_low_rank(ctx, metis_lib):
+    rng = np.random.default_rng(3)
+    r, c, k = 1024, 512, 8
+    M = rng.standard_normal((r, k)) @ (np.geomspace(50, 5, k)[:, None] * rng.standard_normal((k, c)))
+    Mt = torch.from_numpy(M).to(torch.bfloat16)
+    Mb = Mt.double().numpy()
+    f = _gpu_decompose(ctx, Mt.cuda(), k, 4, 128, 0, 0)
+    _, _, Vt = np.linalg.svd(Mb)
+    assert linalg.principal_cosines(f.V.cpu().double().numpy(), Vt[:k].T).min() > 1 - 1e-5
+    low = (f.U.cpu().double().numpy() * f.S.cpu().double().numpy()[:k]) @ f.V.cpu().double().numpy().T
+    assert np.linalg.norm(Mb - low) / np.linalg.norm(Mb) < 1e-3
+
+
+def test_zero_and_nonfinite_inputs(ctx, metis_lib):
+    Z = torch.zeros(256, 256, dtype=torch.bfloat16, device="cuda")
+    f = _gpu_decompose(ctx, Z, 4, 4, 32, 0, 0)
+    assert ctx.poll_device_status() == 0
+    for t in (f.U, f.V, f.S):
+        assert torch.isfinite(t).all()
+    assert not f.S.any() and not f.U.any()
+    N = torch.ones(256, 256, dtype=torch.bfloat16, device="cuda")
+    N[3, 5] = float("nan")
+    _gpu_decompose(ctx, N, 4, 4, 256, 0, 0)
+    assert ctx.poll_device_status() & metis_lib.DEV_NONFINITE
+
+
+def test_decompose_validation(ctx, metis_lib):
+    M = torch.zeros(256, 256, dtype=torch.bfloat16, device="cuda")
+    f = ctx.new_factors(256, 256, 4)
+    with pytest.raises(metis_lib.MetisError):
+        ctx.decompose(M, k=4, s=200, l_k=32, seed=0, operand_id=0, refresh=True, step=0, factors=f)
+    with pytest.raises(metis_lib.MetisError):
+        ctx.decompose(M, k=4, s=4, l_k=4, seed=0, operand_id=0, refresh=True, step=0, factors=f)
