@@ -1,0 +1,374 @@
+"""Benchmark of the Metis W4A4G4 linear layer (fwd + dX + dW) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config llama3_8b_mlp_up] [--no-cpu-baseline]
+
+One step is the whole hot path on one batch: the randomized decomposition of
+X, W and D (refreshed every 8 steps, reused otherwise), the residual NVFP4
+quantization of each in both orientations, and the three fused GeMMs.  The
+metric is effective TFLOP/s = 6 l m n / step time (useful GeMM flops only).
+
+Workload: LLaMA-3 8B MLP up-projection at 8192 tokens (X 8192 x 4096,
+W 4096 x 14336, D 8192 x 14336, k = 64, s = 8, l_k = 82, stochastic rounding),
+synthetic anisotropic bf16 inputs.  The inputs (419 MB) exceed the 126 MB L2.
+
+With N > 1 (launched by torch.distributed.run) every rank runs its own batch
+of X and D with the shared W: weak scaling, no collective in the data path;
+the time is the maximum over ranks.
+
+``--impl reference`` times the CPU oracle on a bounded row sample of the same
+workload (rank 0 only).
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import synth  # noqa: E402
+
+NVFP4_OVER_BF16 = 9.0 / 2.25      # nominal dense tensor-core throughput ratio
+DEFAULT_CONFIG = "llama3_8b_mlp_up"
+METRIC = "effective TFLOP/s of Metis W4A4G4 linear fwd+bwd; % of NVFP4 MMA peak"
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.ident = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            self.ident = str(device.index)
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.ident}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ our arm
+class Layer:
+    """Device state of one Metis linear layer and its step."""
+
+    def __init__(self, lib, ctx, cfg, X, W, D):
+        self.lib, self.ctx, self.cfg = lib, ctx, cfg
+        self.rounding = 1 if cfg["rounding"] == "sr" else 0
+        self.mats = {"X": X, "W": W, "D": D}
+        k, s = cfg["k"], cfg["s"]
+        self.l_k = {"X": cfg["l_k"], "W": cfg["m"], "D": cfg["l_k"]}
+        self.ops = {}
+        for name, M in self.mats.items():
+            rows, cols = M.shape
+            f = ctx.new_factors(rows, cols, k, s)
+            row, col = ctx.new_nvfp4(rows, cols), ctx.new_nvfp4(cols, rows)
+            self.ops[name] = (f, row, col, ctx.operand(row, col, f))
+        l, m, n = cfg["l"], cfg["m"], cfg["n"]
+        self.Y = torch.empty(l, n, dtype=torch.float32, device=X.device)
+        self.dX = torch.empty(l, m, dtype=torch.float32, device=X.device)
+        self.dW = torch.empty(m, n, dtype=torch.float32, device=X.device)
+
+    def step(self, t):
+        cfg, ctx = self.cfg, self.ctx
+        refresh = t % cfg["refresh_every"] == 0
+        for i, name in enumerate(("X", "W", "D")):
+            f, row, col, _ = self.ops[name]
+            M = self.mats[name]
+            ctx.decompose(M, k=cfg["k"], s=cfg["s"], l_k=self.l_k[name], seed=cfg["seed"], operand_id=i,
+                          refresh=refresh, step=t, factors=f, rounding=self.rounding)
+            ctx.residual_quantize_nvfp4(M, f, row, col, rounding=self.rounding, seed=cfg["seed"], operand_id=i,
+                                        step=t)
+        ctx.linear_fwd(self.ops["X"][3], self.ops["W"][3], self.Y)
+        ctx.linear_bwd(self.ops["X"][3], self.ops["W"][3], self.ops["D"][3], self.dX, self.dW)
+
+
+def run_ours(args, rank, world, device):
+    import spectral_quantized_gemm_b200 as lib
+    cfg = synth.CONFIGS[args.config]
+    l, m, n = cfg["l"], cfg["m"], cfg["n"]
+    flops_per_step = 6.0 * l * m * n
+    # weak scaling: each rank its own tokens (X, D), the shared weight W
+    rcfg = dict(cfg, seed=cfg["seed"] + 1000 * rank)
+    host = {"X": synth.operand_matrix(rcfg, "X").pin_memory(), "W": synth.operand_matrix(cfg, "W").pin_memory(),
+            "D": synth.operand_matrix(rcfg, "D").pin_memory()}
+    dev = {k: v.to(device) for k, v in host.items()}
+    ctx = lib.Context(device.index)
+    layer = Layer(lib, ctx, cfg, dev["X"], dev["W"], dev["D"])
+    stream = torch.cuda.current_stream(device)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for t in range(args.warmup):
+        layer.step(t)
+    torch.cuda.synchronize(device)
+    status = ctx.poll_device_status()
+    if status:
+        raise RuntimeError(f"device status bits {status} after warm-up")
+
+    # ---- timed region: inputs resident in HBM
+    clocks = ClockSampler(device)
+    clocks.start()
+    time.sleep(0.3)
+    ctx.profile_enable(True)
+    launches0 = lib.kernel_launches()
+    barrier()
+    torch.cuda.synchronize(device)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for t in range(args.warmup, args.warmup + args.steps):
+        layer.step(t)
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    launches = lib.kernel_launches() - launches0
+    gemm_ms, gemm_n, gemm_flops = ctx.profile_read()
+    ctx.profile_enable(False)
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t_ = torch.tensor([ms], device=device)
+        torch.distributed.all_reduce(t_, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t_.item())
+    ms_per_step = ms / args.steps
+    value = world * flops_per_step / (ms_per_step * 1e-3) / 1e12
+
+    # ---- end to end through the public API: host inputs in, host results out
+    out_host = {"Y": torch.empty_like(layer.Y, device="cpu").pin_memory(),
+                "dX": torch.empty_like(layer.dX, device="cpu").pin_memory(),
+                "dW": torch.empty_like(layer.dW, device="cpu").pin_memory()}
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = sum(v.numel() * v.element_size() for v in out_host.values())
+    e2e_steps = max(2, min(args.steps, 6))
+    barrier()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for t in range(args.warmup + args.steps, args.warmup + args.steps + e2e_steps):
+        for k_ in ("X", "W", "D"):
+            dev[k_].copy_(host[k_], non_blocking=True)
+        layer.step(t)
+        out_host["Y"].copy_(layer.Y, non_blocking=True)
+        out_host["dX"].copy_(layer.dX, non_blocking=True)
+        out_host["dW"].copy_(layer.dW, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t_ = torch.tensor([e2e_ms], device=device)
+        torch.distributed.all_reduce(t_, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t_.item())
+    e2e_value = world * flops_per_step / (e2e_ms / e2e_steps * 1e-3) / 1e12
+    status = ctx.poll_device_status()
+
+    peaks, kind = measured_peaks()
+    peak = peaks["bf16_tflops_sustained"] * NVFP4_OVER_BF16
+    achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, ue4m3 scales; fp32 accumulate)",
+        "data": "synthetic anisotropic bf16 (spikes on 2% of hidden dims + N(0,1) bulk), seeded",
+        "config": {"workload": f"{args.config}: X {l}x{m}, W {m}x{n}, D {l}x{n}, k={cfg['k']}, s={cfg['s']}, "
+                               f"l_k={cfg['l_k']}, refresh every {cfg['refresh_every']}, {cfg['rounding']} rounding",
+                   "tokens_per_gpu": l, "parallelism": f"replicas x{world} (independent batches, shared W)",
+                   "l2": "inputs (419 MB) larger than the 126 MB L2; no flush",
+                   "pct_of_nvfp4_peak": round(100 * value / (world * peak), 2),
+                   "nvfp4_peak_tflops": round(peak, 1),
+                   "nvfp4_peak_basis": f"bf16_tflops_sustained x {NVFP4_OVER_BF16:.0f} ({kind})"},
+        "roofline": {"bound": "tensor", "kernel": "gemm_nvfp4_kernel<256> (fused FP4 GeMM + fold)",
+                     "achieved": None if achieved is None else round(achieved, 1), "peak": round(peak, 1),
+                     "unit": "TFLOP/s", "frac": None if achieved is None else round(achieved / peak, 4),
+                     "traffic": None, "launches_timed": gemm_n,
+                     "peak_basis": f"{kind} bf16 sustained x {NVFP4_OVER_BF16:.0f} (nominal NVFP4/bf16 ratio)"},
+        "clocks": clk,
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": launches,
+        "device_status": status,
+    }
+    return result
+
+
+# ------------------------------------------------------------------ oracle arm
+def oracle_sample_step(cfg, sample, state, t):
+    """The oracle's work for one step on a bounded sample (rows of X and D, full W)."""
+    from oracle import metis
+    rnd = cfg["rounding"]
+    opx = metis.prepare_operand(sample["X"], state["X"], seed=cfg["seed"], operand_id=0, step=t, rounding=rnd)
+    opw = metis.prepare_operand(sample["W"], state["W"], seed=cfg["seed"], operand_id=1, step=t, rounding=rnd)
+    opd = metis.prepare_operand(sample["D"], state["D"], seed=cfg["seed"], operand_id=2, step=t, rounding=rnd)
+    metis.linear_fwd(opx, opw)
+    metis.linear_bwd(opx, opw, opd)
+
+
+def oracle_setup(cfg, rows, cols):
+    """Bounded sub-problem: the first `rows` token rows of X and D and the first
+    `cols` output columns of W and D (bases refreshed once, untimed)."""
+    from oracle import decompose
+    full = {n: synth.operand_matrix(cfg, n, as_numpy=True) for n in ("X", "W", "D")}
+    sample = {"X": full["X"][:rows], "W": np.ascontiguousarray(full["W"][:, :cols]),
+              "D": np.ascontiguousarray(full["D"][:rows, :cols])}
+    state = {}
+    for i, n in enumerate(("X", "W", "D")):
+        l_k = min(cfg["l_k"], rows) if n != "W" else sample[n].shape[0]
+        state[n] = decompose.refresh_basis(sample[n], cfg["k"], cfg["s"], max(l_k, cfg["k"] + cfg["s"]),
+                                           cfg["seed"], i, 0)["V"]
+    return sample, state
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max((d.get("num_threads", 1) for d in info), default=os.cpu_count())
+    except Exception:
+        return os.cpu_count()
+
+
+def sample_text(cfg, rows, cols, dt):
+    return (f"sub-problem of {rows}/{cfg['l']} token rows x {cols}/{cfg['n']} output columns "
+            f"(X {rows}x{cfg['m']}, W {cfg['m']}x{cols}, D {rows}x{cols}): per-step factors, residual NVFP4 "
+            f"in both orientations, fwd, dX, dW; {dt:.1f} s per step; value = 6*rows*m*cols / time")
+
+
+def cpu_baseline(cfg, rows, cols, steps=1):
+    sample, state = oracle_setup(cfg, rows, cols)
+    t0 = time.perf_counter()
+    for t in range(steps):
+        oracle_sample_step(cfg, sample, state, t)
+    dt = (time.perf_counter() - t0) / steps
+    flops = 6.0 * rows * cfg["m"] * cols
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": sample_text(cfg, rows, cols, dt)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    cfg = synth.CONFIGS[args.config]
+    rows, cols = args.ref_rows, args.ref_cols
+    sample, state = oracle_setup(cfg, rows, cols)
+    for t in range(args.warmup):
+        oracle_sample_step(cfg, sample, state, t)
+    t0 = time.perf_counter()
+    for t in range(args.warmup, args.warmup + args.steps):
+        oracle_sample_step(cfg, sample, state, t)
+    dt = (time.perf_counter() - t0) / args.steps
+    flops = 6.0 * rows * cfg["m"] * cols
+    value = flops / dt / 1e12
+    l, m, n = cfg["l"], cfg["m"], cfg["n"]
+    cb = {"value": round(value, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+          "sample": sample_text(cfg, rows, cols, dt)}
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic anisotropic bf16, seeded",
+            "config": {"workload": f"{args.config}: X {l}x{m}, W {m}x{n}, D {l}x{n}, k={cfg['k']}",
+                       "sample_rows": rows, "sample_cols": cols},
+            "cpu_baseline": cb, "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                                        "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=16)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(synth.CONFIGS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-rows", type=int, default=256, help="token rows of the oracle's bounded sample")
+    ap.add_argument("--ref-cols", type=int, default=1024, help="output columns of the oracle's bounded sample")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("need at least 3 warm-up steps")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=300))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    res = run_ours(args, rank, world, device)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(synth.CONFIGS[args.config], args.ref_rows, args.ref_cols)
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -223,6 +223,20 @@ metis_status metis_linear_bwd(metis_ctx* ctx, const metis_operand* X, const meti
                               const metis_operand* D, void* dX, int64_t lddx, int32_t dx_dtype,
                               float* dW, int64_t lddw);
 
+/*
+ * Instrumentation (the notes have no counterpart; used by the benchmark).
+ * metis_kernel_launches: number of kernels libmetis has launched in this process.
+ * metis_profile_enable: when on, every main GeMM launch (the fused FP4 + fold
+ *   kernel of the layer calls and metis_gemm_nvfp4 with n_cols >= 256) is
+ *   bracketed by CUDA events on the context's stream.
+ * metis_profile_read: synchronizes the stream and returns the summed event time
+ *   (ms), the number of timed launches and their algorithmic flops 2*p*q*K, then
+ *   resets the record.
+ */
+uint64_t metis_kernel_launches(void);
+metis_status metis_profile_enable(metis_ctx* ctx, int on);
+metis_status metis_profile_read(metis_ctx* ctx, double* ms, int64_t* launches, double* flops);
+
 #ifdef __cplusplus
 }
 #endif

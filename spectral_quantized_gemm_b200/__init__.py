@@ -24,7 +24,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmetis.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing; build it with `python -m spectral_quantized_gemm_b200.build`")
+    raise ImportError(f"{LIB_PATH} is missing; build it with `python spectral_quantized_gemm_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -40,7 +40,8 @@ OUT_F32, OUT_BF16 = 0, 1
 EXPORTED = ["metis_create", "metis_destroy", "metis_set_stream", "metis_status_str", "metis_last_error",
             "metis_poll_device_status", "metis_nvfp4_codes_bytes", "metis_nvfp4_scales_bytes",
             "metis_decompose", "metis_residual_quantize_nvfp4", "metis_quantize_nvfp4_f32", "metis_gemm_nvfp4",
-            "metis_linear_fwd", "metis_linear_bwd"]
+            "metis_linear_fwd", "metis_linear_bwd", "metis_kernel_launches", "metis_profile_enable",
+            "metis_profile_read"]
 
 
 class Matrix(ctypes.Structure):
@@ -98,6 +99,17 @@ _fwd = _sig("metis_linear_fwd", c_i32, c_p, ctypes.POINTER(OperandStruct), ctype
             c_i64, c_i32)
 _bwd = _sig("metis_linear_bwd", c_i32, c_p, ctypes.POINTER(OperandStruct), ctypes.POINTER(OperandStruct),
             ctypes.POINTER(OperandStruct), c_p, c_i64, c_i32, c_p, c_i64)
+
+
+_launches = _sig("metis_kernel_launches", c_u64)
+_prof_enable = _sig("metis_profile_enable", c_i32, c_p, ctypes.c_int)
+_prof_read = _sig("metis_profile_read", c_i32, c_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(c_i64),
+                  ctypes.POINTER(ctypes.c_double))
+
+
+def kernel_launches():
+    """Kernels launched by libmetis in this process so far."""
+    return int(_launches())
 
 
 class MetisError(RuntimeError):
@@ -220,6 +232,15 @@ class Context:
         dtype = OUT_F32 if C.dtype == torch.float32 else OUT_BF16
         self._call(_gemm, ctypes.byref(A.struct), ctypes.byref(B.struct), n_cols, _ptr(Fa), _ptr(Fb), fold_k,
                    _ptr(col_scale), _ptr(C), C.stride(0), dtype)
+
+    def profile_enable(self, on=True):
+        self._call(_prof_enable, int(bool(on)))
+
+    def profile_read(self):
+        """(milliseconds, launches, flops) of the main GeMM launches since the last read."""
+        ms, n, fl = ctypes.c_double(), c_i64(), ctypes.c_double()
+        self._call(_prof_read, ctypes.byref(ms), ctypes.byref(n), ctypes.byref(fl))
+        return ms.value, n.value, fl.value
 
     @staticmethod
     def operand(rowwise=None, colwise=None, factors=None):

@@ -1,6 +1,6 @@
 """Builds libmetis.so (sm_100a) in-tree with nvcc.
 
-    python -m spectral_quantized_gemm_b200.build [-v] [--ptxas-info]
+    python spectral_quantized_gemm_b200/build.py [-v] [--ptxas-info]
 
 Objects go to ``spectral_quantized_gemm_b200/_build``; the shared library is
 ``spectral_quantized_gemm_b200/libmetis.so``.  A source file is recompiled

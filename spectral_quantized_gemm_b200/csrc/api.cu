@@ -296,3 +296,41 @@ metis_status metis_linear_bwd(metis_ctx* ctx, const metis_operand* X, const meti
 }
 
 }  // extern "C"
+
+namespace metis {
+std::atomic<uint64_t> g_launches{0};
+}  // namespace metis
+
+extern "C" {
+
+uint64_t metis_kernel_launches(void) { return metis::g_launches.load(); }
+
+metis_status metis_profile_enable(metis_ctx* ctx, int on) {
+  if (!ctx) return METIS_ERR_ARG;
+  ctx->profiling = on != 0;
+  return METIS_OK;
+}
+
+metis_status metis_profile_read(metis_ctx* ctx, double* ms, int64_t* launches, double* flops) {
+  if (!ctx || !ms || !launches || !flops) return METIS_ERR_ARG;
+  cudaSetDevice(ctx->device);
+  metis_status s = metis::check_cuda(ctx, cudaStreamSynchronize(ctx->stream), "cudaStreamSynchronize");
+  if (s != METIS_OK) return s;
+  double total = 0.0, fl = 0.0;
+  for (size_t i = 0; i < ctx->prof_events.size(); ++i) {
+    float t = 0.0f;
+    cudaEventElapsedTime(&t, ctx->prof_events[i].first, ctx->prof_events[i].second);
+    total += t;
+    fl += ctx->prof_flops[i];
+    cudaEventDestroy(ctx->prof_events[i].first);
+    cudaEventDestroy(ctx->prof_events[i].second);
+  }
+  *ms = total;
+  *launches = (int64_t)ctx->prof_events.size();
+  *flops = fl;
+  ctx->prof_events.clear();
+  ctx->prof_flops.clear();
+  return METIS_OK;
+}
+
+}  // extern "C"

@@ -566,50 +566,50 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
 
   auto gram = [&](const float* A, int64_t n, int width) {
     const int nb = (int)((n + kGramRows - 1) / kGramRows);
-    gram_partial_kernel<<<nb, 256, 0, st>>>(A, n, width, gpart, ctx->status);
-    gram_reduce_kernel<<<blocks_for((int64_t)width * width), 256, 0, st>>>(gpart, nb, width, G);
+    gram_partial_kernel<<<nb, 256, 0, st>>>(A, n, width, gpart, ctx->status); count_launch();
+    gram_reduce_kernel<<<blocks_for((int64_t)width * width), 256, 0, st>>>(gpart, nb, width, G); count_launch();
   };
   auto rows_times = [&](const int32_t* rowmap, int64_t nr, const float* B, int width, float* out) {
     dim3 grid(blocks_for(nr, kRowsPerBlock), nsplit);
     rows_times_matrix_kernel<<<grid, 256, 0, st>>>(Mb, M->ld, rowmap, nr, c, B, width, split_len, partial,
-                                                   ctx->status);
-    sum_splits_kernel<<<blocks_for(nr * width), 256, 0, st>>>(partial, nsplit, nr * width, out);
+                                                   ctx->status); count_launch();
+    sum_splits_kernel<<<blocks_for(nr * width), 256, 0, st>>>(partial, nsplit, nr * width, out); count_launch();
   };
 
   if (refresh) {
     const bool sampled = lk < r;
     if (sampled) {
       sample_keys_kernel<<<blocks_for(r), 256, 0, st>>>(r, p->seed, stream_tag(p->operand_id, kPurposeSample, 0),
-                                                       step, keys);
-      sample_select_kernel<<<1, 1024, 0, st>>>(keys, r, (int)lk, idx);
+                                                       step, keys); count_launch();
+      sample_select_kernel<<<1, 1024, 0, st>>>(keys, r, (int)lk, idx); count_launch();
     } else {
-      iota_kernel<<<blocks_for(lk), 256, 0, st>>>(lk, idx);
+      iota_kernel<<<blocks_for(lk), 256, 0, st>>>(lk, idx); count_launch();
     }
     if (f->sampled_rows)
       cudaMemcpyAsync(f->sampled_rows, idx, (size_t)lk * 4, cudaMemcpyDeviceToDevice, st);
     omega_kernel<<<blocks_for(((int64_t)c * w + 3) / 4), 256, 0, st>>>((int64_t)c * w, p->seed,
                                                                       stream_tag(p->operand_id, kPurposeOmega, 0),
-                                                                      step, omega, f->omega);
+                                                                      step, omega, f->omega); count_launch();
     // Y = M_s Omega ; Q = Y R^+
     rows_times(idx, lk, omega, w, Y);
     gram(Y, lk, w);
-    small_solver_kernel<<<1, 1024, small_smem, st>>>(G, w, k, 0, so, ctx->status);
-    times_small_kernel<<<blocks_for(lk * w), 256, 0, st>>>(Y, lk, w, T, w, Q);
+    small_solver_kernel<<<1, 1024, small_smem, st>>>(G, w, k, 0, so, ctx->status); count_launch();
+    times_small_kernel<<<blocks_for(lk * w), 256, 0, st>>>(Y, lk, w, T, w, Q); count_launch();
     // Bm^T = M_s^T Q ; R2 = chol(Bm Bm^T) ; SVD(R2^T) ; V = Bm^T R2^+ W'[:, :k]
-    cols_times_matrix_kernel<<<blocks_for(c, 64), 256, 0, st>>>(Mb, M->ld, idx, lk, c, Q, w, Bt);
+    cols_times_matrix_kernel<<<blocks_for(c, 64), 256, 0, st>>>(Mb, M->ld, idx, lk, c, Q, w, Bt); count_launch();
     gram(Bt, c, w);
-    small_solver_kernel<<<1, 1024, small_smem, st>>>(G, w, k, 1, so, ctx->status);
-    times_small_kernel<<<blocks_for(c * k), 256, 0, st>>>(Bt, c, w, T, k, f->V);
+    small_solver_kernel<<<1, 1024, small_smem, st>>>(G, w, k, 1, so, ctx->status); count_launch();
+    times_small_kernel<<<blocks_for(c * k), 256, 0, st>>>(Bt, c, w, T, k, f->V); count_launch();
   }
   // per step: P = M V ; R = chol(P^T P) ; SVD(R) ; U = P R^+ U_r ; V <- V V_r
   rows_times(nullptr, r, f->V, k, Y);
   gram(Y, r, k);
-  small_solver_kernel<<<1, 1024, small_smem, st>>>(G, k, k, 2, so, ctx->status);
-  times_small_kernel<<<blocks_for(r * k), 256, 0, st>>>(Y, r, k, T, k, Q);     // U (unsigned)
-  times_small_kernel<<<blocks_for(c * k), 256, 0, st>>>(f->V, c, k, Vr, k, Bt);  // V V_r
-  sign_pick_kernel<<<k, 256, 0, st>>>(Bt, c, k, flip);
-  apply_flip_kernel<<<blocks_for(c * k), 256, 0, st>>>(Bt, c, k, flip, f->V);
-  apply_flip_kernel<<<blocks_for(r * k), 256, 0, st>>>(Q, r, k, flip, f->U);
+  small_solver_kernel<<<1, 1024, small_smem, st>>>(G, k, k, 2, so, ctx->status); count_launch();
+  times_small_kernel<<<blocks_for(r * k), 256, 0, st>>>(Y, r, k, T, k, Q); count_launch();     // U (unsigned)
+  times_small_kernel<<<blocks_for(c * k), 256, 0, st>>>(f->V, c, k, Vr, k, Bt); count_launch();  // V V_r
+  sign_pick_kernel<<<k, 256, 0, st>>>(Bt, c, k, flip); count_launch();
+  apply_flip_kernel<<<blocks_for(c * k), 256, 0, st>>>(Bt, c, k, flip, f->V); count_launch();
+  apply_flip_kernel<<<blocks_for(r * k), 256, 0, st>>>(Q, r, k, flip, f->U); count_launch();
   cudaMemcpyAsync(f->S, Sw, (size_t)k * 4, cudaMemcpyDeviceToDevice, st);
   if ((s = check_cuda(ctx, cudaGetLastError(), "decompose")) != METIS_OK) return s;
   // factor quantization (blocks along the long dimension, power-of-two tensor scale)

@@ -371,7 +371,19 @@ metis_status launch_bn(metis_ctx* ctx, const GemmArgs& a) {
   if (e != cudaSuccess) return check_cuda(ctx, e, "cudaFuncSetAttribute(gemm)");
   const int tiles = prm.m_tiles * prm.n_tiles;
   const int grid = std::min(tiles, ctx->sm_count);
-  kern<<<grid, kThreads, C::SMEM, ctx->stream>>>(mA, mB, mFa, mFb, prm);
+  const bool prof = ctx->profiling && q_cols >= 256;
+  cudaEvent_t ev0 = nullptr, ev1 = nullptr;
+  if (prof) {
+    cudaEventCreate(&ev0);
+    cudaEventCreate(&ev1);
+    cudaEventRecord(ev0, ctx->stream);
+  }
+  kern<<<grid, kThreads, C::SMEM, ctx->stream>>>(mA, mB, mFa, mFb, prm); count_launch();
+  if (prof) {
+    cudaEventRecord(ev1, ctx->stream);
+    ctx->prof_events.emplace_back(ev0, ev1);
+    ctx->prof_flops.push_back(2.0 * (double)p_rows * (double)q_cols * (double)K);
+  }
   return check_cuda(ctx, cudaGetLastError(), "gemm_nvfp4 launch");
 }
 

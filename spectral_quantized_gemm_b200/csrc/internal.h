@@ -4,8 +4,10 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <string>
+#include <vector>
 
 #include "../../include/metis.h"
 
@@ -17,9 +19,16 @@ struct metis_ctx {
   char* ws = nullptr;          // device workspace, grown on demand
   size_t ws_bytes = 0;
   std::string last_error;
+  bool profiling = false;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> prof_events;
+  std::vector<double> prof_flops;
 };
 
 namespace metis {
+
+// Process-wide count of kernels launched by libmetis.
+extern std::atomic<uint64_t> g_launches;
+inline void count_launch(uint64_t n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
 // Sub-allocator over the context workspace: hands out 256-byte aligned slices.
 struct Workspace {

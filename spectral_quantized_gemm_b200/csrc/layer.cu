@@ -189,12 +189,12 @@ metis_status run_linear(metis_ctx* ctx, const metis_operand* A, const metis_nvfp
   if (kA) {
     vLA = {LAq->codes, LAq->scales, LAq->tensor_scale, LAq->inner, kA};
     vRA = {RAq->codes, RAq->scales, RAq->tensor_scale, RAq->inner, kA};
-    pad_sigma_kernel<<<1, 64, 0, st>>>(fa->S, kA, kpA, SAp);
+    pad_sigma_kernel<<<1, 64, 0, st>>>(fa->S, kA, kpA, SAp); count_launch();
   }
   if (kB) {
     vLB = {LBq->codes, LBq->scales, LBq->tensor_scale, LBq->inner, kB};
     vRB = {RBq->codes, RBq->scales, RBq->tensor_scale, RBq->inner, kB};
-    pad_sigma_kernel<<<1, 64, 0, st>>>(fb->S, kB, kpB, SBp);
+    pad_sigma_kernel<<<1, 64, 0, st>>>(fb->S, kB, kpB, SBp); count_launch();
   }
   // T_B = Q(A_R) Q(L_B) S_B  (p x kpB, fp32)
   if (kB) {
@@ -208,14 +208,14 @@ metis_status run_linear(metis_ctx* ctx, const metis_operand* A, const metis_nvfp
   }
   // Z = Q(R_A)^T Q(L_B)  (kA x kB over the contraction length K)
   if (kA && kB) {
-    z_partial_kernel<<<nchunks, 256, 0, st>>>(vRA, vLB, Zp);
-    z_reduce_kernel<<<16, 256, 0, st>>>(Zp, nchunks, Z);
+    z_partial_kernel<<<nchunks, 256, 0, st>>>(vRA, vLB, Zp); count_launch();
+    z_reduce_kernel<<<16, 256, 0, st>>>(Zp, nchunks, Z); count_launch();
   }
   if (kA || kB) {
     fold_b_kernel<<<(unsigned)((q * fold_k + 255) / 256), 256, 0, st>>>(TA32, kpA, kA, vRB, kpB, SAp, SBp, Z, q,
-                                                                        fold_k, Fb);
+                                                                        fold_k, Fb); count_launch();
     fold_a_kernel<<<(unsigned)((p * fold_k + 255) / 256), 256, 0, st>>>(TB32, kpB, kB, vLA, kpA, p, fold_k,
-                                                                        A_res->tensor_scale, B_res->tensor_scale, Fa);
+                                                                        A_res->tensor_scale, B_res->tensor_scale, Fa); count_launch();
   }
   if ((s = check_cuda(ctx, cudaGetLastError(), "fold preparation")) != METIS_OK) return s;
   GemmArgs g{A_res, B_res, Fa, Fb, fold_k, nullptr, C, ldc, c_dtype, 1.0f, q};

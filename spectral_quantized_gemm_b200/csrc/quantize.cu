@@ -239,13 +239,13 @@ cudaError_t launch_quantize_f32(const float* R, int64_t rows, int64_t cols, int6
     const int64_t n = rows * (cols / 16);
     quantize_rowwise_f32_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, st>>>(
         R, rows, cols, ld, q.tensor_scale, q.rounding, q.seed, stream_tag(q.operand_id, kPurposeSR, kSrRowwise),
-        q.step, rowwise->codes, rowwise->scales, rowwise->tensor_scale, status);
+        q.step, rowwise->codes, rowwise->scales, rowwise->tensor_scale, status); count_launch();
   }
   if (colwise) {
     const int64_t n = (rows / 16) * cols;
     quantize_colwise_f32_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, st>>>(
         R, rows, cols, ld, q.tensor_scale, q.rounding, q.seed, stream_tag(q.operand_id, kPurposeSR, kSrColwise),
-        q.step, colwise->codes, colwise->scales, colwise->tensor_scale, status);
+        q.step, colwise->codes, colwise->scales, colwise->tensor_scale, status); count_launch();
   }
   return cudaGetLastError();
 }
@@ -256,7 +256,7 @@ cudaError_t launch_residual_f32(const void* M_bf16, int64_t rows, int64_t cols, 
   (void)status;
   dim3 grid((unsigned)(cols / 64), (unsigned)(rows / 64));
   residual_f32_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(M_bf16), rows, cols, ld, U, S,
-                                            V, k, out);
+                                            V, k, out); count_launch();
   return cudaGetLastError();
 }
 
@@ -268,11 +268,11 @@ cudaError_t launch_quantize_factor(const float* F, int64_t longdim, int32_t k, i
   if (e != cudaSuccess) return e;
   const int64_t n = longdim * k;
   const int blocks = (int)std::min<int64_t>((n + 255) / 256, 1024);
-  absmax_kernel<<<blocks, 256, 0, st>>>(F, n, amax_bits, status);
+  absmax_kernel<<<blocks, 256, 0, st>>>(F, n, amax_bits, status); count_launch();
   const int64_t nthreads = 128 * (longdim / 16);
   quantize_factor_kernel<<<(unsigned)((nthreads + 255) / 256), 256, 0, st>>>(
       F, longdim, k, rounding, seed, stream_tag(operand_id, kPurposeSR, sub), step, amax_bits, out->codes,
-      out->scales, out->tensor_scale);
+      out->scales, out->tensor_scale); count_launch();
   return cudaGetLastError();
 }
 

@@ -107,10 +107,13 @@ def test_planted_low_rank(ctx, metis_lib):
     Mt = torch.from_numpy(M).to(torch.bfloat16)
     Mb = Mt.double().numpy()
     f = _gpu_decompose(ctx, Mt.cuda(), k, 4, 128, 0, 0)
-    _, _, Vt = np.linalg.svd(Mb)
+    Us, sv, Vt = np.linalg.svd(Mb, full_matrices=False)
     assert linalg.principal_cosines(f.V.cpu().double().numpy(), Vt[:k].T).min() > 1 - 1e-5
     low = (f.U.cpu().double().numpy() * f.S.cpu().double().numpy()[:k]) @ f.V.cpu().double().numpy().T
-    assert np.linalg.norm(Mb - low) / np.linalg.norm(Mb) < 1e-3
+    # bf16 rounding of the planted matrix adds a small full-rank part; the split must
+    # leave no more than the best rank-k approximation does (Eckart-Young)
+    best = np.sqrt(np.sum(sv[k:] ** 2))
+    assert np.linalg.norm(Mb - low) <= 1.01 * best + 1e-6 * np.linalg.norm(Mb)
 
 
 def test_zero_and_nonfinite_inputs(ctx, metis_lib):

@@ -146,6 +146,9 @@ def test_llama_up_full_size_sampled(ctx, metis_lib):
 def test_layer_validation(ctx, metis_lib):
     cfg = synth.CONFIGS["tiny_fwd"]
     res = _layer(ctx, cfg, fwd_only=True)
-    Y = torch.empty(cfg["l"], cfg["n"] + 4, device="cuda")[:, :cfg["n"] - 1]
-    with pytest.raises(metis_lib.MetisError):
+    Y = torch.empty(cfg["l"], cfg["n"] - 4, device="cuda")       # leading dimension < n
+    with pytest.raises(metis_lib.MetisError) as e:
         ctx.linear_fwd(res["X"].struct, res["W"].struct, Y)
+    assert e.value.status == 3
+    with pytest.raises(metis_lib.MetisError) as e:                # X and D swapped: K mismatch
+        ctx.linear_fwd(res["W"].struct, res["W"].struct, torch.empty(cfg["m"], cfg["n"], device="cuda"))
