@@ -14,7 +14,8 @@ ones; row j of R and column j of Q are then set to zero (so Q R reproduces Y
 up to the dropped, numerically null, components).
 
 One-sided (Hestenes) Jacobi SVD: columns p < q of A are rotated in cyclic
-order until every pair satisfies |a_p . a_q| <= tol * |a_p| |a_q| (tol 1e-15);
+order until every pair satisfies |a_p . a_q| <= tol * |a_p| |a_q| (tol 1e-12: at 1e-15 fp64
+rounding noise of length-64 dot products keeps pairs above the bound);
 the accumulated rotations are V, the column norms are the singular values and
 the normalised columns are U.
 
@@ -27,7 +28,7 @@ repeated and zero singular values, and on diagonal matrices.
 import numpy as np
 
 DROP_TOL = 1e-12
-JACOBI_TOL = 1e-15
+JACOBI_TOL = 1e-12
 JACOBI_MAX_SWEEPS = 60
 
 

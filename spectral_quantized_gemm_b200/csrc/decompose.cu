@@ -25,7 +25,7 @@ namespace metis {
 namespace {
 
 constexpr double kDropTol = 1e-12;
-constexpr double kJacobiTol = 1e-15;
+constexpr double kJacobiTol = 1e-12;
 constexpr int kJacobiMaxSweeps = 40;
 constexpr int kMaxW = 128;
 

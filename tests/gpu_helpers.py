@@ -63,3 +63,32 @@ def rel_fro(a, b):
 
 def bf16_round(a):
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64)).to(torch.bfloat16).double().numpy()
+
+
+def hat_select(op, orientation, rows=None, cols=None):
+    """Rows or columns of the dense operand hat Q(U) S Q(V)^T + Q(M_R) (oracle layout op).
+
+    orientation "row": the residual quantized along columns (stored rows x cols);
+    "col": along rows (stored transposed).  Only the requested slice is decoded.
+    """
+    from oracle import metis
+    codes, scales, g = op[orientation]
+    if orientation == "row":
+        sel = slice(None) if rows is None else rows
+        part = nvfp4.dequantize_blocks(codes[sel], scales[sel], g)
+        if cols is not None:
+            part = part[:, cols]
+    else:
+        sel = slice(None) if cols is None else cols
+        part = nvfp4.dequantize_blocks(codes[sel], scales[sel], g).T
+        if rows is not None:
+            part = part[rows]
+    if op.get("U") is not None:
+        U = metis.dequant_factor(op["Uq"])
+        V = metis.dequant_factor(op["Vq"])
+        if rows is not None:
+            U = U[rows]
+        if cols is not None:
+            V = V[cols]
+        part = part + (U * np.asarray(op["S"], dtype=np.float64)[None, :]) @ V.T
+    return part

@@ -150,5 +150,57 @@ def test_layer_validation(ctx, metis_lib):
     with pytest.raises(metis_lib.MetisError) as e:
         ctx.linear_fwd(res["X"].struct, res["W"].struct, Y)
     assert e.value.status == 3
-    with pytest.raises(metis_lib.MetisError) as e:                # X and D swapped: K mismatch
-        ctx.linear_fwd(res["W"].struct, res["W"].struct, torch.empty(cfg["m"], cfg["n"], device="cuda"))
+    no_colwise = ctx.operand(res["W"].row, None, res["W"].f)       # forward needs W column-wise
+    with pytest.raises(metis_lib.MetisError) as e:
+        ctx.linear_fwd(res["X"].struct, no_colwise, torch.empty(cfg["l"], cfg["n"], device="cuda"))
+    assert e.value.status == 1
+
+
+def _sampled_parity(res, l, m, nsample=192, seed=0):
+    from tests.gpu_helpers import hat_select
+    ox, ow, od = res["X"].oracle(), res["W"].oracle(), res["D"].oracle()
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(l, nsample, replace=False))
+    y = hat_select(ox, "row", rows=rows) @ hat_select(ow, "col")
+    e_y = rel_fro(res["Y"][rows].double().cpu().numpy(), y)
+    dx = hat_select(od, "row", rows=rows) @ hat_select(ow, "row").T
+    e_dx = rel_fro(res["dX"][rows].double().cpu().numpy(), dx)
+    cols = np.sort(rng.choice(m, nsample, replace=False))
+    dw = hat_select(ox, "col", cols=cols).T @ hat_select(od, "col")
+    e_dw = rel_fro(res["dW"][cols].double().cpu().numpy(), dw)
+    return e_y, e_dx, e_dw
+
+
+def test_llama_down_reuse_eight_steps(ctx, metis_lib):
+    """LLaMA-3 8B down-projection: decompose once, then 8 fwd+bwd steps on inputs
+    perturbed by 1e-2 relative noise with the factors reused (key design 3)."""
+    cfg = synth.CONFIGS["llama3_8b_down_reuse"]
+    base = {n: synth.operand_matrix(cfg, n) for n in ("X", "W", "D")}
+    k, s = cfg["k"], cfg["s"]
+    facs = {}
+    for step in range(cfg["steps"]):
+        mats = {n: (base[n] if step == 0 else synth.perturbed(cfg, n, base[n], step)).cuda() for n in base}
+        ops = {}
+        for i, n in enumerate(("X", "W", "D")):
+            l_k = cfg["l_k"] if n != "W" else cfg["m"]
+            ops[n] = GpuOperand(ctx, mats[n], k, s, l_k, cfg["seed"], i, 1, step=step, refresh=(step == 0),
+                                factors=facs.get(n))
+            facs[n] = ops[n].f
+        Y = torch.empty(cfg["l"], cfg["n"], device="cuda")
+        dX = torch.empty(cfg["l"], cfg["m"], device="cuda")
+        dW = torch.empty(cfg["m"], cfg["n"], device="cuda")
+        ctx.linear_fwd(ops["X"].struct, ops["W"].struct, Y)
+        ctx.linear_bwd(ops["X"].struct, ops["W"].struct, ops["D"].struct, dX, dW)
+        torch.cuda.synchronize()
+        assert ctx.poll_device_status() == 0
+        if step in (0, 7):
+            errs = _sampled_parity(dict(ops, Y=Y, dX=dX, dW=dW), cfg["l"], cfg["m"], 128, step)
+            assert max(errs) <= TOL, (step, errs)
+
+
+def test_long_token_stress(ctx, metis_lib):
+    """Long-token stress: X 65536 x 4096, l_k = 655, refreshed every step."""
+    cfg = synth.CONFIGS["long_token_stress"]
+    res = _layer(ctx, cfg)
+    errs = _sampled_parity(res, cfg["l"], cfg["m"], 128, 1)
+    assert max(errs) <= TOL, errs
