@@ -470,6 +470,43 @@ __global__ void __launch_bounds__(1024) small_solver_kernel(const double* __rest
   }
 }
 
+// ------------------------------------------- tensor-core projection helpers
+// out (2kp x n, bf16 row-major): row j < k = hi(F[:, j]), row kp + j = lo(F[:, j]) with
+// hi = bf16(F), lo = bf16(F - hi); other rows zero.  F is n x k fp32 row-major.
+__global__ void split_hi_lo_t_kernel(const float* __restrict__ F, int64_t n, int k, int kp,
+                                     __nv_bfloat16* __restrict__ out) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (int64_t)2 * kp * n) return;
+  const int j = (int)(e / n);
+  const int64_t i = e - (int64_t)j * n;
+  const int jj = j < kp ? j : j - kp;
+  float v = 0.0f;
+  if (jj < k) {
+    const float f = F[i * k + jj];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(f);
+    v = j < kp ? __bfloat162float(hi) : f - __bfloat162float(hi);
+  }
+  out[e] = __float2bfloat16_rn(v);
+}
+
+// out[i][j] = sum over splits (in order) of partial[s][i][j] + partial[s][i][kp + j],  j < k.
+__global__ void reduce_hi_lo_kernel(const float* __restrict__ partial, int splits, int64_t rows, int kp, int k,
+                                    float* __restrict__ out) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= rows * k) return;
+  const int64_t i = e / k;
+  const int j = (int)(e - i * k);
+  const int64_t stride = rows * 2 * kp;
+  float a = 0.0f;
+  for (int sp = 0; sp < splits; ++sp) {
+    const float* row = partial + sp * stride + i * 2 * kp;
+    a += row[j] + row[kp + j];
+  }
+  out[e] = a;
+}
+
+int pad_width(int w) { return w <= 16 ? 16 : w <= 32 ? 32 : w <= 64 ? 64 : 128; }
+
 // ------------------------------------------------------------- sign fix
 // flip[j] = 1 if the largest-|.| entry of column j of V (first index on ties) is negative.
 __global__ void sign_pick_kernel(const float* __restrict__ V, int64_t n, int k, int* flip) {
@@ -536,6 +573,11 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
   need += (size_t)((std::max(rows_needed, c) + kGramRows - 1) / kGramRows) * w * w * 8 + 256;  // gram partials
   need += (size_t)kMaxW * kMaxW * 8 * 5 + 2048;                   // G, T, Vr, Rinv, Vt
   need += 64 * 4 * 3 + 1024;                                      // S, flags, flips
+  const int kpw = pad_width(std::max(w, k));
+  need += (size_t)2 * kpw * c * 2 + 256;                          // hi/lo transposed operand
+  const int splits_est = normalize_splits(c, bf16_splits(ctx, r, c));
+  const size_t tc_partial_bytes = (size_t)splits_est * r * 2 * kpw * 4;
+  need += tc_partial_bytes + 256;                                 // split partials
   metis_status s = ensure_workspace(ctx, need);
   if (s != METIS_OK) return s;
   Workspace ws{ctx->ws, ctx->ws_bytes};
@@ -556,7 +598,9 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
   float* Sw = static_cast<float*>(ws.take(64 * 4));
   int* flags = static_cast<int*>(ws.take(64 * 4));
   int* flip = static_cast<int*>(ws.take(64 * 4));
-  if (!flip) return fail(ctx, METIS_ERR_WORKSPACE, "decompose workspace layout");
+  __nv_bfloat16* bt2 = static_cast<__nv_bfloat16*>(ws.take((size_t)2 * kpw * c * 2));
+  float* tc_partial = static_cast<float*>(ws.take(tc_partial_bytes));
+  if (!tc_partial) return fail(ctx, METIS_ERR_WORKSPACE, "decompose workspace layout");
 
   const size_t small_smem = (size_t)kMaxW * kMaxW * 8;
   cudaError_t e = cudaFuncSetAttribute(small_solver_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -568,6 +612,18 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
     const int nb = (int)((n + kGramRows - 1) / kGramRows);
     gram_partial_kernel<<<nb, 256, 0, st>>>(A, n, width, gpart, ctx->status); count_launch();
     gram_reduce_kernel<<<blocks_for((int64_t)width * width), 256, 0, st>>>(gpart, nb, width, G); count_launch();
+  };
+  // out (r x width) = M B on the tensor cores: B (c x width fp32) as a bf16 hi/lo pair
+  auto project = [&](const float* B, int width, float* out) -> metis_status {
+    const int kp = pad_width(width);
+    split_hi_lo_t_kernel<<<blocks_for((int64_t)2 * kp * c), 256, 0, st>>>(B, c, width, kp, bt2); count_launch();
+    const int splits = normalize_splits(c, bf16_splits(ctx, r, c));
+    if ((size_t)splits * r * 2 * kp * 4 > tc_partial_bytes)
+      return fail(ctx, METIS_ERR_WORKSPACE, "projection partials exceed workspace");
+    metis_status st2 = launch_gemm_bf16(ctx, Mb, M->ld, r, bt2, c, 2 * kp, c, tc_partial, 2 * kp, splits);
+    if (st2 != METIS_OK) return st2;
+    reduce_hi_lo_kernel<<<blocks_for(r * width), 256, 0, st>>>(tc_partial, splits, r, kp, width, out); count_launch();
+    return METIS_OK;
   };
   auto rows_times = [&](const int32_t* rowmap, int64_t nr, const float* B, int width, float* out) {
     dim3 grid(blocks_for(nr, kRowsPerBlock), nsplit);
@@ -591,7 +647,11 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
                                                                       stream_tag(p->operand_id, kPurposeOmega, 0),
                                                                       step, omega, f->omega); count_launch();
     // Y = M_s Omega ; Q = Y R^+
-    rows_times(idx, lk, omega, w, Y);
+    if (sampled) {
+      rows_times(idx, lk, omega, w, Y);
+    } else if ((s = project(omega, w, Y)) != METIS_OK) {
+      return s;
+    }
     gram(Y, lk, w);
     small_solver_kernel<<<1, 1024, small_smem, st>>>(G, w, k, 0, so, ctx->status); count_launch();
     times_small_kernel<<<blocks_for(lk * w), 256, 0, st>>>(Y, lk, w, T, w, Q); count_launch();
@@ -602,7 +662,7 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
     times_small_kernel<<<blocks_for(c * k), 256, 0, st>>>(Bt, c, w, T, k, f->V); count_launch();
   }
   // per step: P = M V ; R = chol(P^T P) ; SVD(R) ; U = P R^+ U_r ; V <- V V_r
-  rows_times(nullptr, r, f->V, k, Y);
+  if ((s = project(f->V, k, Y)) != METIS_OK) return s;
   gram(Y, r, k);
   small_solver_kernel<<<1, 1024, small_smem, st>>>(G, k, k, 2, so, ctx->status); count_launch();
   times_small_kernel<<<blocks_for(r * k), 256, 0, st>>>(Y, r, k, T, k, Q); count_launch();     // U (unsigned)

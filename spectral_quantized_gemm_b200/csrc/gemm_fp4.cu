@@ -43,7 +43,7 @@ struct Cfg {
   static constexpr int SFB_BYTES = SFB_ATOMS * 4 * 512;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int SF_STAGE_BYTES = SFA_BYTES + SFB_BYTES;
-  static constexpr int STAGES = BN > 128 ? 4 : 6;
+  static constexpr int STAGES = BN > 128 ? 4 : (BN == 128 ? 6 : 6);
   static constexpr int ACC_COLS = BN;
   static constexpr int SFA_COL = ACC_COLS;                // 4 columns per MMA k-step
   static constexpr int SFB_COLS_PER_K = SFB_ATOMS * 4;
@@ -69,6 +69,8 @@ struct Params {
   int c_dtype;
   int m_tiles, n_tiles;
   int k_stages, fold_stages;
+  int k_splits;            // work units per output tile along K (split-K), >= 1
+  int64_t split_stride;    // elements between the partial outputs of consecutive splits
   uint32_t* status;
 };
 
@@ -122,16 +124,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int num_tiles = p.m_tiles * p.n_tiles;
   const int total_stages = p.k_stages + p.fold_stages;
+  const int num_units = num_tiles * p.k_splits;
+  const int per_split = (total_stages + p.k_splits - 1) / p.k_splits;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
+      for (int unit = blockIdx.x; unit < num_units && !*abort_flag; unit += gridDim.x) {
+        const int tile = unit % num_tiles;
         const int mb = tile % p.m_tiles;
         const int nb = tile / p.m_tiles;
-        for (int kk = 0; kk < total_stages; ++kk) {
+        const int s0 = (unit / num_tiles) * per_split, s1 = min(total_stages, s0 + per_split);
+        for (int kk = s0; kk < s1; ++kk) {
           if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             *abort_flag = 1;
             raise_status(p.status, METIS_DEV_TIMEOUT);
@@ -176,14 +182,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t t_acc = tmem;
       const uint32_t t_sfa = tmem + C::SFA_COL;
       const uint32_t t_sfb = tmem + C::SFB_COL;
-      for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
+      for (int unit = blockIdx.x; unit < num_units && !*abort_flag; unit += gridDim.x) {
+        const int s0 = (unit / num_tiles) * per_split, s1 = min(total_stages, s0 + per_split);
         if (!tc::mbar_wait(tmem_empty, acc_phase ^ 1u, abort_flag)) {
           *abort_flag = 1;
           raise_status(p.status, METIS_DEV_TIMEOUT);
           break;
         }
         tc::tc_fence_after();
-        for (int kk = 0; kk < total_stages; ++kk) {
+        for (int kk = s0; kk < s1; ++kk) {
           if (!tc::mbar_wait(&full[stage], phase, abort_flag)) {
             *abort_flag = 1;
             raise_status(p.status, METIS_DEV_TIMEOUT);
@@ -208,11 +215,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               tc::mma_nvf4(t_acc, adesc + 2 * j, bdesc + 2 * j, id_fp4, t_sfa + 4 * j,
-                           t_sfb + C::SFB_COLS_PER_K * j, (kk | j) ? 1u : 0u);
+                           t_sfb + C::SFB_COLS_PER_K * j, (kk != s0 || j) ? 1u : 0u);
           } else {
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              tc::mma_bf16(t_acc, adesc + 2 * j, bdesc + 2 * j, id_bf16, (kk | j) ? 1u : 0u);
+              tc::mma_bf16(t_acc, adesc + 2 * j, bdesc + 2 * j, id_bf16, (kk != s0 || j) ? 1u : 0u);
           }
           tc::tc_commit(&empty[stage]);
           if (++stage == C::STAGES) {
@@ -235,9 +242,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int h = (warp - 2) >> 2;          // column half
     constexpr int kColsPerWarp = BN >= 64 ? BN / 2 : BN;
     const bool active = BN >= 64 || h == 0;
-    const float alpha = (*p.ga) * (*p.gb) * p.alpha_extra;
+    const float alpha = (p.ga ? *p.ga : 1.0f) * (p.gb ? *p.gb : 1.0f) * p.alpha_extra;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    for (int unit = blockIdx.x; unit < num_units; unit += gridDim.x) {
+      const int tile = unit % num_tiles;
+      float* const split_out = reinterpret_cast<float*>(p.C) + (int64_t)(unit / num_tiles) * p.split_stride;
       const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(tmem_full, acc_phase, abort_flag));
       if (!ok) {
         if (lane == 0) {
@@ -278,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t row = (int64_t)mb * 128 + q * 32 + lane;
         const int64_t cbase = (int64_t)nb * BN + col0;
         if (p.c_dtype == METIS_OUT_F32) {
-          float* dst = reinterpret_cast<float*>(p.C) + row * p.ldc + cbase;
+          float* dst = split_out + row * p.ldc + cbase;
 #pragma unroll
           for (int c = 0; c < kColsPerWarp; c += 4) {
             float4 o;
@@ -331,8 +340,32 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, u
 }
 
 template <int BN>
-metis_status launch_bn(metis_ctx* ctx, const GemmArgs& a) {
+metis_status launch_spec(metis_ctx* ctx, const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mFa,
+                         const CUtensorMap& mFb, Params prm, double flops, bool profiled) {
   using C = Cfg<BN>;
+  auto kern = gemm_nvfp4_kernel<BN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  if (e != cudaSuccess) return check_cuda(ctx, e, "cudaFuncSetAttribute(gemm)");
+  const int units = prm.m_tiles * prm.n_tiles * prm.k_splits;
+  const int grid = std::min(units, ctx->sm_count);
+  const bool prof = ctx->profiling && profiled;
+  cudaEvent_t ev0 = nullptr, ev1 = nullptr;
+  if (prof) {
+    cudaEventCreate(&ev0);
+    cudaEventCreate(&ev1);
+    cudaEventRecord(ev0, ctx->stream);
+  }
+  kern<<<grid, kThreads, C::SMEM, ctx->stream>>>(mA, mB, mFa, mFb, prm); count_launch();
+  if (prof) {
+    cudaEventRecord(ev1, ctx->stream);
+    ctx->prof_events.emplace_back(ev0, ev1);
+    ctx->prof_flops.push_back(flops);
+  }
+  return check_cuda(ctx, cudaGetLastError(), "gemm launch");
+}
+
+template <int BN>
+metis_status launch_bn(metis_ctx* ctx, const GemmArgs& a) {
   const int64_t p_rows = a.A->outer;
   const int64_t K = a.A->inner;
   const int64_t q_cols = a.q_cols;
@@ -365,29 +398,60 @@ metis_status launch_bn(metis_ctx* ctx, const GemmArgs& a) {
   prm.n_tiles = (int)(q_cols / BN);
   prm.k_stages = (int)(K / 256);
   prm.fold_stages = a.fold_k / 64;
+  prm.k_splits = 1;
+  prm.split_stride = 0;
   prm.status = ctx->status;
-  auto kern = gemm_nvfp4_kernel<BN>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-  if (e != cudaSuccess) return check_cuda(ctx, e, "cudaFuncSetAttribute(gemm)");
-  const int tiles = prm.m_tiles * prm.n_tiles;
-  const int grid = std::min(tiles, ctx->sm_count);
-  const bool prof = ctx->profiling && q_cols >= 256;
-  cudaEvent_t ev0 = nullptr, ev1 = nullptr;
-  if (prof) {
-    cudaEventCreate(&ev0);
-    cudaEventCreate(&ev1);
-    cudaEventRecord(ev0, ctx->stream);
-  }
-  kern<<<grid, kThreads, C::SMEM, ctx->stream>>>(mA, mB, mFa, mFb, prm); count_launch();
-  if (prof) {
-    cudaEventRecord(ev1, ctx->stream);
-    ctx->prof_events.emplace_back(ev0, ev1);
-    ctx->prof_flops.push_back(2.0 * (double)p_rows * (double)q_cols * (double)K);
-  }
-  return check_cuda(ctx, cudaGetLastError(), "gemm_nvfp4 launch");
+  return launch_spec<BN>(ctx, mA, mB, mFa, mFb, prm, 2.0 * (double)p_rows * (double)q_cols * (double)K,
+                         q_cols >= 256);
+}
+
+template <int BN>
+metis_status launch_bf16_bn(metis_ctx* ctx, const void* A, int64_t lda, int64_t rows, const void* B, int64_t ldb,
+                            int64_t K, float* C, int64_t ldc, int splits) {
+  CUtensorMap mFa, mFb;
+  if (!make_map_2d(&mFa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, K, rows, (uint64_t)lda * 2, 64, 128) ||
+      !make_map_2d(&mFb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, K, BN, (uint64_t)ldb * 2, 64, BN))
+    return fail(ctx, METIS_ERR_CUDA, "cuTensorMapEncodeTiled failed for the bf16 operands");
+  Params prm{};
+  prm.kb_tiles = 0;
+  prm.alpha_extra = 1.0f;
+  prm.C = C;
+  prm.ldc = ldc;
+  prm.c_dtype = METIS_OUT_F32;
+  prm.m_tiles = (int)(rows / 128);
+  prm.n_tiles = 1;
+  prm.k_stages = 0;
+  prm.fold_stages = (int)(K / 64);
+  prm.k_splits = normalize_splits(K, splits);  // no empty split
+  prm.split_stride = rows * ldc;
+  prm.status = ctx->status;
+  return launch_spec<BN>(ctx, mFa, mFb, mFa, mFb, prm, 2.0 * (double)rows * BN * (double)K, false);
 }
 
 }  // namespace
+
+int bf16_splits(metis_ctx* ctx, int64_t rows, int64_t K) {
+  const int tiles = (int)(rows / 128);
+  const int stages = (int)(K / 64);
+  const int want = (2 * ctx->sm_count + tiles - 1) / tiles;
+  return std::max(1, std::min(want, stages / 4));
+}
+
+metis_status launch_gemm_bf16(metis_ctx* ctx, const void* A, int64_t lda, int64_t rows, const void* B, int64_t ldb,
+                              int n, int64_t K, float* C, int64_t ldc, int splits) {
+  if (rows % 128 || K % 64 || lda % 8 || ldb % 8)
+    return fail(ctx, METIS_ERR_SHAPE, "bf16 GeMM needs rows % 128, K % 64 and 16-byte row strides");
+  if (splits < 1) splits = bf16_splits(ctx, rows, K);
+  if (splits > 1 && (int64_t)splits * rows * ldc > (int64_t(1) << 40))
+    return fail(ctx, METIS_ERR_SHAPE, "split output too large");
+  switch (n) {
+    case 32: return launch_bf16_bn<32>(ctx, A, lda, rows, B, ldb, K, C, ldc, splits);
+    case 64: return launch_bf16_bn<64>(ctx, A, lda, rows, B, ldb, K, C, ldc, splits);
+    case 128: return launch_bf16_bn<128>(ctx, A, lda, rows, B, ldb, K, C, ldc, splits);
+    case 256: return launch_bf16_bn<256>(ctx, A, lda, rows, B, ldb, K, C, ldc, splits);
+    default: return fail(ctx, METIS_ERR_SHAPE, "bf16 GeMM width must be 32, 64, 128 or 256");
+  }
+}
 
 metis_status launch_gemm_nvfp4(metis_ctx* ctx, const GemmArgs& a) {
   if (a.q_cols % 256 == 0) return launch_bn<256>(ctx, a);

@@ -79,6 +79,17 @@ struct GemmArgs {
   int64_t q_cols;     // output columns: a multiple of 256, or 16 / 32 / 64 (thin)
 };
 metis_status launch_gemm_nvfp4(metis_ctx* ctx, const GemmArgs& a);
+// C[s] (rows x n, fp32, split s at C + s * rows * ldc) = A (rows x K bf16, lda) * B^T
+// (B: n x K bf16, ldb) over the s-th share of K.  splits < 1 picks a split count;
+int bf16_splits(metis_ctx* ctx, int64_t rows, int64_t K);
+// Split count with no empty share of the K / 64 stages (what the launch uses).
+inline int normalize_splits(int64_t K, int splits) {
+  const int stages = (int)(K / 64);
+  const int per = (stages + splits - 1) / splits;
+  return (stages + per - 1) / per;
+}
+metis_status launch_gemm_bf16(metis_ctx* ctx, const void* A, int64_t lda, int64_t rows, const void* B, int64_t ldb,
+                              int n, int64_t K, float* C, int64_t ldc, int splits);
 
 // ---- decompose.cu ----
 metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_decomp_params* p, int refresh,

@@ -77,36 +77,50 @@ __global__ void z_reduce_kernel(const float* partial, int nchunks, float* Z) {
 }
 
 // Fb rows: [T_A^T hi | T_A^T lo | Q(R_B) | Q(R_B)] with
-// T_A^T[i][j] = TA32[i][j] + sum_t Q(R_B)[i][t] S_B[t] Z[j][t] S_A[j]   (Z = Q(R_A)^T Q(L_B)).
-// One thread per (row, fold column).
+// T_A^T[i][j] = TA32[i][j] + sum_u Q(R_B)[i][u] S_B[u] Z[j][u] S_A[j]   (Z = Q(R_A)^T Q(L_B)).
+// One block per 32 rows: the decoded rows of Q(R_B) and the k x k correction
+// C2[u][j] = S_B[u] Z[j][u] S_A[j] are staged once in shared memory.
+constexpr int kFoldRows = 32;
 __global__ void fold_b_kernel(const float* __restrict__ TA32, int kpA, int kA, FactorView RB, int kpB,
                               const float* __restrict__ SA, const float* __restrict__ SB, const float* __restrict__ Z,
                               int64_t q, int fold_k, __nv_bfloat16* __restrict__ Fb) {
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= q * fold_k) return;
-  const int64_t i = idx / fold_k;
-  const int c = (int)(idx - i * fold_k);
-  float out = 0.0f;
-  if (c < 2 * kpA) {
-    const int j = c < kpA ? c : c - kpA;
-    float t = 0.0f;
-    if (j < kA) {
-      t = TA32[i * kpA + j];
-      if (RB.k > 0) {
-        const float gr = *RB.g;
-        float acc = 0.0f;
-        for (int u = 0; u < RB.k; ++u)
-          acc = fmaf(factor_value(RB.codes, RB.scales, gr, RB.len, u, i) * SB[u], Z[j * 64 + u], acc);
-        t = fmaf(acc, SA[j], t);
-      }
-    }
-    const __nv_bfloat16 hi = __float2bfloat16_rn(t);
-    out = c < kpA ? __bfloat162float(hi) : t - __bfloat162float(hi);
-  } else if (c < 2 * kpA + 2 * kpB) {
-    const int u = (c - 2 * kpA) % kpB;
-    out = u < RB.k ? factor_value(RB.codes, RB.scales, *RB.g, RB.len, u, i) : 0.0f;
+  __shared__ float qrb[kFoldRows][65];
+  __shared__ float c2[64][65];
+  const int64_t i0 = (int64_t)blockIdx.x * kFoldRows;
+  const float gr = RB.k > 0 ? *RB.g : 0.0f;
+  for (int e = threadIdx.x; e < kFoldRows * 64; e += blockDim.x) {
+    const int r = e / 64, u = e % 64;
+    qrb[r][u] = (u < RB.k) ? factor_value(RB.codes, RB.scales, gr, RB.len, u, i0 + r) : 0.0f;
   }
-  Fb[i * fold_k + c] = __float2bfloat16_rn(out);
+  if (RB.k > 0 && kA > 0) {
+    for (int e = threadIdx.x; e < 64 * 64; e += blockDim.x) {
+      const int u = e / 64, j = e % 64;
+      c2[u][j] = (u < RB.k && j < kA) ? SB[u] * Z[j * 64 + u] * SA[j] : 0.0f;
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < kFoldRows * fold_k; e += blockDim.x) {
+    const int r = e / fold_k, c = e % fold_k;
+    const int64_t i = i0 + r;
+    float out = 0.0f;
+    if (c < 2 * kpA) {
+      const int j = c < kpA ? c : c - kpA;
+      float t = 0.0f;
+      if (j < kA) {
+        t = TA32[i * kpA + j];
+        if (RB.k > 0) {
+          float acc = 0.0f;
+          for (int u = 0; u < RB.k; ++u) acc = fmaf(qrb[r][u], c2[u][j], acc);
+          t += acc;
+        }
+      }
+      const __nv_bfloat16 hi = __float2bfloat16_rn(t);
+      out = c < kpA ? __bfloat162float(hi) : t - __bfloat162float(hi);
+    } else if (c < 2 * kpA + 2 * kpB) {
+      out = qrb[r][(c - 2 * kpA) % kpB];
+    }
+    Fb[i * fold_k + c] = __float2bfloat16_rn(out);
+  }
 }
 
 // Fa rows: [Q(L_A) | Q(L_A) | T_B hi | T_B lo] / alpha.
@@ -212,8 +226,8 @@ metis_status run_linear(metis_ctx* ctx, const metis_operand* A, const metis_nvfp
     z_reduce_kernel<<<16, 256, 0, st>>>(Zp, nchunks, Z); count_launch();
   }
   if (kA || kB) {
-    fold_b_kernel<<<(unsigned)((q * fold_k + 255) / 256), 256, 0, st>>>(TA32, kpA, kA, vRB, kpB, SAp, SBp, Z, q,
-                                                                        fold_k, Fb); count_launch();
+    fold_b_kernel<<<(unsigned)(q / kFoldRows), 256, 0, st>>>(TA32, kpA, kA, vRB, kpB, SAp, SBp, Z, q, fold_k,
+                                                             Fb); count_launch();
     fold_a_kernel<<<(unsigned)((p * fold_k + 255) / 256), 256, 0, st>>>(TB32, kpB, kB, vLA, kpA, p, fold_k,
                                                                         A_res->tensor_scale, B_res->tensor_scale, Fa); count_launch();
   }
