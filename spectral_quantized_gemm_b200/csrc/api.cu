@@ -218,6 +218,8 @@ metis_status metis_residual_quantize_nvfp4(metis_ctx* ctx, const metis_matrix* M
   if (!rowwise && !colwise) return fail(ctx, METIS_ERR_ARG, "no output orientation requested");
   if ((s = check_nvfp4(ctx, rowwise, M->rows, M->cols, "rowwise")) != METIS_OK) return s;
   if ((s = check_nvfp4(ctx, colwise, M->cols, M->rows, "colwise")) != METIS_OK) return s;
+  if (rowwise && colwise) return run_residual_quantize(ctx, M, f, q, rowwise, colwise);
+  // one orientation only: fp32 residual in the workspace, then the quantizer
   const size_t bytes = (size_t)M->rows * M->cols * sizeof(float);
   if ((s = ensure_workspace(ctx, bytes + 256)) != METIS_OK) return s;
   float* R = reinterpret_cast<float*>(ctx->ws);

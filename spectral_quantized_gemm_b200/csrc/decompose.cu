@@ -28,6 +28,7 @@ constexpr double kDropTol = 1e-12;
 constexpr double kJacobiTol = 1e-12;
 constexpr int kJacobiMaxSweeps = 40;
 constexpr int kMaxW = 128;
+constexpr size_t kSmallSmemMax = 200 * 1024;  // dynamic shared memory of the small solver
 
 // ---------------------------------------------------------------- sampling
 __global__ void sample_keys_kernel(int64_t rows, uint64_t seed, uint32_t tag, uint32_t step, uint64_t* keys) {
@@ -251,27 +252,48 @@ __global__ void times_small_kernel(const float* __restrict__ A, int64_t n, int k
 }
 
 // --------------------------------------------------------------- Gram (fp64)
-// partial[block] = A_chunk^T A_chunk, A fp32 n x w; upper triangle, full w x w storage.
+// partial[block] = A_rows^T A_rows over the block's rows (chunks of 32 staged in
+// shared memory); upper triangle, full w x w storage.  Each thread keeps its
+// (a, b) sums in registers across the chunks.
 constexpr int kGramRows = 32;
-__global__ void gram_partial_kernel(const float* __restrict__ A, int64_t n, int w, double* partial,
-                                    uint32_t* status) {
+constexpr int kGramPer = 64;   // (w*w)/256 for w <= 128
+__global__ void gram_partial_kernel(const float* __restrict__ A, int64_t n, int w, int64_t rows_per_block,
+                                    double* partial, uint32_t* status) {
   __shared__ double sa[kGramRows][kMaxW + 1];
-  const int64_t r0 = (int64_t)blockIdx.x * kGramRows;
+  const int64_t r_begin = (int64_t)blockIdx.x * rows_per_block;
+  const int64_t r_end = min(n, r_begin + rows_per_block);
+  double acc[kGramPer];
+#pragma unroll
+  for (int i = 0; i < kGramPer; ++i) acc[i] = 0.0;
   bool finite = true;
-  for (int e = threadIdx.x; e < kGramRows * w; e += blockDim.x) {
-    const int r = e / w, j = e % w;
-    float v = (r0 + r < n) ? A[(r0 + r) * w + j] : 0.0f;
-    finite &= isfinite(v);
-    sa[r][j] = v;
+  for (int64_t r0 = r_begin; r0 < r_end; r0 += kGramRows) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < kGramRows * w; e += blockDim.x) {
+      const int r = e / w, j = e % w;
+      const float v = (r0 + r < r_end) ? A[(r0 + r) * w + j] : 0.0f;
+      finite &= isfinite(v);
+      sa[r][j] = v;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kGramPer; ++i) {
+      const int e = threadIdx.x + i * 256;
+      if (e < w * w) {
+        const int a = e / w, b = e % w;
+        if (a <= b) {
+          double s2 = acc[i];
+#pragma unroll 8
+          for (int r = 0; r < kGramRows; ++r) s2 = fma(sa[r][a], sa[r][b], s2);
+          acc[i] = s2;
+        }
+      }
+    }
   }
   if (!finite) raise_status(status, METIS_DEV_NONFINITE);
-  __syncthreads();
-  for (int e = threadIdx.x; e < w * w; e += blockDim.x) {
-    const int a = e / w, b = e % w;
-    double acc = 0.0;
-    if (a <= b)
-      for (int r = 0; r < kGramRows; ++r) acc = fma(sa[r][a], sa[r][b], acc);
-    partial[(int64_t)blockIdx.x * w * w + e] = acc;
+#pragma unroll
+  for (int i = 0; i < kGramPer; ++i) {
+    const int e = threadIdx.x + i * 256;
+    if (e < w * w) partial[(int64_t)blockIdx.x * w * w + e] = acc[i];
   }
 }
 
@@ -313,7 +335,12 @@ __global__ void __launch_bounds__(1024) small_solver_kernel(const double* __rest
   const int ld = ne;
   double* R = At;                     // R[i * ld + j], upper triangular
   double* Rinv = out.Rinv;            // ld kMaxW
-  double* Vt = out.Vt;                // Vt[col * kMaxW + row]
+  // accumulated rotations by columns: in shared memory after the matrix when
+  // both fit, else in the (L2-resident) workspace
+  const bool vt_shared = (size_t)2 * ld * ld * sizeof(double) <= kSmallSmemMax;
+  double* Vt = vt_shared ? At + ld * ld : out.Vt;
+  const int vld = vt_shared ? ld : kMaxW;
+  __shared__ double nrm[kMaxW];
 
   for (int e = tid; e < ld * ld; e += nt) R[e] = 0.0;
   for (int e = tid; e < kMaxW * kMaxW; e += nt) Rinv[e] = 0.0;
@@ -372,13 +399,20 @@ __global__ void __launch_bounds__(1024) small_solver_kernel(const double* __rest
       }
     }
   }
-  for (int e = tid; e < kMaxW * kMaxW; e += nt) Vt[e] = ((e / kMaxW) == (e % kMaxW) && (e / kMaxW) < ne) ? 1.0 : 0.0;
+  for (int e = tid; e < vld * vld; e += nt) Vt[e] = ((e / vld) == (e % vld) && (e / vld) < ne) ? 1.0 : 0.0;
   __syncthreads();
   const int warp = tid >> 5, lane = tid & 31, nwarps = nt >> 5;
   const int npairs = ne / 2;
   int sweep = 0;
   for (; sweep < kJacobiMaxSweeps; ++sweep) {
     if (tid == 0) any_rot = 0;
+    // exact column norms at the start of every sweep; within the sweep they are
+    // updated with each rotation (||a_p||^2 -= t g, ||a_q||^2 += t g)
+    for (int j = tid; j < ne; j += nt) {
+      double s2 = 0.0;
+      for (int r = 0; r < ne; ++r) s2 = fma(At[j * ld + r], At[j * ld + r], s2);
+      nrm[j] = s2;
+    }
     __syncthreads();
     for (int round = 0; round < ne - 1; ++round) {
       for (int pr = warp; pr < npairs; pr += nwarps) {
@@ -393,25 +427,17 @@ __global__ void __launch_bounds__(1024) small_solver_kernel(const double* __rest
         }
         double* cp = At + p * ld;
         double* cq = At + q * ld;
-        double al = 0.0, be = 0.0, ga = 0.0;
-        for (int r = lane; r < ne; r += 32) {
-          const double x = cp[r], y = cq[r];
-          al = fma(x, x, al);
-          be = fma(y, y, be);
-          ga = fma(x, y, ga);
-        }
+        const double al = nrm[p], be = nrm[q];
+        double ga = 0.0;
+        for (int r = lane; r < ne; r += 32) ga = fma(cp[r], cq[r], ga);
 #pragma unroll
-        for (int off = 16; off; off >>= 1) {
-          al += __shfl_xor_sync(0xffffffffu, al, off);
-          be += __shfl_xor_sync(0xffffffffu, be, off);
-          ga += __shfl_xor_sync(0xffffffffu, ga, off);
-        }
+        for (int off = 16; off; off >>= 1) ga += __shfl_xor_sync(0xffffffffu, ga, off);
         if (ga != 0.0 && fabs(ga) > kJacobiTol * sqrt(al * be)) {
           const double zeta = (be - al) / (2.0 * ga);
           const double t = (zeta >= 0.0 ? 1.0 : -1.0) / (fabs(zeta) + sqrt(1.0 + zeta * zeta));
           const double c = 1.0 / sqrt(1.0 + t * t), s = c * t;
-          double* vp = Vt + p * kMaxW;
-          double* vq = Vt + q * kMaxW;
+          double* vp = Vt + p * vld;
+          double* vq = Vt + q * vld;
           for (int r = lane; r < ne; r += 32) {
             const double x = cp[r], y = cq[r];
             cp[r] = c * x - s * y;
@@ -420,7 +446,11 @@ __global__ void __launch_bounds__(1024) small_solver_kernel(const double* __rest
             vp[r] = c * vx - s * vy;
             vq[r] = s * vx + c * vy;
           }
-          if (lane == 0) any_rot = 1;
+          if (lane == 0) {
+            any_rot = 1;
+            nrm[p] = al - t * ga;
+            nrm[q] = be + t * ga;
+          }
         }
       }
       __syncthreads();
@@ -449,7 +479,7 @@ __global__ void __launch_bounds__(1024) small_solver_kernel(const double* __rest
     // T = R^+ W'[:, top k]  (n x k), W' the accumulated rotations
     for (int e = tid; e < n * k; e += nt) {
       const int i = e / k, c = e % k;
-      const double* wcol = Vt + order[c] * kMaxW;
+      const double* wcol = Vt + order[c] * vld;
       double a = 0.0;
       for (int t = 0; t < n; ++t) a = fma(Rinv[i * kMaxW + t], wcol[t], a);
       out.T[i * kMaxW + c] = a;
@@ -464,7 +494,7 @@ __global__ void __launch_bounds__(1024) small_solver_kernel(const double* __rest
       if (sg > 0.0)
         for (int t = 0; t < n; ++t) a = fma(Rinv[i * kMaxW + t], At[src * ld + t] / sg, a);
       out.T[i * kMaxW + c] = a;
-      out.Vr[i * kMaxW + c] = Vt[src * kMaxW + i];
+      out.Vr[i * kMaxW + c] = Vt[src * vld + i];
     }
     for (int c = tid; c < k; c += nt) out.S[c] = (float)sig[order[c]];
   }
@@ -602,15 +632,19 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
   float* tc_partial = static_cast<float*>(ws.take(tc_partial_bytes));
   if (!tc_partial) return fail(ctx, METIS_ERR_WORKSPACE, "decompose workspace layout");
 
-  const size_t small_smem = (size_t)kMaxW * kMaxW * 8;
+  const int ne_max = ((std::max(w, k) + 1) & ~1);
+  const size_t small_smem = std::max((size_t)ne_max * ne_max * 8,
+                                     std::min(kSmallSmemMax, (size_t)2 * ne_max * ne_max * 8));
   cudaError_t e = cudaFuncSetAttribute(small_solver_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)small_smem);
   if (e != cudaSuccess) return check_cuda(ctx, e, "cudaFuncSetAttribute(small solver)");
   SmallOut so{T, Vr, Sw, flags, Rinv, Vt};
 
   auto gram = [&](const float* A, int64_t n, int width) {
-    const int nb = (int)((n + kGramRows - 1) / kGramRows);
-    gram_partial_kernel<<<nb, 256, 0, st>>>(A, n, width, gpart, ctx->status); count_launch();
+    const int64_t chunks = (n + kGramRows - 1) / kGramRows;
+    const int64_t per_block = ((chunks + ctx->sm_count - 1) / ctx->sm_count) * kGramRows;
+    const int nb = (int)((n + per_block - 1) / per_block);
+    gram_partial_kernel<<<nb, 256, 0, st>>>(A, n, width, per_block, gpart, ctx->status); count_launch();
     gram_reduce_kernel<<<blocks_for((int64_t)width * width), 256, 0, st>>>(gpart, nb, width, G); count_launch();
   };
   // out (r x width) = M B on the tensor cores: B (c x width fp32) as a bf16 hi/lo pair

@@ -64,6 +64,10 @@ cudaError_t launch_quantize_factor(const float* F, int64_t longdim, int32_t k, i
                                    uint32_t operand_id, uint32_t sub, uint32_t step, const metis_nvfp4* out,
                                    float* amax_scratch, uint32_t* status, cudaStream_t st);
 
+// ---- resquant.cu ----
+metis_status run_residual_quantize(metis_ctx* ctx, const metis_matrix* M, const metis_factors* f,
+                                   const metis_quant_params* q, const metis_nvfp4* row, const metis_nvfp4* col);
+
 // ---- gemm_fp4.cu ----
 struct GemmArgs {
   const metis_nvfp4* A;

@@ -1,0 +1,462 @@
+// Fused residual + NVFP4 quantization in both orientations (one read of M).
+//
+// Method: "Metis: Training LLMs with FP4 Quantization" (papernotes.org notes),
+// key design 1: M = U S V^T + M_R with the residual M_R quantized to NVFP4
+// (background section: E2M1, 16-element blocks, E4M3 block scale; training
+// strategy: stochastic rounding).  Every residual is quantized twice, with
+// blocks along each GeMM contraction dimension that reads it.
+//
+// Per 128 x 128 tile of M (persistent CTAs, contiguous row-block-major ranges):
+//   warp 0      TMA: the U*S rows of the row block (kept while the block lasts),
+//               then per tile the V rows and the two 64-column boxes of M
+//   warp 1      tensor-memory owner; one thread issues tcgen05.mma kind::tf32
+//               (U S)(V)^T -> fp32 reconstruction in a double-buffered accumulator
+//   warps 2..9  residual = M - reconstruction (fp32), row-wise quantization from
+//               registers, the tile staged in XOR-swizzled shared memory, then
+//               column-wise quantization; codes and tiled scales go straight to HBM
+// All mbarrier waits are bounded (METIS_DEV_TIMEOUT on expiry).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "device_common.cuh"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace metis {
+namespace {
+
+constexpr int kRqThreads = 320;
+constexpr int kRqEpiThreads = 256;
+
+template <int KK>
+struct RqCfg {
+  static constexpr int A_BYTES = 128 * KK * 4;   // KK/32 swizzle atoms of 128 rows x 128 B
+  static constexpr int V_BYTES = 128 * KK * 4;
+  static constexpr int M_BYTES = 128 * 128 * 2;  // two 64-column boxes of 16 KB
+  static constexpr int STAGE_BYTES = V_BYTES + M_BYTES;
+  static constexpr int STAGES = 2;
+  static constexpr int R_BYTES = 128 * 128 * 4;
+  static constexpr size_t SMEM = (size_t)A_BYTES + STAGES * STAGE_BYTES + R_BYTES + 1024 + 256;
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+struct RqParams {
+  int64_t rows, cols;
+  int n_cb, n_units;
+  float g;
+  int rounding;
+  uint64_t seed;
+  uint32_t tag_row, tag_col, step;
+  uint8_t* row_codes;
+  uint8_t* row_scales;
+  uint8_t* col_codes;
+  uint8_t* col_scales;
+  float* row_g;
+  float* col_g;
+  uint32_t* status;
+};
+
+__host__ __device__ __forceinline__ uint32_t idesc_tf32(uint32_t n) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((n >> 3) << 17) | ((128u >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// One 16-element block: scale code and packed codes (RN or SR with the Philox
+// stream of element index e0 .. e0 + 15 in the orientation's blocked order).
+__device__ __forceinline__ uint2 quantize16(const float (&v)[16], float g, int rounding, uint64_t seed,
+                                            uint32_t tag, uint32_t step, uint64_t e0, uint32_t& scale_code) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const BlockScale bs = block_scale(amax, g);
+  float x[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) x[i] = __fmul_rn(v[i], bs.rcp);
+  float u[16];
+  if (rounding) {
+    const Words4 w0 = stream_call(seed, tag, step, e0 >> 3);
+    const Words4 w1 = stream_call(seed, tag, step, (e0 >> 3) + 1);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      u[i] = sr_uniform_from_words(w0, i);
+      u[8 + i] = sr_uniform_from_words(w1, i);
+    }
+  }
+  uint2 packed = encode16(x, rounding, u);
+  if (bs.code == 0) packed = make_uint2(0, 0);
+  scale_code = bs.code;
+  return packed;
+}
+
+__device__ __forceinline__ void named_sync_epilogue() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// OR of a predicate over the 256 epilogue threads (a barrier: all must call it), so
+// every epilogue thread takes the same branch after a bounded wait.
+__device__ __forceinline__ bool epilogue_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\tbar.red.or.pred p, 1, 256, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
+template <int KK>
+__global__ void __launch_bounds__(kRqThreads, 1)
+    resquant_kernel(const __grid_constant__ CUtensorMap mapM, const __grid_constant__ CUtensorMap mapUS,
+                    const __grid_constant__ CUtensorMap mapV, const RqParams p) {
+  using C = RqCfg<KK>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sStage = sA + C::A_BYTES;
+  float* sR = reinterpret_cast<float*>(sStage + C::STAGES * C::STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sR) + C::R_BYTES);
+  uint64_t* a_full = bars;
+  uint64_t* a_empty = bars + 1;
+  uint64_t* full = bars + 2;                 // [STAGES]
+  uint64_t* empty = full + C::STAGES;        // [STAGES]
+  uint64_t* acc_full = empty + C::STAGES;    // [2]
+  uint64_t* acc_empty = acc_full + 2;        // [2]
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int per = (p.n_units + gridDim.x - 1) / gridDim.x;
+  const int u_begin = blockIdx.x * per;
+  const int u_end = min(p.n_units, u_begin + per);
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(a_full, 1);
+    tc::mbar_init(a_empty, 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1 + kRqEpiThreads / 32);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&acc_full[b], 1);
+      tc::mbar_init(&acc_empty[b], kRqEpiThreads / 32);
+    }
+    tc::mbar_init(drain, 1);
+    *abort_flag = 0;
+    tc::fence_barrier_init();
+    if (blockIdx.x == 0) {
+      *p.row_g = p.g;
+      *p.col_g = p.g;
+    }
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, 256);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto fail_wait = [&]() {
+    *abort_flag = 1;
+    raise_status(p.status, METIS_DEV_TIMEOUT);
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, a_phase = 0;
+      int cur_rb = -1;
+      for (int u = u_begin; u < u_end && !*abort_flag; ++u) {
+        const int rb = u / p.n_cb, cb = u % p.n_cb;
+        if (rb != cur_rb) {
+          if (!tc::mbar_wait(a_empty, a_phase ^ 1u, abort_flag)) { fail_wait(); break; }
+          tc::mbar_expect_tx(a_full, C::A_BYTES);
+#pragma unroll
+          for (int ch = 0; ch < KK / 32; ++ch) tc::tma_load_2d(sA + ch * 16384, &mapUS, a_full, ch * 32, rb * 128);
+          a_phase ^= 1u;
+          cur_rb = rb;
+        }
+        if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { fail_wait(); break; }
+        uint8_t* sV = sStage + stage * C::STAGE_BYTES;
+        uint8_t* sM = sV + C::V_BYTES;
+        tc::mbar_expect_tx(&full[stage], C::STAGE_BYTES);
+#pragma unroll
+        for (int ch = 0; ch < KK / 32; ++ch) tc::tma_load_2d(sV + ch * 16384, &mapV, &full[stage], ch * 32, cb * 128);
+        tc::tma_load_2d(sM, &mapM, &full[stage], cb * 128, rb * 128);
+        tc::tma_load_2d(sM + 16384, &mapM, &full[stage], cb * 128 + 64, rb * 128);
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, a_phase = 0;
+      int cur_rb = -1;
+      int it = 0;
+      const uint32_t idesc = idesc_tf32(128);
+      for (int u = u_begin; u < u_end && !*abort_flag; ++u, ++it) {
+        const int rb = u / p.n_cb;
+        if (rb != cur_rb) {
+          if (cur_rb >= 0) tc::tc_commit(a_empty);  // the old U*S rows are no longer read
+          if (!tc::mbar_wait(a_full, a_phase, abort_flag)) { fail_wait(); break; }
+          a_phase ^= 1u;
+          cur_rb = rb;
+        }
+        const int b = it & 1;
+        const uint32_t use = (uint32_t)(it >> 1);
+        if (!tc::mbar_wait(&full[stage], phase, abort_flag)) { fail_wait(); break; }
+        if (!tc::mbar_wait(&acc_empty[b], (use & 1u) ^ 1u, abort_flag)) { fail_wait(); break; }
+        tc::tc_fence_after();
+        const uint8_t* sV = sStage + stage * C::STAGE_BYTES;
+#pragma unroll
+        for (int ch = 0; ch < KK / 32; ++ch) {
+          const uint64_t ad = tc::sdesc_sw128(tc::smem_addr(sA + ch * 16384));
+          const uint64_t bd = tc::sdesc_sw128(tc::smem_addr(sV + ch * 16384));
+#pragma unroll
+          for (int j = 0; j < 4; ++j) mma_tf32(tmem + b * 128, ad + 2 * j, bd + 2 * j, idesc, (ch | j) ? 1u : 0u);
+        }
+        tc::tc_commit(&empty[stage]);
+        tc::tc_commit(&acc_full[b]);
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      tc::tc_commit(drain);
+      tc::mbar_wait(drain, 0, nullptr);
+    }
+    __syncwarp();
+  } else {
+    const int et = threadIdx.x - 64;   // epilogue thread 0..255
+    const int q = warp & 3;            // tensor-memory lane quarter
+    const int h = (warp - 2) >> 2;     // column half of the tile
+    const int r = q * 32 + lane;       // tile row of this thread in the row pass
+    int stage = 0;
+    uint32_t phase = 0;
+    int it = 0;
+    for (int u = u_begin; u < u_end; ++u, ++it) {
+      const int rb = u / p.n_cb, cb = u % p.n_cb;
+      const int b = it & 1;
+      const uint32_t use = (uint32_t)(it >> 1);
+      bool ok = tc::mbar_wait(&acc_full[b], use & 1u, abort_flag);
+      ok = ok && tc::mbar_wait(&full[stage], phase, abort_flag);
+      if (epilogue_any(!ok)) {
+        if (et == 0) fail_wait();
+        break;
+      }
+      tc::tc_fence_after();
+      // reconstruction of this thread's row, 64 columns
+      float v[64];
+      {
+        float t[32];
+        tc::tmem_load_32cols(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * 128 + h * 64), t);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = t[i];
+        tc::tmem_load_32cols(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * 128 + h * 64 + 32), t);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[32 + i] = t[i];
+      }
+      tc::tmem_load_wait();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&acc_empty[b]);
+      // residual = M - reconstruction (M from the 128B-swizzled box of this half)
+      const uint8_t* sM = sStage + stage * C::STAGE_BYTES + C::V_BYTES + h * 16384;
+      bool finite = true;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(sM + r * 128 + ((c ^ (r & 7)) << 4));
+        const __nv_bfloat162* pr = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(pr[i]);
+          v[c * 8 + 2 * i] = f.x - v[c * 8 + 2 * i];
+          v[c * 8 + 2 * i + 1] = f.y - v[c * 8 + 2 * i + 1];
+        }
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&empty[stage]);   // this warp is done with M
+#pragma unroll
+      for (int i = 0; i < 64; ++i) finite &= isfinite(v[i]);
+      if (!finite) raise_status(p.status, METIS_DEV_NONFINITE);
+      // stage the residual row half in shared memory (16-byte chunks XOR-swizzled by row)
+#pragma unroll
+      for (int t4 = 0; t4 < 16; ++t4) {
+        const int cc = h * 16 + t4;
+        *reinterpret_cast<float4*>(sR + r * 128 + ((cc ^ (r & 7)) << 2)) =
+            make_float4(v[4 * t4], v[4 * t4 + 1], v[4 * t4 + 2], v[4 * t4 + 3]);
+      }
+      // row-wise quantization (blocks along columns) straight from registers
+      {
+        const int64_t grow = (int64_t)rb * 128 + r;
+        const int64_t gcol = (int64_t)cb * 128 + h * 64;
+        uint32_t sc = 0;
+        uint4 out0, out1;
+        uint32_t* o = reinterpret_cast<uint32_t*>(&out0);
+        uint32_t* o1 = reinterpret_cast<uint32_t*>(&out1);
+#pragma unroll
+        for (int blk = 0; blk < 4; ++blk) {
+          float x[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) x[i] = v[blk * 16 + i];
+          uint32_t code;
+          const uint2 pk = quantize16(x, p.g, p.rounding, p.seed, p.tag_row, p.step,
+                                      (uint64_t)grow * (uint64_t)p.cols + (uint64_t)(gcol + blk * 16), code);
+          sc |= code << (8 * blk);
+          uint32_t* dst = blk < 2 ? o : o1;
+          dst[(blk & 1) * 2] = pk.x;
+          dst[(blk & 1) * 2 + 1] = pk.y;
+        }
+        uint8_t* cdst = p.row_codes + grow * (p.cols / 2) + gcol / 2;
+        reinterpret_cast<uint4*>(cdst)[0] = out0;
+        reinterpret_cast<uint4*>(cdst)[1] = out1;
+        *reinterpret_cast<uint32_t*>(p.row_scales + scale_offset(grow, gcol / 16, p.cols / 64)) = sc;
+      }
+      named_sync_epilogue();
+      // column-wise quantization (blocks along rows) from the staged tile
+      {
+        const int j = et & 127, hh = et >> 7;
+        const int64_t gcolj = (int64_t)cb * 128 + j;
+        const int64_t grow0 = (int64_t)rb * 128 + hh * 64;
+        uint32_t sc = 0;
+        uint4 out0, out1;
+        uint32_t* o = reinterpret_cast<uint32_t*>(&out0);
+        uint32_t* o1 = reinterpret_cast<uint32_t*>(&out1);
+#pragma unroll
+        for (int blk = 0; blk < 4; ++blk) {
+          float x[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int rr = hh * 64 + blk * 16 + i;
+            x[i] = sR[rr * 128 + ((((j >> 2) ^ (rr & 7))) << 2) + (j & 3)];
+          }
+          uint32_t code;
+          const uint2 pk = quantize16(x, p.g, p.rounding, p.seed, p.tag_col, p.step,
+                                      (uint64_t)gcolj * (uint64_t)p.rows + (uint64_t)(grow0 + blk * 16), code);
+          sc |= code << (8 * blk);
+          uint32_t* dst = blk < 2 ? o : o1;
+          dst[(blk & 1) * 2] = pk.x;
+          dst[(blk & 1) * 2 + 1] = pk.y;
+        }
+        uint8_t* cdst = p.col_codes + gcolj * (p.rows / 2) + grow0 / 2;
+        reinterpret_cast<uint4*>(cdst)[0] = out0;
+        reinterpret_cast<uint4*>(cdst)[1] = out1;
+        *reinterpret_cast<uint32_t*>(p.col_scales + scale_offset(gcolj, grow0 / 16, p.rows / 64)) = sc;
+      }
+      named_sync_epilogue();
+      if (++stage == C::STAGES) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 256);
+  }
+}
+
+// US (rows x KK) = U diag(S) and Vp (cols x KK) = V, zero-padded to KK columns.
+__global__ void pad_factors_kernel(const float* __restrict__ U, const float* __restrict__ S,
+                                   const float* __restrict__ V, int64_t rows, int64_t cols, int k, int KK,
+                                   float* __restrict__ US, float* __restrict__ Vp) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t nu = rows * KK;
+  if (e < nu) {
+    const int64_t i = e / KK;
+    const int j = (int)(e - i * KK);
+    US[e] = (j < k) ? U[i * k + j] * S[j] : 0.0f;
+  } else if (e < nu + cols * KK) {
+    const int64_t f = e - nu;
+    const int64_t i = f / KK;
+    const int j = (int)(f - i * KK);
+    Vp[f] = (j < k) ? V[i * k + j] : 0.0f;
+  }
+}
+
+bool map2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t inner, uint64_t outer,
+           uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  EncodeTiledFn enc = encode_tiled();
+  return enc && enc(map, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int KK>
+metis_status launch_kk(metis_ctx* ctx, const metis_matrix* M, const float* US, const float* Vp,
+                       const metis_quant_params* q, const metis_nvfp4* row, const metis_nvfp4* col) {
+  using C = RqCfg<KK>;
+  CUtensorMap mM, mU, mV;
+  if (!map2d(&mM, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, M->data, M->cols, M->rows, (uint64_t)M->ld * 2, 64, 128) ||
+      !map2d(&mU, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, US, KK, M->rows, (uint64_t)KK * 4, 32, 128) ||
+      !map2d(&mV, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Vp, KK, M->cols, (uint64_t)KK * 4, 32, 128))
+    return fail(ctx, METIS_ERR_CUDA, "cuTensorMapEncodeTiled failed (residual quantization)");
+  RqParams prm;
+  prm.rows = M->rows;
+  prm.cols = M->cols;
+  prm.n_cb = (int)(M->cols / 128);
+  prm.n_units = (int)((M->rows / 128) * prm.n_cb);
+  prm.g = q->tensor_scale;
+  prm.rounding = q->rounding;
+  prm.seed = q->seed;
+  prm.tag_row = stream_tag(q->operand_id, kPurposeSR, kSrRowwise);
+  prm.tag_col = stream_tag(q->operand_id, kPurposeSR, kSrColwise);
+  prm.step = q->step;
+  prm.row_codes = row->codes;
+  prm.row_scales = row->scales;
+  prm.col_codes = col->codes;
+  prm.col_scales = col->scales;
+  prm.row_g = row->tensor_scale;
+  prm.col_g = col->tensor_scale;
+  prm.status = ctx->status;
+  auto kern = resquant_kernel<KK>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  if (e != cudaSuccess) return check_cuda(ctx, e, "cudaFuncSetAttribute(resquant)");
+  const int grid = std::min(prm.n_units, ctx->sm_count);
+  kern<<<grid, kRqThreads, C::SMEM, ctx->stream>>>(mM, mU, mV, prm); count_launch();
+  return check_cuda(ctx, cudaGetLastError(), "resquant launch");
+}
+
+}  // namespace
+
+metis_status run_residual_quantize(metis_ctx* ctx, const metis_matrix* M, const metis_factors* f,
+                                   const metis_quant_params* q, const metis_nvfp4* row, const metis_nvfp4* col) {
+  const int k = (f && f->k > 0) ? f->k : 0;
+  const int KK = k <= 32 ? 32 : 64;
+  const size_t need = (size_t)(M->rows + M->cols) * KK * 4 + 1024;
+  metis_status s = ensure_workspace(ctx, need);
+  if (s != METIS_OK) return s;
+  Workspace ws{ctx->ws, ctx->ws_bytes};
+  float* US = static_cast<float*>(ws.take((size_t)M->rows * KK * 4));
+  float* Vp = static_cast<float*>(ws.take((size_t)M->cols * KK * 4));
+  const int64_t n = (M->rows + M->cols) * KK;
+  pad_factors_kernel<<<(unsigned)((n + 255) / 256), 256, 0, ctx->stream>>>(
+      k ? f->U : nullptr, k ? f->S : nullptr, k ? f->V : nullptr, M->rows, M->cols, k, KK, US, Vp); count_launch();
+  if ((s = check_cuda(ctx, cudaGetLastError(), "pad factors")) != METIS_OK) return s;
+  return KK == 32 ? launch_kk<32>(ctx, M, US, Vp, q, row, col) : launch_kk<64>(ctx, M, US, Vp, q, row, col);
+}
+
+}  // namespace metis
