@@ -100,7 +100,7 @@ def jacobi_svd(A, tol=JACOBI_TOL, max_sweeps=JACOBI_MAX_SWEEPS):
                     continue
                 rotated = True
                 zeta = (beta - alpha) / (2.0 * gamma)
-                t = (1.0 if zeta >= 0 else -1.0) / (abs(zeta) + np.sqrt(1.0 + zeta * zeta))
+                t = (1.0 if zeta >= 0 else -1.0) / (abs(zeta) + np.hypot(1.0, zeta))
                 c = 1.0 / np.sqrt(1.0 + t * t)
                 s = c * t
                 up = U[:, p].copy()
