@@ -44,9 +44,12 @@ struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int SF_STAGE_BYTES = SFA_BYTES + SFB_BYTES;
   static constexpr int STAGES = BN > 128 ? 4 : (BN == 128 ? 6 : 6);
-  static constexpr int ACC_COLS = BN;
-  static constexpr int SFA_COL = ACC_COLS;                // 4 columns per MMA k-step
   static constexpr int SFB_COLS_PER_K = SFB_ATOMS * 4;
+  // two accumulator buffers (epilogue of tile t overlaps the MMAs of tile t+1)
+  // whenever they fit next to the scale columns in the 512 tensor-memory columns
+  static constexpr int ACC_BUFS = (2 * BN + 16 + 4 * SFB_COLS_PER_K) <= 512 ? 2 : 1;
+  static constexpr int ACC_COLS = BN * ACC_BUFS;
+  static constexpr int SFA_COL = ACC_COLS;                // 4 columns per MMA k-step
   static constexpr int SFB_COL = SFA_COL + 16;
   static constexpr int USED_COLS = SFB_COL + 4 * SFB_COLS_PER_K;
   static constexpr int TMEM_COLS = USED_COLS <= 32 ? 32 : USED_COLS <= 64 ? 64 : USED_COLS <= 128 ? 128
@@ -87,10 +90,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sf + C::STAGES * C::SF_STAGE_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + C::STAGES;
-  uint64_t* tmem_full = bars + 2 * C::STAGES;
-  uint64_t* tmem_empty = tmem_full + 1;
-  uint64_t* drain = tmem_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_full + 3);
+  uint64_t* tmem_full = bars + 2 * C::STAGES;   // [2]
+  uint64_t* tmem_empty = tmem_full + 2;         // [2]
+  uint64_t* drain = tmem_full + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_full + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -101,8 +104,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(&full[s], 1);
       tc::mbar_init(&empty[s], 1);
     }
-    tc::mbar_init(tmem_full, 1);
-    tc::mbar_init(tmem_empty, kEpiWarps);
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&tmem_full[b], 1);
+      tc::mbar_init(&tmem_empty[b], kEpiWarps);
+    }
     tc::mbar_init(drain, 1);
     *abort_flag = 0;
     tc::fence_barrier_init();
@@ -176,15 +181,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t acc_phase = 0;
+      int it = 0;
       const uint32_t id_fp4 = tc::idesc_nvf4(BN);
       const uint32_t id_bf16 = tc::idesc_bf16(BN);
-      const uint32_t t_acc = tmem;
       const uint32_t t_sfa = tmem + C::SFA_COL;
       const uint32_t t_sfb = tmem + C::SFB_COL;
-      for (int unit = blockIdx.x; unit < num_units && !*abort_flag; unit += gridDim.x) {
+      for (int unit = blockIdx.x; unit < num_units && !*abort_flag; unit += gridDim.x, ++it) {
         const int s0 = (unit / num_tiles) * per_split, s1 = min(total_stages, s0 + per_split);
-        if (!tc::mbar_wait(tmem_empty, acc_phase ^ 1u, abort_flag)) {
+        const int ab = it % C::ACC_BUFS;
+        const uint32_t use = (uint32_t)(it / C::ACC_BUFS);
+        const uint32_t t_acc = tmem + ab * BN;
+        if (!tc::mbar_wait(&tmem_empty[ab], (use & 1u) ^ 1u, abort_flag)) {
           *abort_flag = 1;
           raise_status(p.status, METIS_DEV_TIMEOUT);
           break;
@@ -228,8 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (*abort_flag) break;
-        tc::tc_commit(tmem_full);
-        acc_phase ^= 1u;
+        tc::tc_commit(&tmem_full[ab]);
       }
       // let every issued tensor-core operation finish before the memory is released
       tc::tc_commit(drain);
@@ -243,11 +249,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kColsPerWarp = BN >= 64 ? BN / 2 : BN;
     const bool active = BN >= 64 || h == 0;
     const float alpha = (p.ga ? *p.ga : 1.0f) * (p.gb ? *p.gb : 1.0f) * p.alpha_extra;
-    uint32_t acc_phase = 0;
-    for (int unit = blockIdx.x; unit < num_units; unit += gridDim.x) {
+    int it = 0;
+    for (int unit = blockIdx.x; unit < num_units; unit += gridDim.x, ++it) {
       const int tile = unit % num_tiles;
+      const int ab = it % C::ACC_BUFS;
+      const uint32_t use = (uint32_t)(it / C::ACC_BUFS);
       float* const split_out = reinterpret_cast<float*>(p.C) + (int64_t)(unit / num_tiles) * p.split_stride;
-      const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(tmem_full, acc_phase, abort_flag));
+      const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&tmem_full[ab], use & 1u, abort_flag));
       if (!ok) {
         if (lane == 0) {
           *abort_flag = 1;
@@ -265,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < kColsPerWarp; c += 16) {
           float t[16];
           uint32_t r[16];
-          const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(col0 + c);
+          const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * BN + col0 + c);
           asm volatile(
               "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
               "%13, %14, %15}, [%16];"
@@ -282,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(tmem_empty);
+      if (lane == 0) tc::mbar_arrive(&tmem_empty[ab]);
       if (active) {
         const int64_t row = (int64_t)mb * 128 + q * 32 + lane;
         const int64_t cbase = (int64_t)nb * BN + col0;
@@ -314,7 +322,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      acc_phase ^= 1u;
     }
   }
 
@@ -455,6 +462,7 @@ metis_status launch_gemm_bf16(metis_ctx* ctx, const void* A, int64_t lda, int64_
 
 metis_status launch_gemm_nvfp4(metis_ctx* ctx, const GemmArgs& a) {
   if (a.q_cols % 256 == 0) return launch_bn<256>(ctx, a);
+  if (a.q_cols == 128) return launch_bn<128>(ctx, a);
   if (a.q_cols == 64) return launch_bn<64>(ctx, a);
   if (a.q_cols == 32) return launch_bn<32>(ctx, a);
   if (a.q_cols == 16) return launch_bn<16>(ctx, a);
