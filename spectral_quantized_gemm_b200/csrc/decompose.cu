@@ -28,7 +28,7 @@ constexpr double kDropTol = 1e-12;
 constexpr double kJacobiTol = 1e-12;
 constexpr int kJacobiMaxSweeps = 40;
 constexpr int kMaxW = 128;
-constexpr size_t kSmallSmemMax = 200 * 1024;  // dynamic shared memory of the small solver
+constexpr int kSmallMaxN = 96;                 // sketch width limit of the one-CTA solver
 
 // ---------------------------------------------------------------- sampling
 __global__ void sample_keys_kernel(int64_t rows, uint64_t seed, uint32_t tag, uint32_t step, uint64_t* keys) {
@@ -128,58 +128,55 @@ __global__ void omega_kernel(int64_t n, uint64_t seed, uint32_t tag, uint32_t st
 
 // ------------------------------------------------ skinny products (fp32 accumulate)
 // Partial C[r][j] = sum_{c in chunk} M[rowmap[r]][c] * B[c][j]   (M bf16, B fp32 n x w)
-// grid: (ceil(nr/64), nsplit), block 256; partial layout [split][nr][w]
+// grid: (ceil(nr/64), nsplit), block 256; partial layout [split][nr][w].
+// Thread t owns row r = t % 64 and the outputs j = t / 64 + 4 i (registers).
 constexpr int kRowsPerBlock = 64;
 constexpr int kColChunk = 32;
-__global__ void rows_times_matrix_kernel(const __nv_bfloat16* __restrict__ M, int64_t ld, const int32_t* rowmap,
-                                         int64_t nr, int64_t ncols, const float* __restrict__ B, int w,
-                                         int64_t split_len, float* __restrict__ partial, uint32_t* status) {
+constexpr int kPerThread = kMaxW / 4;
+__global__ void __launch_bounds__(256) rows_times_matrix_kernel(
+    const __nv_bfloat16* __restrict__ M, int64_t ld, const int32_t* rowmap, int64_t nr, int64_t ncols,
+    const float* __restrict__ B, int w, int64_t split_len, float* __restrict__ partial, uint32_t* status) {
   __shared__ float sm[kRowsPerBlock][kColChunk + 1];
   __shared__ float sb[kColChunk][kMaxW];
   const int64_t r0 = (int64_t)blockIdx.x * kRowsPerBlock;
   const int64_t c_begin = (int64_t)blockIdx.y * split_len;
   const int64_t c_end = min(ncols, c_begin + split_len);
-  const int nout = kRowsPerBlock * w;
-  float acc[(kRowsPerBlock * kMaxW) / 256];
-  const int per = (nout + 255) / 256;
-  for (int i = 0; i < per; ++i) acc[i] = 0.0f;
+  const int r = threadIdx.x & 63, j0 = threadIdx.x >> 6;
+  float acc[kPerThread];
+#pragma unroll
+  for (int i = 0; i < kPerThread; ++i) acc[i] = 0.0f;
   bool finite = true;
   for (int64_t c0 = c_begin; c0 < c_end; c0 += kColChunk) {
     for (int e = threadIdx.x; e < kRowsPerBlock * kColChunk; e += blockDim.x) {
-      const int r = e / kColChunk, c = e % kColChunk;
-      const int64_t row = r0 + r;
+      const int rr = e / kColChunk, c = e % kColChunk;
+      const int64_t row = r0 + rr;
       float v = 0.0f;
       if (row < nr && c0 + c < c_end) {
         const int64_t src = rowmap ? rowmap[row] : row;
         v = __bfloat162float(M[src * ld + c0 + c]);
         finite &= isfinite(v);
       }
-      sm[r][c] = v;
+      sm[rr][c] = v;
     }
-    for (int e = threadIdx.x; e < kColChunk * w; e += blockDim.x) {
-      const int c = e / w, j = e % w;
-      sb[c][j] = (c0 + c < c_end) ? B[(c0 + c) * w + j] : 0.0f;
+    for (int e = threadIdx.x; e < kColChunk * kMaxW; e += blockDim.x) {
+      const int c = e / kMaxW, j = e % kMaxW;
+      sb[c][j] = (c0 + c < c_end && j < w) ? B[(c0 + c) * w + j] : 0.0f;
     }
     __syncthreads();
-    for (int i = 0; i < per; ++i) {
-      const int o = threadIdx.x + i * 256;
-      if (o < nout) {
-        const int r = o / w, j = o % w;
-        float a = acc[i];
-#pragma unroll 8
-        for (int c = 0; c < kColChunk; ++c) a = fmaf(sm[r][c], sb[c][j], a);
-        acc[i] = a;
-      }
+#pragma unroll 4
+    for (int c = 0; c < kColChunk; ++c) {
+      const float a = sm[r][c];
+#pragma unroll
+      for (int i = 0; i < kPerThread; ++i) acc[i] = fmaf(a, sb[c][j0 + 4 * i], acc[i]);
     }
     __syncthreads();
   }
   if (!finite) raise_status(status, METIS_DEV_NONFINITE);
-  for (int i = 0; i < per; ++i) {
-    const int o = threadIdx.x + i * 256;
-    if (o < nout) {
-      const int r = o / w, j = o % w;
-      if (r0 + r < nr) partial[((int64_t)blockIdx.y * nr + r0 + r) * w + j] = acc[i];
-    }
+  if (r0 + r < nr) {
+    float* dst = partial + ((int64_t)blockIdx.y * nr + r0 + r) * w;
+#pragma unroll
+    for (int i = 0; i < kPerThread; ++i)
+      if (j0 + 4 * i < w) dst[j0 + 4 * i] = acc[i];
   }
 }
 
@@ -193,49 +190,45 @@ __global__ void sum_splits_kernel(const float* partial, int nsplit, int64_t n, f
 }
 
 // Bm^T = M_s^T Q: out[c][j] = sum_r M[rowmap[r]][c] * Q[r][j]   (64 columns of M per block)
-__global__ void cols_times_matrix_kernel(const __nv_bfloat16* __restrict__ M, int64_t ld, const int32_t* rowmap,
-                                         int64_t nr, int64_t ncols, const float* __restrict__ Q, int w,
-                                         float* __restrict__ out) {
+// Thread t owns column c = t % 64 and the outputs j = t / 64 + 4 i (registers).
+__global__ void __launch_bounds__(256) cols_times_matrix_kernel(
+    const __nv_bfloat16* __restrict__ M, int64_t ld, const int32_t* rowmap, int64_t nr, int64_t ncols,
+    const float* __restrict__ Q, int w, float* __restrict__ out) {
   __shared__ float sm[16][65];
   __shared__ float sq[16][kMaxW];
   const int64_t c0 = (int64_t)blockIdx.x * 64;
-  const int nout = 64 * w;
-  const int per = (nout + 255) / 256;
-  float acc[(64 * kMaxW) / 256];
-  for (int i = 0; i < per; ++i) acc[i] = 0.0f;
+  const int c = threadIdx.x & 63, j0 = threadIdx.x >> 6;
+  float acc[kPerThread];
+#pragma unroll
+  for (int i = 0; i < kPerThread; ++i) acc[i] = 0.0f;
   for (int64_t r0 = 0; r0 < nr; r0 += 16) {
     for (int e = threadIdx.x; e < 16 * 64; e += blockDim.x) {
-      const int r = e / 64, c = e % 64;
+      const int rr = e / 64, cc = e % 64;
       float v = 0.0f;
-      if (r0 + r < nr && c0 + c < ncols) {
-        const int64_t src = rowmap ? rowmap[r0 + r] : r0 + r;
-        v = __bfloat162float(M[src * ld + c0 + c]);
+      if (r0 + rr < nr && c0 + cc < ncols) {
+        const int64_t src = rowmap ? rowmap[r0 + rr] : r0 + rr;
+        v = __bfloat162float(M[src * ld + c0 + cc]);
       }
-      sm[r][c] = v;
+      sm[rr][cc] = v;
     }
-    for (int e = threadIdx.x; e < 16 * w; e += blockDim.x) {
-      const int r = e / w, j = e % w;
-      sq[r][j] = (r0 + r < nr) ? Q[(r0 + r) * w + j] : 0.0f;
+    for (int e = threadIdx.x; e < 16 * kMaxW; e += blockDim.x) {
+      const int rr = e / kMaxW, j = e % kMaxW;
+      sq[rr][j] = (r0 + rr < nr && j < w) ? Q[(r0 + rr) * w + j] : 0.0f;
     }
     __syncthreads();
-    for (int i = 0; i < per; ++i) {
-      const int o = threadIdx.x + i * 256;
-      if (o < nout) {
-        const int c = o / w, j = o % w;
-        float a = acc[i];
+#pragma unroll 4
+    for (int rr = 0; rr < 16; ++rr) {
+      const float a = sm[rr][c];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) a = fmaf(sm[r][c], sq[r][j], a);
-        acc[i] = a;
-      }
+      for (int i = 0; i < kPerThread; ++i) acc[i] = fmaf(a, sq[rr][j0 + 4 * i], acc[i]);
     }
     __syncthreads();
   }
-  for (int i = 0; i < per; ++i) {
-    const int o = threadIdx.x + i * 256;
-    if (o < nout) {
-      const int c = o / w, j = o % w;
-      if (c0 + c < ncols) out[(c0 + c) * w + j] = acc[i];
-    }
+  if (c0 + c < ncols) {
+    float* dst = out + (c0 + c) * w;
+#pragma unroll
+    for (int i = 0; i < kPerThread; ++i)
+      if (j0 + 4 * i < w) dst[j0 + 4 * i] = acc[i];
   }
 }
 
@@ -307,196 +300,350 @@ __global__ void gram_reduce_kernel(const double* partial, int nblocks, int w, do
   G[e] = acc;
 }
 
-// ----------------------------------------------------- single-CTA small solver
-// Modes: 0 = CholQR factor only (T = R^+), 1 = refresh SVD (T = R^+ W'[:, :k] with
-// SVD of R^T), 2 = step SVD (T = R^+ U_r[:, :k], Vr, S from SVD of R).
-// Shared memory holds the n x n matrix being orthogonalized, stored by columns;
-// R^+ and the accumulated rotations live in (L2-resident) workspace.
+// ----------------------------------------------------- single-CTA small solvers
+// Both take the Gram matrix G (n x n, fp64) of a tall matrix Y and run in one CTA of
+// a few hundred threads; the problems are a few hundred thousand flops, so the design
+// goal is few barrier-separated steps with independent work inside each.
+//
+// cholqr_solver_kernel: T = R^+ with G = R^T R (Cholesky with dependent-column drop), so
+//   that Q = Y T is the CholQR factor.  Right-looking on unscaled rows
+//   (B_it -= B_ji B_jt / d_j) in panels of kPanel pivots, then R^+ by blocked back
+//   substitution on the identity.
+// eig_solver_kernel: the SVD of Y through the symmetric eigenproblem of G = Y^T Y =
+//   Z Lambda Z^T (two-sided Jacobi, Brent-Luk parallel ordering: a round's disjoint
+//   rotations are applied to H as one step over its 2 x 2 blocks), ordered by
+//   descending eigenvalue: S = sqrt(lambda), Vr = Z[:, :k] and T = Z[:, :k] Lambda^-1/2,
+//   so that Y T are the left singular vectors.  An eigenvalue not above
+//   kDropTol * lambda_max counts as zero (zero column of T, zero singular value).
+constexpr int kSolverThreads = 256;                 // Cholesky solver
+constexpr int kSolverWarps = kSolverThreads / 32;
+constexpr int kEigThreads = 1024;                   // eigensolver: a warp per rotation pair
+constexpr int kPanel = 8;
+constexpr int kLaneRows = (kMaxW + 31) / 32;   // entries of a row or column per lane
+
 struct SmallOut {
   double* T;      // n x kMaxW (row-major, ld kMaxW)
   double* Vr;     // n x kMaxW
   float* S;       // k
-  int* flags;     // [0] = numeric failure
-  double* Rinv;   // kMaxW x kMaxW scratch
-  double* Vt;     // kMaxW x kMaxW scratch: accumulated rotations, by columns
+  int* flags;     // [0] = numeric failure, [1] = Jacobi sweeps of the last solve
+  double* scratch;  // small_solver_doubles(kMaxW), used when the sketch is wider than kSmallMaxN
 };
 
-__global__ void __launch_bounds__(1024) small_solver_kernel(const double* __restrict__ G, int n, int k, int mode,
-                                                            SmallOut out, uint32_t* status) {
-  extern __shared__ double At[];      // ld x ld; Cholesky factor first, then A by columns
-  __shared__ int dropped[kMaxW];
-  __shared__ double gmax_s, pivot_s;
-  __shared__ double sig[kMaxW];
-  __shared__ int order[kMaxW];
-  __shared__ int any_rot;
-  const int tid = threadIdx.x;
-  const int nt = blockDim.x;
-  const int ne = (n + 1) & ~1;
-  const int ld = ne;
-  double* R = At;                     // R[i * ld + j], upper triangular
-  double* Rinv = out.Rinv;            // ld kMaxW
-  // accumulated rotations by columns: in shared memory after the matrix when
-  // both fit, else in the (L2-resident) workspace
-  const bool vt_shared = (size_t)2 * ld * ld * sizeof(double) <= kSmallSmemMax;
-  double* Vt = vt_shared ? At + ld * ld : out.Vt;
-  const int vld = vt_shared ? ld : kMaxW;
-  __shared__ double nrm[kMaxW];
+// fp64 words of shared memory (or scratch) either solver uses for a width ne problem
+__host__ __device__ constexpr size_t small_solver_doubles(int ne) {
+  return (size_t)2 * ne * (ne + 1);
+}
 
-  for (int e = tid; e < ld * ld; e += nt) R[e] = 0.0;
-  for (int e = tid; e < kMaxW * kMaxW; e += nt) Rinv[e] = 0.0;
-  if (tid == 0) {
+__device__ __forceinline__ int rr_index(int pos, int round, int ne) {
+  // position 0 stays; positions 1 .. ne-1 rotate by one each round
+  if (pos == 0) return 0;
+  int v = pos - 1 + round;
+  if (v >= ne - 1) v -= ne - 1;
+  return v + 1;
+}
+
+__device__ __forceinline__ void round_pair(int pr, int round, int ne, int& p, int& q) {
+  p = rr_index(pr, round, ne);
+  q = rr_index(ne - 1 - pr, round, ne);
+  if (p > q) {
+    const int t = p;
+    p = q;
+    q = t;
+  }
+}
+
+template <bool kSmem>
+__global__ void __launch_bounds__(kSolverThreads) cholqr_solver_kernel(const double* __restrict__ G, int n,
+                                                                       SmallOut out) {
+  extern __shared__ double smem_d[];
+  const int ne = (n + 1) & ~1;
+  const int ld = ne;       // R / Cholesky work array, ld x ld
+  const int lp = ne + 1;   // odd column stride of the right-hand sides
+  double* const bR = kSmem ? smem_d : out.scratch;
+  double* const bV = bR + ld * ld;
+  __shared__ int dropped[kMaxW];
+  __shared__ double invd[kMaxW];        // 1 / d_j (0 for a dropped pivot)
+  __shared__ double rinv[kMaxW];        // 1 / R_jj (0 for a dropped pivot)
+  __shared__ double gmax_s;
+  const int tid = threadIdx.x;
+  const int ty = tid >> 5, tx = tid & 31;
+  constexpr int W = kSolverWarps;
+
+  for (int e = tid; e < n * n; e += kSolverThreads) {
+    const int i = e / n, j = e - (e / n) * n;
+    if (j >= i) bR[i * ld + j] = G[e];
+  }
+  if (ty == 0) {
     double g = 0.0;
-    for (int j = 0; j < n; ++j) g = fmax(g, G[j * n + j]);
-    gmax_s = g;
+    for (int j = tx; j < n; j += 32) g = fmax(g, G[j * n + j]);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) g = fmax(g, __shfl_xor_sync(0xffffffffu, g, off));
+    if (tx == 0) gmax_s = g;
   }
   __syncthreads();
   const double tol = kDropTol * gmax_s;
-  // Cholesky G = R^T R with dependent columns dropped (their row of R is zero)
-  for (int j = 0; j < n; ++j) {
-    if (tid == 0) {
-      double d = G[j * n + j];
-      for (int i = 0; i < j; ++i) d -= R[i * ld + j] * R[i * ld + j];
-      const bool drop = !(d > tol) || gmax_s == 0.0;
-      dropped[j] = drop;
-      pivot_s = drop ? 0.0 : sqrt(d);
-      R[j * ld + j] = pivot_s;
-    }
-    __syncthreads();
-    if (!dropped[j]) {
-      for (int t = j + 1 + tid; t < n; t += nt) {
-        double v = G[j * n + t];
-        for (int i = 0; i < j; ++i) v -= R[i * ld + j] * R[i * ld + t];
-        R[j * ld + t] = v / pivot_s;
-      }
-    }
-    __syncthreads();
-  }
-  // R^+: column j solves R x = e_j on the kept indices
-  for (int j = tid; j < n; j += nt) {
-    if (dropped[j]) continue;
-    Rinv[j * kMaxW + j] = 1.0 / R[j * ld + j];
-    for (int i = j - 1; i >= 0; --i) {
-      if (dropped[i]) continue;
-      double acc = 0.0;
-      for (int t = i + 1; t <= j; ++t) acc += R[i * ld + t] * Rinv[t * kMaxW + j];
-      Rinv[i * kMaxW + j] = -acc / R[i * ld + i];
-    }
-  }
-  __syncthreads();
-  if (mode == 0) {
-    for (int e = tid; e < n * n; e += nt) out.T[(e / n) * kMaxW + e % n] = Rinv[(e / n) * kMaxW + e % n];
-    return;
-  }
-  // A by columns: mode 1 takes A = R^T, whose column j is row j of R (already the
-  // layout); mode 2 takes A = R, so transpose in place.
-  if (mode == 2) {
-    for (int e = tid; e < ld * ld; e += nt) {
-      const int i = e / ld, j = e % ld;
-      if (i < j) {
-        const double a = R[i * ld + j];
-        R[i * ld + j] = R[j * ld + i];
-        R[j * ld + i] = a;
-      }
-    }
-  }
-  for (int e = tid; e < vld * vld; e += nt) Vt[e] = ((e / vld) == (e % vld) && (e / vld) < ne) ? 1.0 : 0.0;
-  __syncthreads();
-  const int warp = tid >> 5, lane = tid & 31, nwarps = nt >> 5;
-  const int npairs = ne / 2;
-  int sweep = 0;
-  for (; sweep < kJacobiMaxSweeps; ++sweep) {
-    if (tid == 0) any_rot = 0;
-    // exact column norms at the start of every sweep; within the sweep they are
-    // updated with each rotation (||a_p||^2 -= t g, ||a_q||^2 += t g)
-    for (int j = tid; j < ne; j += nt) {
-      double s2 = 0.0;
-      for (int r = 0; r < ne; ++r) s2 = fma(At[j * ld + r], At[j * ld + r], s2);
-      nrm[j] = s2;
-    }
-    __syncthreads();
-    for (int round = 0; round < ne - 1; ++round) {
-      for (int pr = warp; pr < npairs; pr += nwarps) {
-        // round-robin tournament: position 0 stays, the others rotate each round
-        const int pa = pr, pb = ne - 1 - pr;
-        int p = pa == 0 ? 0 : 1 + (pa - 1 + round) % (ne - 1);
-        int q = pb == 0 ? 0 : 1 + (pb - 1 + round) % (ne - 1);
-        if (p > q) {
-          const int t = p;
-          p = q;
-          q = t;
+
+  // ---- Cholesky in panels: warp 0 factors the panel rows, all threads update the rest
+  for (int jb = 0; jb < n; jb += kPanel) {
+    const int je = min(n, jb + kPanel);
+    if (ty == 0) {
+      for (int j = jb; j < je; ++j) {
+        const double d = bR[j * ld + j];
+        const bool drop = !(d > tol) || gmax_s == 0.0;
+        const double inv_d = drop ? 0.0 : 1.0 / d;
+        if (tx == 0) {
+          dropped[j] = drop;
+          invd[j] = inv_d;
         }
-        double* cp = At + p * ld;
-        double* cq = At + q * ld;
-        const double al = nrm[p], be = nrm[q];
-        double ga = 0.0;
-        for (int r = lane; r < ne; r += 32) ga = fma(cp[r], cq[r], ga);
+        if (!drop) {
+          for (int i = j + 1; i < je; ++i) {
+            const double coef = bR[j * ld + i] * inv_d;
+            for (int t = i + tx; t < n; t += 32) bR[i * ld + t] = fma(-coef, bR[j * ld + t], bR[i * ld + t]);
+          }
+        }
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+    // trailing rows i >= je: B_it -= sum_j B_ji B_jt / d_j over the panel, t >= i
+    const int m = n - je;
+    if (m > 0) {
+      const int np = je - jb;
+      for (int e = tid; e < m * 32; e += kSolverThreads) {
+        const int i = je + e / 32, lane = e & 31;
+        double cf[kPanel];
 #pragma unroll
-        for (int off = 16; off; off >>= 1) ga += __shfl_xor_sync(0xffffffffu, ga, off);
-        if (ga != 0.0 && fabs(ga) > kJacobiTol * sqrt(al * be)) {
-          const double zeta = (be - al) / (2.0 * ga);
-          const double t = (zeta >= 0.0 ? 1.0 : -1.0) / (fabs(zeta) + sqrt(1.0 + zeta * zeta));
-          const double c = 1.0 / sqrt(1.0 + t * t), s = c * t;
-          double* vp = Vt + p * vld;
-          double* vq = Vt + q * vld;
-          for (int r = lane; r < ne; r += 32) {
-            const double x = cp[r], y = cq[r];
-            cp[r] = c * x - s * y;
-            cq[r] = s * x + c * y;
-            const double vx = vp[r], vy = vq[r];
-            vp[r] = c * vx - s * vy;
-            vq[r] = s * vx + c * vy;
-          }
-          if (lane == 0) {
-            any_rot = 1;
-            nrm[p] = al - t * ga;
-            nrm[q] = be + t * ga;
-          }
+        for (int q = 0; q < kPanel; ++q) cf[q] = q < np ? bR[(jb + q) * ld + i] * invd[jb + q] : 0.0;
+        for (int t = i + lane; t < n; t += 32) {
+          double acc = bR[i * ld + t];
+#pragma unroll
+          for (int q = 0; q < kPanel; ++q)
+            if (q < np) acc = fma(-cf[q], bR[(jb + q) * ld + t], acc);
+          bR[i * ld + t] = acc;
         }
       }
-      __syncthreads();
     }
-    if (!any_rot) break;
     __syncthreads();
   }
-  if (sweep == kJacobiMaxSweeps && tid == 0) {
-    raise_status(status, METIS_DEV_NUMERIC);
-    out.flags[0] = 1;
+  for (int j = tid; j < n; j += kSolverThreads) rinv[j] = dropped[j] ? 0.0 : rsqrt(bR[j * ld + j]);
+  __syncthreads();
+  // R (scaled) column-major into the lower part: R[r][i] at bR[i * ld + r]
+  for (int j = ty; j < ne; j += W) {
+    for (int t = j + tx; t < ne; t += 32) {
+      double v = 0.0;
+      if (t < n && j < n && !dropped[j]) v = bR[j * ld + t] * rinv[j];
+      bR[t * ld + j] = v;
+    }
   }
-  // singular values and descending order (ties by index)
-  for (int j = tid; j < ne; j += nt) {
-    double s2 = 0.0;
-    for (int r = 0; r < ne; ++r) s2 = fma(At[j * ld + r], At[j * ld + r], s2);
-    sig[j] = sqrt(s2);
+  // identity right-hand sides, column c at bV + c * lp
+  for (int e = tid; e < ne * lp; e += kSolverThreads) {
+    const int c = e / lp, r = e - c * lp;
+    bV[e] = (c == r && c < n) ? 1.0 : 0.0;
   }
   __syncthreads();
-  for (int j = tid; j < ne; j += nt) {
+
+  // ---- blocked back substitution R X = I; x_i = B_i / R_ii (0 for a dropped pivot)
+  for (int ie = n; ie > 0; ie -= kPanel) {
+    const int ib = max(0, ie - kPanel);
+    for (int c = tid; c < n; c += kSolverThreads) {   // diagonal block, a thread per column
+      double* col = bV + c * lp;
+      for (int i = ie - 1; i >= ib; --i) {
+        const double x = col[i] * rinv[i];
+        col[i] = x;
+        for (int r = ib; r < i; ++r) col[r] = fma(-bR[i * ld + r], x, col[r]);
+      }
+    }
+    __syncthreads();
+    if (ib > 0) {   // rows above the block: B_r -= sum_i R[r][i] x_i
+      const int nb = ie - ib;
+      for (int c = ty; c < n; c += W) {
+        double* col = bV + c * lp;
+        double x[kPanel];
+#pragma unroll
+        for (int q = 0; q < kPanel; ++q) x[q] = q < nb ? col[ib + q] : 0.0;
+        for (int r = tx; r < ib; r += 32) {
+          double acc = col[r];
+#pragma unroll
+          for (int q = 0; q < kPanel; ++q)
+            if (q < nb) acc = fma(-bR[(ib + q) * ld + r], x[q], acc);
+          col[r] = acc;
+        }
+      }
+    }
+    __syncthreads();
+  }
+  for (int e = tid; e < n * n; e += kSolverThreads) {
+    const int i = e / n, c = e - (e / n) * n;
+    out.T[i * kMaxW + c] = bV[c * lp + i];
+  }
+}
+
+// mode 1: T only (refresh basis); mode 2: T, Vr and S (per-step factors)
+template <bool kSmem>
+__global__ void __launch_bounds__(kEigThreads) eig_solver_kernel(const double* __restrict__ G, int n, int k,
+                                                                    int mode, SmallOut out, uint32_t* status) {
+  extern __shared__ double smem_d[];
+  const int ne = (n + 1) & ~1;
+  const int ld = ne + 1;   // odd stride: rows and columns of H, columns of Z, all conflict-free
+  double* const H = kSmem ? smem_d : out.scratch;   // H[i * ld + j], symmetric
+  double* const Z = H + ne * ld;                     // column c at Z + c * ld
+  __shared__ double lam[kMaxW];
+  __shared__ int order[kMaxW];
+  __shared__ double rot_c[kMaxW / 2], rot_s[kMaxW / 2];
+  // flags double-buffered by parity: a flag is cleared one step before it is set and
+  // read, so no thread clears it while another still reads it
+  __shared__ int any_rot[2], round_rot[2], need_rot;
+  const int tid = threadIdx.x;
+  const int ty = tid >> 5, tx = tid & 31;
+  constexpr int W = kEigThreads / 32;
+  constexpr int LR = kSmem ? (kSmallMaxN + 31) / 32 : kLaneRows;   // entries of a row or column per lane
+
+  for (int e = tid; e < ne * ld; e += kEigThreads) {
+    const int i = e / ld, j = e - (e / ld) * ld;
+    H[e] = (i < n && j < n) ? G[i * n + j] : 0.0;
+    Z[e] = (i == j) ? 1.0 : 0.0;
+  }
+  if (tid == 0) {
+    need_rot = 0;
+    any_rot[0] = 0;
+    round_rot[0] = 0;
+  }
+  __syncthreads();
+  const int npairs = ne / 2;
+  const double tol2 = kJacobiTol * kJacobiTol;
+  {  // every pair checked at once: none above the tolerance means no sweep rotates
+    bool need = false;
+    for (int p = ty; p < ne && !need; p += W)
+      for (int q = p + 1 + tx; q < ne; q += 32) {
+        const double ga = H[p * ld + q];
+        need = need || (ga != 0.0 && ga * ga > tol2 * (H[p * ld + p] * H[q * ld + q]));
+      }
+    if (need) need_rot = 1;
+  }
+  __syncthreads();
+  int sweep = 0;
+  if (need_rot) {
+    for (; sweep < kJacobiMaxSweeps; ++sweep) {
+      if (tid == 0) round_rot[0] = 0;   // last read before the previous round's barrier
+      __syncthreads();
+      for (int round = 0; round < ne - 1; ++round) {
+        if (tid == 0) {
+          round_rot[(round + 1) & 1] = 0;                // last read in round - 1
+          if (round == 0) any_rot[(sweep + 1) & 1] = 0;  // last read after sweep - 1
+        }
+        // (1) rotation parameters, a thread per pair: with al = H_pp, be = H_qq,
+        // ga = H_pq, t = sign(zeta) / (|zeta| + sqrt(1 + zeta^2)), zeta = (be - al) / (2 ga),
+        // c = 1 / sqrt(1 + t^2), s = c t (written without divisions)
+        for (int pr = tid; pr < npairs; pr += kEigThreads) {
+          int p, q;
+          round_pair(pr, round, ne, p, q);
+          const double al = H[p * ld + p], be = H[q * ld + q], ga = H[p * ld + q];
+          double c = 1.0, s = 0.0;
+          if (ga != 0.0 && ga * ga > tol2 * (al * be)) {
+            const double dd = be - al;
+            const double g2 = 2.0 * ga;
+            const double x = fma(dd, dd, g2 * g2);
+            const double rt = x * rsqrt(x);
+            const double den = fabs(dd) + rt;
+            const double rho = rsqrt(fma(den, den, g2 * g2));
+            const double sgn = (dd == 0.0) ? 1.0 : copysign(1.0, dd) * copysign(1.0, ga);
+            c = den * rho;
+            s = sgn * fabs(g2) * rho;
+            round_rot[round & 1] = 1;
+            any_rot[sweep & 1] = 1;
+          }
+          rot_c[pr] = c;
+          rot_s[pr] = s;
+        }
+        __syncthreads();
+        if (round_rot[round & 1]) {   // uniform
+          // (2) H <- J^T H J and Z <- Z J with J the round's disjoint rotations: a thread per
+          // 2 x 2 block (rows p_i, q_i; columns p_j, q_j), all reads of a block before
+          // its writes; a warp per column pair of Z
+          for (int e = tid; e < npairs * npairs; e += kEigThreads) {
+            const int i = e / npairs, j = e - (e / npairs) * npairs;
+            const double si = rot_s[i], sj = rot_s[j];
+            if (si == 0.0 && sj == 0.0) continue;
+            const double ci = rot_c[i], cj = rot_c[j];
+            int pa, pb, qa, qb;
+            round_pair(i, round, ne, pa, pb);
+            round_pair(j, round, ne, qa, qb);
+            const double h00 = H[pa * ld + qa], h01 = H[pa * ld + qb];
+            const double h10 = H[pb * ld + qa], h11 = H[pb * ld + qb];
+            const double r00 = ci * h00 - si * h10, r10 = si * h00 + ci * h10;   // rows
+            const double r01 = ci * h01 - si * h11, r11 = si * h01 + ci * h11;
+            H[pa * ld + qa] = cj * r00 - sj * r01;                                 // columns
+            H[pa * ld + qb] = sj * r00 + cj * r01;
+            H[pb * ld + qa] = cj * r10 - sj * r11;
+            H[pb * ld + qb] = sj * r10 + cj * r11;
+          }
+          for (int pr = ty; pr < npairs; pr += W) {
+            const double s = rot_s[pr];
+            if (s == 0.0) continue;
+            const double c = rot_c[pr];
+            int p, q;
+            round_pair(pr, round, ne, p, q);
+            double* zp = Z + p * ld;
+            double* zq = Z + q * ld;
+            double za[LR], zb[LR];
+#pragma unroll
+            for (int u = 0; u < LR; ++u) {
+              const int x = tx + 32 * u;
+              if (x < ne) {
+                za[u] = zp[x];
+                zb[u] = zq[x];
+              }
+            }
+#pragma unroll
+            for (int u = 0; u < LR; ++u) {
+              const int x = tx + 32 * u;
+              if (x < ne) {
+                zp[x] = c * za[u] - s * zb[u];
+                zq[x] = s * za[u] + c * zb[u];
+              }
+            }
+          }
+        }
+        __syncthreads();
+      }
+      if (!any_rot[sweep & 1]) break;
+    }
+  }
+  if (tid == 0) {
+    out.flags[1] = sweep;   // sweeps taken (diagnostic)
+    if (sweep == kJacobiMaxSweeps) {
+      raise_status(status, METIS_DEV_NUMERIC);
+      out.flags[0] = 1;
+    }
+  }
+  // eigenvalues and descending order (ties by index; a NaN sorts last)
+  for (int j = tid; j < ne; j += kEigThreads) {
+    const double l = H[j * ld + j];
+    lam[j] = (l == l) ? l : -HUGE_VAL;
+  }
+  __syncthreads();
+  for (int j = tid; j < ne; j += kEigThreads) {
     int rank = 0;
-    for (int i = 0; i < ne; ++i) rank += (sig[i] > sig[j]) || (sig[i] == sig[j] && i < j);
+    for (int i = 0; i < ne; ++i) rank += (lam[i] > lam[j]) || (lam[i] == lam[j] && i < j);
     order[rank] = j;
   }
   __syncthreads();
-  if (mode == 1) {
-    // T = R^+ W'[:, top k]  (n x k), W' the accumulated rotations
-    for (int e = tid; e < n * k; e += nt) {
-      const int i = e / k, c = e % k;
-      const double* wcol = Vt + order[c] * vld;
-      double a = 0.0;
-      for (int t = 0; t < n; ++t) a = fma(Rinv[i * kMaxW + t], wcol[t], a);
-      out.T[i * kMaxW + c] = a;
+  const double lmax = fmax(lam[order[0]], 0.0);
+  const double thr = kDropTol * lmax;
+  for (int e = tid; e < n * k; e += kEigThreads) {
+    const int i = e / k, c = e - (e / k) * k;
+    const int src = order[c];
+    const double l = lam[src];
+    const bool keep = l > thr && lmax > 0.0;
+    const double z = Z[src * ld + i];
+    out.T[i * kMaxW + c] = keep ? z * rsqrt(l) : 0.0;
+    if (mode == 2) out.Vr[i * kMaxW + c] = z;
+  }
+  if (mode == 2) {
+    for (int c = tid; c < k; c += kEigThreads) {
+      const double l = lam[order[c]];
+      out.S[c] = (l > thr && lmax > 0.0) ? (float)sqrt(l) : 0.0f;
     }
-  } else {
-    // U_r = A / sigma (zero column for sigma == 0); T = R^+ U_r[:, top k]; Vr; S
-    for (int e = tid; e < n * k; e += nt) {
-      const int i = e / k, c = e % k;
-      const int src = order[c];
-      const double sg = sig[src];
-      double a = 0.0;
-      if (sg > 0.0)
-        for (int t = 0; t < n; ++t) a = fma(Rinv[i * kMaxW + t], At[src * ld + t] / sg, a);
-      out.T[i * kMaxW + c] = a;
-      out.Vr[i * kMaxW + c] = Vt[src * vld + i];
-    }
-    for (int c = tid; c < k; c += nt) out.S[c] = (float)sig[order[c]];
   }
 }
 
@@ -601,7 +748,7 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
   need += (size_t)rows_needed * std::max(w, k) * 4 + 256;         // Q / U
   need += (size_t)c * std::max(w, k) * 4 + 256;                   // Bm^T / V new
   need += (size_t)((std::max(rows_needed, c) + kGramRows - 1) / kGramRows) * w * w * 8 + 256;  // gram partials
-  need += (size_t)kMaxW * kMaxW * 8 * 5 + 2048;                   // G, T, Vr, Rinv, Vt
+  need += (size_t)kMaxW * kMaxW * 8 * 3 + small_solver_doubles(kMaxW) * 8 + 2048;  // G, T, Vr, solver scratch
   need += 64 * 4 * 3 + 1024;                                      // S, flags, flips
   const int kpw = pad_width(std::max(w, k));
   need += (size_t)2 * kpw * c * 2 + 256;                          // hi/lo transposed operand
@@ -623,8 +770,7 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
   double* G = static_cast<double*>(ws.take((size_t)kMaxW * kMaxW * 8));
   double* T = static_cast<double*>(ws.take((size_t)kMaxW * kMaxW * 8));
   double* Vr = static_cast<double*>(ws.take((size_t)kMaxW * kMaxW * 8));
-  double* Rinv = static_cast<double*>(ws.take((size_t)kMaxW * kMaxW * 8));
-  double* Vt = static_cast<double*>(ws.take((size_t)kMaxW * kMaxW * 8));
+  double* sscratch = static_cast<double*>(ws.take(small_solver_doubles(kMaxW) * 8));
   float* Sw = static_cast<float*>(ws.take(64 * 4));
   int* flags = static_cast<int*>(ws.take(64 * 4));
   int* flip = static_cast<int*>(ws.take(64 * 4));
@@ -632,13 +778,27 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
   float* tc_partial = static_cast<float*>(ws.take(tc_partial_bytes));
   if (!tc_partial) return fail(ctx, METIS_ERR_WORKSPACE, "decompose workspace layout");
 
-  const int ne_max = ((std::max(w, k) + 1) & ~1);
-  const size_t small_smem = std::max((size_t)ne_max * ne_max * 8,
-                                     std::min(kSmallSmemMax, (size_t)2 * ne_max * ne_max * 8));
-  cudaError_t e = cudaFuncSetAttribute(small_solver_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)small_smem);
+  cudaError_t e = cudaFuncSetAttribute(cholqr_solver_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)(small_solver_doubles(kSmallMaxN) * 8));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(eig_solver_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(small_solver_doubles(kSmallMaxN) * 8));
   if (e != cudaSuccess) return check_cuda(ctx, e, "cudaFuncSetAttribute(small solver)");
-  SmallOut so{T, Vr, Sw, flags, Rinv, Vt};
+  SmallOut so{T, Vr, Sw, flags, sscratch};
+  // mode 0: CholQR factor T = R^+; modes 1 and 2: SVD through the eigenproblem of G
+  auto solve = [&](int n, int mode) {
+    const int ne = (n + 1) & ~1;
+    const bool in_smem = ne <= kSmallMaxN;
+    const size_t smem = in_smem ? small_solver_doubles(ne) * 8 : 0;
+    if (mode == 0) {
+      if (in_smem) cholqr_solver_kernel<true><<<1, kSolverThreads, smem, st>>>(G, n, so);
+      else cholqr_solver_kernel<false><<<1, kSolverThreads, 0, st>>>(G, n, so);
+    } else {
+      if (in_smem) eig_solver_kernel<true><<<1, kEigThreads, smem, st>>>(G, n, k, mode, so, ctx->status);
+      else eig_solver_kernel<false><<<1, kEigThreads, 0, st>>>(G, n, k, mode, so, ctx->status);
+    }
+    count_launch();
+  };
 
   auto gram = [&](const float* A, int64_t n, int width) {
     const int64_t chunks = (n + kGramRows - 1) / kGramRows;
@@ -687,18 +847,18 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
       return s;
     }
     gram(Y, lk, w);
-    small_solver_kernel<<<1, 1024, small_smem, st>>>(G, w, k, 0, so, ctx->status); count_launch();
+    solve(w, 0);
     times_small_kernel<<<blocks_for(lk * w), 256, 0, st>>>(Y, lk, w, T, w, Q); count_launch();
     // Bm^T = M_s^T Q ; R2 = chol(Bm Bm^T) ; SVD(R2^T) ; V = Bm^T R2^+ W'[:, :k]
     cols_times_matrix_kernel<<<blocks_for(c, 64), 256, 0, st>>>(Mb, M->ld, idx, lk, c, Q, w, Bt); count_launch();
     gram(Bt, c, w);
-    small_solver_kernel<<<1, 1024, small_smem, st>>>(G, w, k, 1, so, ctx->status); count_launch();
+    solve(w, 1);
     times_small_kernel<<<blocks_for(c * k), 256, 0, st>>>(Bt, c, w, T, k, f->V); count_launch();
   }
   // per step: P = M V ; R = chol(P^T P) ; SVD(R) ; U = P R^+ U_r ; V <- V V_r
   if ((s = project(f->V, k, Y)) != METIS_OK) return s;
   gram(Y, r, k);
-  small_solver_kernel<<<1, 1024, small_smem, st>>>(G, k, k, 2, so, ctx->status); count_launch();
+  solve(k, 2);
   times_small_kernel<<<blocks_for(r * k), 256, 0, st>>>(Y, r, k, T, k, Q); count_launch();     // U (unsigned)
   times_small_kernel<<<blocks_for(c * k), 256, 0, st>>>(f->V, c, k, Vr, k, Bt); count_launch();  // V V_r
   sign_pick_kernel<<<k, 256, 0, st>>>(Bt, c, k, flip); count_launch();
