@@ -174,6 +174,28 @@ metis_status metis_quantize_nvfp4_f32(metis_ctx* ctx, const float* R, int64_t ro
                                       int64_t ld, const metis_quant_params* q,
                                       metis_nvfp4* rowwise, metis_nvfp4* colwise);
 
+/*
+ * Allocation-free residual quantization (no counterpart in the paper).
+ * Same computation and results as metis_residual_quantize_nvfp4 with both
+ * orientations, for callers that may not allocate device memory while they run:
+ * a step being captured into a CUDA graph cannot call cudaMalloc, and a
+ * framework that manages device memory through its own caching allocator must
+ * not have a library allocate behind it.  This call allocates nothing: its
+ * scratch (rank-padded copies of U diag(S) and V) is a fixed 6 MiB device array
+ * inside libmetis, present on every GPU that loads the library until the process
+ * exits.  The caller still provides every input and output.
+ *   - rows + cols must not exceed 24576 (k <= 64); larger shapes return
+ *     METIS_ERR_SHAPE with a message.  rowwise and colwise are both required.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device); make that first call before any stream capture begins.
+ *   - All calls share the one array and it keeps the last call's contents (every
+ *     call overwrites the part it reads first).  Calls whose GPU work overlaps --
+ *     e.g. issued on two streams without ordering -- race on it.
+ */
+metis_status metis_residual_quantize_nvfp4_noalloc(metis_ctx* ctx, const metis_matrix* M,
+                                                   const metis_factors* f, const metis_quant_params* q,
+                                                   metis_nvfp4* rowwise, metis_nvfp4* colwise);
+
 /* Output element types. */
 #define METIS_OUT_F32  0
 #define METIS_OUT_BF16 1

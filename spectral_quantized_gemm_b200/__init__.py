@@ -41,7 +41,7 @@ EXPORTED = ["metis_create", "metis_destroy", "metis_set_stream", "metis_status_s
             "metis_poll_device_status", "metis_nvfp4_codes_bytes", "metis_nvfp4_scales_bytes",
             "metis_decompose", "metis_residual_quantize_nvfp4", "metis_quantize_nvfp4_f32", "metis_gemm_nvfp4",
             "metis_linear_fwd", "metis_linear_bwd", "metis_kernel_launches", "metis_profile_enable",
-            "metis_profile_read"]
+            "metis_profile_read", "metis_residual_quantize_nvfp4_noalloc"]
 
 
 class Matrix(ctypes.Structure):
@@ -91,6 +91,9 @@ _decompose = _sig("metis_decompose", c_i32, c_p, ctypes.POINTER(Matrix), ctypes.
                   ctypes.c_int, c_u32, ctypes.POINTER(FactorsStruct))
 _resq = _sig("metis_residual_quantize_nvfp4", c_i32, c_p, ctypes.POINTER(Matrix), ctypes.POINTER(FactorsStruct),
              ctypes.POINTER(QuantParams), ctypes.POINTER(Nvfp4Struct), ctypes.POINTER(Nvfp4Struct))
+_resq_noalloc = _sig("metis_residual_quantize_nvfp4_noalloc", c_i32, c_p, ctypes.POINTER(Matrix),
+                     ctypes.POINTER(FactorsStruct), ctypes.POINTER(QuantParams), ctypes.POINTER(Nvfp4Struct),
+                     ctypes.POINTER(Nvfp4Struct))
 _quant_f32 = _sig("metis_quantize_nvfp4_f32", c_i32, c_p, c_p, c_i64, c_i64, c_i64, ctypes.POINTER(QuantParams),
                   ctypes.POINTER(Nvfp4Struct), ctypes.POINTER(Nvfp4Struct))
 _gemm = _sig("metis_gemm_nvfp4", c_i32, c_p, ctypes.POINTER(Nvfp4Struct), ctypes.POINTER(Nvfp4Struct), c_i64, c_p,
@@ -217,6 +220,14 @@ class Context:
         self._call(_resq, ctypes.byref(_matrix(M)), None if factors is None else ctypes.byref(factors.struct),
                    ctypes.byref(q), None if rowwise is None else ctypes.byref(rowwise.struct),
                    None if colwise is None else ctypes.byref(colwise.struct))
+
+    def residual_quantize_nvfp4_noalloc(self, M, factors, rowwise, colwise, rounding=0, seed=0, operand_id=0,
+                                        step=0, tensor_scale=1.0):
+        """Allocation-free residual quantization: libmetis calls no cudaMalloc here
+        (fixed 6 MiB device scratch; rows + cols <= 24576)."""
+        q = QuantParams(rounding, seed, operand_id, step, tensor_scale)
+        self._call(_resq_noalloc, ctypes.byref(_matrix(M)), None if factors is None else ctypes.byref(factors.struct),
+                   ctypes.byref(q), ctypes.byref(rowwise.struct), ctypes.byref(colwise.struct))
 
     def quantize_nvfp4_f32(self, R, rowwise=None, colwise=None, rounding=0, seed=0, operand_id=0, step=0,
                            tensor_scale=1.0):

@@ -336,3 +336,26 @@ metis_status metis_profile_read(metis_ctx* ctx, double* ms, int64_t* launches, d
 }
 
 }  // extern "C"
+
+extern "C" metis_status metis_residual_quantize_nvfp4_noalloc(metis_ctx* ctx, const metis_matrix* M,
+                                                               const metis_factors* f, const metis_quant_params* q,
+                                                               metis_nvfp4* rowwise, metis_nvfp4* colwise) {
+  metis_status s = enter(ctx);
+  if (s != METIS_OK) return s;
+  if (!M || !M->data) return fail(ctx, METIS_ERR_ARG, "null matrix");
+  if ((s = check_dims(ctx, M->rows, M->cols)) != METIS_OK) return s;
+  if (M->rows + M->cols > kNoAllocMaxRowsPlusCols)
+    return fail(ctx, METIS_ERR_SHAPE, "rows + cols = " + std::to_string(M->rows + M->cols) +
+                                          " exceeds the allocation-free limit of " +
+                                          std::to_string(kNoAllocMaxRowsPlusCols));
+  if (M->ld < M->cols || M->ld % 8 || !aligned16(M->data))
+    return fail(ctx, METIS_ERR_ALIGN, "bf16 matrix needs 16-byte alignment and ld % 8 == 0");
+  if ((s = check_quant(ctx, q)) != METIS_OK) return s;
+  if ((s = check_factors(ctx, f, M->rows, M->cols)) != METIS_OK) return s;
+  if (!rowwise || !colwise) return fail(ctx, METIS_ERR_ARG, "the allocation-free path writes both orientations");
+  if ((s = check_nvfp4(ctx, rowwise, M->rows, M->cols, "rowwise")) != METIS_OK) return s;
+  if ((s = check_nvfp4(ctx, colwise, M->cols, M->rows, "colwise")) != METIS_OK) return s;
+  float* scratch = noalloc_scratch(ctx, &s);
+  if (!scratch) return s;
+  return run_residual_quantize_into(ctx, M, f, q, rowwise, colwise, scratch);
+}

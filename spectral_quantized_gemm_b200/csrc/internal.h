@@ -68,6 +68,15 @@ cudaError_t launch_quantize_factor(const float* F, int64_t longdim, int32_t k, i
 metis_status run_residual_quantize(metis_ctx* ctx, const metis_matrix* M, const metis_factors* f,
                                    const metis_quant_params* q, const metis_nvfp4* row, const metis_nvfp4* col);
 
+// ---- noalloc.cu ----
+// Limits of the allocation-free residual quantizer's fixed scratch.
+constexpr int64_t kNoAllocMaxRowsPlusCols = 24576;
+constexpr int kNoAllocWidth = 64;
+float* noalloc_scratch(metis_ctx* ctx, metis_status* st);
+metis_status run_residual_quantize_into(metis_ctx* ctx, const metis_matrix* M, const metis_factors* f,
+                                        const metis_quant_params* q, const metis_nvfp4* row, const metis_nvfp4* col,
+                                        float* scratch);
+
 // ---- gemm_fp4.cu ----
 struct GemmArgs {
   const metis_nvfp4* A;

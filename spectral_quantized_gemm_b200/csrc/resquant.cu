@@ -460,3 +460,25 @@ metis_status run_residual_quantize(metis_ctx* ctx, const metis_matrix* M, const 
 }
 
 }  // namespace metis
+
+namespace metis {
+
+// Same work as run_residual_quantize, with the padded factor copies written to
+// caller-provided device scratch of (rows + cols) * 64 floats instead of the
+// context workspace.
+metis_status run_residual_quantize_into(metis_ctx* ctx, const metis_matrix* M, const metis_factors* f,
+                                        const metis_quant_params* q, const metis_nvfp4* row, const metis_nvfp4* col,
+                                        float* scratch) {
+  const int k = (f && f->k > 0) ? f->k : 0;
+  const int KK = k <= 32 ? 32 : 64;
+  float* US = scratch;
+  float* Vp = scratch + M->rows * KK;
+  const int64_t n = (M->rows + M->cols) * KK;
+  pad_factors_kernel<<<(unsigned)((n + 255) / 256), 256, 0, ctx->stream>>>(
+      k ? f->U : nullptr, k ? f->S : nullptr, k ? f->V : nullptr, M->rows, M->cols, k, KK, US, Vp); count_launch();
+  metis_status s = check_cuda(ctx, cudaGetLastError(), "pad factors");
+  if (s != METIS_OK) return s;
+  return KK == 32 ? launch_kk<32>(ctx, M, US, Vp, q, row, col) : launch_kk<64>(ctx, M, US, Vp, q, row, col);
+}
+
+}  // namespace metis
