@@ -20,18 +20,24 @@ block v with decode tensor scale g (a power of two):
 
 Stochastic rounding (R4 of the build's readings): with a = |x|, if a >= 6 the
 magnitude is 6; otherwise lo <= a < hi are the neighbouring E2M1 magnitudes,
-p = (a - lo) / (hi - lo) (exact in fp32: a - lo is exact by Sterbenz, hi - lo
-is a power of two) and the magnitude rounds up to hi iff u < p, where u is
-the element's 16-bit uniform from ``philox.sr_uniforms``.  The sign of x is
-kept.  Scales are always rounded to nearest.
+p = (a - lo) / (hi - lo) (exact: a - lo is exact by Sterbenz, hi - lo is a
+power of two) and the magnitude rounds up to hi iff
+
+    floor(p * 2^16) + F >= 2^16,
+
+F being the element's 16-bit random field from ``philox.sr_fields`` (so the
+chance of rounding up is floor(p * 2^16) / 2^16: unbiased to within 2^-16 of a
+grid step).  The sign of x is kept, so a negative value that rounds to zero
+gives -0.  Scales are always rounded to nearest.
 
 Readings that go beyond the pages are listed in the design doc: the per-tensor
 decode scale g (1.0 for residuals unless the caller sets one), the reciprocal
-multiply in step 5-6, and the SR uniform layout.
+multiply in step 5-6, and the SR random-field layout.
 
 Pins (tests/test_oracle_nvfp4.py): round trips of values already on the
 grid, the scale rule against hand-computed blocks, dequantization error
-bounded by half a grid step, SR unbiasedness over many seeds, the all-zero
+bounded by half a grid step, SR: the exact count of up-roundings over all
+2^16 fields, unbiasedness over many seeds, a hand-worked block; the all-zero
 block, saturation, and the packed layout.
 """
 
@@ -54,17 +60,18 @@ def _scale_codes(amax, g):
     return codes
 
 
-def _sr_magnitude(a, u):
-    """Stochastic rounding of magnitudes a in [0, 6) onto the E2M1 grid."""
+def _sr_magnitude(a, fields):
+    """Stochastic rounding of magnitudes a in [0, 6) onto the E2M1 grid (index of the result)."""
     grid = formats.E2M1_MAGNITUDES
     lo_idx = np.searchsorted(grid, a, side="right") - 1       # grid[lo_idx] <= a < grid[lo_idx+1]
     lo = grid[lo_idx]
     hi = grid[lo_idx + 1]
     p = (a - lo) / (hi - lo)
-    return np.where(u < p, lo_idx + 1, lo_idx)
+    up = np.floor(p * 65536.0) + np.asarray(fields, dtype=np.float64) >= 65536.0
+    return np.where(up, lo_idx + 1, lo_idx)
 
 
-def quantize_blocks(M, g=1.0, rounding="rn", u=None):
+def quantize_blocks(M, g=1.0, rounding="rn", fields=None):
     """Quantize ``M`` (outer x inner, fp32 values) with 16-blocks along inner.
 
     Returns (codes, scale_codes): codes is uint8 (outer x inner) holding one
@@ -90,12 +97,12 @@ def quantize_blocks(M, g=1.0, rounding="rn", u=None):
     if rounding == "rn":
         codes = formats.e2m1_encode_rn(x.astype(np.float64))
     elif rounding == "sr":
-        if u is None:
-            raise ValueError("stochastic rounding needs uniforms")
-        u = np.asarray(u, dtype=np.float64).reshape(outer, inner // BLOCK, BLOCK)
+        if fields is None:
+            raise ValueError("stochastic rounding needs random fields")
+        fields = np.asarray(fields, dtype=np.int64).reshape(outer, inner // BLOCK, BLOCK)
         a = np.abs(x.astype(np.float64))
         saturated = a >= 6.0
-        mag_idx = np.where(saturated, 7, _sr_magnitude(np.where(saturated, 0.0, a), u))
+        mag_idx = np.where(saturated, 7, _sr_magnitude(np.where(saturated, 0.0, a), fields))
         codes = (mag_idx.astype(np.uint8) | (np.signbit(x).astype(np.uint8) << 3))
     else:
         raise ValueError(rounding)
@@ -131,16 +138,16 @@ def quantize_oriented(M, orientation, g=1.0, rounding="rn", seed=0, operand_id=0
 
     Column-wise quantization is row-wise quantization of M^T, so both return
     ``outer x inner`` codes with inner the blocked (contraction) dimension.
-    SR uniforms follow the blocked-contiguous element order e = i*inner + j
+    SR fields follow the blocked-contiguous element order e = i*inner + j
     of the oriented view, from sub-stream ``sr_sub`` (default: 0 for
     row-wise, 1 for column-wise).
     """
     M = np.asarray(M, dtype=np.float32)
     view = M if orientation == "row" else M.T
     view = np.ascontiguousarray(view)
-    u = None
+    fields = None
     if rounding == "sr":
         if sr_sub is None:
             sr_sub = philox.SR_SUB_ROWWISE if orientation == "row" else philox.SR_SUB_COLWISE
-        u = philox.sr_uniforms(seed, operand_id, sr_sub, step, view.size).reshape(view.shape)
-    return quantize_blocks(view, g, rounding, u)
+        fields = philox.sr_fields(seed, operand_id, sr_sub, step, view.size).reshape(view.shape)
+    return quantize_blocks(view, g, rounding, fields)

@@ -96,12 +96,12 @@ def test_quantizer_full_size_sampled_rows(ctx, metis_lib):
     R = dev.cpu().numpy()
     codes = row.codes.view(rows, cols // 2)
     for i in np.random.default_rng(0).choice(rows, 24, replace=False):
-        u = philox.sr_uniforms_at(2, 2, philox.SR_SUB_ROWWISE, 9, np.arange(i * cols, (i + 1) * cols))
+        u = philox.sr_fields_at(2, 2, philox.SR_SUB_ROWWISE, 9, np.arange(i * cols, (i + 1) * cols))
         want_c, _ = nvfp4.quantize_blocks(R[i:i + 1], 1.0, "sr", u[None, :])
         assert np.array_equal(nvfp4.unpack_codes(codes[i:i + 1].cpu().numpy()), want_c)
     colcodes = col.codes.view(cols, rows // 2)
     for j in np.random.default_rng(1).choice(cols, 24, replace=False):
-        u = philox.sr_uniforms_at(2, 2, philox.SR_SUB_COLWISE, 9, np.arange(j * rows, (j + 1) * rows))
+        u = philox.sr_fields_at(2, 2, philox.SR_SUB_COLWISE, 9, np.arange(j * rows, (j + 1) * rows))
         want_c, _ = nvfp4.quantize_blocks(np.ascontiguousarray(R[:, j][None, :]), 1.0, "sr", u[None, :])
         assert np.array_equal(nvfp4.unpack_codes(colcodes[j:j + 1].cpu().numpy()), want_c)
 

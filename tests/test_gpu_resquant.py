@@ -84,7 +84,7 @@ def test_full_size_gradient_shape(ctx, metis_lib):
     codes = nvfp4.unpack_codes(row.codes.view(rows, cols // 2)[torch.from_numpy(pick)].cpu().numpy())
     agree = []
     for a, i in enumerate(pick):
-        u = philox.sr_uniforms_at(2, 2, philox.SR_SUB_ROWWISE, 0, np.arange(i * cols, (i + 1) * cols))
+        u = philox.sr_fields_at(2, 2, philox.SR_SUB_ROWWISE, 0, np.arange(i * cols, (i + 1) * cols))
         wc, _ = nvfp4.quantize_blocks(R[a:a + 1], 1.0, "sr", u[None, :])
         agree.append(np.mean(codes[a] == wc[0]))
     assert np.mean(agree) > 0.99

@@ -18,7 +18,7 @@ def _golden_blocks(golden_dir):
             cases.append(dict(
                 name=name, rounding=rounding, g=float(g),
                 v=np.array([float(x) for x in vals.split()], dtype=np.float32),
-                u=None if us == "-" else np.array([float(x) for x in us.split()]),
+                fields=None if us == "-" else np.array([int(x) for x in us.split()]),
                 scale=int(scale, 16), codes=[int(c, 16) for c in codes.split()]))
     return cases
 
@@ -27,8 +27,8 @@ def test_hand_worked_blocks(golden_dir):
     cases = _golden_blocks(golden_dir)
     assert len(cases) == 7
     for c in cases:
-        u = None if c["u"] is None else c["u"][None, :]
-        codes, scales = nvfp4.quantize_blocks(c["v"][None, :], c["g"], c["rounding"], u)
+        fields = None if c["fields"] is None else c["fields"][None, :]
+        codes, scales = nvfp4.quantize_blocks(c["v"][None, :], c["g"], c["rounding"], fields)
         assert int(scales[0, 0]) == c["scale"], c["name"]
         assert [int(x) for x in codes[0]] == c["codes"], c["name"]
 
@@ -77,6 +77,28 @@ def test_non_finite_is_rejected():
         nvfp4.quantize_blocks(v)
 
 
+def test_sr_up_count_over_all_fields():
+    # over the 2^16 equally likely fields an element between grid points rounds up
+    # exactly floor(p 2^16) times, p its fractional position
+    rng = np.random.default_rng(7)
+    F = np.arange(65536)
+    for x in np.concatenate([rng.uniform(0, 5.99, 12), [0.25, 0.3, 1.75, 3.999, 4.0000005, 5.5]]).astype(np.float32):
+        v = np.zeros((65536, 16), dtype=np.float32)
+        v[:, 0] = 6.0                           # scale code 0x38: d = 1, x = v
+        v[:, 1] = x
+        f = np.zeros((65536, 16), dtype=np.int64)
+        f[:, 1] = F
+        codes, scales = nvfp4.quantize_blocks(v, 1.0, "sr", f)
+        assert np.all(scales == 0x38)
+        mags = formats.E2M1_MAGNITUDES[codes[:, 1] & 7]
+        grid = formats.E2M1_MAGNITUDES
+        lo = grid[np.searchsorted(grid, float(x), "right") - 1]
+        hi = grid[np.searchsorted(grid, float(x), "right")]
+        p = (float(x) - lo) / (hi - lo)
+        assert set(np.unique(mags)) <= {lo, hi}
+        assert int(np.sum(mags == hi)) == int(np.floor(p * 65536))
+
+
 def test_sr_is_unbiased():
     rng = np.random.default_rng(2)
     v = rng.uniform(-5.9, 5.9, size=(1, 16)).astype(np.float32)
@@ -121,7 +143,7 @@ def test_orientation_and_packing():
 def test_sr_uses_the_orientation_stream():
     rng = np.random.default_rng(6)
     M = rng.standard_normal((16, 16)).astype(np.float32)
-    u = philox.sr_uniforms(9, 2, philox.SR_SUB_COLWISE, 4, 256).reshape(16, 16)
-    want, _ = nvfp4.quantize_blocks(np.ascontiguousarray(M.T), 1.0, "sr", u)
+    f = philox.sr_fields(9, 2, philox.SR_SUB_COLWISE, 4, 256).reshape(16, 16)
+    want, _ = nvfp4.quantize_blocks(np.ascontiguousarray(M.T), 1.0, "sr", f)
     got, _ = nvfp4.quantize_oriented(M, "col", rounding="sr", seed=9, operand_id=2, step=4)
     assert np.array_equal(want, got)

@@ -44,16 +44,38 @@ def test_element_words_layout():
         assert int(w[e]) == int(calls[e >> 2][e & 3])
 
 
-def test_sr_uniform_layout_and_range():
+def test_sr_field_layout():
+    # element e: counter e >> 4, word (e >> 2) & 3, position e & 3 of the word's group
     n = 40
-    u = philox.sr_uniforms(3, 1, philox.SR_SUB_COLWISE, 9, n)
+    f = philox.sr_fields(3, 1, philox.SR_SUB_COLWISE, 9, n)
     calls = philox.stream_words(3, philox.tag(1, philox.PURPOSE_SR, philox.SR_SUB_COLWISE), 9,
-                                np.arange(5, dtype=np.uint64))
+                                np.arange(3, dtype=np.uint64))
     for e in range(n):
-        word = int(calls[e >> 3][(e >> 1) & 3])
-        half = (word >> (16 * (e & 1))) & 0xFFFF
-        assert u[e] == half / 65536.0
-    assert np.all((u >= 0) & (u < 1))
+        word = int(calls[e >> 4][(e >> 2) & 3])
+        assert int(f[e]) == int(philox.fields_from_words(np.uint64(word), e & 3))
+    assert np.all((f >= 0) & (f < 65536))
+    at = philox.sr_fields_at(3, 1, philox.SR_SUB_COLWISE, 9, np.array([39, 0, 17]))
+    assert [int(x) for x in at] == [int(f[39]), int(f[0]), int(f[17])]
+
+
+def test_sr_fields_of_a_word_by_hand():
+    # W = 0x12345678: b0 = 0x78, b1 = 0x56, b2 = 0x34, b3 = 0x12
+    # position 0: b2:b0 = 0x3478; 1: 0x3478 bit-reversed = 0x1E2C;
+    # position 2: b3:b1 = 0x1256; 3: 0x1256 bit-reversed = 0x6A48
+    w = np.uint64(0x12345678)
+    got = [int(philox.fields_from_words(w, p)) for p in range(4)]
+    assert got == [0x3478, 0x1E2C, 0x1256, 0x6A48]
+
+
+def test_sr_fields_are_uniform_per_position():
+    # 2^14 groups: the high byte of every position's field is uniform (chi-square,
+    # 255 dof, mean 255, sd ~22.6)
+    f = philox.sr_fields(11, 0, philox.SR_SUB_ROWWISE, 0, 1 << 16).reshape(-1, 4)
+    for p in range(4):
+        counts = np.bincount((f[:, p] >> 8).astype(np.int64), minlength=256)
+        expected = f.shape[0] / 256
+        chi2 = float(np.sum((counts - expected) ** 2 / expected))
+        assert 150 < chi2 < 380, p
 
 
 def test_uniformity_chi_square():
