@@ -735,8 +735,9 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
   const __nv_bfloat16* Mb = static_cast<const __nv_bfloat16*>(M->data);
   cudaStream_t st = ctx->stream;
 
-  // split the long dimension of the skinny products into chunks of ~1024 columns
-  const int64_t split_len = 1024;
+  // split the long dimension of the sampled sketch into chunks of 128 columns, so that
+  // (row blocks x chunks) fills the GPU even with l_k = 82 rows
+  const int64_t split_len = 128;
   const int nsplit = (int)((c + split_len - 1) / split_len);
   const int64_t rows_needed = std::max(r, lk);
   size_t need = 0;

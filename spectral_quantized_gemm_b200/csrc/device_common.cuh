@@ -90,30 +90,16 @@ __device__ __forceinline__ uint32_t e2m1x2_rn(float lo, float hi) {
   return r;
 }
 
-// Stochastic rounding of a scaled value onto the E2M1 grid (sign kept):
-// magnitude a >= 6 gives 6; otherwise lo <= a < hi are grid neighbours and the
-// magnitude rounds up iff u < (a - lo) / (hi - lo).  All steps are exact.
-__device__ __forceinline__ float e2m1_sr_value(float x, float u) {
-  const float a = fabsf(x);
-  float q;
-  if (a >= 6.0f) {
-    q = 6.0f;
-  } else {
-    const float h = a < 2.0f ? 0.5f : (a < 4.0f ? 1.0f : 2.0f);
-    const float inv_h = a < 2.0f ? 2.0f : (a < 4.0f ? 1.0f : 0.5f);
-    const float t = a * inv_h;
-    const float fl = floorf(t);
-    const float p = t - fl;
-    q = (u < p ? fl + 1.0f : fl) * h;
-  }
-  return copysignf(q, x);
-}
-
-// Uniform of element e (16-bit half e&1 of word (e>>1)&3 of counter e>>3).
-__device__ __forceinline__ float sr_uniform_from_words(const Words4& w, uint32_t e_in_call) {
-  const uint32_t word = w.w[(e_in_call >> 1) & 3u];
-  const uint32_t half = (e_in_call & 1u) ? (word >> 16) : (word & 0xFFFFu);
-  return (float)half * (1.0f / 65536.0f);
+// Stochastic rounding of four scaled values onto the E2M1 grid with 32 random bits w
+// (codes of x0..x3 in bits 0-3 .. 12-15).  Per element, sign kept and |x| >= 6 giving 6:
+// with lo <= |x| < hi the neighbouring magnitudes and p = (|x| - lo) / (hi - lo), the
+// magnitude rounds up iff floor(p * 2^16) + F >= 2^16, where F is the element's 16-bit
+// field of w: x0 takes bytes b2:b0, x1 the same 16 bits reversed, x2 takes b3:b1, x3
+// those reversed.  The conversion instruction applies exactly this rule.
+__device__ __forceinline__ uint32_t e2m1x4_sr(float x0, float x1, float x2, float x3, uint32_t w) {
+  uint16_t r;
+  asm("cvt.rs.satfinite.e2m1x4.f32 %0, {%1, %2, %3, %4}, %5;" : "=h"(r) : "f"(x3), "f"(x2), "f"(x1), "f"(x0), "r"(w));
+  return (uint32_t)r;
 }
 
 // Byte offset of the scale of (row o, block b) inside the tiled scale array of
@@ -141,22 +127,24 @@ __device__ __forceinline__ BlockScale block_scale(float amax, float g) {
   return bs;
 }
 
-// Encodes 16 fp32 values of one block (already multiplied by the reciprocal
-// scale) into 8 bytes (two uint32).  rounding: 0 RN, 1 SR with uniforms u.
-__device__ __forceinline__ uint2 encode16(const float (&x)[16], int rounding, const float* u) {
-  uint32_t b[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    float lo = x[2 * i], hi = x[2 * i + 1];
-    if (rounding) {
-      lo = e2m1_sr_value(lo, u[2 * i]);
-      hi = e2m1_sr_value(hi, u[2 * i + 1]);
-    }
-    b[i] = e2m1x2_rn(lo, hi);
-  }
+// Codes of one 16-element block whose values are already multiplied by the block's
+// reciprocal scale, packed two per byte (element 2i in the low nibble of byte i).
+// rounding 0: round to nearest even; 1: stochastic, with the four words of the Philox
+// call of counter e0 / 16 (e0 = the block's first element index, a multiple of 16).
+__device__ __forceinline__ uint2 encode_block16(const float (&x)[16], int rounding, uint64_t seed, uint32_t tag,
+                                                uint32_t step, uint64_t e0) {
   uint2 r;
-  r.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
-  r.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+  if (rounding) {
+    const Words4 w = stream_call(seed, tag, step, e0 >> 4);
+    r.x = e2m1x4_sr(x[0], x[1], x[2], x[3], w.w[0]) | (e2m1x4_sr(x[4], x[5], x[6], x[7], w.w[1]) << 16);
+    r.y = e2m1x4_sr(x[8], x[9], x[10], x[11], w.w[2]) | (e2m1x4_sr(x[12], x[13], x[14], x[15], w.w[3]) << 16);
+  } else {
+    uint32_t b[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) b[i] = e2m1x2_rn(x[2 * i], x[2 * i + 1]);
+    r.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+    r.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+  }
   return r;
 }
 

@@ -50,18 +50,8 @@ __global__ void quantize_rowwise_f32_kernel(const float* __restrict__ R, int64_t
   float x[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) x[i] = __fmul_rn(v[i], bs.rcp);
-  float u[16];
-  if (rounding) {
-    const uint64_t e0 = (uint64_t)o * (uint64_t)cols + (uint64_t)b * 16;
-    const Words4 w0 = stream_call(seed, tag, step, e0 >> 3);
-    const Words4 w1 = stream_call(seed, tag, step, (e0 >> 3) + 1);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      u[i] = sr_uniform_from_words(w0, i);
-      u[8 + i] = sr_uniform_from_words(w1, i);
-    }
-  }
-  uint2 packed = encode16(x, rounding, u);
+  const uint64_t e0 = (uint64_t)o * (uint64_t)cols + (uint64_t)b * 16;
+  uint2 packed = encode_block16(x, rounding, seed, tag, step, e0);
   if (bs.code == 0) packed = make_uint2(0, 0);
   *reinterpret_cast<uint2*>(codes + o * (cols / 2) + b * 8) = packed;
   scales[scale_offset(o, b, cols / 64)] = (uint8_t)bs.code;
@@ -94,18 +84,8 @@ __global__ void quantize_colwise_f32_kernel(const float* __restrict__ R, int64_t
   float x[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) x[i] = __fmul_rn(v[i], bs.rcp);
-  float u[16];
-  if (rounding) {
-    const uint64_t e0 = (uint64_t)j * (uint64_t)rows + (uint64_t)b * 16;
-    const Words4 w0 = stream_call(seed, tag, step, e0 >> 3);
-    const Words4 w1 = stream_call(seed, tag, step, (e0 >> 3) + 1);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      u[i] = sr_uniform_from_words(w0, i);
-      u[8 + i] = sr_uniform_from_words(w1, i);
-    }
-  }
-  uint2 packed = encode16(x, rounding, u);
+  const uint64_t e0 = (uint64_t)j * (uint64_t)rows + (uint64_t)b * 16;
+  uint2 packed = encode_block16(x, rounding, seed, tag, step, e0);
   if (bs.code == 0) packed = make_uint2(0, 0);
   *reinterpret_cast<uint2*>(codes + j * (rows / 2) + b * 8) = packed;
   scales[scale_offset(j, b, rows / 64)] = (uint8_t)bs.code;
@@ -210,18 +190,8 @@ __global__ void quantize_factor_kernel(const float* __restrict__ F, int64_t long
     float x[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) x[i] = __fmul_rn(v[i], bs.rcp);
-    float u[16];
-    if (rounding) {
-      const uint64_t e0 = (uint64_t)j * (uint64_t)longdim + (uint64_t)b * 16;
-      const Words4 w0 = stream_call(seed, tag, step, e0 >> 3);
-      const Words4 w1 = stream_call(seed, tag, step, (e0 >> 3) + 1);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        u[i] = sr_uniform_from_words(w0, i);
-        u[8 + i] = sr_uniform_from_words(w1, i);
-      }
-    }
-    packed = encode16(x, rounding, u);
+    const uint64_t e0 = (uint64_t)j * (uint64_t)longdim + (uint64_t)b * 16;
+    packed = encode_block16(x, rounding, seed, tag, step, e0);
     if (bs.code == 0) packed = make_uint2(0, 0);
     code = bs.code;
   }

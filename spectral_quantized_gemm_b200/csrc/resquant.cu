@@ -83,17 +83,7 @@ __device__ __forceinline__ uint2 quantize16(const float (&v)[16], float g, int r
   float x[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) x[i] = __fmul_rn(v[i], bs.rcp);
-  float u[16];
-  if (rounding) {
-    const Words4 w0 = stream_call(seed, tag, step, e0 >> 3);
-    const Words4 w1 = stream_call(seed, tag, step, (e0 >> 3) + 1);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      u[i] = sr_uniform_from_words(w0, i);
-      u[8 + i] = sr_uniform_from_words(w1, i);
-    }
-  }
-  uint2 packed = encode16(x, rounding, u);
+  uint2 packed = encode_block16(x, rounding, seed, tag, step, e0);
   if (bs.code == 0) packed = make_uint2(0, 0);
   scale_code = bs.code;
   return packed;
