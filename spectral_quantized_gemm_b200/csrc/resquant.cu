@@ -11,9 +11,10 @@
 //               then per tile the V rows and the two 64-column boxes of M
 //   warp 1      tensor-memory owner; one thread issues tcgen05.mma kind::tf32
 //               (U S)(V)^T -> fp32 reconstruction in a double-buffered accumulator
-//   warps 2..9  residual = M - reconstruction (fp32), row-wise quantization from
-//               registers, the tile staged in XOR-swizzled shared memory, then
-//               column-wise quantization; codes and tiled scales go straight to HBM
+//   warps 2..17 residual = M - reconstruction (fp32), row-wise quantization from
+//               registers (a warp per 32 rows x 32 columns), the tile staged in
+//               XOR-swizzled shared memory, then column-wise quantization (a thread per
+//               32 rows of a column); codes and tiled scales go straight to HBM
 // All mbarrier waits are bounded (METIS_DEV_TIMEOUT on expiry).
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -28,8 +29,9 @@
 namespace metis {
 namespace {
 
-constexpr int kRqThreads = 320;
-constexpr int kRqEpiThreads = 256;
+constexpr int kRqEpiWarps = 16;                 // 4 per tensor-memory lane quarter
+constexpr int kRqEpiThreads = kRqEpiWarps * 32;
+constexpr int kRqThreads = 64 + kRqEpiThreads;
 
 template <int KK>
 struct RqCfg {
@@ -89,16 +91,16 @@ __device__ __forceinline__ uint2 quantize16(const float (&v)[16], float g, int r
   return packed;
 }
 
-__device__ __forceinline__ void named_sync_epilogue() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ void named_sync_epilogue() { asm volatile("bar.sync 1, %0;" ::"n"(kRqEpiThreads) : "memory"); }
 
-// OR of a predicate over the 256 epilogue threads (a barrier: all must call it), so
+// OR of a predicate over the epilogue threads (a barrier: all must call it), so
 // every epilogue thread takes the same branch after a bounded wait.
 __device__ __forceinline__ bool epilogue_any(bool v) {
   uint32_t r;
   asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\tbar.red.or.pred p, 1, 256, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\tbar.red.or.pred p, 1, %2, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)v)
+      : "r"((uint32_t)v), "n"(kRqEpiThreads)
       : "memory");
   return r != 0;
 }
@@ -233,9 +235,9 @@ __global__ void __launch_bounds__(kRqThreads, 1)
     }
     __syncwarp();
   } else {
-    const int et = threadIdx.x - 64;   // epilogue thread 0..255
+    const int et = threadIdx.x - 64;   // epilogue thread 0 .. kRqEpiThreads - 1
     const int q = warp & 3;            // tensor-memory lane quarter
-    const int h = (warp - 2) >> 2;     // column half of the tile
+    const int h = (warp - 2) >> 2;     // 32-column quarter of the tile in the row pass
     const int r = q * 32 + lane;       // tile row of this thread in the row pass
     int stage = 0;
     uint32_t phase = 0;
@@ -251,57 +253,50 @@ __global__ void __launch_bounds__(kRqThreads, 1)
         break;
       }
       tc::tc_fence_after();
-      // reconstruction of this thread's row, 64 columns
-      float v[64];
-      {
-        float t[32];
-        tc::tmem_load_32cols(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * 128 + h * 64), t);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = t[i];
-        tc::tmem_load_32cols(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * 128 + h * 64 + 32), t);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[32 + i] = t[i];
-      }
+      // reconstruction of this thread's row, 32 columns
+      float v[32];
+      tc::tmem_load_32cols(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * 128 + h * 32), v);
       tc::tmem_load_wait();
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&acc_empty[b]);
-      // residual = M - reconstruction (M from the 128B-swizzled box of this half)
-      const uint8_t* sM = sStage + stage * C::STAGE_BYTES + C::V_BYTES + h * 16384;
+      // residual = M - reconstruction (M from the 128B-swizzled 64-column box holding
+      // this quarter: chunks (h & 1) * 4 .. + 3 of box h >> 1)
+      const uint8_t* sM = sStage + stage * C::STAGE_BYTES + C::V_BYTES + (h >> 1) * 16384;
       bool finite = true;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int cc = 0; cc < 4; ++cc) {
+        const int c = (h & 1) * 4 + cc;
         const uint4 raw = *reinterpret_cast<const uint4*>(sM + r * 128 + ((c ^ (r & 7)) << 4));
         const __nv_bfloat162* pr = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float2 f = __bfloat1622float2(pr[i]);
-          v[c * 8 + 2 * i] = f.x - v[c * 8 + 2 * i];
-          v[c * 8 + 2 * i + 1] = f.y - v[c * 8 + 2 * i + 1];
+          v[cc * 8 + 2 * i] = f.x - v[cc * 8 + 2 * i];
+          v[cc * 8 + 2 * i + 1] = f.y - v[cc * 8 + 2 * i + 1];
         }
       }
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&empty[stage]);   // this warp is done with M
 #pragma unroll
-      for (int i = 0; i < 64; ++i) finite &= isfinite(v[i]);
+      for (int i = 0; i < 32; ++i) finite &= isfinite(v[i]);
       if (!finite) raise_status(p.status, METIS_DEV_NONFINITE);
-      // stage the residual row half in shared memory (16-byte chunks XOR-swizzled by row)
+      // stage the residual row quarter in shared memory (16-byte chunks XOR-swizzled by row)
 #pragma unroll
-      for (int t4 = 0; t4 < 16; ++t4) {
-        const int cc = h * 16 + t4;
+      for (int t4 = 0; t4 < 8; ++t4) {
+        const int cc = h * 8 + t4;
         *reinterpret_cast<float4*>(sR + r * 128 + ((cc ^ (r & 7)) << 2)) =
             make_float4(v[4 * t4], v[4 * t4 + 1], v[4 * t4 + 2], v[4 * t4 + 3]);
       }
       // row-wise quantization (blocks along columns) straight from registers
       {
         const int64_t grow = (int64_t)rb * 128 + r;
-        const int64_t gcol = (int64_t)cb * 128 + h * 64;
+        const int64_t gcol = (int64_t)cb * 128 + h * 32;
         uint32_t sc = 0;
-        uint4 out0, out1;
-        uint32_t* o = reinterpret_cast<uint32_t*>(&out0);
-        uint32_t* o1 = reinterpret_cast<uint32_t*>(&out1);
+        uint4 out;
+        uint32_t* o = reinterpret_cast<uint32_t*>(&out);
 #pragma unroll
-        for (int blk = 0; blk < 4; ++blk) {
+        for (int blk = 0; blk < 2; ++blk) {
           float x[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) x[i] = v[blk * 16 + i];
@@ -309,45 +304,39 @@ __global__ void __launch_bounds__(kRqThreads, 1)
           const uint2 pk = quantize16(x, p.g, p.rounding, p.seed, p.tag_row, p.step,
                                       (uint64_t)grow * (uint64_t)p.cols + (uint64_t)(gcol + blk * 16), code);
           sc |= code << (8 * blk);
-          uint32_t* dst = blk < 2 ? o : o1;
-          dst[(blk & 1) * 2] = pk.x;
-          dst[(blk & 1) * 2 + 1] = pk.y;
+          o[2 * blk] = pk.x;
+          o[2 * blk + 1] = pk.y;
         }
-        uint8_t* cdst = p.row_codes + grow * (p.cols / 2) + gcol / 2;
-        reinterpret_cast<uint4*>(cdst)[0] = out0;
-        reinterpret_cast<uint4*>(cdst)[1] = out1;
-        *reinterpret_cast<uint32_t*>(p.row_scales + scale_offset(grow, gcol / 16, p.cols / 64)) = sc;
+        *reinterpret_cast<uint4*>(p.row_codes + grow * (p.cols / 2) + gcol / 2) = out;
+        *reinterpret_cast<uint16_t*>(p.row_scales + scale_offset(grow, gcol / 16, p.cols / 64)) = (uint16_t)sc;
       }
       named_sync_epilogue();
-      // column-wise quantization (blocks along rows) from the staged tile
+      // column-wise quantization (blocks along rows) from the staged tile: column j,
+      // rows hh * 32 .. + 31
       {
         const int j = et & 127, hh = et >> 7;
         const int64_t gcolj = (int64_t)cb * 128 + j;
-        const int64_t grow0 = (int64_t)rb * 128 + hh * 64;
+        const int64_t grow0 = (int64_t)rb * 128 + hh * 32;
         uint32_t sc = 0;
-        uint4 out0, out1;
-        uint32_t* o = reinterpret_cast<uint32_t*>(&out0);
-        uint32_t* o1 = reinterpret_cast<uint32_t*>(&out1);
+        uint4 out;
+        uint32_t* o = reinterpret_cast<uint32_t*>(&out);
 #pragma unroll
-        for (int blk = 0; blk < 4; ++blk) {
+        for (int blk = 0; blk < 2; ++blk) {
           float x[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int rr = hh * 64 + blk * 16 + i;
+            const int rr = hh * 32 + blk * 16 + i;
             x[i] = sR[rr * 128 + ((((j >> 2) ^ (rr & 7))) << 2) + (j & 3)];
           }
           uint32_t code;
           const uint2 pk = quantize16(x, p.g, p.rounding, p.seed, p.tag_col, p.step,
                                       (uint64_t)gcolj * (uint64_t)p.rows + (uint64_t)(grow0 + blk * 16), code);
           sc |= code << (8 * blk);
-          uint32_t* dst = blk < 2 ? o : o1;
-          dst[(blk & 1) * 2] = pk.x;
-          dst[(blk & 1) * 2 + 1] = pk.y;
+          o[2 * blk] = pk.x;
+          o[2 * blk + 1] = pk.y;
         }
-        uint8_t* cdst = p.col_codes + gcolj * (p.rows / 2) + grow0 / 2;
-        reinterpret_cast<uint4*>(cdst)[0] = out0;
-        reinterpret_cast<uint4*>(cdst)[1] = out1;
-        *reinterpret_cast<uint32_t*>(p.col_scales + scale_offset(gcolj, grow0 / 16, p.rows / 64)) = sc;
+        *reinterpret_cast<uint4*>(p.col_codes + gcolj * (p.rows / 2) + grow0 / 2) = out;
+        *reinterpret_cast<uint16_t*>(p.col_scales + scale_offset(gcolj, grow0 / 16, p.rows / 64)) = (uint16_t)sc;
       }
       named_sync_epilogue();
       if (++stage == C::STAGES) {
