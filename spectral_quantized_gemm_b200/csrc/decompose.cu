@@ -492,7 +492,7 @@ __global__ void __launch_bounds__(kEigThreads) eig_solver_kernel(const double* _
   __shared__ double rot_c[kMaxW / 2], rot_s[kMaxW / 2];
   // flags double-buffered by parity: a flag is cleared one step before it is set and
   // read, so no thread clears it while another still reads it
-  __shared__ int any_rot[2], round_rot[2], need_rot;
+  __shared__ int round_rot[2], need_rot[2];
   const int tid = threadIdx.x;
   const int ty = tid >> 5, tx = tid & 31;
   constexpr int W = kEigThreads / 32;
@@ -503,110 +503,104 @@ __global__ void __launch_bounds__(kEigThreads) eig_solver_kernel(const double* _
     H[e] = (i < n && j < n) ? G[i * n + j] : 0.0;
     Z[e] = (i == j) ? 1.0 : 0.0;
   }
-  if (tid == 0) {
-    need_rot = 0;
-    any_rot[0] = 0;
-    round_rot[0] = 0;
-  }
+  if (tid == 0) need_rot[0] = 0;
   __syncthreads();
   const int npairs = ne / 2;
   const double tol2 = kJacobiTol * kJacobiTol;
-  {  // every pair checked at once: none above the tolerance means no sweep rotates
-    bool need = false;
-    for (int p = ty; p < ne && !need; p += W)
-      for (int q = p + 1 + tx; q < ne; q += 32) {
-        const double ga = H[p * ld + q];
-        need = need || (ga != 0.0 && ga * ga > tol2 * (H[p * ld + p] * H[q * ld + q]));
-      }
-    if (need) need_rot = 1;
-  }
-  __syncthreads();
+  // A sweep that would rotate no pair ends the iteration; so before each sweep every
+  // pair is checked at once (one step instead of a sweep of rounds that rotates nothing).
   int sweep = 0;
-  if (need_rot) {
-    for (; sweep < kJacobiMaxSweeps; ++sweep) {
-      if (tid == 0) round_rot[0] = 0;   // last read before the previous round's barrier
-      __syncthreads();
-      for (int round = 0; round < ne - 1; ++round) {
-        if (tid == 0) {
-          round_rot[(round + 1) & 1] = 0;                // last read in round - 1
-          if (round == 0) any_rot[(sweep + 1) & 1] = 0;  // last read after sweep - 1
+  for (; sweep < kJacobiMaxSweeps; ++sweep) {
+    {
+      bool need = false;
+      for (int p = ty; p < ne && !need; p += W)
+        for (int q = p + 1 + tx; q < ne; q += 32) {
+          const double ga = H[p * ld + q];
+          need = need || (ga != 0.0 && ga * ga > tol2 * (H[p * ld + p] * H[q * ld + q]));
         }
-        // (1) rotation parameters, a thread per pair: with al = H_pp, be = H_qq,
-        // ga = H_pq, t = sign(zeta) / (|zeta| + sqrt(1 + zeta^2)), zeta = (be - al) / (2 ga),
-        // c = 1 / sqrt(1 + t^2), s = c t (written without divisions)
-        for (int pr = tid; pr < npairs; pr += kEigThreads) {
+      if (need) need_rot[sweep & 1] = 1;
+      if (tid == 0) {
+        need_rot[(sweep + 1) & 1] = 0;   // last read after the previous sweep's check
+        round_rot[0] = 0;                // last read before the previous round's barrier
+      }
+    }
+    __syncthreads();
+    if (!need_rot[sweep & 1]) break;
+    for (int round = 0; round < ne - 1; ++round) {
+      if (tid == 0) round_rot[(round + 1) & 1] = 0;   // last read in round - 1
+      // (1) rotation parameters, a thread per pair: with al = H_pp, be = H_qq,
+      // ga = H_pq, t = sign(zeta) / (|zeta| + sqrt(1 + zeta^2)), zeta = (be - al) / (2 ga),
+      // c = 1 / sqrt(1 + t^2), s = c t (written without divisions)
+      for (int pr = tid; pr < npairs; pr += kEigThreads) {
+        int p, q;
+        round_pair(pr, round, ne, p, q);
+        const double al = H[p * ld + p], be = H[q * ld + q], ga = H[p * ld + q];
+        double c = 1.0, s = 0.0;
+        if (ga != 0.0 && ga * ga > tol2 * (al * be)) {
+          const double dd = be - al;
+          const double g2 = 2.0 * ga;
+          const double x = fma(dd, dd, g2 * g2);
+          const double rt = x * rsqrt(x);
+          const double den = fabs(dd) + rt;
+          const double rho = rsqrt(fma(den, den, g2 * g2));
+          const double sgn = (dd == 0.0) ? 1.0 : copysign(1.0, dd) * copysign(1.0, ga);
+          c = den * rho;
+          s = sgn * fabs(g2) * rho;
+          round_rot[round & 1] = 1;
+        }
+        rot_c[pr] = c;
+        rot_s[pr] = s;
+      }
+      __syncthreads();
+      if (round_rot[round & 1]) {   // uniform
+        // (2) H <- J^T H J and Z <- Z J with J the round's disjoint rotations: a thread per
+        // 2 x 2 block (rows p_i, q_i; columns p_j, q_j), all reads of a block before
+        // its writes; a warp per column pair of Z
+        for (int e = tid; e < npairs * npairs; e += kEigThreads) {
+          const int i = e / npairs, j = e - (e / npairs) * npairs;
+          const double si = rot_s[i], sj = rot_s[j];
+          if (si == 0.0 && sj == 0.0) continue;
+          const double ci = rot_c[i], cj = rot_c[j];
+          int pa, pb, qa, qb;
+          round_pair(i, round, ne, pa, pb);
+          round_pair(j, round, ne, qa, qb);
+          const double h00 = H[pa * ld + qa], h01 = H[pa * ld + qb];
+          const double h10 = H[pb * ld + qa], h11 = H[pb * ld + qb];
+          const double r00 = ci * h00 - si * h10, r10 = si * h00 + ci * h10;   // rows
+          const double r01 = ci * h01 - si * h11, r11 = si * h01 + ci * h11;
+          H[pa * ld + qa] = cj * r00 - sj * r01;                                 // columns
+          H[pa * ld + qb] = sj * r00 + cj * r01;
+          H[pb * ld + qa] = cj * r10 - sj * r11;
+          H[pb * ld + qb] = sj * r10 + cj * r11;
+        }
+        for (int pr = ty; pr < npairs; pr += W) {
+          const double s = rot_s[pr];
+          if (s == 0.0) continue;
+          const double c = rot_c[pr];
           int p, q;
           round_pair(pr, round, ne, p, q);
-          const double al = H[p * ld + p], be = H[q * ld + q], ga = H[p * ld + q];
-          double c = 1.0, s = 0.0;
-          if (ga != 0.0 && ga * ga > tol2 * (al * be)) {
-            const double dd = be - al;
-            const double g2 = 2.0 * ga;
-            const double x = fma(dd, dd, g2 * g2);
-            const double rt = x * rsqrt(x);
-            const double den = fabs(dd) + rt;
-            const double rho = rsqrt(fma(den, den, g2 * g2));
-            const double sgn = (dd == 0.0) ? 1.0 : copysign(1.0, dd) * copysign(1.0, ga);
-            c = den * rho;
-            s = sgn * fabs(g2) * rho;
-            round_rot[round & 1] = 1;
-            any_rot[sweep & 1] = 1;
-          }
-          rot_c[pr] = c;
-          rot_s[pr] = s;
-        }
-        __syncthreads();
-        if (round_rot[round & 1]) {   // uniform
-          // (2) H <- J^T H J and Z <- Z J with J the round's disjoint rotations: a thread per
-          // 2 x 2 block (rows p_i, q_i; columns p_j, q_j), all reads of a block before
-          // its writes; a warp per column pair of Z
-          for (int e = tid; e < npairs * npairs; e += kEigThreads) {
-            const int i = e / npairs, j = e - (e / npairs) * npairs;
-            const double si = rot_s[i], sj = rot_s[j];
-            if (si == 0.0 && sj == 0.0) continue;
-            const double ci = rot_c[i], cj = rot_c[j];
-            int pa, pb, qa, qb;
-            round_pair(i, round, ne, pa, pb);
-            round_pair(j, round, ne, qa, qb);
-            const double h00 = H[pa * ld + qa], h01 = H[pa * ld + qb];
-            const double h10 = H[pb * ld + qa], h11 = H[pb * ld + qb];
-            const double r00 = ci * h00 - si * h10, r10 = si * h00 + ci * h10;   // rows
-            const double r01 = ci * h01 - si * h11, r11 = si * h01 + ci * h11;
-            H[pa * ld + qa] = cj * r00 - sj * r01;                                 // columns
-            H[pa * ld + qb] = sj * r00 + cj * r01;
-            H[pb * ld + qa] = cj * r10 - sj * r11;
-            H[pb * ld + qb] = sj * r10 + cj * r11;
-          }
-          for (int pr = ty; pr < npairs; pr += W) {
-            const double s = rot_s[pr];
-            if (s == 0.0) continue;
-            const double c = rot_c[pr];
-            int p, q;
-            round_pair(pr, round, ne, p, q);
-            double* zp = Z + p * ld;
-            double* zq = Z + q * ld;
-            double za[LR], zb[LR];
+          double* zp = Z + p * ld;
+          double* zq = Z + q * ld;
+          double za[LR], zb[LR];
 #pragma unroll
-            for (int u = 0; u < LR; ++u) {
-              const int x = tx + 32 * u;
-              if (x < ne) {
-                za[u] = zp[x];
-                zb[u] = zq[x];
-              }
+          for (int u = 0; u < LR; ++u) {
+            const int x = tx + 32 * u;
+            if (x < ne) {
+              za[u] = zp[x];
+              zb[u] = zq[x];
             }
+          }
 #pragma unroll
-            for (int u = 0; u < LR; ++u) {
-              const int x = tx + 32 * u;
-              if (x < ne) {
-                zp[x] = c * za[u] - s * zb[u];
-                zq[x] = s * za[u] + c * zb[u];
-              }
+          for (int u = 0; u < LR; ++u) {
+            const int x = tx + 32 * u;
+            if (x < ne) {
+              zp[x] = c * za[u] - s * zb[u];
+              zq[x] = s * za[u] + c * zb[u];
             }
           }
         }
-        __syncthreads();
       }
-      if (!any_rot[sweep & 1]) break;
+      __syncthreads();
     }
   }
   if (tid == 0) {

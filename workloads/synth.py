@@ -98,6 +98,33 @@ def operand_matrix(cfg, name, as_numpy=False):
     return t.double().numpy() if as_numpy else t
 
 
+def batch_matrix(cfg, name, batch):
+    """Operand of training batch ``batch`` (bf16, CPU): a new draw of the tokens.
+
+    The layer's persistent structure -- the spike directions (outlier channels or
+    dense directions) and their magnitudes -- comes from a generator seeded by
+    (seed, operand); the token content -- the spike coefficients P and the N(0, 1)
+    bulk -- from one seeded by (seed, operand, batch).  So consecutive batches share
+    their dominant subspace, as the notes observe for activations and gradients
+    (关键设计 3), while no two batches have the same values.
+    """
+    rows, cols = operand_shape(cfg, name)
+    n_spike = cfg["spikes"][name] if cfg.get("spikes") else n_spikes(rows, cols)
+    srng = np.random.default_rng([cfg["seed"], OPERAND_IDS[name], 7])
+    crng = np.random.default_rng([cfg["seed"], OPERAND_IDS[name], 100 + int(batch)])
+    out = crng.standard_normal((rows, cols))
+    if n_spike > 0:
+        sigma = cfg["sigma0"] * cfg["rho"] ** np.arange(n_spike) * np.sqrt(rows)
+        P = crng.standard_normal((rows, n_spike)) / np.sqrt(rows)
+        if cfg.get("directions", "dense") == "dense":
+            Q, _ = np.linalg.qr(srng.standard_normal((cols, n_spike)))
+            out += (P * sigma[None, :]) @ Q.T
+        else:
+            channels = srng.choice(cols, size=n_spike, replace=False)
+            out[:, channels] += P * sigma[None, :]
+    return to_bf16(out)
+
+
 def perturbed(cfg, name, base, step):
     """base + perturb * rms(base) * N(0,1), fresh noise per step (bf16)."""
     rng = np.random.default_rng([cfg["seed"], OPERAND_IDS[name], 1000 + int(step)])
