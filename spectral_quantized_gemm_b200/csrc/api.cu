@@ -255,7 +255,7 @@ metis_status metis_gemm_nvfp4(metis_ctx* ctx, const metis_nvfp4* A, const metis_
   if (c_dtype != METIS_OUT_F32 && c_dtype != METIS_OUT_BF16) return fail(ctx, METIS_ERR_ARG, "bad output dtype");
   if (ldc < n_cols || ldc % (c_dtype == METIS_OUT_F32 ? 4 : 8) || !aligned16(C))
     return fail(ctx, METIS_ERR_ALIGN, "output needs 16-byte alignment and a 16-byte multiple leading dimension");
-  GemmArgs a{A, B, fold_k ? Fa : nullptr, fold_k ? Fb : nullptr, fold_k, col_scale, C, ldc, c_dtype, 1.0f, n_cols};
+  GemmArgs a{A, B, fold_k ? Fa : nullptr, fold_k ? Fb : nullptr, fold_k, col_scale, C, ldc, c_dtype, 1.0f, n_cols, 1, 0};
   return launch_gemm_nvfp4(ctx, a);
 }
 

@@ -478,14 +478,13 @@ __global__ void __launch_bounds__(kSolverThreads) cholqr_solver_kernel(const dou
   }
 }
 
-// mode 1: T only (refresh basis); mode 2: T, Vr and S (per-step factors)
-template <bool kSmem>
+// mode 1: T only (refresh basis); mode 2: T, Vr and S (per-step factors).  Works in global
+// scratch; used for sketches wider than the two-kernel solver below takes.
 __global__ void __launch_bounds__(kEigThreads) eig_solver_kernel(const double* __restrict__ G, int n, int k,
                                                                     int mode, SmallOut out, uint32_t* status) {
-  extern __shared__ double smem_d[];
   const int ne = (n + 1) & ~1;
   const int ld = ne + 1;   // odd stride: rows and columns of H, columns of Z, all conflict-free
-  double* const H = kSmem ? smem_d : out.scratch;   // H[i * ld + j], symmetric
+  double* const H = out.scratch;                     // H[i * ld + j], symmetric
   double* const Z = H + ne * ld;                     // column c at Z + c * ld
   __shared__ double lam[kMaxW];
   __shared__ int order[kMaxW];
@@ -496,7 +495,7 @@ __global__ void __launch_bounds__(kEigThreads) eig_solver_kernel(const double* _
   const int tid = threadIdx.x;
   const int ty = tid >> 5, tx = tid & 31;
   constexpr int W = kEigThreads / 32;
-  constexpr int LR = kSmem ? (kSmallMaxN + 31) / 32 : kLaneRows;   // entries of a row or column per lane
+  constexpr int LR = kLaneRows;   // entries of a row or column per lane
 
   for (int e = tid; e < ne * ld; e += kEigThreads) {
     const int i = e / ld, j = e - (e / ld) * ld;
@@ -641,6 +640,340 @@ __global__ void __launch_bounds__(kEigThreads) eig_solver_kernel(const double* _
   }
 }
 
+// ------------------------------------------- two-kernel Jacobi eigensolver (ne <= 88)
+// The eigenproblem of G (n x n, fp64) by cyclic two-sided Jacobi in the round-robin
+// (circle) ordering, split in two launches:
+//
+// jacobi_rounds_kernel (one CTA): the matrix is kept in slot order -- slot pair a =
+//   (2a, 2a+1) is the rotation pair of the current round -- and after each round every
+//   element moves to its next slot (jac_dest), written into the other of two shared-memory
+//   buffers.  Only the upper triangle is kept; a thread owns one 2 x 2 block (a <= b) of
+//   the slot grid.  The rotation of the NEXT round's pair a' is computed in the same step
+//   by the owner of the block that holds that pair's off-diagonal element; the two new
+//   diagonal entries it needs are recomputed from the old diagonal blocks with the same
+//   correctly rounded arithmetic the diagonal owners use.  One barrier per round.  Each
+//   round's rotations (c, s) go to global memory; after a whole number of sweeps every
+//   element is back in its own slot, so the diagonal is the spectrum in index order.
+// jacobi_replay_kernel (a warp per row of Z): applies the recorded rotations and slot
+//   moves to one row of the identity, giving the eigenvector matrix row by row, and
+//   writes T = Z Lambda^-1/2 and Vr = Z in descending eigenvalue order.
+constexpr int kJacMaxNE = 88;          // m(m - 1)/2 off-diagonal blocks fit in 32 - ceil(m/32) warps, m = ne/2
+constexpr int kJacThreads = 1024;
+constexpr int kJacChunk = 16;          // replay: rounds of rotations staged per chunk
+constexpr int kJacRowsPerCta = 4;      // replay: rows (warps) per CTA
+
+__host__ __device__ constexpr int jac_ne(int n) { return n < 4 ? 4 : (n + 1) & ~1; }
+__host__ __device__ constexpr size_t jac_rot_entries(int n) {
+  return ((size_t)kJacobiMaxSweeps * (jac_ne(n) - 1) + 1) * (jac_ne(n) / 2);
+}
+__host__ __device__ constexpr size_t jac_smem_bytes(int ne) {
+  return (size_t)2 * ne * ne * sizeof(double) + (size_t)2 * (ne / 2) * (2 * sizeof(double2) + sizeof(double));
+}
+
+// slot an element moves to after a round: top of pair 0 stays; the other 2m - 1 slots
+// form a ring top_1 -> top_2 -> ... -> top_{m-1} -> bot_{m-1} -> ... -> bot_0 -> top_1
+__device__ __forceinline__ int jac_dest(int s, int m) {
+  if (s == 0) return 0;
+  const int a = s >> 1;
+  if ((s & 1) == 0) return a <= m - 2 ? 2 * (a + 1) : 2 * m - 1;
+  return a >= 1 ? 2 * a - 1 : 2;
+}
+__device__ __forceinline__ int jac_src(int s, int m) {
+  if (s == 0) return 0;
+  const int a = s >> 1;
+  if ((s & 1) == 0) return a == 1 ? 1 : 2 * a - 2;
+  return a == m - 1 ? 2 * m - 2 : 2 * a + 3;
+}
+
+// rotation (c, s) that annihilates ga in [[al, ga], [ga, be]] (x_p' = c x_p - s x_q,
+// x_q' = s x_p + c x_q), or the identity when |ga| is below tol * sqrt(al be)
+__device__ __forceinline__ double2 jac_rotation(double al, double be, double ga, double tol2) {
+  double c = 1.0, s = 0.0;
+  if (ga != 0.0 && ga * ga > tol2 * (al * be)) {
+    const double dd = be - al;
+    const double g2 = 2.0 * ga;
+    const double x = fma(dd, dd, g2 * g2);
+    const double rt = x * rsqrt(x);
+    const double den = fabs(dd) + rt;
+    const double rho = rsqrt(fma(den, den, g2 * g2));
+    const double sgn = (dd == 0.0) ? 1.0 : copysign(1.0, dd) * copysign(1.0, ga);
+    c = den * rho;
+    s = sgn * fabs(g2) * rho;
+  }
+  return make_double2(c, s);
+}
+
+// new diagonal of a rotated pair; correctly rounded operations only, so every thread
+// that evaluates it for the same pair gets the same bits
+__device__ __forceinline__ void jac_diag(double al, double be, double ga, double2 cs, double& d0, double& d1) {
+  const double cc = __dmul_rn(cs.x, cs.x), ss = __dmul_rn(cs.y, cs.y);
+  const double x = __dmul_rn(__dmul_rn(__dmul_rn(2.0, cs.x), cs.y), ga);
+  d0 = __fma_rn(cc, al, __fma_rn(ss, be, -x));
+  d1 = __fma_rn(ss, al, __fma_rn(cc, be, x));
+}
+
+struct JacOut {
+  double2* rot;      // jac_rot_entries(n) rotations, round-major
+  int* info;         // [0] rounds recorded
+  int* order;        // k source slots, descending eigenvalue
+  double* inv_sqrt;  // k factors lambda^-1/2 (0 for a dropped eigenvalue)
+};
+
+__global__ void __launch_bounds__(kJacThreads, 1) jacobi_rounds_kernel(const double* __restrict__ G, int n, int k,
+                                                                       int mode, JacOut jo, SmallOut out,
+                                                                       uint32_t* status) {
+  extern __shared__ double smem_d[];
+  const int ne = jac_ne(n), m = ne / 2;
+  double* Hbuf0 = smem_d;                       // off-diagonal blocks of the slot grid, upper triangle
+  double* Hbuf1 = smem_d + ne * ne;
+  double2* prm = reinterpret_cast<double2*>(smem_d + 2 * ne * ne);   // [2][m] rotation (c, s) of pair p
+  double2* dgn = prm + 2 * m;                                          // [2][m] diagonal (al, be) of pair p
+  double* dof = reinterpret_cast<double*>(dgn + 2 * m);               // [2][m] off-diagonal ga of pair p
+  __shared__ double lam[kJacMaxNE];
+  __shared__ int order[kJacMaxNE];
+  const int tid = threadIdx.x;
+  const double tol2 = kJacobiTol * kJacobiTol;
+
+  for (int e = tid; e < ne * ne; e += kJacThreads) {
+    const int i = e / ne, j = e - (e / ne) * ne;
+    Hbuf0[e] = (i < n && j < n && i <= j) ? G[i * n + j] : 0.0;
+  }
+  // Roles, warp-aligned so that each warp runs one instruction stream.  The pair warps
+  // (ceil(m / 32) of them, warps 0, 4, ...) own pair p: its 2 x 2 diagonal block, kept in
+  // dgn/dof, and the rotation of the next round's pair p -- the chain that bounds a round --
+  // so they sit on the SM sub-partition of warps 0 mod 4, which the block warps fill last.
+  // The block warps own the off-diagonal blocks (a < b), warps not 0 mod 4 first.
+  const int warp = tid >> 5, lane = tid & 31;
+  const int n_pair_warps = (m + 31) / 32;
+  const bool pair_warp = (warp & 3) == 0 && (warp >> 2) < n_pair_warps;
+  int off_rank;   // position of this warp among the block warps
+  if ((warp & 3) != 0) off_rank = warp - (warp >> 2) - 1;
+  else off_rank = 24 + (warp >> 2) - n_pair_warps;
+  const int n_off = m * (m - 1) / 2;
+  const int e_off = off_rank * 32 + lane;
+  const bool is_off = !pair_warp && e_off < n_off;
+  const int p = pair_warp ? (warp >> 2) * 32 + lane : -1;
+  const bool is_pair = pair_warp && p < m;
+  int a = 0, b = 0;
+  int wr[4] = {0, 0, 0, 0};
+  int lo = 0, hi = 0, su = 0, sv = 0, x = 0, y = 0;
+  if (is_off) {
+    int rem = e_off;
+    while (rem >= m - 1 - a) {
+      rem -= m - 1 - a;
+      ++a;
+    }
+    b = a + 1 + rem;
+    const int da0 = jac_dest(2 * a, m), da1 = jac_dest(2 * a + 1, m);
+    const int db0 = jac_dest(2 * b, m), db1 = jac_dest(2 * b + 1, m);
+    wr[0] = min(da0, db0) * ne + max(da0, db0);
+    wr[1] = min(da0, db1) * ne + max(da0, db1);
+    wr[2] = min(da1, db0) * ne + max(da1, db0);
+    wr[3] = min(da1, db1) * ne + max(da1, db1);
+  } else if (is_pair) {
+    const int d0 = jac_dest(2 * p, m), d1 = jac_dest(2 * p + 1, m);
+    wr[0] = min(d0, d1) * ne + max(d0, d1);   // where this pair's off-diagonal element goes
+    // the next round's pair p is (su, sv) in the current slots; its off-diagonal element
+    // lies in block (lo, hi), at (x, y) within it
+    su = jac_src(2 * p, m);
+    sv = jac_src(2 * p + 1, m);
+    const bool fwd = (su >> 1) < (sv >> 1);
+    lo = fwd ? su >> 1 : sv >> 1;
+    hi = fwd ? sv >> 1 : su >> 1;
+    x = fwd ? su & 1 : sv & 1;
+    y = fwd ? sv & 1 : su & 1;
+  }
+  __syncthreads();
+  double own_ga = 0.0;
+  double2 own_cs = make_double2(1.0, 0.0);
+  if (is_pair) {
+    const double al = Hbuf0[2 * p * ne + 2 * p], be = Hbuf0[(2 * p + 1) * ne + 2 * p + 1];
+    own_ga = Hbuf0[2 * p * ne + 2 * p + 1];
+    own_cs = jac_rotation(al, be, own_ga, tol2);
+    prm[p] = own_cs;
+    dgn[p] = make_double2(al, be);
+    dof[p] = own_ga;
+    jo.rot[p] = own_cs;
+  }
+  const double* Hr = Hbuf0;
+  double* Hw = Hbuf1;
+  int round = 0, sweep = 0;
+  for (;; ++sweep) {
+    // converged when no pair of the current matrix would rotate
+    const double2* Dc = dgn + (round & 1) * m;
+    bool need = false;
+    if (is_off) {
+      const double2 da = Dc[a], db = Dc[b];
+      const double h00 = Hr[2 * a * ne + 2 * b], h01 = Hr[2 * a * ne + 2 * b + 1];
+      const double h10 = Hr[(2 * a + 1) * ne + 2 * b], h11 = Hr[(2 * a + 1) * ne + 2 * b + 1];
+      need = (h00 != 0.0 && h00 * h00 > tol2 * (da.x * db.x)) || (h01 != 0.0 && h01 * h01 > tol2 * (da.x * db.y)) ||
+             (h10 != 0.0 && h10 * h10 > tol2 * (da.y * db.x)) || (h11 != 0.0 && h11 * h11 > tol2 * (da.y * db.y));
+    } else if (is_pair) {
+      const double2 d = Dc[p];
+      need = own_ga != 0.0 && own_ga * own_ga > tol2 * (d.x * d.y);
+    }
+    if (!__syncthreads_or(need)) break;
+    if (sweep == kJacobiMaxSweeps) {
+      if (tid == 0) {
+        raise_status(status, METIS_DEV_NUMERIC);
+        out.flags[0] = 1;
+      }
+      break;
+    }
+    for (int r = 0; r < ne - 1; ++r, ++round) {
+      const int cur = (round & 1) * m, nxt = m - cur;
+      if (is_off) {
+        const double2 ca = prm[cur + a], cb = prm[cur + b];
+        const double2 top = *reinterpret_cast<const double2*>(Hr + 2 * a * ne + 2 * b);
+        const double2 bot = *reinterpret_cast<const double2*>(Hr + (2 * a + 1) * ne + 2 * b);
+        const double r00 = ca.x * top.x - ca.y * bot.x, r10 = ca.y * top.x + ca.x * bot.x;
+        const double r01 = ca.x * top.y - ca.y * bot.y, r11 = ca.y * top.y + ca.x * bot.y;
+        Hw[wr[0]] = cb.x * r00 - cb.y * r01;
+        Hw[wr[1]] = cb.y * r00 + cb.x * r01;
+        Hw[wr[2]] = cb.x * r10 - cb.y * r11;
+        Hw[wr[3]] = cb.y * r10 + cb.x * r11;
+      } else if (is_pair) {
+        const int pu = su >> 1, pv = sv >> 1;
+        const double2 ru = *reinterpret_cast<const double2*>(Hr + (2 * lo + x) * ne + 2 * hi);
+        const double2 rl = *reinterpret_cast<const double2*>(Hr + (2 * lo + 1 - x) * ne + 2 * hi);
+        const double2 clo = prm[cur + lo], chi = prm[cur + hi], cu = prm[cur + pu], cv = prm[cur + pv];
+        const double2 du = dgn[cur + pu], dv = dgn[cur + pv];
+        const double gu = dof[cur + pu], gv = dof[cur + pv];
+        // this pair's own off-diagonal element: annihilated when it rotates
+        Hw[wr[0]] = (own_cs.y != 0.0) ? 0.0 : own_ga;
+        // next round's pair p: new diagonal entries of its two slots and its rotated
+        // off-diagonal element; rotated row x = c (row x) -+ s (other row), minus for the top
+        double u0, u1, v0, v1;
+        jac_diag(du.x, du.y, gu, cu, u0, u1);
+        jac_diag(dv.x, dv.y, gv, cv, v0, v1);
+        const double gx = x ? clo.y : -clo.y;
+        const double q0 = clo.x * ru.x + gx * rl.x, q1 = clo.x * ru.y + gx * rl.y;   // columns 2hi, 2hi + 1
+        own_ga = y ? (chi.y * q0 + chi.x * q1) : (chi.x * q0 - chi.y * q1);
+        const double nal = (su & 1) ? u1 : u0, nbe = (sv & 1) ? v1 : v0;
+        own_cs = jac_rotation(nal, nbe, own_ga, tol2);
+        prm[nxt + p] = own_cs;
+        dgn[nxt + p] = make_double2(nal, nbe);
+        dof[nxt + p] = own_ga;
+        jo.rot[(size_t)(round + 1) * m + p] = own_cs;
+      }
+      __syncthreads();
+      const double* t = Hr;
+      Hr = Hw;
+      Hw = const_cast<double*>(t);
+    }
+  }
+  // after whole sweeps every element is in its own slot: the diagonal is the spectrum
+  const double2* Dc = dgn + (round & 1) * m;
+  for (int j = tid; j < ne; j += kJacThreads) {
+    const double l = (j & 1) ? Dc[j >> 1].y : Dc[j >> 1].x;
+    lam[j] = (l == l) ? l : -HUGE_VAL;
+  }
+  __syncthreads();
+  for (int j = tid; j < ne; j += kJacThreads) {
+    int rank = 0;
+    for (int i = 0; i < ne; ++i) rank += (lam[i] > lam[j]) || (lam[i] == lam[j] && i < j);
+    order[rank] = j;
+  }
+  __syncthreads();
+  const double lmax = fmax(lam[order[0]], 0.0);
+  const double thr = kDropTol * lmax;
+  for (int c = tid; c < k; c += kJacThreads) {
+    const double l = lam[order[c]];
+    const bool keep = l > thr && lmax > 0.0;
+    jo.order[c] = order[c];
+    jo.inv_sqrt[c] = keep ? rsqrt(l) : 0.0;
+    if (mode == 2) out.S[c] = keep ? (float)sqrt(l) : 0.0f;
+  }
+  if (tid == 0) {
+    jo.info[0] = round;
+    out.flags[1] = sweep;
+  }
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+
+// One warp per row of Z.  Lane l holds the row's entries at the slots of pairs l and
+// l + 32; a round rotates each pair and moves every entry one step along the slot ring
+// (two shuffles per set of pairs).  The recorded rotations are staged through shared
+// memory in chunks of kJacChunk rounds, the next chunk copied while this one is applied.
+__global__ void __launch_bounds__(32 * kJacRowsPerCta) jacobi_replay_kernel(const double2* __restrict__ rot,
+                                                                            const int* __restrict__ info, int n,
+                                                                            int k, int mode,
+                                                                            const int* __restrict__ order,
+                                                                            const double* __restrict__ inv_sqrt,
+                                                                            SmallOut out) {
+  __shared__ __align__(16) double2 chunk[2][kJacChunk * (kJacMaxNE / 2)];
+  __shared__ double zrow[kJacRowsPerCta][kJacMaxNE];
+  constexpr unsigned kFull = 0xffffffffu;
+  const int ne = jac_ne(n), m = ne / 2;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * kJacRowsPerCta + warp;
+  const int rounds = info[0];
+  const int a0 = lane, a1 = lane + 32;
+  double t0 = (2 * a0 == row) ? 1.0 : 0.0, b0 = (2 * a0 + 1 == row) ? 1.0 : 0.0;
+  double t1 = (2 * a1 == row) ? 1.0 : 0.0, b1 = (2 * a1 + 1 == row) ? 1.0 : 0.0;
+  const int nchunks = (rounds + kJacChunk - 1) / kJacChunk;
+  auto stage = [&](int ch) {
+    const int r0 = ch * kJacChunk;
+    const int cnt = (min(rounds, r0 + kJacChunk) - r0) * m;
+    double2* dst = chunk[ch & 1];
+    const double2* src = rot + (size_t)r0 * m;
+    for (int e = threadIdx.x; e < cnt; e += blockDim.x) cp_async16(dst + e, src + e);
+    cp_async_commit();
+  };
+  if (nchunks > 0) stage(0);
+  for (int ch = 0; ch < nchunks; ++ch) {
+    cp_async_wait_all();
+    __syncthreads();                       // chunk ch visible; chunk ch - 1 no longer read
+    if (ch + 1 < nchunks) stage(ch + 1);
+    const double2* cr = chunk[ch & 1];
+    const int nr = min(rounds, (ch + 1) * kJacChunk) - ch * kJacChunk;
+    for (int rr = 0; rr < nr; ++rr, cr += m) {
+      const double2 c0 = a0 < m ? cr[a0] : make_double2(1.0, 0.0);
+      const double2 c1 = a1 < m ? cr[a1] : make_double2(1.0, 0.0);
+      const double rt0 = c0.x * t0 - c0.y * b0, rb0 = c0.y * t0 + c0.x * b0;
+      const double rt1 = c1.x * t1 - c1.y * b1, rb1 = c1.y * t1 + c1.x * b1;
+      // new top[a] = a == 0 ? top[0] : a == 1 ? bot[0] : top[a - 1]
+      // new bot[a] = a == m - 1 ? top[m - 1] : bot[a + 1]
+      const double up_t0 = __shfl_up_sync(kFull, rt0, 1);
+      const double dn_b0 = __shfl_down_sync(kFull, rb0, 1);
+      const double bot_0 = __shfl_sync(kFull, rb0, 0);
+      double up_t1 = 0.0, dn_b1 = 0.0, w_t0 = 0.0, w_b1 = 0.0;
+      if (m > 32) {
+        up_t1 = __shfl_up_sync(kFull, rt1, 1);
+        dn_b1 = __shfl_down_sync(kFull, rb1, 1);
+        w_t0 = __shfl_sync(kFull, rt0, 31);
+        w_b1 = __shfl_sync(kFull, rb1, 0);
+      }
+      t0 = lane == 0 ? rt0 : (lane == 1 ? bot_0 : up_t0);
+      b0 = a0 == m - 1 ? rt0 : (lane == 31 ? w_b1 : dn_b0);
+      t1 = lane == 0 ? w_t0 : up_t1;
+      b1 = a1 == m - 1 ? rt1 : dn_b1;
+    }
+  }
+  if (a0 < m) {
+    zrow[warp][2 * a0] = t0;
+    zrow[warp][2 * a0 + 1] = b0;
+  }
+  if (a1 < m) {
+    zrow[warp][2 * a1] = t1;
+    zrow[warp][2 * a1 + 1] = b1;
+  }
+  __syncwarp();
+  if (row < n) {
+    for (int c = lane; c < k; c += 32) {
+      const double z = zrow[warp][order[c]];
+      out.T[row * kMaxW + c] = z * inv_sqrt[c];
+      if (mode == 2) out.Vr[row * kMaxW + c] = z;
+    }
+  }
+}
+
 // ------------------------------------------- tensor-core projection helpers
 // out (2kp x n, bf16 row-major): row j < k = hi(F[:, j]), row kp + j = lo(F[:, j]) with
 // hi = bf16(F), lo = bf16(F - hi); other rows zero.  F is n x k fp32 row-major.
@@ -745,6 +1078,8 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
   need += (size_t)((std::max(rows_needed, c) + kGramRows - 1) / kGramRows) * w * w * 8 + 256;  // gram partials
   need += (size_t)kMaxW * kMaxW * 8 * 3 + small_solver_doubles(kMaxW) * 8 + 2048;  // G, T, Vr, solver scratch
   need += 64 * 4 * 3 + 1024;                                      // S, flags, flips
+  need += jac_rot_entries(kJacMaxNE) * sizeof(double2) + 256;     // recorded Jacobi rotations
+  need += (size_t)kMaxW * (4 + 8) + 1024;                          // Jacobi order, lambda^-1/2, info
   const int kpw = pad_width(std::max(w, k));
   need += (size_t)2 * kpw * c * 2 + 256;                          // hi/lo transposed operand
   const int splits_est = normalize_splits(c, bf16_splits(ctx, r, c));
@@ -769,6 +1104,10 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
   float* Sw = static_cast<float*>(ws.take(64 * 4));
   int* flags = static_cast<int*>(ws.take(64 * 4));
   int* flip = static_cast<int*>(ws.take(64 * 4));
+  double2* jrot = static_cast<double2*>(ws.take(jac_rot_entries(kJacMaxNE) * sizeof(double2)));
+  int* jorder = static_cast<int*>(ws.take((size_t)kMaxW * 4));
+  double* jinv = static_cast<double*>(ws.take((size_t)kMaxW * 8));
+  int* jinfo = static_cast<int*>(ws.take(64));
   __nv_bfloat16* bt2 = static_cast<__nv_bfloat16*>(ws.take((size_t)2 * kpw * c * 2));
   float* tc_partial = static_cast<float*>(ws.take(tc_partial_bytes));
   if (!tc_partial) return fail(ctx, METIS_ERR_WORKSPACE, "decompose workspace layout");
@@ -776,10 +1115,11 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
   cudaError_t e = cudaFuncSetAttribute(cholqr_solver_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)(small_solver_doubles(kSmallMaxN) * 8));
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(eig_solver_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(small_solver_doubles(kSmallMaxN) * 8));
+    e = cudaFuncSetAttribute(jacobi_rounds_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)jac_smem_bytes(kJacMaxNE));
   if (e != cudaSuccess) return check_cuda(ctx, e, "cudaFuncSetAttribute(small solver)");
   SmallOut so{T, Vr, Sw, flags, sscratch};
+  JacOut jo{jrot, jinfo, jorder, jinv};
   // mode 0: CholQR factor T = R^+; modes 1 and 2: SVD through the eigenproblem of G
   auto solve = [&](int n, int mode) {
     const int ne = (n + 1) & ~1;
@@ -788,9 +1128,13 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
     if (mode == 0) {
       if (in_smem) cholqr_solver_kernel<true><<<1, kSolverThreads, smem, st>>>(G, n, so);
       else cholqr_solver_kernel<false><<<1, kSolverThreads, 0, st>>>(G, n, so);
+    } else if (jac_ne(n) <= kJacMaxNE) {
+      jacobi_rounds_kernel<<<1, kJacThreads, jac_smem_bytes(jac_ne(n)), st>>>(G, n, k, mode, jo, so, ctx->status);
+      count_launch();
+      jacobi_replay_kernel<<<(n + kJacRowsPerCta - 1) / kJacRowsPerCta, 32 * kJacRowsPerCta, 0, st>>>(
+          jrot, jinfo, n, k, mode, jorder, jinv, so);
     } else {
-      if (in_smem) eig_solver_kernel<true><<<1, kEigThreads, smem, st>>>(G, n, k, mode, so, ctx->status);
-      else eig_solver_kernel<false><<<1, kEigThreads, 0, st>>>(G, n, k, mode, so, ctx->status);
+      eig_solver_kernel<<<1, kEigThreads, 0, st>>>(G, n, k, mode, so, ctx->status);
     }
     count_launch();
   };

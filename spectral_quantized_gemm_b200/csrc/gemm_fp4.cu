@@ -407,6 +407,13 @@ metis_status launch_bn(metis_ctx* ctx, const GemmArgs& a) {
   prm.fold_stages = a.fold_k / 64;
   prm.k_splits = 1;
   prm.split_stride = 0;
+  if (a.k_splits > 1) {
+    if (a.c_dtype != METIS_OUT_F32) return fail(ctx, METIS_ERR_ARG, "split-K partials are fp32");
+    const int total = prm.k_stages + prm.fold_stages;
+    const int per = (total + a.k_splits - 1) / a.k_splits;
+    prm.k_splits = (total + per - 1) / per;
+    prm.split_stride = a.split_stride;
+  }
   prm.status = ctx->status;
   return launch_spec<BN>(ctx, mA, mB, mFa, mFb, prm, 2.0 * (double)p_rows * (double)q_cols * (double)K,
                          q_cols >= 256);
@@ -436,6 +443,13 @@ metis_status launch_bf16_bn(metis_ctx* ctx, const void* A, int64_t lda, int64_t 
 }
 
 }  // namespace
+
+int fp4_splits(metis_ctx* ctx, int64_t tiles, int stages) {
+  const int64_t want = (2 * (int64_t)ctx->sm_count + tiles - 1) / tiles;
+  const int s = (int)std::max<int64_t>(1, std::min<int64_t>(want, stages));
+  const int per = (stages + s - 1) / s;
+  return (stages + per - 1) / per;
+}
 
 int bf16_splits(metis_ctx* ctx, int64_t rows, int64_t K) {
   const int tiles = (int)(rows / 128);

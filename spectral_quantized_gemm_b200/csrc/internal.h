@@ -90,7 +90,12 @@ struct GemmArgs {
   int32_t c_dtype;
   float alpha_extra;  // multiplies alpha = gA * gB (1.0 normally)
   int64_t q_cols;     // output columns: a multiple of 256, or 16 / 32 / 64 (thin)
+  int32_t k_splits;       // > 1: split-K over the FP4 + fold stages, partial s at C + s * split_stride (fp32)
+  int64_t split_stride;   // elements between consecutive partial outputs
 };
+// Split count for an FP4 GeMM of `tiles` output tiles and `stages` K stages: about two
+// work units per SM, no empty share.
+int fp4_splits(metis_ctx* ctx, int64_t tiles, int stages);
 metis_status launch_gemm_nvfp4(metis_ctx* ctx, const GemmArgs& a);
 // C[s] (rows x n, fp32, split s at C + s * rows * ldc) = A (rows x K bf16, lda) * B^T
 // (B: n x K bf16, ldb) over the s-th share of K.  splits < 1 picks a split count;

@@ -45,108 +45,121 @@ struct FactorView {
   int k;
 };
 
-// Partial Z = Q(L)^T Q(R) over one chunk of the shared length (kL x kR).
-constexpr int kZChunk = 64;
-__global__ void z_partial_kernel(FactorView L, FactorView R, float* partial) {
-  __shared__ float sl[64][kZChunk + 1];
-  __shared__ float sr[64][kZChunk + 1];
-  const int64_t i0 = (int64_t)blockIdx.x * kZChunk;
-  const float gl = *L.g, gr = *R.g;
-  for (int e = threadIdx.x; e < 64 * kZChunk; e += blockDim.x) {
-    const int t = e / kZChunk, c = e % kZChunk;
-    sl[t][c] = t < L.k ? factor_value(L.codes, L.scales, gl, L.len, t, i0 + c) : 0.0f;
-    sr[t][c] = t < R.k ? factor_value(R.codes, R.scales, gr, R.len, t, i0 + c) : 0.0f;
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < 64 * 64; e += blockDim.x) {
-    const int a = e / 64, b = e % 64;
-    float acc = 0.0f;
-    if (a < L.k && b < R.k)
-      for (int c = 0; c < kZChunk; ++c) acc = fmaf(sl[a][c], sr[b][c], acc);
-    partial[(int64_t)blockIdx.x * 4096 + e] = acc;
-  }
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// Z[a][b] = sum over chunks in a fixed order (deterministic).
-__global__ void z_reduce_kernel(const float* partial, int nchunks, float* Z) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= 4096) return;
-  float acc = 0.0f;
-  for (int c = 0; c < nchunks; ++c) acc += partial[(int64_t)c * 4096 + e];
-  Z[e] = acc;
-}
-
-// Fb rows: [T_A^T hi | T_A^T lo | Q(R_B) | Q(R_B)] with
-// T_A^T[i][j] = TA32[i][j] + sum_u Q(R_B)[i][u] S_B[u] Z[j][u] S_A[j]   (Z = Q(R_A)^T Q(L_B)).
-// One block per 32 rows: the decoded rows of Q(R_B) and the k x k correction
-// C2[u][j] = S_B[u] Z[j][u] S_A[j] are staged once in shared memory.
-constexpr int kFoldRows = 32;
-__global__ void fold_b_kernel(const float* __restrict__ TA32, int kpA, int kA, FactorView RB, int kpB,
-                              const float* __restrict__ SA, const float* __restrict__ SB, const float* __restrict__ Z,
-                              int64_t q, int fold_k, __nv_bfloat16* __restrict__ Fb) {
-  __shared__ float qrb[kFoldRows][65];
-  __shared__ float c2[64][65];
-  const int64_t i0 = (int64_t)blockIdx.x * kFoldRows;
-  const float gr = RB.k > 0 ? *RB.g : 0.0f;
-  for (int e = threadIdx.x; e < kFoldRows * 64; e += blockDim.x) {
-    const int r = e / 64, u = e % 64;
-    qrb[r][u] = (u < RB.k) ? factor_value(RB.codes, RB.scales, gr, RB.len, u, i0 + r) : 0.0f;
-  }
-  if (RB.k > 0 && kA > 0) {
-    for (int e = threadIdx.x; e < 64 * 64; e += blockDim.x) {
-      const int u = e / 64, j = e % 64;
-      c2[u][j] = (u < RB.k && j < kA) ? SB[u] * Z[j * 64 + u] * SA[j] : 0.0f;
+// Operands of the correction folded into the T_A GeMM (the second term of
+// T_A^T = Q(B_R)^T Q(R_A) S_A + Q(R_B) S_B Z^T S_A, Z = Q(R_A)^T Q(L_B)):
+//   blocks [0, zblocks):  FbZ (128 x fz_k; rows a < kA) = [Z S_B / alpha_TA hi | lo | 0],
+//                         alpha_TA the T_A GeMM's tensor scales; a thread per (a, u)
+//   blocks [zblocks, ..): FaZ rows = [Q(R_B) | Q(R_B) | 0] (bf16, exact), and the same two
+//                         copies of Q(R_B) into the main fold operand Fb at [2 kpA, 2 kpA + 2 kpB)
+// Z arrives as zsplits split-K partials of 128 x kpB, summed in order.  FbZ / FaZ are null
+// when A has no factors (no correction, zblocks = 0).
+constexpr int kRowsPerBlock = 32;
+__global__ void __launch_bounds__(256) zfold_kernel(const float* __restrict__ Zp, int zsplits, int zblocks, int kA,
+                                                    int kB, int kpA, int kpB, const float* __restrict__ SB,
+                                                    const float* gBres, const float* gRA, FactorView RB, int fz_k,
+                                                    __nv_bfloat16* __restrict__ FbZ, __nv_bfloat16* __restrict__ FaZ,
+                                                    __nv_bfloat16* __restrict__ Fb, int fold_k, int64_t q) {
+  if ((int)blockIdx.x < zblocks) {
+    const int t = blockIdx.x * 256 + threadIdx.x;
+    if (t >= 128 * kpB) return;
+    const int a = t / kpB, u = t - (t / kpB) * kpB;
+    float hi = 0.0f, lo = 0.0f;
+    if (a < kA && u < kB) {
+      const float inv_alpha = 1.0f / ((*gBres) * (*gRA));   // exact: powers of two
+      float z = 0.0f;
+      for (int s = 0; s < zsplits; ++s) z += Zp[((int64_t)s * 128 + a) * kpB + u];
+      const float v = z * SB[u] * inv_alpha;
+      hi = __bfloat162float(__float2bfloat16_rn(v));
+      lo = v - hi;
     }
+    FbZ[a * fz_k + u] = __float2bfloat16_rn(hi);
+    FbZ[a * fz_k + kpB + u] = __float2bfloat16_rn(lo);
+    for (int c = 2 * kpB + u; c < fz_k; c += kpB) FbZ[a * fz_k + c] = __float2bfloat16_rn(0.0f);
+    return;
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < kFoldRows * fold_k; e += blockDim.x) {
-    const int r = e / fold_k, c = e % fold_k;
+  const int64_t i0 = (int64_t)(blockIdx.x - zblocks) * kRowsPerBlock;
+  const float g = *RB.g;
+  for (int e = threadIdx.x; e < kRowsPerBlock * kpB; e += blockDim.x) {
+    const int r = e / kpB, u = e - (e / kpB) * kpB;
     const int64_t i = i0 + r;
-    float out = 0.0f;
-    if (c < 2 * kpA) {
-      const int j = c < kpA ? c : c - kpA;
-      float t = 0.0f;
-      if (j < kA) {
-        t = TA32[i * kpA + j];
-        if (RB.k > 0) {
-          float acc = 0.0f;
-          for (int u = 0; u < RB.k; ++u) acc = fmaf(qrb[r][u], c2[u][j], acc);
-          t += acc;
-        }
-      }
-      const __nv_bfloat16 hi = __float2bfloat16_rn(t);
-      out = c < kpA ? __bfloat162float(hi) : t - __bfloat162float(hi);
-    } else if (c < 2 * kpA + 2 * kpB) {
-      out = qrb[r][(c - 2 * kpA) % kpB];
+    if (i >= q) continue;
+    const __nv_bfloat16 v = __float2bfloat16_rn(u < kB ? factor_value(RB.codes, RB.scales, g, RB.len, u, i) : 0.0f);
+    Fb[i * fold_k + 2 * kpA + u] = v;
+    Fb[i * fold_k + 2 * kpA + kpB + u] = v;
+    if (FaZ) {
+      FaZ[i * fz_k + u] = v;
+      FaZ[i * fz_k + kpB + u] = v;
+      for (int c = 2 * kpB + u; c < fz_k; c += kpB) FaZ[i * fz_k + c] = __float2bfloat16_rn(0.0f);
     }
-    Fb[i * fold_k + c] = __float2bfloat16_rn(out);
   }
 }
 
-// Fa rows: [Q(L_A) | Q(L_A) | T_B hi | T_B lo] / alpha.
-__global__ void fold_a_kernel(const float* __restrict__ TB32, int kpB, int kB, FactorView LA, int kpA, int64_t p,
-                              int fold_k, const float* ga, const float* gb, __nv_bfloat16* __restrict__ Fa) {
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= p * fold_k) return;
-  const int64_t i = idx / fold_k;
-  const int c = (int)(idx - i * fold_k);
-  const float inv_alpha = 1.0f / ((*ga) * (*gb));  // exact: a power of two
-  float out = 0.0f;
-  if (c < 2 * kpA) {
-    const int u = c % kpA;
-    out = u < LA.k ? factor_value(LA.codes, LA.scales, *LA.g, LA.len, u, i) * inv_alpha : 0.0f;
-  } else if (c < 2 * kpA + 2 * kpB) {
-    const int j = (c - 2 * kpA) % kpB;
-    const float t = j < kB ? TB32[i * kpB + j] * inv_alpha : 0.0f;
-    const __nv_bfloat16 hi = __float2bfloat16_rn(t);
-    out = (c - 2 * kpA) < kpB ? __bfloat162float(hi) : t - __bfloat162float(hi);
+// The main GeMM's fold operands, one warp per output row:
+//   Fa rows i < p:  [Q(L_A) | Q(L_A) | T_B hi | T_B lo | 0] / alpha,  T_B = (sum of splits) S_B
+//   Fb rows i < q:  [T_A^T hi | T_A^T lo | (Q(R_B) copies, written by zfold_kernel) | 0],
+//                   T_A^T = (sum of splits) S_A
+// alpha = gA * gB, the tensor scales of the main FP4 GeMM.  A lane owns columns j and j + 1
+// of a kp-wide part and writes both of its copies (hi and lo, or the two Q(L_A) copies).
+__global__ void __launch_bounds__(256) assemble_kernel(const float* __restrict__ TB, int bsplits, int64_t tb_stride,
+                                                       const float* __restrict__ TA, int asplits, int64_t ta_stride,
+                                                       const float* __restrict__ SA, const float* __restrict__ SB,
+                                                       int kA, int kB, int kpA, int kpB, FactorView LA, int64_t p,
+                                                       int64_t q, int fold_k, const float* ga, const float* gb,
+                                                       __nv_bfloat16* __restrict__ Fa, __nv_bfloat16* __restrict__ Fb) {
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= p + q) return;
+  const bool is_a = row < p;
+  const int64_t i = is_a ? row : row - p;
+  __nv_bfloat16* dst = (is_a ? Fa : Fb) + i * fold_k;
+  const float inv_alpha = is_a ? 1.0f / ((*ga) * (*gb)) : 1.0f;   // exact: a power of two
+  // part 1 (columns [0, 2 kpA)): Q(L_A) copies on Fa rows, T_A^T hi / lo on Fb rows
+  for (int j = 2 * lane; j < kpA; j += 64) {
+    float v0 = 0.0f, v1 = 0.0f;
+    if (is_a) {
+      const float gl = *LA.g;
+      if (j < kA) v0 = factor_value(LA.codes, LA.scales, gl, LA.len, j, i) * inv_alpha;
+      if (j + 1 < kA) v1 = factor_value(LA.codes, LA.scales, gl, LA.len, j + 1, i) * inv_alpha;
+      const uint32_t w = pack_bf16x2(v0, v1);
+      *reinterpret_cast<uint32_t*>(dst + j) = w;
+      *reinterpret_cast<uint32_t*>(dst + kpA + j) = w;
+    } else {
+      for (int s = 0; s < asplits; ++s) {
+        const float2 t = *reinterpret_cast<const float2*>(TA + s * ta_stride + i * kpA + j);
+        v0 += t.x;
+        v1 += t.y;
+      }
+      v0 = j < kA ? v0 * SA[j] : 0.0f;
+      v1 = j + 1 < kA ? v1 * SA[j + 1] : 0.0f;
+      const float h0 = __bfloat162float(__float2bfloat16_rn(v0)), h1 = __bfloat162float(__float2bfloat16_rn(v1));
+      *reinterpret_cast<uint32_t*>(dst + j) = pack_bf16x2(h0, h1);
+      *reinterpret_cast<uint32_t*>(dst + kpA + j) = pack_bf16x2(v0 - h0, v1 - h1);
+    }
   }
-  Fa[i * fold_k + c] = __float2bfloat16_rn(out);
-}
-
-__global__ void pad_sigma_kernel(const float* S, int k, int kp, float* out) {
-  const int i = threadIdx.x;
-  if (i < kp) out[i] = i < k ? S[i] : 0.0f;
+  // part 2 (columns [2 kpA, 2 kpA + 2 kpB)): T_B hi / lo on Fa rows (zfold_kernel fills Fb's)
+  if (is_a) {
+    for (int j = 2 * lane; j < kpB; j += 64) {
+      float v0 = 0.0f, v1 = 0.0f;
+      for (int s = 0; s < bsplits; ++s) {
+        const float2 t = *reinterpret_cast<const float2*>(TB + s * tb_stride + i * kpB + j);
+        v0 += t.x;
+        v1 += t.y;
+      }
+      v0 = j < kB ? v0 * SB[j] * inv_alpha : 0.0f;
+      v1 = j + 1 < kB ? v1 * SB[j + 1] * inv_alpha : 0.0f;
+      const float h0 = __bfloat162float(__float2bfloat16_rn(v0)), h1 = __bfloat162float(__float2bfloat16_rn(v1));
+      *reinterpret_cast<uint32_t*>(dst + 2 * kpA + j) = pack_bf16x2(h0, h1);
+      *reinterpret_cast<uint32_t*>(dst + 2 * kpA + kpB + j) = pack_bf16x2(v0 - h0, v1 - h1);
+    }
+  }
+  // padding columns
+  for (int c = 2 * kpA + 2 * kpB + 2 * lane; c < fold_k; c += 64)
+    *reinterpret_cast<uint32_t*>(dst + c) = 0u;
 }
 
 int pad_rank(int k) { return k == 0 ? 0 : k <= 16 ? 16 : k <= 32 ? 32 : 64; }
@@ -180,59 +193,61 @@ metis_status run_linear(metis_ctx* ctx, const metis_operand* A, const metis_nvfp
   const int fold_k = (kA || kB) ? ((2 * kpA + 2 * kpB + 63) / 64) * 64 : 0;
 
   if (fold_k == 0) {
-    GemmArgs g{A_res, B_res, nullptr, nullptr, 0, nullptr, C, ldc, c_dtype, 1.0f, q};
+    GemmArgs g{A_res, B_res, nullptr, nullptr, 0, nullptr, C, ldc, c_dtype, 1.0f, q, 1, 0};
     return launch_gemm_nvfp4(ctx, g);
   }
 
-  const int nchunks = (int)(K / kZChunk);
-  const size_t need = 256 * 12 + (size_t)p * kpB * 4 + (size_t)q * kpA * 4 + (size_t)nchunks * 4096 * 4 + 4096 * 4 +
-                      2 * 64 * 4 + (size_t)p * fold_k * 2 + (size_t)q * fold_k * 2;
+  const bool corr = kA && kB;   // T_A picks up the correction Q(R_B) S_B Z^T S_A
+  const int stagesK = (int)(K / 256);
+  const int fz_k = corr ? ((2 * kpB + 63) / 64) * 64 : 0;
+  const int zsplits = corr ? fp4_splits(ctx, 1, stagesK) : 0;
+  const int bsplits = kB ? fp4_splits(ctx, p / 128, stagesK) : 0;
+  const int asplits = kA ? fp4_splits(ctx, q / 128, stagesK + fz_k / 64) : 0;
+  const size_t need = 256 * 12 + (size_t)bsplits * p * kpB * 4 + (size_t)asplits * q * kpA * 4 +
+                      (size_t)zsplits * 128 * kpB * 4 + (size_t)q * fz_k * 2 + (size_t)128 * fz_k * 2 +
+                      (size_t)p * fold_k * 2 + (size_t)q * fold_k * 2;
   if ((s = ensure_workspace(ctx, need)) != METIS_OK) return s;
   Workspace ws{ctx->ws, ctx->ws_bytes};
-  float* TB32 = static_cast<float*>(ws.take((size_t)p * std::max(kpB, 1) * 4));
-  float* TA32 = static_cast<float*>(ws.take((size_t)q * std::max(kpA, 1) * 4));
-  float* Zp = static_cast<float*>(ws.take((size_t)nchunks * 4096 * 4));
-  float* Z = static_cast<float*>(ws.take(4096 * 4));
-  float* SAp = static_cast<float*>(ws.take(64 * 4));
-  float* SBp = static_cast<float*>(ws.take(64 * 4));
+  float* TB32 = static_cast<float*>(ws.take((size_t)std::max(bsplits, 1) * p * std::max(kpB, 1) * 4));
+  float* TA32 = static_cast<float*>(ws.take((size_t)std::max(asplits, 1) * q * std::max(kpA, 1) * 4));
+  float* Zp = static_cast<float*>(ws.take((size_t)std::max(zsplits, 1) * 128 * std::max(kpB, 1) * 4));
+  __nv_bfloat16* FaZ = static_cast<__nv_bfloat16*>(ws.take((size_t)q * std::max(fz_k, 64) * 2));
+  __nv_bfloat16* FbZ = static_cast<__nv_bfloat16*>(ws.take((size_t)128 * std::max(fz_k, 64) * 2));
   __nv_bfloat16* Fa = static_cast<__nv_bfloat16*>(ws.take((size_t)p * fold_k * 2));
   __nv_bfloat16* Fb = static_cast<__nv_bfloat16*>(ws.take((size_t)q * fold_k * 2));
+  if (!Fb) return fail(ctx, METIS_ERR_WORKSPACE, "fold workspace layout");
   cudaStream_t st = ctx->stream;
 
-  FactorView vLA{}, vRA{}, vLB{}, vRB{};
-  if (kA) {
-    vLA = {LAq->codes, LAq->scales, LAq->tensor_scale, LAq->inner, kA};
-    vRA = {RAq->codes, RAq->scales, RAq->tensor_scale, RAq->inner, kA};
-    pad_sigma_kernel<<<1, 64, 0, st>>>(fa->S, kA, kpA, SAp); count_launch();
-  }
-  if (kB) {
-    vLB = {LBq->codes, LBq->scales, LBq->tensor_scale, LBq->inner, kB};
-    vRB = {RBq->codes, RBq->scales, RBq->tensor_scale, RBq->inner, kB};
-    pad_sigma_kernel<<<1, 64, 0, st>>>(fb->S, kB, kpB, SBp); count_launch();
-  }
-  // T_B = Q(A_R) Q(L_B) S_B  (p x kpB, fp32)
-  if (kB) {
-    GemmArgs g{A_res, LBq, nullptr, nullptr, 0, SBp, TB32, kpB, METIS_OUT_F32, 1.0f, kpB};
+  FactorView vLA{}, vRB{};
+  if (kA) vLA = {LAq->codes, LAq->scales, LAq->tensor_scale, LAq->inner, kA};
+  if (kB) vRB = {RBq->codes, RBq->scales, RBq->tensor_scale, RBq->inner, kB};
+  // Z = Q(R_A)^T Q(L_B) on the tensor cores (128 x kpB, split-K over the contraction length)
+  if (corr) {
+    GemmArgs g{RAq, LBq, nullptr, nullptr, 0, nullptr, Zp, kpB, METIS_OUT_F32, 1.0f, kpB, zsplits, 128 * kpB};
     if ((s = launch_gemm_nvfp4(ctx, g)) != METIS_OK) return s;
   }
-  // first part of T_A^T = Q(B_R)^T Q(R_A) S_A  (q x kpA, fp32)
-  if (kA) {
-    GemmArgs g{B_res, RAq, nullptr, nullptr, 0, SAp, TA32, kpA, METIS_OUT_F32, 1.0f, kpA};
+  if (kB) {
+    const int zblocks = corr ? (128 * kpB + 255) / 256 : 0;
+    zfold_kernel<<<(unsigned)(zblocks + (q + kRowsPerBlock - 1) / kRowsPerBlock), 256, 0, st>>>(
+        Zp, zsplits, zblocks, kA, kB, kpA, kpB, fb->S, B_res->tensor_scale, corr ? RAq->tensor_scale : nullptr,
+        vRB, fz_k, corr ? FbZ : nullptr, corr ? FaZ : nullptr, Fb, fold_k, q); count_launch();
+    // T_B = Q(A_R) Q(L_B)  (p x kpB partials; S_B applied when assembling)
+    GemmArgs g{A_res, LBq, nullptr, nullptr, 0, nullptr, TB32, kpB, METIS_OUT_F32, 1.0f, kpB, bsplits,
+               p * kpB};
     if ((s = launch_gemm_nvfp4(ctx, g)) != METIS_OK) return s;
   }
-  // Z = Q(R_A)^T Q(L_B)  (kA x kB over the contraction length K)
-  if (kA && kB) {
-    z_partial_kernel<<<nchunks, 256, 0, st>>>(vRA, vLB, Zp); count_launch();
-    z_reduce_kernel<<<16, 256, 0, st>>>(Zp, nchunks, Z); count_launch();
+  // T_A^T / S_A = Q(B_R)^T Q(R_A) + [Q(R_B) | Q(R_B)] [Z S_B hi | lo]^T / alpha_TA  (q x kpA partials)
+  if (kA) {
+    GemmArgs g{B_res, RAq, corr ? FaZ : nullptr, corr ? FbZ : nullptr, fz_k, nullptr, TA32, kpA, METIS_OUT_F32,
+               1.0f, kpA, asplits, q * kpA};
+    if ((s = launch_gemm_nvfp4(ctx, g)) != METIS_OK) return s;
   }
-  if (kA || kB) {
-    fold_b_kernel<<<(unsigned)(q / kFoldRows), 256, 0, st>>>(TA32, kpA, kA, vRB, kpB, SAp, SBp, Z, q, fold_k,
-                                                             Fb); count_launch();
-    fold_a_kernel<<<(unsigned)((p * fold_k + 255) / 256), 256, 0, st>>>(TB32, kpB, kB, vLA, kpA, p, fold_k,
-                                                                        A_res->tensor_scale, B_res->tensor_scale, Fa); count_launch();
-  }
+  assemble_kernel<<<(unsigned)((p + q + 7) / 8), 256, 0, st>>>(TB32, bsplits, p * kpB, TA32, asplits, q * kpA,
+                                                               kA ? fa->S : nullptr, kB ? fb->S : nullptr, kA, kB,
+                                                               kpA, kpB, vLA, p, q, fold_k, A_res->tensor_scale,
+                                                               B_res->tensor_scale, Fa, Fb); count_launch();
   if ((s = check_cuda(ctx, cudaGetLastError(), "fold preparation")) != METIS_OK) return s;
-  GemmArgs g{A_res, B_res, Fa, Fb, fold_k, nullptr, C, ldc, c_dtype, 1.0f, q};
+  GemmArgs g{A_res, B_res, Fa, Fb, fold_k, nullptr, C, ldc, c_dtype, 1.0f, q, 1, 0};
   return launch_gemm_nvfp4(ctx, g);
 }
 
