@@ -245,59 +245,87 @@ __global__ void times_small_kernel(const float* __restrict__ A, int64_t n, int k
 }
 
 // --------------------------------------------------------------- Gram (fp64)
-// partial[block] = A_rows^T A_rows over the block's rows (chunks of 32 staged in
-// shared memory); upper triangle, full w x w storage.  Each thread keeps its
-// (a, b) sums in registers across the chunks.
+// partial[block] = A_rows^T A_rows over the block's rows, rows staged 32 at a time in
+// shared memory as fp64; a thread owns 4 x 4 tiles (ta <= tb) of the upper triangle
+// and keeps their 16 sums in registers.  TPT = tiles per thread (1 covers w <= 64).
 constexpr int kGramRows = 32;
-constexpr int kGramPer = 64;   // (w*w)/256 for w <= 128
-__global__ void gram_partial_kernel(const float* __restrict__ A, int64_t n, int w, int64_t rows_per_block,
-                                    double* partial, uint32_t* status) {
-  __shared__ double sa[kGramRows][kMaxW + 1];
+template <int TPT>
+__global__ void __launch_bounds__(256) gram_partial_kernel(const float* __restrict__ A, int64_t n, int w,
+                                                           int64_t rows_per_block, double* partial,
+                                                           uint32_t* status) {
+  __shared__ __align__(16) double sa[kGramRows][kMaxW + 2];
   const int64_t r_begin = (int64_t)blockIdx.x * rows_per_block;
   const int64_t r_end = min(n, r_begin + rows_per_block);
-  double acc[kGramPer];
+  const int nt = (w + 3) / 4;
+  int ta[TPT], tb[TPT];
+  double acc[TPT][16];
 #pragma unroll
-  for (int i = 0; i < kGramPer; ++i) acc[i] = 0.0;
+  for (int u = 0; u < TPT; ++u) {
+    const int t = threadIdx.x + u * 256;
+    ta[u] = t / nt;
+    tb[u] = t - (t / nt) * nt;
+    if (ta[u] >= nt || ta[u] > tb[u]) ta[u] = -1;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) acc[u][e] = 0.0;
+  }
   bool finite = true;
+  const int wp = nt * 4;
   for (int64_t r0 = r_begin; r0 < r_end; r0 += kGramRows) {
     __syncthreads();
-    for (int e = threadIdx.x; e < kGramRows * w; e += blockDim.x) {
-      const int r = e / w, j = e % w;
-      const float v = (r0 + r < r_end) ? A[(r0 + r) * w + j] : 0.0f;
+    for (int e = threadIdx.x; e < kGramRows * wp; e += 256) {
+      const int r = e / wp, j = e - (e / wp) * wp;
+      const float v = (r0 + r < r_end && j < w) ? A[(r0 + r) * w + j] : 0.0f;
       finite &= isfinite(v);
       sa[r][j] = v;
     }
     __syncthreads();
 #pragma unroll
-    for (int i = 0; i < kGramPer; ++i) {
-      const int e = threadIdx.x + i * 256;
-      if (e < w * w) {
-        const int a = e / w, b = e % w;
-        if (a <= b) {
-          double s2 = acc[i];
-#pragma unroll 8
-          for (int r = 0; r < kGramRows; ++r) s2 = fma(sa[r][a], sa[r][b], s2);
-          acc[i] = s2;
-        }
+    for (int u = 0; u < TPT; ++u) {
+      if (ta[u] < 0) continue;
+      const double* pa = &sa[0][4 * ta[u]];
+      const double* pb = &sa[0][4 * tb[u]];
+#pragma unroll 4
+      for (int r = 0; r < kGramRows; ++r) {
+        const double2 a01 = *reinterpret_cast<const double2*>(pa + r * (kMaxW + 2));
+        const double2 a23 = *reinterpret_cast<const double2*>(pa + r * (kMaxW + 2) + 2);
+        const double2 b01 = *reinterpret_cast<const double2*>(pb + r * (kMaxW + 2));
+        const double2 b23 = *reinterpret_cast<const double2*>(pb + r * (kMaxW + 2) + 2);
+        const double av[4] = {a01.x, a01.y, a23.x, a23.y}, bv[4] = {b01.x, b01.y, b23.x, b23.y};
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+          for (int y = 0; y < 4; ++y) acc[u][x * 4 + y] = fma(av[x], bv[y], acc[u][x * 4 + y]);
       }
     }
   }
   if (!finite) raise_status(status, METIS_DEV_NONFINITE);
+  double* out = partial + (int64_t)blockIdx.x * w * w;
 #pragma unroll
-  for (int i = 0; i < kGramPer; ++i) {
-    const int e = threadIdx.x + i * 256;
-    if (e < w * w) partial[(int64_t)blockIdx.x * w * w + e] = acc[i];
+  for (int u = 0; u < TPT; ++u) {
+    if (ta[u] < 0) continue;
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int y = 0; y < 4; ++y) {
+        const int a = 4 * ta[u] + x, b = 4 * tb[u] + y;
+        if (a < w && b < w && a <= b) out[a * w + b] = acc[u][x * 4 + y];
+      }
   }
 }
 
-__global__ void gram_reduce_kernel(const double* partial, int nblocks, int w, double* G) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+// G (w x w, full) = sum of the blocks' upper triangles, a warp per entry: lane l adds
+// blocks l, l + 32, ... in order, then a fixed shuffle tree (deterministic).
+__global__ void gram_reduce_kernel(const double* __restrict__ partial, int nblocks, int w, double* __restrict__ G) {
+  const int e = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
   if (e >= w * w) return;
-  const int a = e / w, b = e % w;
-  double acc = 0.0;
+  const int a = e / w, b = e - (e / w) * w;
   const int src = a <= b ? e : b * w + a;
-  for (int c = 0; c < nblocks; ++c) acc += partial[(int64_t)c * w * w + src];
-  G[e] = acc;
+  double acc = 0.0;
+  for (int c = lane; c < nblocks; c += 32) acc += partial[(int64_t)c * w * w + src];
+#pragma unroll
+  for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) G[e] = acc;
 }
 
 // ----------------------------------------------------- single-CTA small solvers
@@ -1011,43 +1039,128 @@ __global__ void reduce_hi_lo_kernel(const float* __restrict__ partial, int split
 
 int pad_width(int w) { return w <= 16 ? 16 : w <= 32 ? 32 : w <= 64 ? 64 : 128; }
 
-// ------------------------------------------------------------- sign fix
-// flip[j] = 1 if the largest-|.| entry of column j of V (first index on ties) is negative.
-__global__ void sign_pick_kernel(const float* __restrict__ V, int64_t n, int k, int* flip) {
-  const int j = blockIdx.x;
-  float best = -1.0f;
-  int64_t bi = 0;
-  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
-    const float a = fabsf(V[i * k + j]);
-    if (a > best) {
-      best = a;
-      bi = i;
-    }
+// ---------------------------------------------------- per-step factor finalization
+// Counters gathered while the new factors are formed (zeroed before): the largest |.| of
+// U and of V (float bits; order-independent atomicMax), and per column j of V V_r the key
+// (|v| bits << 32 | ~row) of its largest-|.| entry, first row on ties.
+struct FactorStats {
+  unsigned long long* amax;   // [0] U, [1] V
+  unsigned long long* key;    // k
+};
+
+// Uraw (r x k) = P T and Vn (c x k) = V Vr, T and Vr fp64 (ld kMaxW), k <= 64.  A block
+// owns 32 rows of one product: the k x k matrix and the rows are staged in shared memory
+// (fp64) and each thread forms up to 8 outputs of one row in fp64.
+constexpr int kFpRows = 32;
+__global__ void __launch_bounds__(256) factor_products_kernel(const float* __restrict__ P, int64_t r,
+                                                              const double* __restrict__ T,
+                                                              const float* __restrict__ V, int64_t c,
+                                                              const double* __restrict__ Vr, int k,
+                                                              float* __restrict__ Uraw, float* __restrict__ Vn,
+                                                              FactorStats fs, uint32_t* status) {
+  __shared__ double sm[64][64];
+  __shared__ float sr[kFpRows][64];
+  __shared__ float so[kFpRows][64];
+  const int64_t nbu = (r + kFpRows - 1) / kFpRows;
+  const bool is_u = blockIdx.x < nbu;
+  const int64_t i0 = (int64_t)(is_u ? blockIdx.x : blockIdx.x - nbu) * kFpRows;
+  const int64_t n = is_u ? r : c;
+  const float* src = is_u ? P : V;
+  const double* M = is_u ? T : Vr;
+  float* dst = is_u ? Uraw : Vn;
+  for (int e = threadIdx.x; e < k * k; e += 256) sm[e / k][e % k] = M[(e / k) * kMaxW + e % k];
+  for (int e = threadIdx.x; e < kFpRows * k; e += 256) {
+    const int rr = e / k, j = e % k;
+    sr[rr][j] = (i0 + rr < n) ? src[(i0 + rr) * k + j] : 0.0f;
   }
-  __shared__ float sb[256];
-  __shared__ int64_t si[256];
-  sb[threadIdx.x] = best;
-  si[threadIdx.x] = bi;
   __syncthreads();
-  for (int s = blockDim.x / 2; s; s >>= 1) {
-    if (threadIdx.x < s) {
-      const float ob = sb[threadIdx.x + s];
-      const int64_t oi = si[threadIdx.x + s];
-      if (ob > sb[threadIdx.x] || (ob == sb[threadIdx.x] && oi < si[threadIdx.x])) {
-        sb[threadIdx.x] = ob;
-        si[threadIdx.x] = oi;
+  const int rr = threadIdx.x >> 3, j0 = threadIdx.x & 7;
+  const int64_t i = i0 + rr;
+  float amax = 0.0f;
+  bool finite = true;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    const int j = j0 + 8 * t;
+    if (j < k) {
+      double a = 0.0;
+      for (int u = 0; u < k; ++u) a = fma((double)sr[rr][u], sm[u][j], a);
+      const float v = (float)a;
+      finite &= isfinite(v);
+      so[rr][j] = v;
+      if (i < n) {
+        dst[i * k + j] = v;
+        amax = fmaxf(amax, fabsf(v));
       }
     }
-    __syncthreads();
   }
-  if (threadIdx.x == 0) flip[j] = V[si[0] * k + j] < 0.0f;
+  if (!finite && i < n) raise_status(status, METIS_DEV_NONFINITE);
+#pragma unroll
+  for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  if ((threadIdx.x & 31) == 0) atomicMax(&fs.amax[is_u ? 0 : 1], (unsigned long long)__float_as_uint(amax));
+  if (!is_u) {
+    __syncthreads();
+    for (int j = threadIdx.x; j < k; j += 256) {
+      unsigned long long best = 0;
+      for (int q = 0; q < kFpRows && i0 + q < n; ++q) {
+        const float a = fabsf(so[q][j]);
+        if (!(a <= 3.402823466e38f)) continue;   // not finite
+        const unsigned long long key =
+            ((unsigned long long)__float_as_uint(a) << 32) | (0xFFFFFFFFu - (uint32_t)(i0 + q));
+        best = key > best ? key : best;
+      }
+      atomicMax(&fs.key[j], best);
+    }
+  }
 }
 
-__global__ void apply_flip_kernel(const float* __restrict__ src, int64_t n, int k, const int* flip, float* dst) {
-  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= n * k) return;
-  const int j = (int)(e % k);
-  dst[e] = flip[j] ? -src[e] : src[e];
+// U, V (fp32 caller state) = the products with the sign convention applied (column j
+// flipped when the largest-|.| entry of Vn's column j is negative), and their NVFP4
+// copies: the transposes, blocks of 16 along the long dimension, outer padded to 128 with
+// zeros, tensor scale pow2_ceil(max / 2688).  A thread per (16-row block, column < 128).
+__global__ void __launch_bounds__(256) factor_finalize_kernel(const float* __restrict__ Uraw, int64_t r,
+                                                              const float* __restrict__ Vn, int64_t c, int k,
+                                                              FactorStats fs, int rounding, uint64_t seed,
+                                                              uint32_t tag_u, uint32_t tag_v, uint32_t step,
+                                                              float* __restrict__ U, float* __restrict__ V,
+                                                              metis_nvfp4 uq, metis_nvfp4 vq) {
+  const int64_t nu = 128 * (r / 16);
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= nu + 128 * (c / 16)) return;
+  const bool is_u = idx < nu;
+  const int64_t t = is_u ? idx : idx - nu;
+  const int j = (int)(t & 127);
+  const int64_t b = t >> 7;
+  const int64_t len = is_u ? r : c;
+  const metis_nvfp4& q = is_u ? uq : vq;
+  const float g = pow2_ceil(__fdiv_rn(__uint_as_float((uint32_t)fs.amax[is_u ? 0 : 1]), 2688.0f));
+  if (t == 0) *q.tensor_scale = g;
+  uint2 packed = make_uint2(0, 0);
+  uint32_t code = 0;
+  if (j < k) {
+    const unsigned long long key = fs.key[j];   // 0 only when the column has no finite entry
+    const int64_t pivot = key ? (int64_t)(0xFFFFFFFFu - (uint32_t)key) : 0;
+    const bool flip = pivot < c && Vn[pivot * k + j] < 0.0f;
+    const float* src = is_u ? Uraw : Vn;
+    float* dst = is_u ? U : V;
+    float v[16];
+    float amax = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float x = src[(b * 16 + e) * k + j];
+      v[e] = flip ? -x : x;
+      dst[(b * 16 + e) * k + j] = v[e];
+      amax = fmaxf(amax, fabsf(v[e]));
+    }
+    const BlockScale bs = block_scale(amax, g);
+    float x[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) x[e] = __fmul_rn(v[e], bs.rcp);
+    packed = encode_block16(x, rounding, seed, is_u ? tag_u : tag_v, step, (uint64_t)j * (uint64_t)len + b * 16);
+    if (bs.code == 0) packed = make_uint2(0, 0);
+    code = bs.code;
+  }
+  *reinterpret_cast<uint2*>(q.codes + j * (len / 2) + b * 8) = packed;
+  q.scales[scale_offset(j, b, len / 64)] = (uint8_t)code;
 }
 
 unsigned blocks_for(int64_t n, int t = 256) { return (unsigned)((n + t - 1) / t); }
@@ -1077,7 +1190,7 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
   need += (size_t)c * std::max(w, k) * 4 + 256;                   // Bm^T / V new
   need += (size_t)((std::max(rows_needed, c) + kGramRows - 1) / kGramRows) * w * w * 8 + 256;  // gram partials
   need += (size_t)kMaxW * kMaxW * 8 * 3 + small_solver_doubles(kMaxW) * 8 + 2048;  // G, T, Vr, solver scratch
-  need += 64 * 4 * 3 + 1024;                                      // S, flags, flips
+  need += 64 * 4 * 2 + (2 + kMaxW) * 8 + 1024;                    // S, flags, factor stats
   need += jac_rot_entries(kJacMaxNE) * sizeof(double2) + 256;     // recorded Jacobi rotations
   need += (size_t)kMaxW * (4 + 8) + 1024;                          // Jacobi order, lambda^-1/2, info
   const int kpw = pad_width(std::max(w, k));
@@ -1103,7 +1216,7 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
   double* sscratch = static_cast<double*>(ws.take(small_solver_doubles(kMaxW) * 8));
   float* Sw = static_cast<float*>(ws.take(64 * 4));
   int* flags = static_cast<int*>(ws.take(64 * 4));
-  int* flip = static_cast<int*>(ws.take(64 * 4));
+  unsigned long long* stats = static_cast<unsigned long long*>(ws.take((2 + kMaxW) * sizeof(unsigned long long)));
   double2* jrot = static_cast<double2*>(ws.take(jac_rot_entries(kJacMaxNE) * sizeof(double2)));
   int* jorder = static_cast<int*>(ws.take((size_t)kMaxW * 4));
   double* jinv = static_cast<double*>(ws.take((size_t)kMaxW * 8));
@@ -1143,8 +1256,10 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
     const int64_t chunks = (n + kGramRows - 1) / kGramRows;
     const int64_t per_block = ((chunks + ctx->sm_count - 1) / ctx->sm_count) * kGramRows;
     const int nb = (int)((n + per_block - 1) / per_block);
-    gram_partial_kernel<<<nb, 256, 0, st>>>(A, n, width, per_block, gpart, ctx->status); count_launch();
-    gram_reduce_kernel<<<blocks_for((int64_t)width * width), 256, 0, st>>>(gpart, nb, width, G); count_launch();
+    if (width <= 64) gram_partial_kernel<1><<<nb, 256, 0, st>>>(A, n, width, per_block, gpart, ctx->status);
+    else gram_partial_kernel<4><<<nb, 256, 0, st>>>(A, n, width, per_block, gpart, ctx->status);
+    count_launch();
+    gram_reduce_kernel<<<(unsigned)((width * width + 7) / 8), 256, 0, st>>>(gpart, nb, width, G); count_launch();
   };
   // out (r x width) = M B on the tensor cores: B (c x width fp32) as a bf16 hi/lo pair
   auto project = [&](const float* B, int width, float* out) -> metis_status {
@@ -1197,22 +1312,19 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
   // per step: P = M V ; R = chol(P^T P) ; SVD(R) ; U = P R^+ U_r ; V <- V V_r
   if ((s = project(f->V, k, Y)) != METIS_OK) return s;
   gram(Y, r, k);
+  so.S = f->S;
   solve(k, 2);
-  times_small_kernel<<<blocks_for(r * k), 256, 0, st>>>(Y, r, k, T, k, Q); count_launch();     // U (unsigned)
-  times_small_kernel<<<blocks_for(c * k), 256, 0, st>>>(f->V, c, k, Vr, k, Bt); count_launch();  // V V_r
-  sign_pick_kernel<<<k, 256, 0, st>>>(Bt, c, k, flip); count_launch();
-  apply_flip_kernel<<<blocks_for(c * k), 256, 0, st>>>(Bt, c, k, flip, f->V); count_launch();
-  apply_flip_kernel<<<blocks_for(r * k), 256, 0, st>>>(Q, r, k, flip, f->U); count_launch();
-  cudaMemcpyAsync(f->S, Sw, (size_t)k * 4, cudaMemcpyDeviceToDevice, st);
-  if ((s = check_cuda(ctx, cudaGetLastError(), "decompose")) != METIS_OK) return s;
-  // factor quantization (blocks along the long dimension, power-of-two tensor scale)
-  float* amax = reinterpret_cast<float*>(flags + 8);
-  e = launch_quantize_factor(f->U, r, k, p->rounding, p->seed, p->operand_id, kSrLeft, step, &f->Uq, amax,
-                             ctx->status, st);
-  if (e != cudaSuccess) return check_cuda(ctx, e, "factor quantization");
-  e = launch_quantize_factor(f->V, c, k, p->rounding, p->seed, p->operand_id, kSrRight, step, &f->Vq, amax + 1,
-                             ctx->status, st);
-  return check_cuda(ctx, e, "factor quantization");
+  // U = P T and V V_r, then the sign convention and the NVFP4 copies (blocks along the long
+  // dimension, power-of-two tensor scale)
+  FactorStats fs{stats, stats + 2};
+  e = cudaMemsetAsync(stats, 0, (size_t)(2 + k) * sizeof(unsigned long long), st);
+  if (e != cudaSuccess) return check_cuda(ctx, e, "cudaMemsetAsync(factor stats)");
+  factor_products_kernel<<<(unsigned)((r + kFpRows - 1) / kFpRows + (c + kFpRows - 1) / kFpRows), 256, 0, st>>>(
+      Y, r, T, f->V, c, Vr, k, Q, Bt, fs, ctx->status); count_launch();
+  factor_finalize_kernel<<<(unsigned)((128 * (r / 16) + 128 * (c / 16) + 255) / 256), 256, 0, st>>>(
+      Q, r, Bt, c, k, fs, p->rounding, p->seed, stream_tag(p->operand_id, kPurposeSR, kSrLeft),
+      stream_tag(p->operand_id, kPurposeSR, kSrRight), step, f->U, f->V, f->Uq, f->Vq); count_launch();
+  return check_cuda(ctx, cudaGetLastError(), "decompose");
 }
 
 }  // namespace metis

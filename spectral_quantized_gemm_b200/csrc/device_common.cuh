@@ -148,6 +148,22 @@ __device__ __forceinline__ uint2 encode_block16(const float (&x)[16], int roundi
   return r;
 }
 
+// Tensor scale of a factor: g = pow2_ceil(max|F| / (6 * 448)), so that every block scale
+// fits E4M3 and dequantized factors stay exact in bf16.
+// Smallest power of two >= t (t >= 0 finite); 1 for t == 0.
+__device__ __forceinline__ float pow2_ceil(float t) {
+  if (!(t > 0.0f)) return 1.0f;
+  const uint32_t bits = __float_as_uint(t);
+  const uint32_t e = bits >> 23, m = bits & 0x7FFFFFu;
+  if (e == 0) {  // subnormal: t = m * 2^-149
+    const uint32_t top = 31u - __clz(m);
+    const uint32_t p = (m & (m - 1)) ? top + 1 : top;
+    return p >= 23 ? __uint_as_float(1u << 23) : __uint_as_float(1u << p);
+  }
+  if (m == 0) return t;
+  return __uint_as_float((e + 1) << 23);
+}
+
 __device__ __forceinline__ void raise_status(uint32_t* status, uint32_t bits) {
   if (status) atomicOr(status, bits);
 }

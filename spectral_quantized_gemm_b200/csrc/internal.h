@@ -60,9 +60,6 @@ cudaError_t launch_quantize_f32(const float* R, int64_t rows, int64_t cols, int6
 cudaError_t launch_residual_f32(const void* M_bf16, int64_t rows, int64_t cols, int64_t ld, const float* U,
                                 const float* S, const float* V, int32_t k, float* out, uint32_t* status,
                                 cudaStream_t st);
-cudaError_t launch_quantize_factor(const float* F, int64_t longdim, int32_t k, int32_t rounding, uint64_t seed,
-                                   uint32_t operand_id, uint32_t sub, uint32_t step, const metis_nvfp4* out,
-                                   float* amax_scratch, uint32_t* status, cudaStream_t st);
 
 // ---- resquant.cu ----
 metis_status run_residual_quantize(metis_ctx* ctx, const metis_matrix* M, const metis_factors* f,

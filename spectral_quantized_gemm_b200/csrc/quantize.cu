@@ -134,71 +134,6 @@ __global__ void residual_f32_kernel(const __nv_bfloat16* __restrict__ M, int64_t
   }
 }
 
-__global__ void absmax_kernel(const float* __restrict__ F, int64_t n, unsigned int* amax_bits, uint32_t* status) {
-  float m = 0.0f;
-  bool finite = true;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-    const float v = F[i];
-    finite &= isfinite(v);
-    m = fmaxf(m, fabsf(v));
-  }
-  if (!finite) raise_status(status, METIS_DEV_NONFINITE);
-#pragma unroll
-  for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-  if ((threadIdx.x & 31) == 0) atomicMax(amax_bits, __float_as_uint(m));
-}
-
-// Smallest power of two >= t (t >= 0 finite); 1 for t == 0.
-__device__ __forceinline__ float pow2_ceil(float t) {
-  if (!(t > 0.0f)) return 1.0f;
-  const uint32_t bits = __float_as_uint(t);
-  const uint32_t e = bits >> 23, m = bits & 0x7FFFFFu;
-  if (e == 0) {  // subnormal: t = m * 2^-149
-    const uint32_t top = 31u - __clz(m);
-    const uint32_t p = (m & (m - 1)) ? top + 1 : top;
-    return p >= 23 ? __uint_as_float(1u << 23) : __uint_as_float(1u << p);
-  }
-  if (m == 0) return t;
-  return __uint_as_float((e + 1) << 23);
-}
-
-// Factor F (long x k, fp32 row-major) -> NVFP4 of F^T (outer 128, inner long),
-// rows >= k written as zeros.  One thread per (row of F^T, 16-block).
-__global__ void quantize_factor_kernel(const float* __restrict__ F, int64_t longdim, int k, int rounding,
-                                       uint64_t seed, uint32_t tag, uint32_t step,
-                                       const unsigned int* __restrict__ amax_bits, uint8_t* __restrict__ codes,
-                                       uint8_t* __restrict__ scales, float* tensor_scale) {
-  const float amax_all = __uint_as_float(*amax_bits);
-  const float g = pow2_ceil(__fdiv_rn(amax_all, 2688.0f));
-  const int64_t nblk = longdim / 16;
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx == 0) *tensor_scale = g;
-  if (idx >= 128 * nblk) return;
-  const int64_t j = idx / nblk;
-  const int64_t b = idx - j * nblk;
-  uint2 packed = make_uint2(0, 0);
-  uint32_t code = 0;
-  if (j < k) {
-    float v[16];
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      v[i] = F[(b * 16 + i) * k + j];
-      amax = fmaxf(amax, fabsf(v[i]));
-    }
-    const BlockScale bs = block_scale(amax, g);
-    float x[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) x[i] = __fmul_rn(v[i], bs.rcp);
-    const uint64_t e0 = (uint64_t)j * (uint64_t)longdim + (uint64_t)b * 16;
-    packed = encode_block16(x, rounding, seed, tag, step, e0);
-    if (bs.code == 0) packed = make_uint2(0, 0);
-    code = bs.code;
-  }
-  *reinterpret_cast<uint2*>(codes + j * (longdim / 2) + b * 8) = packed;
-  scales[scale_offset(j, b, longdim / 64)] = (uint8_t)code;
-}
-
 }  // namespace
 
 cudaError_t launch_quantize_f32(const float* R, int64_t rows, int64_t cols, int64_t ld,
@@ -230,20 +165,5 @@ cudaError_t launch_residual_f32(const void* M_bf16, int64_t rows, int64_t cols, 
   return cudaGetLastError();
 }
 
-cudaError_t launch_quantize_factor(const float* F, int64_t longdim, int32_t k, int32_t rounding, uint64_t seed,
-                                   uint32_t operand_id, uint32_t sub, uint32_t step, const metis_nvfp4* out,
-                                   float* amax_scratch, uint32_t* status, cudaStream_t st) {
-  unsigned int* amax_bits = reinterpret_cast<unsigned int*>(amax_scratch);
-  cudaError_t e = cudaMemsetAsync(amax_bits, 0, sizeof(unsigned int), st);
-  if (e != cudaSuccess) return e;
-  const int64_t n = longdim * k;
-  const int blocks = (int)std::min<int64_t>((n + 255) / 256, 1024);
-  absmax_kernel<<<blocks, 256, 0, st>>>(F, n, amax_bits, status); count_launch();
-  const int64_t nthreads = 128 * (longdim / 16);
-  quantize_factor_kernel<<<(unsigned)((nthreads + 255) / 256), 256, 0, st>>>(
-      F, longdim, k, rounding, seed, stream_tag(operand_id, kPurposeSR, sub), step, amax_bits, out->codes,
-      out->scales, out->tensor_scale); count_launch();
-  return cudaGetLastError();
-}
 
 }  // namespace metis
