@@ -148,8 +148,10 @@ class Layer:
             row, col = ctx.new_nvfp4(rows, cols), ctx.new_nvfp4(cols, rows)
             self.ops[name] = (f, row, col, ctx.operand(row, col, f))
         l, m, n = cfg["l"], cfg["m"], cfg["n"]
-        self.Y = torch.empty(l, n, dtype=torch.float32, device=dev)
-        self.dX = torch.empty(l, m, dtype=torch.float32, device=dev)
+        # activations and input gradients in bf16, the weight gradient in fp32 (the
+        # boundary's output types; the GeMMs accumulate in fp32 either way)
+        self.Y = torch.empty(l, n, dtype=torch.bfloat16, device=dev)
+        self.dX = torch.empty(l, m, dtype=torch.bfloat16, device=dev)
         self.dW = torch.empty(m, n, dtype=torch.float32, device=dev)
 
     def step(self, t):
@@ -286,6 +288,7 @@ def run_ours(args, rank, world, device):
                    "l2": "each step's inputs (419 MB) larger than the 126 MB L2; no flush",
                    "batches": args.batches,
                    "streams": "X, W and D decomposed and quantized on three streams; the GeMMs on one",
+                   "outputs": "Y and dX bf16, dW fp32 (fp32 accumulation)",
                    "pct_of_nvfp4_peak": round(100 * value / (world * peak), 2),
                    "nvfp4_peak_tflops": round(peak, 1),
                    "nvfp4_peak_basis": f"bf16_tflops_sustained x {NVFP4_OVER_BF16:.0f} ({kind})"},

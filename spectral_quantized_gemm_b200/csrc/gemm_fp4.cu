@@ -45,13 +45,16 @@ struct Cfg {
   static constexpr int SF_STAGE_BYTES = SFA_BYTES + SFB_BYTES;
   static constexpr int STAGES = BN > 128 ? 4 : (BN == 128 ? 6 : 6);
   static constexpr int SFB_COLS_PER_K = SFB_ATOMS * 4;
+  // scale columns of one stage: SFA (4 per MMA k-step) then SFB
+  static constexpr int SF_SET_COLS = 16 + 4 * SFB_COLS_PER_K;
   // two accumulator buffers (epilogue of tile t overlaps the MMAs of tile t+1)
-  // whenever they fit next to the scale columns in the 512 tensor-memory columns
-  static constexpr int ACC_BUFS = (2 * BN + 16 + 4 * SFB_COLS_PER_K) <= 512 ? 2 : 1;
+  // whenever they fit next to two sets of scale columns in the 512 tensor-memory columns
+  static constexpr int ACC_BUFS = (2 * BN + 2 * SF_SET_COLS) <= 512 ? 2 : 1;
   static constexpr int ACC_COLS = BN * ACC_BUFS;
-  static constexpr int SFA_COL = ACC_COLS;                // 4 columns per MMA k-step
-  static constexpr int SFB_COL = SFA_COL + 16;
-  static constexpr int USED_COLS = SFB_COL + 4 * SFB_COLS_PER_K;
+  // one set of scale columns per ring stage, so the copy of stage s + 1's scales never
+  // waits for the MMAs of stage s to finish reading theirs
+  static constexpr int SF_SETS = STAGES;
+  static constexpr int USED_COLS = ACC_COLS + SF_SETS * SF_SET_COLS;
   static constexpr int TMEM_COLS = USED_COLS <= 32 ? 32 : USED_COLS <= 64 ? 64 : USED_COLS <= 128 ? 128
                                    : USED_COLS <= 256 ? 256 : 512;
   static constexpr size_t SMEM = (size_t)STAGES * (STAGE_BYTES + SF_STAGE_BYTES) + 1024 + 256;
@@ -184,8 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0;
       const uint32_t id_fp4 = tc::idesc_nvf4(BN);
       const uint32_t id_bf16 = tc::idesc_bf16(BN);
-      const uint32_t t_sfa = tmem + C::SFA_COL;
-      const uint32_t t_sfb = tmem + C::SFB_COL;
+
       for (int unit = blockIdx.x; unit < num_units && !*abort_flag; unit += gridDim.x, ++it) {
         const int s0 = (unit / num_tiles) * per_split, s1 = min(total_stages, s0 + per_split);
         const int ab = it % C::ACC_BUFS;
@@ -211,6 +213,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (kk < p.k_stages) {
             const uint8_t* sSFA = sf + stage * C::SF_STAGE_BYTES;
             const uint8_t* sSFB = sSFA + C::SFA_BYTES;
+            const uint32_t t_sfa = tmem + C::ACC_COLS + stage * C::SF_SET_COLS;
+            const uint32_t t_sfb = t_sfa + 16;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               tc::tc_copy_32x128b_x4(t_sfa + 4 * j, tc::sdesc_scales(tc::smem_addr(sSFA + 512 * j)));
