@@ -15,6 +15,9 @@
 //   warp 0      TMA producer: A/B tiles (128-byte swizzle), scale tiles (bulk copy)
 //   warp 1      tensor-memory owner and MMA issuer (one thread)
 //   warps 2..9  epilogue: tcgen05.ld of the accumulator, scale, store
+//   warps 10-11 scale copies (shared -> tensor memory) of each stage, split between
+//               two issuing threads: issued from the MMA thread they serialized with
+//               the MMAs and cost about a quarter of the kernel's time
 // Every mbarrier wait is bounded; on expiry the CTA raises METIS_DEV_TIMEOUT,
 // stops issuing work and exits after releasing its tensor memory.
 #include <cuda.h>
@@ -30,7 +33,7 @@
 namespace metis {
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 constexpr int kEpiWarps = 8;
 
 template <int BN>
@@ -96,7 +99,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* tmem_full = bars + 2 * C::STAGES;   // [2]
   uint64_t* tmem_empty = tmem_full + 2;         // [2]
   uint64_t* drain = tmem_full + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_full + 5);
+  uint64_t* sf_ready = tmem_full + 5;           // [STAGES] the stage's scales are in tensor memory
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_ready + C::STAGES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -106,6 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < C::STAGES; ++s) {
       tc::mbar_init(&full[s], 1);
       tc::mbar_init(&empty[s], 1);
+      tc::mbar_init(&sf_ready[s], 2);
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&tmem_full[b], 1);
@@ -200,7 +205,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc::tc_fence_after();
         for (int kk = s0; kk < s1; ++kk) {
-          if (!tc::mbar_wait(&full[stage], phase, abort_flag)) {
+          if (!tc::mbar_wait(&full[stage], phase, abort_flag) ||
+              !tc::mbar_wait(&sf_ready[stage], phase, abort_flag)) {
             *abort_flag = 1;
             raise_status(p.status, METIS_DEV_TIMEOUT);
             break;
@@ -211,18 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t adesc = tc::sdesc_sw128(tc::smem_addr(sA));
           const uint64_t bdesc = tc::sdesc_sw128(tc::smem_addr(sB));
           if (kk < p.k_stages) {
-            const uint8_t* sSFA = sf + stage * C::SF_STAGE_BYTES;
-            const uint8_t* sSFB = sSFA + C::SFA_BYTES;
             const uint32_t t_sfa = tmem + C::ACC_COLS + stage * C::SF_SET_COLS;
             const uint32_t t_sfb = t_sfa + 16;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              tc::tc_copy_32x128b_x4(t_sfa + 4 * j, tc::sdesc_scales(tc::smem_addr(sSFA + 512 * j)));
-#pragma unroll
-              for (int a = 0; a < C::SFB_ATOMS; ++a)
-                tc::tc_copy_32x128b_x4(t_sfb + C::SFB_COLS_PER_K * j + 4 * a,
-                                       tc::sdesc_scales(tc::smem_addr(sSFB + 2048 * a + 512 * j)));
-            }
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               tc::mma_nvf4(t_acc, adesc + 2 * j, bdesc + 2 * j, id_fp4, t_sfa + 4 * j,
@@ -244,6 +240,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       // let every issued tensor-core operation finish before the memory is released
       tc::tc_commit(drain);
       tc::mbar_wait(drain, 0, nullptr);
+    }
+    __syncwarp();
+  } else if (warp >= 10) {
+    // ------------------------------------------------------------ scale copies
+    // Thread 0 of warp 10 copies SFA and the first 128-row atom of SFB, thread 0 of
+    // warp 11 the second SFB atom; both commit to the stage's sf_ready (count 2), for
+    // fold stages too, so its phases follow the ring.  A stage's scale columns are
+    // free again once the stage is refilled (its previous MMAs committed empty).
+    const int part = warp - 10;
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int unit = blockIdx.x; unit < num_units && !*abort_flag; unit += gridDim.x) {
+        const int s0 = (unit / num_tiles) * per_split, s1 = min(total_stages, s0 + per_split);
+        for (int kk = s0; kk < s1; ++kk) {
+          if (!tc::mbar_wait(&full[stage], phase, abort_flag)) {
+            *abort_flag = 1;
+            raise_status(p.status, METIS_DEV_TIMEOUT);
+            break;
+          }
+          tc::tc_fence_after();
+          if (kk < p.k_stages) {
+            const uint8_t* sSFA = sf + stage * C::SF_STAGE_BYTES;
+            const uint8_t* sSFB = sSFA + C::SFA_BYTES;
+            const uint32_t t_sfa = tmem + C::ACC_COLS + stage * C::SF_SET_COLS;
+            const uint32_t t_sfb = t_sfa + 16;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              if (part == 0) tc::tc_copy_32x128b_x4(t_sfa + 4 * j, tc::sdesc_scales(tc::smem_addr(sSFA + 512 * j)));
+#pragma unroll
+              for (int a = 0; a < C::SFB_ATOMS; ++a)
+                if (a == part || (C::SFB_ATOMS == 1 && part == 0))
+                  tc::tc_copy_32x128b_x4(t_sfb + C::SFB_COLS_PER_K * j + 4 * a,
+                                         tc::sdesc_scales(tc::smem_addr(sSFB + 2048 * a + 512 * j)));
+            }
+          }
+          tc::tc_commit(&sf_ready[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
     }
     __syncwarp();
   } else {
