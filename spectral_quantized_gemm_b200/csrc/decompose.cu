@@ -1163,6 +1163,31 @@ __global__ void __launch_bounds__(256) factor_finalize_kernel(const float* __res
   q.scales[scale_offset(j, b, len / 64)] = (uint8_t)code;
 }
 
+// Mt (c x r, bf16, row-major) = M^T for M (r x c, leading dimension ld), r and c multiples
+// of 64: 64 x 64 tiles through shared memory, rows read and written as 128-byte lines.
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(const __nv_bfloat16* __restrict__ M, int64_t ld,
+                                                             int64_t r, __nv_bfloat16* __restrict__ Mt) {
+  __shared__ __nv_bfloat16 t[64][66];
+  const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int row = ty + 8 * i;
+    const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(M + (r0 + row) * ld + c0 + 2 * tx);
+    t[row][2 * tx] = v.x;
+    t[row][2 * tx + 1] = v.y;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int col = ty + 8 * i;
+    __nv_bfloat162 v;
+    v.x = t[2 * tx][col];
+    v.y = t[2 * tx + 1][col];
+    *reinterpret_cast<__nv_bfloat162*>(Mt + (c0 + col) * r + r0 + 2 * tx) = v;
+  }
+}
+
 unsigned blocks_for(int64_t n, int t = 256) { return (unsigned)((n + t - 1) / t); }
 
 }  // namespace
@@ -1194,10 +1219,13 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
   need += jac_rot_entries(kJacMaxNE) * sizeof(double2) + 256;     // recorded Jacobi rotations
   need += (size_t)kMaxW * (4 + 8) + 1024;                          // Jacobi order, lambda^-1/2, info
   const int kpw = pad_width(std::max(w, k));
-  need += (size_t)2 * kpw * c * 2 + 256;                          // hi/lo transposed operand
-  const int splits_est = normalize_splits(c, bf16_splits(ctx, r, c));
-  const size_t tc_partial_bytes = (size_t)splits_est * r * 2 * kpw * 4;
+  const bool unsampled = lk >= r;   // the refresh's Bm^T = M^T Q then runs on M^T (tensor cores)
+  need += (size_t)2 * kpw * std::max(r, c) * 2 + 256;             // hi/lo transposed operand
+  const int splits_est = std::max(normalize_splits(c, bf16_splits(ctx, r, c)),
+                                  unsampled ? normalize_splits(r, bf16_splits(ctx, c, r)) : 1);
+  const size_t tc_partial_bytes = (size_t)splits_est * std::max(r, c) * 2 * kpw * 4;
   need += tc_partial_bytes + 256;                                 // split partials
+  if (unsampled) need += (size_t)r * c * 2 + 256;                 // M^T
   metis_status s = ensure_workspace(ctx, need);
   if (s != METIS_OK) return s;
   Workspace ws{ctx->ws, ctx->ws_bytes};
@@ -1221,8 +1249,9 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
   int* jorder = static_cast<int*>(ws.take((size_t)kMaxW * 4));
   double* jinv = static_cast<double*>(ws.take((size_t)kMaxW * 8));
   int* jinfo = static_cast<int*>(ws.take(64));
-  __nv_bfloat16* bt2 = static_cast<__nv_bfloat16*>(ws.take((size_t)2 * kpw * c * 2));
+  __nv_bfloat16* bt2 = static_cast<__nv_bfloat16*>(ws.take((size_t)2 * kpw * std::max(r, c) * 2));
   float* tc_partial = static_cast<float*>(ws.take(tc_partial_bytes));
+  __nv_bfloat16* Mt = unsampled ? static_cast<__nv_bfloat16*>(ws.take((size_t)r * c * 2)) : nullptr;
   if (!tc_partial) return fail(ctx, METIS_ERR_WORKSPACE, "decompose workspace layout");
 
   cudaError_t e = cudaFuncSetAttribute(cholqr_solver_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1262,16 +1291,24 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
     gram_reduce_kernel<<<(unsigned)((width * width + 7) / 8), 256, 0, st>>>(gpart, nb, width, G); count_launch();
   };
   // out (r x width) = M B on the tensor cores: B (c x width fp32) as a bf16 hi/lo pair
-  auto project = [&](const float* B, int width, float* out) -> metis_status {
+  // out (rows x width) = A B on the tensor cores: A bf16 (rows x K, leading dimension lda),
+  // B fp32 (K x width) as a bf16 hi/lo pair, split-K partials summed in order
+  auto project_on = [&](const __nv_bfloat16* A, int64_t lda, int64_t rows, int64_t K, const float* B, int width,
+                        float* out) -> metis_status {
     const int kp = pad_width(width);
-    split_hi_lo_t_kernel<<<blocks_for((int64_t)2 * kp * c), 256, 0, st>>>(B, c, width, kp, bt2); count_launch();
-    const int splits = normalize_splits(c, bf16_splits(ctx, r, c));
-    if ((size_t)splits * r * 2 * kp * 4 > tc_partial_bytes)
+    split_hi_lo_t_kernel<<<blocks_for((int64_t)2 * kp * K), 256, 0, st>>>(B, K, width, kp, bt2); count_launch();
+    const int splits = normalize_splits(K, bf16_splits(ctx, rows, K));
+    if ((size_t)splits * rows * 2 * kp * 4 > tc_partial_bytes)
       return fail(ctx, METIS_ERR_WORKSPACE, "projection partials exceed workspace");
-    metis_status st2 = launch_gemm_bf16(ctx, Mb, M->ld, r, bt2, c, 2 * kp, c, tc_partial, 2 * kp, splits);
+    metis_status st2 = launch_gemm_bf16(ctx, A, lda, rows, bt2, K, 2 * kp, K, tc_partial, 2 * kp, splits);
     if (st2 != METIS_OK) return st2;
-    reduce_hi_lo_kernel<<<blocks_for(r * width), 256, 0, st>>>(tc_partial, splits, r, kp, width, out); count_launch();
+    reduce_hi_lo_kernel<<<blocks_for(rows * width), 256, 0, st>>>(tc_partial, splits, rows, kp, width, out);
+    count_launch();
     return METIS_OK;
+  };
+  // out (r x width) = M B
+  auto project = [&](const float* B, int width, float* out) -> metis_status {
+    return project_on(Mb, M->ld, r, c, B, width, out);
   };
   auto rows_times = [&](const int32_t* rowmap, int64_t nr, const float* B, int width, float* out) {
     dim3 grid(blocks_for(nr, kRowsPerBlock), nsplit);
@@ -1304,7 +1341,14 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
     solve(w, 0);
     times_small_kernel<<<blocks_for(lk * w), 256, 0, st>>>(Y, lk, w, T, w, Q); count_launch();
     // Bm^T = M_s^T Q ; R2 = chol(Bm Bm^T) ; SVD(R2^T) ; V = Bm^T R2^+ W'[:, :k]
-    cols_times_matrix_kernel<<<blocks_for(c, 64), 256, 0, st>>>(Mb, M->ld, idx, lk, c, Q, w, Bt); count_launch();
+    if (unsampled) {
+      // all rows: Bm^T = M^T Q on the tensor cores, from one transposed copy of M
+      dim3 tgrid((unsigned)(c / 64), (unsigned)(r / 64));
+      transpose_bf16_kernel<<<tgrid, 256, 0, st>>>(Mb, M->ld, r, Mt); count_launch();
+      if ((s = project_on(Mt, r, c, r, Q, w, Bt)) != METIS_OK) return s;
+    } else {
+      cols_times_matrix_kernel<<<blocks_for(c, 64), 256, 0, st>>>(Mb, M->ld, idx, lk, c, Q, w, Bt); count_launch();
+    }
     gram(Bt, c, w);
     solve(w, 1);
     times_small_kernel<<<blocks_for(c * k), 256, 0, st>>>(Bt, c, w, T, k, f->V); count_launch();
