@@ -41,7 +41,7 @@ struct RqCfg {
   static constexpr int STAGE_BYTES = V_BYTES + M_BYTES;
   static constexpr int STAGES = 2;
   static constexpr int R_BYTES = 128 * 128 * 4;
-  static constexpr size_t SMEM = (size_t)A_BYTES + STAGES * STAGE_BYTES + R_BYTES + 1024 + 256;
+  static constexpr size_t SMEM = (size_t)A_BYTES + STAGES * STAGE_BYTES + R_BYTES + 1024 + 256 + 512;
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -74,14 +74,37 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64
       : "memory");
 }
 
+// The block rule of block_scale() with two exact shortcuts for this kernel:
+//  * target = RN(amax / (6 g)).  For g = 1 it is formed as q0 = RN(amax * RN(1/6)) corrected
+//    by one fused multiply-add, q0 + RN(amax - 6 q0) * RN(1/6); checked exhaustively on the
+//    CPU to equal the IEEE quotient for every finite amax >= 2^-125, and below that both
+//    round to E4M3 code 0.  Other g use the IEEE division.
+//  * rcp = RN(1 / (s g)) depends only on the scale code: a per-CTA table of 128 entries
+//    built with the same operations.
+__device__ __forceinline__ BlockScale block_scale_fast(float amax, float g, const float* rcp_table) {
+  float target;
+  if (g == 1.0f) {
+    const float r6 = 1.0f / 6.0f;
+    const float q0 = __fmul_rn(amax, r6);
+    target = __fmaf_rn(__fmaf_rn(-6.0f, q0, amax), r6, q0);
+  } else {
+    target = __fdiv_rn(amax, __fmul_rn(6.0f, g));
+  }
+  uint32_t code = e4m3_code_rn(target);
+  if (amax > 0.0f && code == 0) code = 1;  // smallest E4M3 value 2^-9
+  BlockScale bs;
+  bs.code = code;
+  bs.rcp = rcp_table[code & 127u];
+  return bs;
+}
+
 // One 16-element block: scale code and packed codes (RN or SR with the Philox
-// stream of element index e0 .. e0 + 15 in the orientation's blocked order).
-__device__ __forceinline__ uint2 quantize16(const float (&v)[16], float g, int rounding, uint64_t seed,
-                                            uint32_t tag, uint32_t step, uint64_t e0, uint32_t& scale_code) {
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-  const BlockScale bs = block_scale(amax, g);
+// stream of element index e0 .. e0 + 15 in the orientation's blocked order).  amax is
+// the block's largest |v| (computed by the caller).
+__device__ __forceinline__ uint2 quantize16(const float (&v)[16], float amax, float g, const float* rcp_table,
+                                            int rounding, uint64_t seed, uint32_t tag, uint32_t step, uint64_t e0,
+                                            uint32_t& scale_code) {
+  const BlockScale bs = block_scale_fast(amax, g, rcp_table);
   float x[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) x[i] = __fmul_rn(v[i], bs.rcp);
@@ -125,6 +148,10 @@ __global__ void __launch_bounds__(kRqThreads, 1)
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* rcp_table = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);   // 128 entries
+
+  for (int c = threadIdx.x; c < 128; c += blockDim.x)
+    rcp_table[c] = c ? __frcp_rn(__fmul_rn(e4m3_value((uint32_t)c), p.g)) : 0.0f;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -263,7 +290,6 @@ __global__ void __launch_bounds__(kRqThreads, 1)
       // residual = M - reconstruction (M from the 128B-swizzled 64-column box holding
       // this quarter: chunks (h & 1) * 4 .. + 3 of box h >> 1)
       const uint8_t* sM = sStage + stage * C::STAGE_BYTES + C::V_BYTES + (h >> 1) * 16384;
-      bool finite = true;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         const int c = (h & 1) * 4 + cc;
@@ -278,9 +304,6 @@ __global__ void __launch_bounds__(kRqThreads, 1)
       }
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&empty[stage]);   // this warp is done with M
-#pragma unroll
-      for (int i = 0; i < 32; ++i) finite &= isfinite(v[i]);
-      if (!finite) raise_status(p.status, METIS_DEV_NONFINITE);
       // stage the residual row quarter in shared memory (16-byte chunks XOR-swizzled by row)
 #pragma unroll
       for (int t4 = 0; t4 < 8; ++t4) {
@@ -295,18 +318,25 @@ __global__ void __launch_bounds__(kRqThreads, 1)
         uint32_t sc = 0;
         uint4 out;
         uint32_t* o = reinterpret_cast<uint32_t*>(&out);
+        bool finite = true;
 #pragma unroll
         for (int blk = 0; blk < 2; ++blk) {
           float x[16];
+          uint32_t abits = 0;   // largest |x| as a bit pattern: an integer max keeps Inf and NaN visible
 #pragma unroll
-          for (int i = 0; i < 16; ++i) x[i] = v[blk * 16 + i];
+          for (int i = 0; i < 16; ++i) {
+            x[i] = v[blk * 16 + i];
+            abits = max(abits, __float_as_uint(x[i]) & 0x7FFFFFFFu);
+          }
+          finite &= abits < 0x7F800000u;
           uint32_t code;
-          const uint2 pk = quantize16(x, p.g, p.rounding, p.seed, p.tag_row, p.step,
-                                      (uint64_t)grow * (uint64_t)p.cols + (uint64_t)(gcol + blk * 16), code);
+          const uint2 pk = quantize16(x, __uint_as_float(abits), p.g, rcp_table, p.rounding, p.seed, p.tag_row,
+                                      p.step, (uint64_t)grow * (uint64_t)p.cols + (uint64_t)(gcol + blk * 16), code);
           sc |= code << (8 * blk);
           o[2 * blk] = pk.x;
           o[2 * blk + 1] = pk.y;
         }
+        if (!finite) raise_status(p.status, METIS_DEV_NONFINITE);
         *reinterpret_cast<uint4*>(p.row_codes + grow * (p.cols / 2) + gcol / 2) = out;
         *reinterpret_cast<uint16_t*>(p.row_scales + scale_offset(grow, gcol / 16, p.cols / 64)) = (uint16_t)sc;
       }
@@ -323,13 +353,15 @@ __global__ void __launch_bounds__(kRqThreads, 1)
 #pragma unroll
         for (int blk = 0; blk < 2; ++blk) {
           float x[16];
+          float amax = 0.0f;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int rr = hh * 32 + blk * 16 + i;
             x[i] = sR[rr * 128 + ((((j >> 2) ^ (rr & 7))) << 2) + (j & 3)];
+            amax = fmaxf(amax, fabsf(x[i]));
           }
           uint32_t code;
-          const uint2 pk = quantize16(x, p.g, p.rounding, p.seed, p.tag_col, p.step,
+          const uint2 pk = quantize16(x, amax, p.g, rcp_table, p.rounding, p.seed, p.tag_col, p.step,
                                       (uint64_t)gcolj * (uint64_t)p.rows + (uint64_t)(grow0 + blk * 16), code);
           sc |= code << (8 * blk);
           o[2 * blk] = pk.x;
