@@ -224,12 +224,18 @@ def run_ours(args, rank, world, device):
     barrier()
     torch.cuda.synchronize(device)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ev0.record(stream)
-    for t in range(args.warmup, args.warmup + args.steps):
+    for i, t in enumerate(range(args.warmup, args.warmup + args.steps)):
+        step_ev[i].record(stream)     # a step's operand work starts after the previous step's GeMMs
         layer.step(t)
     ev1.record(stream)
     torch.cuda.synchronize(device)
     barrier()
+    bounds = step_ev + [ev1]
+    step_ms = [bounds[i].elapsed_time(bounds[i + 1]) for i in range(args.steps)]
+    refresh_ms = [d for i, d in enumerate(step_ms) if (args.warmup + i) % cfg["refresh_every"] == 0]
+    normal_ms = [d for i, d in enumerate(step_ms) if (args.warmup + i) % cfg["refresh_every"] != 0]
     launches = lib.kernel_launches() - launches0
     gemm_ms, gemm_n, gemm_flops = ctx.profile_read()
     ctx.profile_enable(False)
@@ -297,6 +303,15 @@ def run_ours(args, rank, world, device):
                      "unit": "TFLOP/s", "frac": None if achieved is None else round(achieved / peak, 4),
                      "traffic": None, "launches_timed": gemm_n,
                      "peak_basis": f"{kind} bf16 sustained x {NVFP4_OVER_BF16:.0f} (nominal NVFP4/bf16 ratio)"},
+        "decomposition": {
+            "refresh_every": cfg["refresh_every"],
+            "refresh_steps_timed": len(refresh_ms),
+            "refresh_step_ms": round(statistics.mean(refresh_ms), 4) if refresh_ms else None,
+            "reuse_step_ms": round(statistics.median(normal_ms), 4) if normal_ms else None,
+            "amortised_share": (round((statistics.mean(refresh_ms) - statistics.median(normal_ms))
+                                      / (cfg["refresh_every"] * statistics.median(normal_ms)), 4)
+                                if refresh_ms and normal_ms else None),
+            "basis": "(refresh step - reuse step) / (refresh_every x reuse step), CUDA events per step"},
         "clocks": clk,
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
