@@ -43,6 +43,11 @@ from workloads import synth  # noqa: E402
 NVFP4_OVER_BF16 = 9.0 / 2.25      # nominal dense tensor-core throughput ratio
 DEFAULT_CONFIG = "llama3_8b_mlp_up"
 METRIC = "effective TFLOP/s of Metis W4A4G4 linear fwd+bwd; % of NVFP4 MMA peak"
+# DRAM bytes (read + write) of one launch of the fused GeMM at the forward shape
+# (8192 x 14336 x 4096, fold 256, bf16 out), from one ncu capture of this kernel version
+# (profile_case.py gemm --bf16; summarized in profiles/gemm_nvfp4_fused_llama3_8b_mlp_up.md).
+# Must be retaken whenever the kernel changes.
+GEMM_FWD_DRAM_BYTES = 73.269504e6 + 188.533248e6
 
 
 def measured_peaks():
@@ -301,7 +306,10 @@ def run_ours(args, rank, world, device):
         "roofline": {"bound": "tensor", "kernel": "gemm_nvfp4_kernel<256> (fused FP4 GeMM + fold)",
                      "achieved": None if achieved is None else round(achieved, 1), "peak": round(peak, 1),
                      "unit": "TFLOP/s", "frac": None if achieved is None else round(achieved / peak, 4),
-                     "traffic": None, "launches_timed": gemm_n,
+                     "traffic": round(GEMM_FWD_DRAM_BYTES),
+                     "traffic_basis": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one forward-shape "
+                                      "launch (bytes); the timed launches are the fwd, dX and dW GeMMs",
+                     "launches_timed": gemm_n,
                      "peak_basis": f"{kind} bf16 sustained x {NVFP4_OVER_BF16:.0f} (nominal NVFP4/bf16 ratio)"},
         "decomposition": {
             "refresh_every": cfg["refresh_every"],
