@@ -1052,18 +1052,21 @@ struct FactorStats {
 };
 
 // Uraw (r x k) = P T and Vn (c x k) = V Vr, T and Vr fp64 (ld kMaxW), k <= 64.  A block
-// owns 32 rows of one product: the k x k matrix and the rows are staged in shared memory
-// (fp64) and each thread forms up to 8 outputs of one row in fp64.
-constexpr int kFpRows = 32;
+// owns 64 rows of one product: the k x k matrix (fp64) and the rows (fp32) are staged in
+// shared memory, and each thread forms a 4 x 4 tile of outputs in fp64 (6 loads per 16
+// fused multiply-adds).
+constexpr int kFpRows = 64;
+constexpr size_t kFpSmem = (size_t)64 * 64 * 8 + (size_t)kFpRows * 64 * 4 * 2;
 __global__ void __launch_bounds__(256) factor_products_kernel(const float* __restrict__ P, int64_t r,
                                                               const double* __restrict__ T,
                                                               const float* __restrict__ V, int64_t c,
                                                               const double* __restrict__ Vr, int k,
                                                               float* __restrict__ Uraw, float* __restrict__ Vn,
                                                               FactorStats fs, uint32_t* status) {
-  __shared__ double sm[64][64];
-  __shared__ float sr[kFpRows][64];
-  __shared__ float so[kFpRows][64];
+  extern __shared__ __align__(16) uint8_t fp_smem[];
+  double* sm = reinterpret_cast<double*>(fp_smem);                  // [64][64]
+  float* sr = reinterpret_cast<float*>(fp_smem + 64 * 64 * 8);      // [kFpRows][64]
+  float* so = sr + kFpRows * 64;                                      // [kFpRows][64]
   const int64_t nbu = (r + kFpRows - 1) / kFpRows;
   const bool is_u = blockIdx.x < nbu;
   const int64_t i0 = (int64_t)(is_u ? blockIdx.x : blockIdx.x - nbu) * kFpRows;
@@ -1071,32 +1074,50 @@ __global__ void __launch_bounds__(256) factor_products_kernel(const float* __res
   const float* src = is_u ? P : V;
   const double* M = is_u ? T : Vr;
   float* dst = is_u ? Uraw : Vn;
-  for (int e = threadIdx.x; e < k * k; e += 256) sm[e / k][e % k] = M[(e / k) * kMaxW + e % k];
-  for (int e = threadIdx.x; e < kFpRows * k; e += 256) {
-    const int rr = e / k, j = e % k;
-    sr[rr][j] = (i0 + rr < n) ? src[(i0 + rr) * k + j] : 0.0f;
+  for (int e = threadIdx.x; e < 64 * 64; e += 256) {
+    const int u = e >> 6, j = e & 63;
+    sm[e] = (u < k && j < k) ? M[u * kMaxW + j] : 0.0;
+  }
+  for (int e = threadIdx.x; e < kFpRows * 64; e += 256) {
+    const int rr = e >> 6, j = e & 63;
+    sr[e] = (i0 + rr < n && j < k) ? src[(i0 + rr) * k + j] : 0.0f;
   }
   __syncthreads();
-  const int rr = threadIdx.x >> 3, j0 = threadIdx.x & 7;
-  const int64_t i = i0 + rr;
+  const int rg = threadIdx.x >> 4, cg = threadIdx.x & 15;   // rows 4 rg .. +3, columns 4 cg .. +3
+  double acc[4][4];
+#pragma unroll
+  for (int x = 0; x < 4; ++x)
+#pragma unroll
+    for (int y = 0; y < 4; ++y) acc[x][y] = 0.0;
+  for (int u = 0; u < k; ++u) {
+    const double2 b01 = *reinterpret_cast<const double2*>(sm + u * 64 + 4 * cg);
+    const double2 b23 = *reinterpret_cast<const double2*>(sm + u * 64 + 4 * cg + 2);
+    const double bv[4] = {b01.x, b01.y, b23.x, b23.y};
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const double a = (double)sr[(4 * rg + x) * 64 + u];
+#pragma unroll
+      for (int y = 0; y < 4; ++y) acc[x][y] = fma(a, bv[y], acc[x][y]);
+    }
+  }
   float amax = 0.0f;
   bool finite = true;
 #pragma unroll
-  for (int t = 0; t < 8; ++t) {
-    const int j = j0 + 8 * t;
-    if (j < k) {
-      double a = 0.0;
-      for (int u = 0; u < k; ++u) a = fma((double)sr[rr][u], sm[u][j], a);
-      const float v = (float)a;
-      finite &= isfinite(v);
-      so[rr][j] = v;
-      if (i < n) {
+  for (int x = 0; x < 4; ++x) {
+    const int64_t i = i0 + 4 * rg + x;
+#pragma unroll
+    for (int y = 0; y < 4; ++y) {
+      const int j = 4 * cg + y;
+      const float v = (float)acc[x][y];
+      so[(4 * rg + x) * 64 + j] = v;
+      if (i < n && j < k) {
         dst[i * k + j] = v;
+        finite &= isfinite(v);
         amax = fmaxf(amax, fabsf(v));
       }
     }
   }
-  if (!finite && i < n) raise_status(status, METIS_DEV_NONFINITE);
+  if (!finite) raise_status(status, METIS_DEV_NONFINITE);
 #pragma unroll
   for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
   if ((threadIdx.x & 31) == 0) atomicMax(&fs.amax[is_u ? 0 : 1], (unsigned long long)__float_as_uint(amax));
@@ -1105,7 +1126,7 @@ __global__ void __launch_bounds__(256) factor_products_kernel(const float* __res
     for (int j = threadIdx.x; j < k; j += 256) {
       unsigned long long best = 0;
       for (int q = 0; q < kFpRows && i0 + q < n; ++q) {
-        const float a = fabsf(so[q][j]);
+        const float a = fabsf(so[q * 64 + j]);
         if (!(a <= 3.402823466e38f)) continue;   // not finite
         const unsigned long long key =
             ((unsigned long long)__float_as_uint(a) << 32) | (0xFFFFFFFFu - (uint32_t)(i0 + q));
@@ -1366,8 +1387,10 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
   FactorStats fs{stats, stats + 2};
   e = cudaMemsetAsync(stats, 0, (size_t)(2 + k) * sizeof(unsigned long long), st);
   if (e != cudaSuccess) return check_cuda(ctx, e, "cudaMemsetAsync(factor stats)");
-  factor_products_kernel<<<(unsigned)((r + kFpRows - 1) / kFpRows + (c + kFpRows - 1) / kFpRows), 256, 0, st>>>(
-      Y, r, T, f->V, c, Vr, k, Q, Bt, fs, ctx->status); count_launch();
+  e = cudaFuncSetAttribute(factor_products_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFpSmem);
+  if (e != cudaSuccess) return check_cuda(ctx, e, "cudaFuncSetAttribute(factor products)");
+  factor_products_kernel<<<(unsigned)((r + kFpRows - 1) / kFpRows + (c + kFpRows - 1) / kFpRows), 256, kFpSmem,
+                           st>>>(Y, r, T, f->V, c, Vr, k, Q, Bt, fs, ctx->status); count_launch();
   factor_finalize_kernel<<<(unsigned)((128 * (r / 16) + 128 * (c / 16) + 255) / 256), 256, 0, st>>>(
       Q, r, Bt, c, k, fs, p->rounding, p->seed, stream_tag(p->operand_id, kPurposeSR, kSrLeft),
       stream_tag(p->operand_id, kPurposeSR, kSrRight), step, f->U, f->V, f->Uq, f->Vq); count_launch();
