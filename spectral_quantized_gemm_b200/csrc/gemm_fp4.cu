@@ -244,10 +244,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp >= 10) {
     // ------------------------------------------------------------ scale copies
-    // Thread 0 of warp 10 copies SFA and the first 128-row atom of SFB, thread 0 of
-    // warp 11 the second SFB atom; both commit to the stage's sf_ready (count 2), for
-    // fold stages too, so its phases follow the ring.  A stage's scale columns are
-    // free again once the stage is refilled (its previous MMAs committed empty).
+    // Thread 0 of warp 10 copies SFA of k-steps 0-1 and the first 128-row atom of SFB,
+    // thread 0 of warp 11 SFA of k-steps 2-3 and the second SFB atom (six copies each
+    // for N = 256); both commit to the stage's sf_ready (count 2), for fold stages too,
+    // so its phases follow the ring.  A stage's scale columns are free again once the
+    // stage is refilled (its previous MMAs committed empty).
     const int part = warp - 10;
     if (lane == 0) {
       int stage = 0;
@@ -268,7 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t t_sfb = t_sfa + 16;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              if (part == 0) tc::tc_copy_32x128b_x4(t_sfa + 4 * j, tc::sdesc_scales(tc::smem_addr(sSFA + 512 * j)));
+              if ((j >> 1) == part)
+                tc::tc_copy_32x128b_x4(t_sfa + 4 * j, tc::sdesc_scales(tc::smem_addr(sSFA + 512 * j)));
 #pragma unroll
               for (int a = 0; a < C::SFB_ATOMS; ++a)
                 if (a == part || (C::SFB_ATOMS == 1 && part == 0))
