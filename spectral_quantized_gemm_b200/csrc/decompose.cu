@@ -336,8 +336,8 @@ __global__ void gram_reduce_kernel(const double* __restrict__ partial, int nbloc
 // a few hundred threads; the problems are a few hundred thousand flops, so the design
 // goal is few barrier-separated steps with independent work inside each.
 //
-// cholqr_solver_kernel: T = R^+ with G = R^T R (Cholesky with dependent-column drop), so
-//   that Q = Y T is the CholQR factor.  Right-looking on unscaled rows
+// cholqr_solver_kernel (sketches wider than kSmallMaxN, global scratch): T = R^+ with
+//   G = R^T R (Cholesky with dependent-column drop), so that Q = Y T is the CholQR factor.  Right-looking on unscaled rows
 //   (B_it -= B_ji B_jt / d_j) in panels of kPanel pivots, then R^+ by blocked back
 //   substitution on the identity.
 // eig_solver_kernel: the SVD of Y through the symmetric eigenproblem of G = Y^T Y =
@@ -383,14 +383,12 @@ __device__ __forceinline__ void round_pair(int pr, int round, int ne, int& p, in
   }
 }
 
-template <bool kSmem>
 __global__ void __launch_bounds__(kSolverThreads) cholqr_solver_kernel(const double* __restrict__ G, int n,
                                                                        SmallOut out) {
-  extern __shared__ double smem_d[];
   const int ne = (n + 1) & ~1;
   const int ld = ne;       // R / Cholesky work array, ld x ld
   const int lp = ne + 1;   // odd column stride of the right-hand sides
-  double* const bR = kSmem ? smem_d : out.scratch;
+  double* const bR = out.scratch;
   double* const bV = bR + ld * ld;
   __shared__ int dropped[kMaxW];
   __shared__ double invd[kMaxW];        // 1 / d_j (0 for a dropped pivot)
@@ -506,6 +504,73 @@ __global__ void __launch_bounds__(kSolverThreads) cholqr_solver_kernel(const dou
   for (int e = tid; e < n * n; e += kSolverThreads) {
     const int i = e / n, c = e - (e / n) * n;
     out.T[i * kMaxW + c] = bV[c * lp + i];
+  }
+}
+
+// T = R^+ for G = R^T R (CholQR of a tall Y with G = Y^T Y), n <= kSmallMaxN, one CTA:
+// right-looking Cholesky of the lower triangle (G = L L^T, L = R^T) on unscaled columns,
+// A_ik -= A_ij A_kj / d_j, two barriers per pivot; a pivot d_j not above
+// kDropTol * max diag(G) drops column j (zero row of R, zero column of Q).  Then
+// X = L^{-1} by forward substitution on the identity, all columns at once, and
+// T = X^T.  A warp per row, lanes along the row: no divisions in the index math.
+constexpr int kCholThreads = 512;
+__host__ __device__ constexpr size_t chol_smem_bytes(int n) { return (size_t)2 * n * (n + 1) * sizeof(double); }
+__global__ void __launch_bounds__(kCholThreads) chol_inverse_kernel(const double* __restrict__ G, int n,
+                                                                    SmallOut out) {
+  extern __shared__ double smem_d[];
+  const int ld = n + 1;
+  double* const A = smem_d;            // A[i * ld + k], k <= i
+  double* const X = smem_d + n * ld;   // L^{-1}, X[i * ld + c], c <= i
+  __shared__ double linv[kMaxW];       // 1 / L_jj = d_j^{-1/2}, 0 for a dropped pivot
+  __shared__ double gmax_s;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  constexpr int W = kCholThreads / 32;
+  for (int e = tid; e < n * n; e += kCholThreads) {
+    const int i = e / n, k = e - (e / n) * n;
+    if (k <= i) A[i * ld + k] = G[e];
+    X[i * ld + k] = (i == k) ? 1.0 : 0.0;
+  }
+  if (warp == 0) {
+    double g = 0.0;
+    for (int j = lane; j < n; j += 32) g = fmax(g, G[j * n + j]);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) g = fmax(g, __shfl_xor_sync(0xffffffffu, g, off));
+    if (lane == 0) gmax_s = g;
+  }
+  __syncthreads();
+  const double tol = kDropTol * gmax_s;
+  for (int j = 0; j < n; ++j) {
+    if (tid == 0) {
+      const double d = A[j * ld + j];
+      const bool drop = !(d > tol) || gmax_s == 0.0;
+      linv[j] = drop ? 0.0 : rsqrt(d);
+    }
+    __syncthreads();
+    const double invd = linv[j] * linv[j];
+    if (invd != 0.0) {
+      for (int i = j + 1 + warp; i < n; i += W) {
+        const double f = A[i * ld + j] * invd;
+        for (int k = j + 1 + lane; k <= i; k += 32) A[i * ld + k] = fma(-f, A[k * ld + j], A[i * ld + k]);
+      }
+    }
+    __syncthreads();
+  }
+  // X = L^{-1}: row i is final once scaled by 1 / L_ii; then rows r > i drop L_ri X_i
+  for (int i = 0; i < n; ++i) {
+    const double s = linv[i];
+    for (int c = tid; c <= i; c += kCholThreads) X[i * ld + c] *= s;
+    __syncthreads();
+    for (int r = i + 1 + warp; r < n; r += W) {
+      const double l = A[r * ld + i] * s;   // L_ri
+      if (l != 0.0)
+        for (int c = lane; c <= i; c += 32) X[r * ld + c] = fma(-l, X[i * ld + c], X[r * ld + c]);
+    }
+    __syncthreads();
+  }
+  for (int e = tid; e < n * n; e += kCholThreads) {
+    const int i = e / n, c = e - (e / n) * n;
+    out.T[i * kMaxW + c] = (i <= c) ? X[c * ld + i] : 0.0;   // T = X^T (upper triangular)
   }
 }
 
@@ -1278,8 +1343,8 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
   __nv_bfloat16* Mt = unsampled ? static_cast<__nv_bfloat16*>(ws.take((size_t)r * c * 2)) : nullptr;
   if (!tc_partial) return fail(ctx, METIS_ERR_WORKSPACE, "decompose workspace layout");
 
-  cudaError_t e = cudaFuncSetAttribute(cholqr_solver_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)(small_solver_doubles(kSmallMaxN) * 8));
+  cudaError_t e = cudaFuncSetAttribute(chol_inverse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)chol_smem_bytes(kSmallMaxN));
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(jacobi_rounds_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)jac_smem_bytes(kJacMaxNE));
@@ -1288,12 +1353,9 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
   JacOut jo{jrot, jinfo, jorder, jinv};
   // mode 0: CholQR factor T = R^+; modes 1 and 2: SVD through the eigenproblem of G
   auto solve = [&](int n, int mode) {
-    const int ne = (n + 1) & ~1;
-    const bool in_smem = ne <= kSmallMaxN;
-    const size_t smem = in_smem ? small_solver_doubles(ne) * 8 : 0;
     if (mode == 0) {
-      if (in_smem) cholqr_solver_kernel<true><<<1, kSolverThreads, smem, st>>>(G, n, so);
-      else cholqr_solver_kernel<false><<<1, kSolverThreads, 0, st>>>(G, n, so);
+      if (n <= kSmallMaxN) chol_inverse_kernel<<<1, kCholThreads, chol_smem_bytes(n), st>>>(G, n, so);
+      else cholqr_solver_kernel<<<1, kSolverThreads, 0, st>>>(G, n, so);
     } else if (jac_ne(n) <= kJacMaxNE) {
       jacobi_rounds_kernel<<<1, kJacThreads, jac_smem_bytes(jac_ne(n)), st>>>(G, n, k, mode, jo, so, ctx->status);
       count_launch();
