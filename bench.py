@@ -132,8 +132,9 @@ class Layer:
 
     NAMES = ("X", "W", "D")
 
-    def __init__(self, lib, ctx, cfg, batches, W):
+    def __init__(self, lib, ctx, cfg, batches, W, plain=False):
         self.lib, self.ctx, self.cfg = lib, ctx, cfg
+        self.plain = plain   # plain NVFP4 (no decomposition, no fold): the baseline Metis improves on
         self.rounding = 1 if cfg["rounding"] == "sr" else 0
         self.batches = batches
         X, D = batches[0]
@@ -149,7 +150,7 @@ class Layer:
         self.ops = {}
         for name, M in self.mats.items():
             rows, cols = M.shape
-            f = ctx.new_factors(rows, cols, k, s)
+            f = None if plain else ctx.new_factors(rows, cols, k, s)
             row, col = ctx.new_nvfp4(rows, cols), ctx.new_nvfp4(cols, rows)
             self.ops[name] = (f, row, col, ctx.operand(row, col, f))
         l, m, n = cfg["l"], cfg["m"], cfg["n"]
@@ -174,8 +175,9 @@ class Layer:
                 ctx = self.ctxs[name]
                 f, row, col, _ = self.ops[name]
                 M = self.mats[name]
-                ctx.decompose(M, k=cfg["k"], s=cfg["s"], l_k=self.l_k[name], seed=cfg["seed"], operand_id=i,
-                              refresh=refresh, step=t, factors=f, rounding=self.rounding)
+                if not self.plain:
+                    ctx.decompose(M, k=cfg["k"], s=cfg["s"], l_k=self.l_k[name], seed=cfg["seed"], operand_id=i,
+                                  refresh=refresh, step=t, factors=f, rounding=self.rounding)
                 ctx.residual_quantize_nvfp4(M, f, row, col, rounding=self.rounding, seed=cfg["seed"],
                                             operand_id=i, step=t)
                 ready[name] = torch.cuda.Event()
@@ -284,6 +286,26 @@ def run_ours(args, rank, world, device):
     e2e_value = world * flops_per_step / (e2e_ms / e2e_steps * 1e-3) / 1e12
     status = layer.poll_device_status()
 
+    # ---- plain NVFP4 on the same batches (no decomposition, no rank fold), same timing
+    plain = Layer(lib, ctx, cfg, dev_batches, dev_W, plain=True)
+    for t in range(3):
+        plain.step(t)
+    barrier()
+    torch.cuda.synchronize(device)
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    for t in range(3, 3 + args.steps):
+        plain.step(t)
+    p1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    plain_ms = p0.elapsed_time(p1) / args.steps
+    if world > 1:
+        t_ = torch.tensor([plain_ms], device=device)
+        torch.distributed.all_reduce(t_, op=torch.distributed.ReduceOp.MAX)
+        plain_ms = float(t_.item())
+    status |= plain.poll_device_status()
+
     peaks, kind = measured_peaks()
     peak = peaks["bf16_tflops_sustained"] * NVFP4_OVER_BF16
     achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
@@ -311,6 +333,12 @@ def run_ours(args, rank, world, device):
                                       "launch (bytes); the timed launches are the fwd, dX and dW GeMMs",
                      "launches_timed": gemm_n,
                      "peak_basis": f"{kind} bf16 sustained x {NVFP4_OVER_BF16:.0f} (nominal NVFP4/bf16 ratio)"},
+        "plain_nvfp4": {
+            "value": round(world * flops_per_step / (plain_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(plain_ms, 4),
+            "metis_over_plain": round(ms_per_step / plain_ms, 4),
+            "what": "the same step with k = 0: residual = operand, plain NVFP4 in both orientations, "
+                    "three FP4 GeMMs without the rank fold"},
         "decomposition": {
             "refresh_every": cfg["refresh_every"],
             "refresh_steps_timed": len(refresh_ms),
