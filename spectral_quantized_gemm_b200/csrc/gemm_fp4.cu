@@ -84,6 +84,62 @@ struct Params {
   uint32_t* status;
 };
 
+// Epilogue store of one warp's 32-row slice: lane t holds row row0 + t, columns
+// [cbase, cbase + COLS) in v.  Chunks of 32 bytes per row (16 bf16 or 8 fp32 columns) go
+// through the warp's 1 KB staging buffer and leave as full 32-byte sectors: lane pairs
+// store the two halves of one row, 16 rows per instruction.  (Storing each lane's own
+// row directly wrote half sectors and cost a fifth of the GeMM's time.)  fp32 output
+// goes to f32_out (a split-K partial or C); bf16 output to C.
+template <int COLS>
+__device__ __forceinline__ void store_rows(const Params& p, const float (&v)[COLS], uint8_t* buf, int lane,
+                                           int64_t row0, int64_t cbase, float alpha, float* f32_out) {
+  uint4* stage_buf = reinterpret_cast<uint4*>(buf);
+  const int half = lane & 1;
+  if (p.c_dtype == METIS_OUT_F32) {
+#pragma unroll
+    for (int c = 0; c < COLS; c += 8) {
+      float o[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = v[c + i] * alpha * (p.col_scale ? p.col_scale[cbase + c + i] : 1.0f);
+      stage_buf[lane * 2] = make_uint4(__float_as_uint(o[0]), __float_as_uint(o[1]), __float_as_uint(o[2]),
+                                       __float_as_uint(o[3]));
+      stage_buf[lane * 2 + 1] = make_uint4(__float_as_uint(o[4]), __float_as_uint(o[5]), __float_as_uint(o[6]),
+                                           __float_as_uint(o[7]));
+      __syncwarp();
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int r = (lane >> 1) + 16 * t;
+        float* dst = f32_out + (row0 + r) * p.ldc + cbase + c + half * 4;
+        *reinterpret_cast<uint4*>(dst) = stage_buf[r * 2 + half];
+      }
+      __syncwarp();
+    }
+  } else {
+    __nv_bfloat16* const out = reinterpret_cast<__nv_bfloat16*>(p.C);
+#pragma unroll
+    for (int c = 0; c < COLS; c += 16) {
+      uint32_t w[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float a = v[c + 2 * i] * alpha * (p.col_scale ? p.col_scale[cbase + c + 2 * i] : 1.0f);
+        const float b = v[c + 2 * i + 1] * alpha * (p.col_scale ? p.col_scale[cbase + c + 2 * i + 1] : 1.0f);
+        const __nv_bfloat162 pr = __floats2bfloat162_rn(a, b);
+        w[i] = *reinterpret_cast<const uint32_t*>(&pr);
+      }
+      stage_buf[lane * 2] = make_uint4(w[0], w[1], w[2], w[3]);
+      stage_buf[lane * 2 + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+      __syncwarp();
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int r = (lane >> 1) + 16 * t;
+        __nv_bfloat16* dst = out + (row0 + r) * p.ldc + cbase + c + half * 8;
+        *reinterpret_cast<uint4*>(dst) = stage_buf[r * 2 + half];
+      }
+      __syncwarp();
+    }
+  }
+}
+
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
@@ -338,60 +394,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&tmem_empty[ab]);
-      if (active) {
-        // Each lane holds one row of the warp's 32-row slice.  Chunks of 32 bytes per row
-        // (16 bf16 or 8 fp32 columns) go through the warp's staging buffer and leave as
-        // full 32-byte sectors: lane pairs store the two halves of one row, 16 rows per
-        // instruction (storing each lane's own row directly wrote half sectors and cost a
-        // fifth of the kernel's time).
-        uint4* stage_buf = reinterpret_cast<uint4*>(epi_smem + (warp - 2) * 1024);
-        const int64_t row0 = (int64_t)mb * 128 + q * 32;
-        const int64_t cbase = (int64_t)nb * BN + col0;
-        const int half = lane & 1;
-        if (p.c_dtype == METIS_OUT_F32) {
-#pragma unroll
-          for (int c = 0; c < kColsPerWarp; c += 8) {
-            float o[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) o[i] = v[c + i] * alpha * (p.col_scale ? p.col_scale[cbase + c + i] : 1.0f);
-            stage_buf[lane * 2] = make_uint4(__float_as_uint(o[0]), __float_as_uint(o[1]), __float_as_uint(o[2]),
-                                             __float_as_uint(o[3]));
-            stage_buf[lane * 2 + 1] = make_uint4(__float_as_uint(o[4]), __float_as_uint(o[5]),
-                                                 __float_as_uint(o[6]), __float_as_uint(o[7]));
-            __syncwarp();
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-              const int r = (lane >> 1) + 16 * t;
-              float* dst = split_out + (row0 + r) * p.ldc + cbase + c + half * 4;
-              *reinterpret_cast<uint4*>(dst) = stage_buf[r * 2 + half];
-            }
-            __syncwarp();
-          }
-        } else {
-          __nv_bfloat16* const out = reinterpret_cast<__nv_bfloat16*>(p.C);
-#pragma unroll
-          for (int c = 0; c < kColsPerWarp; c += 16) {
-            uint32_t w[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float a = v[c + 2 * i] * alpha * (p.col_scale ? p.col_scale[cbase + c + 2 * i] : 1.0f);
-              const float b = v[c + 2 * i + 1] * alpha * (p.col_scale ? p.col_scale[cbase + c + 2 * i + 1] : 1.0f);
-              const __nv_bfloat162 pr = __floats2bfloat162_rn(a, b);
-              w[i] = *reinterpret_cast<const uint32_t*>(&pr);
-            }
-            stage_buf[lane * 2] = make_uint4(w[0], w[1], w[2], w[3]);
-            stage_buf[lane * 2 + 1] = make_uint4(w[4], w[5], w[6], w[7]);
-            __syncwarp();
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-              const int r = (lane >> 1) + 16 * t;
-              __nv_bfloat16* dst = out + (row0 + r) * p.ldc + cbase + c + half * 8;
-              *reinterpret_cast<uint4*>(dst) = stage_buf[r * 2 + half];
-            }
-            __syncwarp();
-          }
-        }
-      }
+      if (active)
+        store_rows(p, v, epi_smem + (warp - 2) * 1024, lane, (int64_t)mb * 128 + q * 32, (int64_t)nb * BN + col0,
+                   alpha, split_out);
     }
   }
 
@@ -400,6 +405,354 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ CTA-pair kernel
+// The large GeMMs (both output dimensions multiples of 256, no split-K) run on CTA
+// pairs: a cluster of two CTAs computes a 256 x 256 output tile with cta_group::2 MMAs
+// (M = 256, N = 256).  Each CTA loads its own 128 rows of A, its 128 rows of B, the
+// scales of its A rows and of all 256 B rows: 38 KB per K stage for the MMA work that
+// takes 54 KB in a single-CTA 128 x 256 tile, and each MMA reads half of B from the
+// other SM's shared memory.
+//   both CTAs, warp 0: TMA loads of the CTA's tiles; the bytes are counted on the even
+//     CTA's stage barrier, so the even CTA learns that the whole pair stage landed
+//   even CTA, warp 1: the pair-wide MMAs; commits free the stage in both CTAs and hand
+//     each CTA its accumulator
+//   even CTA, warps 10-11: pair-wide block-scale copies (each CTA's scales into its own
+//     tensor memory), committed to the stage's sf_ready barrier
+//   both CTAs, warps 2-9: epilogue of the CTA's own 128 rows; the drain is reported to
+//     the even CTA's accumulator-empty barrier
+// Waits are bounded as in the single-CTA kernel, and both CTAs always reach the final
+// cluster barrier before the tensor memory is released.
+struct PairCfg {
+  static constexpr int BN = 256;
+  static constexpr int A_BYTES = 128 * 128;        // this CTA's 128 rows, 256 K elements
+  static constexpr int B_BYTES = 128 * 128;        // this CTA's 128 of the 256 B rows
+  static constexpr int SFA_BYTES = 4 * 512;        // scales of this CTA's A rows
+  static constexpr int SFB_BYTES = 2 * 4 * 512;    // scales of all 256 B rows
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int SF_STAGE_BYTES = SFA_BYTES + SFB_BYTES;
+  static constexpr int STAGES = 5;
+  static constexpr int SFB_COLS_PER_K = 8;
+  static constexpr int SF_SET_COLS = 16 + 4 * SFB_COLS_PER_K;
+  static constexpr int ACC_COLS = 256;
+  static constexpr int USED_COLS = ACC_COLS + STAGES * SF_SET_COLS;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr uint32_t PAIR_TX = 2 * (STAGE_BYTES + SF_STAGE_BYTES);  // an NVFP4 stage of the pair
+  static constexpr uint32_t PAIR_FOLD_TX = 2 * STAGE_BYTES;               // a bf16 fold stage of the pair
+  // output staging: per epilogue warp one 128-byte-swizzled box of 32 rows x 128 bytes
+  static constexpr int EPI_WARP_BYTES = 4096;
+  static constexpr size_t SMEM =
+      (size_t)STAGES * (STAGE_BYTES + SF_STAGE_BYTES) + kEpiWarps * EPI_WARP_BYTES + 1024 + 256;
+  static_assert(USED_COLS <= TMEM_COLS, "tensor memory budget");
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                           const __grid_constant__ CUtensorMap mapFa, const __grid_constant__ CUtensorMap mapFb,
+                           const __grid_constant__ CUtensorMap mapSa, const __grid_constant__ CUtensorMap mapSb,
+                           const __grid_constant__ CUtensorMap mapC, const Params p) {
+  using C = PairCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* tiles = smem;
+  uint8_t* sf = smem + C::STAGES * C::STAGE_BYTES;
+  uint8_t* epi = sf + C::STAGES * C::SF_STAGE_BYTES;   // 1024-byte aligned
+  uint64_t* bars = reinterpret_cast<uint64_t*>(epi + kEpiWarps * C::EPI_WARP_BYTES);
+  uint64_t* full = bars;                          // (even CTA) the pair's stage landed
+  uint64_t* empty = bars + C::STAGES;             // the pair's MMAs are done with the stage
+  uint64_t* sf_ready = bars + 2 * C::STAGES;      // (even CTA) the stage's scales are in tensor memory
+  uint64_t* tmem_full = bars + 3 * C::STAGES;     // this CTA's accumulator is complete
+  uint64_t* tmem_empty = tmem_full + 1;           // (even CTA) both CTAs' epilogues drained
+  uint64_t* drain = tmem_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_full + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = tc::cluster_rank();
+  const bool even = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+      tc::mbar_init(&sf_ready[s], 2);
+    }
+    tc::mbar_init(tmem_full, 1);
+    tc::mbar_init(tmem_empty, 2 * kEpiWarps);
+    tc::mbar_init(drain, 1);
+    *abort_flag = 0;
+    tc::fence_barrier_init();
+    tc::prefetch_tensormap(&mapA);
+    tc::prefetch_tensormap(&mapB);
+    tc::prefetch_tensormap(&mapSa);
+    tc::prefetch_tensormap(&mapSb);
+    tc::prefetch_tensormap(&mapC);
+    if (p.fold_stages) {
+      tc::prefetch_tensormap(&mapFa);
+      tc::prefetch_tensormap(&mapFb);
+    }
+  }
+  if (warp == 1) {
+    tc::tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    tc::tmem_relinquish_pair();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::cluster_sync();   // both CTAs' barriers exist before any cross-CTA arrival
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int num_tiles = p.m_tiles * p.n_tiles;   // m_tiles counts 256-row blocks
+  const int total_stages = p.k_stages + p.fold_stages;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      const uint32_t full0 = tc::cluster_addr(&full[0], 0);   // the even CTA's stage barriers
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = pair; tile < num_tiles && !*abort_flag; tile += npairs) {
+        const int mb = tile % p.m_tiles;
+        const int nb = tile / p.m_tiles;
+        const int arow = mb * 256 + (int)rank * 128;
+        const int brow = nb * C::BN + (int)rank * 128;
+        for (int kk = 0; kk < total_stages; ++kk) {
+          if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+            *abort_flag = 1;
+            raise_status(p.status, METIS_DEV_TIMEOUT);
+            break;
+          }
+          uint8_t* sA = tiles + stage * C::STAGE_BYTES;
+          uint8_t* sB = sA + C::A_BYTES;
+          const uint32_t fb = full0 + 8u * (uint32_t)stage;
+          if (kk < p.k_stages) {
+            uint8_t* sSFA = sf + stage * C::SF_STAGE_BYTES;
+            uint8_t* sSFB = sSFA + C::SFA_BYTES;
+            if (even) tc::mbar_expect_tx(&full[stage], C::PAIR_TX);
+            tc::tma_load_2d_pair(sA, &mapA, fb, kk * 128, arow);
+            tc::tma_load_2d_pair(sB, &mapB, fb, kk * 128, brow);
+            // scale tiles: 512-byte atoms, 4 per stage and 128-row block; 8-byte elements
+            tc::tma_load_1d_pair(sSFA, &mapSa, fb, (int32_t)(((int64_t)(arow / 128) * p.kb_tiles + kk * 4) * 64));
+#pragma unroll
+            for (int a = 0; a < 2; ++a)
+              tc::tma_load_1d_pair(sSFB + a * 2048, &mapSb, fb,
+                                   (int32_t)(((int64_t)(nb * 2 + a) * p.kb_tiles + kk * 4) * 64));
+          } else {
+            const int f = kk - p.k_stages;
+            if (even) tc::mbar_expect_tx(&full[stage], C::PAIR_FOLD_TX);
+            tc::tma_load_2d_pair(sA, &mapFa, fb, f * 64, arow);
+            tc::tma_load_2d_pair(sB, &mapFb, fb, f * 64, brow);
+          }
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && even) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      const uint32_t id_fp4 = tc::idesc_nvf4(C::BN, 256);
+      const uint32_t id_bf16 = tc::idesc_bf16(C::BN, 256);
+      for (int tile = pair; tile < num_tiles && !*abort_flag; tile += npairs, ++it) {
+        if (!tc::mbar_wait(tmem_empty, ((uint32_t)it & 1u) ^ 1u, abort_flag)) {
+          *abort_flag = 1;
+          raise_status(p.status, METIS_DEV_TIMEOUT);
+          break;
+        }
+        tc::tc_fence_after();
+        for (int kk = 0; kk < total_stages; ++kk) {
+          if (!tc::mbar_wait(&full[stage], phase, abort_flag) ||
+              !tc::mbar_wait(&sf_ready[stage], phase, abort_flag)) {
+            *abort_flag = 1;
+            raise_status(p.status, METIS_DEV_TIMEOUT);
+            break;
+          }
+          tc::tc_fence_after();
+          const uint8_t* sA = tiles + stage * C::STAGE_BYTES;
+          const uint8_t* sB = sA + C::A_BYTES;
+          const uint64_t adesc = tc::sdesc_sw128(tc::smem_addr(sA));
+          const uint64_t bdesc = tc::sdesc_sw128(tc::smem_addr(sB));
+          if (kk < p.k_stages) {
+            const uint32_t t_sfa = tmem + C::ACC_COLS + stage * C::SF_SET_COLS;
+            const uint32_t t_sfb = t_sfa + 16;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              tc::mma_nvf4_pair(tmem, adesc + 2 * j, bdesc + 2 * j, id_fp4, t_sfa + 4 * j,
+                                t_sfb + C::SFB_COLS_PER_K * j, (kk || j) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              tc::mma_bf16_pair(tmem, adesc + 2 * j, bdesc + 2 * j, id_bf16, (kk || j) ? 1u : 0u);
+          }
+          tc::tc_commit_pair(&empty[stage], 0x3);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (*abort_flag) break;
+        tc::tc_commit_pair(tmem_full, 0x3);
+      }
+      // let every issued tensor-core operation finish before the memory is released
+      tc::tc_commit_pair(drain, 0x1);
+      tc::mbar_wait(drain, 0, nullptr);
+    }
+    __syncwarp();
+  } else if (warp >= 10) {
+    // ------------------------------------------------------------ scale copies (even CTA)
+    // Warp 10 copies SFA of k-steps 0-1 and the first 128-row atom of SFB, warp 11 SFA
+    // of k-steps 2-3 and the second atom: six pair-wide copies each per stage.
+    const int part = warp - 10;
+    if (lane == 0 && even) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = pair; tile < num_tiles && !*abort_flag; tile += npairs) {
+        for (int kk = 0; kk < total_stages; ++kk) {
+          if (!tc::mbar_wait(&full[stage], phase, abort_flag)) {
+            *abort_flag = 1;
+            raise_status(p.status, METIS_DEV_TIMEOUT);
+            break;
+          }
+          tc::tc_fence_after();
+          if (kk < p.k_stages) {
+            const uint8_t* sSFA = sf + stage * C::SF_STAGE_BYTES;
+            const uint8_t* sSFB = sSFA + C::SFA_BYTES;
+            const uint32_t t_sfa = tmem + C::ACC_COLS + stage * C::SF_SET_COLS;
+            const uint32_t t_sfb = t_sfa + 16;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              if ((j >> 1) == part)
+                tc::tc_copy_32x128b_x4_pair(t_sfa + 4 * j, tc::sdesc_scales(tc::smem_addr(sSFA + 512 * j)));
+              tc::tc_copy_32x128b_x4_pair(t_sfb + C::SFB_COLS_PER_K * j + 4 * part,
+                                          tc::sdesc_scales(tc::smem_addr(sSFB + 2048 * part + 512 * j)));
+            }
+          }
+          tc::tc_commit_pair(&sf_ready[stage], 0x1);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    // The accumulator is loaded into registers and released at once; the scaled tile
+    // goes through the warp's shared-memory boxes (128-byte swizzle, so the row-per-lane
+    // writes are conflict-free) and leaves by TMA stores, which the warp does not wait
+    // for until it reuses the boxes one tile later.
+    const int q = warp & 3;                 // tensor-memory lane quarter of this warp
+    const int h = (warp - 2) >> 2;          // column half
+    constexpr int kColsPerWarp = C::BN / 2;
+    const float alpha = (p.ga ? *p.ga : 1.0f) * (p.gb ? *p.gb : 1.0f) * p.alpha_extra;
+    const uint32_t empty_bar = tc::cluster_addr(tmem_empty, 0);
+    uint8_t* box = epi + (warp - 2) * C::EPI_WARP_BYTES;
+    const bool f32 = p.c_dtype == METIS_OUT_F32;
+    int it = 0;
+    for (int tile = pair; tile < num_tiles; tile += npairs, ++it) {
+      const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(tmem_full, (uint32_t)it & 1u, abort_flag));
+      if (!ok) {
+        if (lane == 0) {
+          *abort_flag = 1;
+          raise_status(p.status, METIS_DEV_TIMEOUT);
+        }
+        break;
+      }
+      tc::tc_fence_after();
+      const int mb = tile % p.m_tiles;
+      const int nb = tile / p.m_tiles;
+      const int col0 = h * kColsPerWarp;
+      float v[kColsPerWarp];
+#pragma unroll
+      for (int c = 0; c < kColsPerWarp; c += 32) {
+        float t[32];
+        tc::tmem_load_32cols(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(col0 + c), t);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[c + i] = t[i];
+      }
+      tc::tmem_load_wait();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive_cluster(empty_bar);
+
+      const int32_t y = mb * 256 + (int)rank * 128 + q * 32;
+      const int32_t x0 = nb * C::BN + col0;
+      // 16-byte chunk j of a 128-byte box row r sits at position j ^ (r mod 8)
+      const int swz = lane & 7;
+      // one box of 128 bytes per row at a time: 64 bf16 or 32 fp32 columns
+      constexpr int kBoxCols16 = 64, kBoxCols32 = 32;
+      if (!f32) {
+#pragma unroll
+        for (int bx = 0; bx < kColsPerWarp / kBoxCols16; ++bx) {
+          if (lane == 0) tc::bulk_wait_read_all();
+          __syncwarp();
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {        // 8 bf16 columns per 16-byte chunk
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int col = kBoxCols16 * bx + 8 * c + 2 * i;
+              const float a = v[col] * alpha * (p.col_scale ? p.col_scale[x0 + col] : 1.0f);
+              const float b = v[col + 1] * alpha * (p.col_scale ? p.col_scale[x0 + col + 1] : 1.0f);
+              const __nv_bfloat162 pr = __floats2bfloat162_rn(a, b);
+              w[i] = *reinterpret_cast<const uint32_t*>(&pr);
+            }
+            *reinterpret_cast<uint4*>(box + lane * 128 + ((c ^ swz) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          tc::fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) {
+            tc::tma_store_2d(&mapC, box, x0 + kBoxCols16 * bx, y);
+            tc::bulk_commit_group();
+          }
+        }
+      } else {
+#pragma unroll
+        for (int bx = 0; bx < kColsPerWarp / kBoxCols32; ++bx) {
+          if (lane == 0) tc::bulk_wait_read_all();
+          __syncwarp();
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {        // 4 fp32 columns per 16-byte chunk
+            const int col = kBoxCols32 * bx + 4 * c;
+            float o[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              o[i] = v[col + i] * alpha * (p.col_scale ? p.col_scale[x0 + col + i] : 1.0f);
+            *reinterpret_cast<uint4*>(box + lane * 128 + ((c ^ swz) << 4)) =
+                make_uint4(__float_as_uint(o[0]), __float_as_uint(o[1]), __float_as_uint(o[2]),
+                           __float_as_uint(o[3]));
+          }
+          tc::fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) {
+            tc::tma_store_2d(&mapC, box, x0 + kBoxCols32 * bx, y);
+            tc::bulk_commit_group();
+          }
+        }
+      }
+    }
+    if (lane == 0) tc::bulk_wait_all();   // stores complete before the boxes go away
+    __syncwarp();
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::cluster_sync();   // no cross-CTA access is outstanding past this point
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc_pair(tmem, C::TMEM_COLS);
   }
 }
 
@@ -413,6 +766,20 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, u
   if (!enc) return false;
   return enc(map, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 1-D map over a scale buffer viewed as 8-byte elements, 2 KB boxes (four 512-byte
+// scale atoms); the buffer start is 16-byte aligned and every box starts on a 2 KB multiple.
+bool make_map_1d_u64(CUtensorMap* map, const void* base, uint64_t bytes) {
+  const cuuint64_t dims[1] = {bytes / 8};
+  const cuuint64_t strides[1] = {bytes};   // unused for one dimension
+  const cuuint32_t box[1] = {256};
+  const cuuint32_t estr[1] = {1};
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 1, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -489,6 +856,74 @@ metis_status launch_bn(metis_ctx* ctx, const GemmArgs& a) {
                          q_cols >= 256);
 }
 
+// Both output dimensions multiples of 256, K a multiple of 256, one split.
+metis_status launch_pair(metis_ctx* ctx, const GemmArgs& a) {
+  using C = PairCfg;
+  const int64_t p_rows = a.A->outer;
+  const int64_t K = a.A->inner;
+  const int64_t q_cols = a.q_cols;
+  const int64_t kb_tiles = K / 64;
+  CUtensorMap mA, mB, mFa, mFb, mSa, mSb;
+  if (!make_map_2d(&mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.A->codes, K / 2, p_rows, K / 2, 128, 128) ||
+      !make_map_2d(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.B->codes, K / 2, a.B->outer, K / 2, 128, 128) ||
+      !make_map_1d_u64(&mSa, a.A->scales, (uint64_t)(p_rows / 128) * kb_tiles * 512) ||
+      !make_map_1d_u64(&mSb, a.B->scales, (uint64_t)((a.B->outer + 127) / 128) * kb_tiles * 512))
+    return fail(ctx, METIS_ERR_CUDA, "cuTensorMapEncodeTiled failed for the NVFP4 operands");
+  if (a.fold_k > 0) {
+    if (!make_map_2d(&mFa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.Fa, a.fold_k, p_rows, (uint64_t)a.fold_k * 2, 64,
+                     128) ||
+        !make_map_2d(&mFb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.Fb, a.fold_k, a.B->outer, (uint64_t)a.fold_k * 2,
+                     64, 128))
+      return fail(ctx, METIS_ERR_CUDA, "cuTensorMapEncodeTiled failed for the fold operands");
+  } else {
+    mFa = mA;
+    mFb = mB;
+  }
+  CUtensorMap mC;
+  const bool f32 = a.c_dtype == METIS_OUT_F32;
+  if (!make_map_2d(&mC, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.C, q_cols,
+                   p_rows, (uint64_t)a.ldc * (f32 ? 4 : 2), f32 ? 32 : 64, 32))
+    return fail(ctx, METIS_ERR_CUDA, "cuTensorMapEncodeTiled failed for the output");
+  Params prm{};
+  prm.sfa = a.A->scales;
+  prm.sfb = a.B->scales;
+  prm.kb_tiles = kb_tiles;
+  prm.ga = a.A->tensor_scale;
+  prm.gb = a.B->tensor_scale;
+  prm.alpha_extra = a.alpha_extra;
+  prm.col_scale = a.col_scale;
+  prm.C = a.C;
+  prm.ldc = a.ldc;
+  prm.c_dtype = a.c_dtype;
+  prm.m_tiles = (int)(p_rows / 256);
+  prm.n_tiles = (int)(q_cols / C::BN);
+  prm.k_stages = (int)(K / 256);
+  prm.fold_stages = a.fold_k / 64;
+  prm.k_splits = 1;
+  prm.split_stride = 0;
+  prm.status = ctx->status;
+  cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)C::SMEM);
+  if (e != cudaSuccess) return check_cuda(ctx, e, "cudaFuncSetAttribute(gemm pair)");
+  const int tiles = prm.m_tiles * prm.n_tiles;
+  const int grid = 2 * std::min(tiles, ctx->sm_count / 2);
+  const bool prof = ctx->profiling;
+  cudaEvent_t ev0 = nullptr, ev1 = nullptr;
+  if (prof) {
+    cudaEventCreate(&ev0);
+    cudaEventCreate(&ev1);
+    cudaEventRecord(ev0, ctx->stream);
+  }
+  gemm_nvfp4_pair_kernel<<<grid, kThreads, C::SMEM, ctx->stream>>>(mA, mB, mFa, mFb, mSa, mSb, mC, prm);
+  count_launch();
+  if (prof) {
+    cudaEventRecord(ev1, ctx->stream);
+    ctx->prof_events.emplace_back(ev0, ev1);
+    ctx->prof_flops.push_back(2.0 * (double)p_rows * (double)q_cols * (double)K);
+  }
+  return check_cuda(ctx, cudaGetLastError(), "gemm pair launch");
+}
+
 template <int BN>
 metis_status launch_bf16_bn(metis_ctx* ctx, const void* A, int64_t lda, int64_t rows, const void* B, int64_t ldb,
                             int64_t K, float* C, int64_t ldc, int splits) {
@@ -545,6 +980,12 @@ metis_status launch_gemm_bf16(metis_ctx* ctx, const void* A, int64_t lda, int64_
 }
 
 metis_status launch_gemm_nvfp4(metis_ctx* ctx, const GemmArgs& a) {
+  // CTA pairs whenever both output dimensions are multiples of 256 (the layer's GeMMs)
+  // (the output leaves by TMA stores: 16-byte aligned base and row pitch)
+  const int64_t out_bytes = a.c_dtype == METIS_OUT_F32 ? 4 : 2;
+  if (a.q_cols % 256 == 0 && a.A->outer % 256 == 0 && a.k_splits <= 1 && ctx->sm_count >= 2 &&
+      reinterpret_cast<uintptr_t>(a.C) % 16 == 0 && (a.ldc * out_bytes) % 16 == 0)
+    return launch_pair(ctx, a);
   if (a.q_cols % 256 == 0) return launch_bn<256>(ctx, a);
   if (a.q_cols == 128) return launch_bn<128>(ctx, a);
   if (a.q_cols == 64) return launch_bn<64>(ctx, a);

@@ -84,6 +84,22 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
+// 2-D TMA tile store shared -> global in the calling thread's bulk group.  The
+// shared-memory source must be made visible to the async proxy first (fence_proxy_async).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_addr(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until this thread's bulk groups have finished reading their shared-memory sources.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until this thread's bulk groups have completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -159,6 +175,93 @@ __device__ __forceinline__ void tmem_load_32cols(uint32_t taddr, float (&v)[32])
 
 __device__ __forceinline__ void tmem_load_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// ---- CTA pairs (a cluster of two CTAs, tcgen05 cta_group::2) ---------------
+// A kernel that uses these issues every tcgen05 instruction with cta_group::2; the
+// even CTA of the pair issues the MMAs, scale copies and commits for both.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Barrier over every thread of both CTAs (release / acquire at cluster scope).
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// shared::cluster address of the object at `p`'s offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+  return r;
+}
+// Arrive (release, cluster scope) on the mbarrier at shared::cluster address `bar`.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// Tile loads into this CTA's shared memory whose bytes are counted on the mbarrier at
+// shared::cluster address `bar`, which may belong to the other CTA of the pair; every
+// CTA loads only its own tiles from this GPU's memory.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar, int32_t x,
+                                                 int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4}], [%2];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_1d_pair(void* dst, const CUtensorMap* map, uint32_t bar, int32_t x) {
+  asm volatile(
+      "cp.async.bulk.tensor.1d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3}], "
+      "[%2];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x)
+      : "memory");
+}
+// Tensor memory of both CTAs, same columns (one warp of each CTA, same warp index).
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(slot)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// Arrive on `bar` (same offset) in each CTA of `mask` once this thread's previously
+// issued pair-wide tcgen05 operations finish.
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_addr(bar)),
+      "h"(mask)
+      : "memory");
+}
+// Pair-wide block-scale copy: each CTA's 32 x 16-byte tile at this shared-memory
+// offset into its own tensor memory, replicated into the four lane quarters.
+__device__ __forceinline__ void tc_copy_32x128b_x4_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+// Pair-wide MMAs, M = 256: rows 0-127 of A from the even CTA's shared memory, rows
+// 128-255 from the odd CTA's (same offset); B's N rows split the same way; each CTA's
+// tensor memory holds the accumulator of its own 128 rows.
+__device__ __forceinline__ void mma_nvf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // ---- descriptors -----------------------------------------------------------
 // Shared-memory matrix descriptor, K-major operand in the 128-byte swizzle
 // layout: rows of 128 bytes, groups of 8 rows 1024 bytes apart.
@@ -183,25 +286,25 @@ __device__ __forceinline__ uint64_t sdesc_scales(uint32_t saddr) {
 }
 
 // Instruction descriptor: block-scaled E2M1 x E2M1, UE4M3 scales, fp32 accumulate,
-// both operands K-major, M = 128.
-__host__ __device__ __forceinline__ uint32_t idesc_nvf4(uint32_t n) {
+// both operands K-major; M = 128 (one CTA) or 256 (a CTA pair).
+__host__ __device__ __forceinline__ uint32_t idesc_nvf4(uint32_t n, uint32_t m = 128) {
   uint32_t d = 0;
   d |= 1u << 7;               // A format: E2M1
   d |= 1u << 10;              // B format: E2M1
   d |= (n >> 3) << 17;        // N / 8
   d |= 0u << 23;              // scale format: UE4M3
-  d |= (128u >> 4) << 24;     // M / 16
+  d |= (m >> 4) << 24;        // M / 16
   return d;
 }
 
-// Instruction descriptor: bf16 x bf16 -> fp32, both K-major, M = 128.
-__host__ __device__ __forceinline__ uint32_t idesc_bf16(uint32_t n) {
+// Instruction descriptor: bf16 x bf16 -> fp32, both K-major; M = 128 or 256.
+__host__ __device__ __forceinline__ uint32_t idesc_bf16(uint32_t n, uint32_t m = 128) {
   uint32_t d = 0;
   d |= 1u << 4;               // D format: fp32
   d |= 1u << 7;               // A format: bf16
   d |= 1u << 10;              // B format: bf16
   d |= (n >> 3) << 17;
-  d |= (128u >> 4) << 24;
+  d |= (m >> 4) << 24;
   return d;
 }
 

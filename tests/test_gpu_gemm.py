@@ -71,6 +71,17 @@ def test_fp4_gemm_many_tiles_per_cta(ctx, metis_lib):
     assert rel_fro(got, want) <= TIGHT
 
 
+def test_pair_tiles_fold_column_scale_bf16(ctx, metis_lib):
+    # CTA-pair path (both output dimensions multiples of 256): 4 x 9 pair tiles, a K loop
+    # that wraps the stage ring, three fold stages, per-column scale, bf16 output
+    got, want, absprod, terms = _run(ctx, 1024, 2304, 1536, fold_k=192, col_scale=True, out=torch.bfloat16,
+                                     seed=21, with_abs=True)
+    assert np.all(np.isfinite(got))
+    # bf16 rounding of each output plus fp32 accumulation
+    bound = np.abs(want) * 2.0 ** -8 + absprod * terms * 2.0 ** -23
+    assert np.all(np.abs(got - want) <= bound)
+
+
 @pytest.mark.parametrize("q", [16, 32, 64])
 def test_thin_gemm_with_column_scale(ctx, metis_lib, q):
     got, want = _run(ctx, 512, q, 1024, thin=True, col_scale=True, seed=q)
