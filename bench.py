@@ -43,11 +43,11 @@ from workloads import synth  # noqa: E402
 NVFP4_OVER_BF16 = 9.0 / 2.25      # nominal dense tensor-core throughput ratio
 DEFAULT_CONFIG = "llama3_8b_mlp_up"
 METRIC = "effective TFLOP/s of Metis W4A4G4 linear fwd+bwd; % of NVFP4 MMA peak"
-# DRAM bytes (read + write) of one launch of the fused GeMM at the forward shape
-# (8192 x 14336 x 4096, fold 256, bf16 out), from one ncu capture of this kernel version
-# (profile_case.py gemm --bf16; summarized in profiles/gemm_nvfp4_fused_llama3_8b_mlp_up.md).
+# DRAM bytes (read + write) of one launch of the fused GeMM (CTA-pair kernel) at the
+# forward shape (8192 x 14336 x 4096, fold 256, bf16 out), from one ncu capture of this
+# kernel version (profile_case.py gemm --bf16; the summary sits under profiles/).
 # Must be retaken whenever the kernel changes.
-GEMM_FWD_DRAM_BYTES = 73.269504e6 + 188.533248e6
+GEMM_FWD_DRAM_BYTES = 69.383424e6 + 192.398336e6
 
 
 def measured_peaks():
@@ -325,7 +325,7 @@ def run_ours(args, rank, world, device):
                    "pct_of_nvfp4_peak": round(100 * value / (world * peak), 2),
                    "nvfp4_peak_tflops": round(peak, 1),
                    "nvfp4_peak_basis": f"bf16_tflops_sustained x {NVFP4_OVER_BF16:.0f} ({kind})"},
-        "roofline": {"bound": "tensor", "kernel": "gemm_nvfp4_kernel<256> (fused FP4 GeMM + fold)",
+        "roofline": {"bound": "tensor", "kernel": "gemm_nvfp4_pair_kernel (fused FP4 GeMM + fold, CTA pairs)",
                      "achieved": None if achieved is None else round(achieved, 1), "peak": round(peak, 1),
                      "unit": "TFLOP/s", "frac": None if achieved is None else round(achieved / peak, 4),
                      "traffic": round(GEMM_FWD_DRAM_BYTES),
