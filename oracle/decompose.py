@@ -9,7 +9,7 @@ Source: "Metis: Training LLMs with FP4 Quantization" (papernotes.org notes):
 * 关键设计 3 -- the low-rank factors are reused across steps and the
   decomposition is refreshed every 8 steps (训练策略: rank 1.5%, refresh 8).
 
-Steps (the build's readings R7, R8, R10, R12 in the design doc):
+Steps (readings R7, R8, R10, R12 of the pages):
 
 refresh_basis (every R steps):
   1. sample l_k distinct rows: each row i gets the Philox word (i & 3) of

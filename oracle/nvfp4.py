@@ -30,9 +30,9 @@ chance of rounding up is floor(p * 2^16) / 2^16: unbiased to within 2^-16 of a
 grid step).  The sign of x is kept, so a negative value that rounds to zero
 gives -0.  Scales are always rounded to nearest.
 
-Readings that go beyond the pages are listed in the design doc: the per-tensor
-decode scale g (1.0 for residuals unless the caller sets one), the reciprocal
-multiply in step 5-6, and the SR random-field layout.
+Readings that go beyond the pages: the per-tensor decode scale g (1.0 for
+residuals unless the caller sets one or asks for ``auto_tensor_scale``), the
+reciprocal multiply in step 5-6, and the SR random-field layout.
 
 Pins (tests/test_oracle_nvfp4.py): round trips of values already on the
 grid, the scale rule against hand-computed blocks, dequantization error
@@ -50,6 +50,33 @@ BLOCK = 16
 
 class NonFiniteInput(ValueError):
     pass
+
+
+E2M1_MAX = 6.0
+E4M3_MAX = 448.0
+
+
+def auto_tensor_scale(M):
+    """The decode tensor scale g chosen from the data (reading R1b): the smallest
+    power of two g with 2 * amax <= 6 * 448 * g, amax = max |M| over the finite
+    entries (so the largest block of M, or of a residual of M up to twice its size,
+    gets an E4M3 block scale of at most 448); 1.0 when M has no nonzero finite entry;
+    the exponent is kept within the normal fp32 range [-126, 127].
+
+    Written as the definition: start from a power of two at or above the bound and
+    step down while the next smaller one still satisfies it."""
+    A = np.abs(np.asarray(M, dtype=np.float64))
+    A = A[np.isfinite(A)]
+    amax = float(A.max()) if A.size else 0.0
+    if amax == 0.0:
+        return 1.0
+    bound = 2.0 * amax / (E2M1_MAX * E4M3_MAX)
+    e = int(np.ceil(np.log2(bound))) + 1
+    while e > -126 and bound <= 2.0 ** (e - 1):
+        e -= 1
+    while bound > 2.0 ** e:
+        e += 1
+    return float(2.0 ** min(max(e, -126), 127))
 
 
 def _scale_codes(amax, g):

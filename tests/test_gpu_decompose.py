@@ -1,6 +1,6 @@
 """GPU randomized decomposition vs the oracle.
 
-Contract (the benchmark spec): identical sampled rows, the same Gaussian test matrix
+Contract: identical sampled rows, the same Gaussian test matrix
 (within 1 fp32 ulp: both sides evaluate Box-Muller in fp64), and subspace
 cosines >= 0.999 for the recovered basis and factors.  Factor quantization is
 bit-exact given the GPU's own fp32 factors.

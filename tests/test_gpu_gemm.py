@@ -2,7 +2,7 @@
 
 The oracle multiplies the dequantized operands in fp64 (FP4 x FP4 products are
 exact); the GPU accumulates in fp32 in tensor memory.  Contract: relative
-Frobenius error <= 2e-3 (the benchmark spec); the expected error is fp32 accumulation
+Frobenius error <= 2e-3 (the parity contract); the expected error is fp32 accumulation
 only, so a much tighter internal bound (1e-4) is checked as well.
 """
 

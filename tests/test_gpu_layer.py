@@ -1,6 +1,6 @@
 """End-to-end Metis linear layer (fwd, dX, dW) on the GPU vs the oracle.
 
-Parity (the benchmark spec): GeMM outputs within relative Frobenius error 2e-3 of the
+Parity contract: GeMM outputs within relative Frobenius error 2e-3 of the
 oracle fed the GPU's own codes, scales and factor copies.  End to end from raw
 bf16 inputs the quantization codes may differ at rounding boundaries, so the
 check there is statistical: GPU and oracle errors against the exact product

@@ -1,6 +1,6 @@
 """GPU NVFP4 quantizer vs the oracle: codes and scales bit-exact on identical fp32 input.
 
-Contract (the benchmark spec): NVFP4 codes and scales bit-exact given an identical fp32
+Contract: NVFP4 codes and scales bit-exact given an identical fp32
 residual input; both orientations; round-to-nearest and stochastic rounding.
 """
 

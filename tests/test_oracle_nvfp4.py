@@ -147,3 +147,40 @@ def test_sr_uses_the_orientation_stream():
     want, _ = nvfp4.quantize_blocks(np.ascontiguousarray(M.T), 1.0, "sr", f)
     got, _ = nvfp4.quantize_oriented(M, "col", rounding="sr", seed=9, operand_id=2, step=4)
     assert np.array_equal(want, got)
+
+
+def test_auto_tensor_scale_closed_forms():
+    # 6 * 448 = 2688: the bound 2 * amax <= 2688 * g is met with equality at amax = 1344 g
+    assert nvfp4.auto_tensor_scale(np.array([[1344.0]])) == 1.0
+    assert nvfp4.auto_tensor_scale(np.array([[1344.5]])) == 2.0
+    assert nvfp4.auto_tensor_scale(np.array([[-2688.0, 3.0]])) == 2.0
+    assert nvfp4.auto_tensor_scale(np.array([[672.0]])) == 0.5
+    assert nvfp4.auto_tensor_scale(np.array([[672.5]])) == 1.0
+    assert nvfp4.auto_tensor_scale(np.zeros((4, 4))) == 1.0
+    assert nvfp4.auto_tensor_scale(np.array([[np.nan, np.inf, 0.0]])) == 1.0
+    # 1e-3: bound 7.44e-7 lies between 2^-21 and 2^-20
+    assert nvfp4.auto_tensor_scale(np.array([[1e-3]])) == 2.0 ** -20
+    # exponent kept in the normal range
+    assert nvfp4.auto_tensor_scale(np.array([[1e-41]])) == 2.0 ** -126
+
+
+def test_auto_tensor_scale_is_the_smallest_admissible_power():
+    rng = np.random.default_rng(5)
+    for amax in np.exp(rng.uniform(-60, 20, 500)):
+        g = nvfp4.auto_tensor_scale(np.array([[amax, -amax / 3]]))
+        assert np.log2(g) == np.round(np.log2(g))            # a power of two
+        assert 2 * amax <= 2688.0 * g                          # admissible
+        assert not 2 * amax <= 2688.0 * g / 2                  # and no smaller one is
+
+
+def test_auto_tensor_scale_keeps_small_gradients():
+    """Gradient-sized data (1e-7) underflows every E4M3 block scale at g = 1; with the
+    chosen g the quantization error is the usual NVFP4 level."""
+    rng = np.random.default_rng(6)
+    M = (rng.standard_normal((32, 64)) * 1e-7).astype(np.float32)
+    c1, s1 = nvfp4.quantize_blocks(M, 1.0)
+    assert np.all(nvfp4.dequantize_blocks(c1, s1, 1.0) == 0.0) or \
+        np.linalg.norm(nvfp4.dequantize_blocks(c1, s1, 1.0) - M) > 0.5 * np.linalg.norm(M)
+    g = nvfp4.auto_tensor_scale(M)
+    c, s = nvfp4.quantize_blocks(M, g)
+    assert np.linalg.norm(nvfp4.dequantize_blocks(c, s, g) - M) < 0.15 * np.linalg.norm(M)
