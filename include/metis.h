@@ -149,7 +149,11 @@ typedef struct {
   uint64_t seed;
   uint32_t operand_id;
   uint32_t step;
-  float tensor_scale;    /* decode-side tensor scale g of the residual (power of two, >0) */
+  float tensor_scale;    /* decode-side tensor scale g (power of two, > 0), or 0: chosen from the
+                            data as the smallest power of two with 2 * amax <= 6 * 448 * g, amax =
+                            max |x| over the finite entries of the input (1 for an all-zero input,
+                            exponent kept in [-126, 127]); costs one extra read of the input.  The
+                            chosen g is written to the outputs' tensor_scale words. */
 } metis_quant_params;
 
 /*

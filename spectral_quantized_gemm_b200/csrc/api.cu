@@ -89,8 +89,8 @@ metis_status check_dims(metis_ctx* ctx, int64_t rows, int64_t cols) {
 metis_status check_quant(metis_ctx* ctx, const metis_quant_params* q) {
   if (!q) return fail(ctx, METIS_ERR_ARG, "null quant params");
   if (q->rounding != 0 && q->rounding != 1) return fail(ctx, METIS_ERR_ARG, "rounding must be 0 (RN) or 1 (SR)");
-  if (!pow2_positive(q->tensor_scale))
-    return fail(ctx, METIS_ERR_ARG, "tensor_scale must be a positive power of two");
+  if (q->tensor_scale != 0.0f && !pow2_positive(q->tensor_scale))
+    return fail(ctx, METIS_ERR_ARG, "tensor_scale must be a positive power of two, or 0 to choose it from the data");
   return METIS_OK;
 }
 
@@ -200,7 +200,16 @@ metis_status metis_quantize_nvfp4_f32(metis_ctx* ctx, const float* R, int64_t ro
   if (!rowwise && !colwise) return fail(ctx, METIS_ERR_ARG, "no output orientation requested");
   if ((s = check_nvfp4(ctx, rowwise, rows, cols, "rowwise")) != METIS_OK) return s;
   if ((s = check_nvfp4(ctx, colwise, cols, rows, "colwise")) != METIS_OK) return s;
-  return check_cuda(ctx, launch_quantize_f32(R, rows, cols, ld, *q, rowwise, colwise, ctx->status, ctx->stream),
+  uint32_t* amax = nullptr;
+  if (q->tensor_scale == 0.0f) {
+    if ((s = ensure_workspace(ctx, 256)) != METIS_OK) return s;
+    amax = reinterpret_cast<uint32_t*>(ctx->ws);
+    if ((s = check_cuda(ctx, launch_amax(R, false, rows, cols, ld, amax, ctx->sm_count, ctx->stream),
+                        "amax launch")) != METIS_OK)
+      return s;
+  }
+  return check_cuda(ctx,
+                    launch_quantize_f32(R, rows, cols, ld, *q, amax, rowwise, colwise, ctx->status, ctx->stream),
                     "quantize launch");
 }
 
@@ -221,8 +230,15 @@ metis_status metis_residual_quantize_nvfp4(metis_ctx* ctx, const metis_matrix* M
   if (rowwise && colwise) return run_residual_quantize(ctx, M, f, q, rowwise, colwise);
   // one orientation only: fp32 residual in the workspace, then the quantizer
   const size_t bytes = (size_t)M->rows * M->cols * sizeof(float);
-  if ((s = ensure_workspace(ctx, bytes + 256)) != METIS_OK) return s;
+  if ((s = ensure_workspace(ctx, bytes + 512)) != METIS_OK) return s;
   float* R = reinterpret_cast<float*>(ctx->ws);
+  uint32_t* amax = nullptr;
+  if (q->tensor_scale == 0.0f) {   // g from the amax of M, as in the two-orientation path
+    amax = reinterpret_cast<uint32_t*>(ctx->ws + ((bytes + 255) & ~size_t(255)));
+    if ((s = check_cuda(ctx, launch_amax(M->data, true, M->rows, M->cols, M->ld, amax, ctx->sm_count, ctx->stream),
+                        "amax launch")) != METIS_OK)
+      return s;
+  }
   const bool lowrank = f && f->k > 0;
   s = check_cuda(ctx,
                  launch_residual_f32(M->data, M->rows, M->cols, M->ld, lowrank ? f->U : nullptr,
@@ -230,7 +246,9 @@ metis_status metis_residual_quantize_nvfp4(metis_ctx* ctx, const metis_matrix* M
                                      ctx->status, ctx->stream),
                  "residual launch");
   if (s != METIS_OK) return s;
-  return check_cuda(ctx, launch_quantize_f32(R, M->rows, M->cols, M->cols, *q, rowwise, colwise, ctx->status, ctx->stream),
+  return check_cuda(ctx,
+                    launch_quantize_f32(R, M->rows, M->cols, M->cols, *q, amax, rowwise, colwise, ctx->status,
+                                        ctx->stream),
                     "quantize launch");
 }
 

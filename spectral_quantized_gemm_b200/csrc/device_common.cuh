@@ -148,6 +148,20 @@ __device__ __forceinline__ uint2 encode_block16(const float (&x)[16], int roundi
   return r;
 }
 
+// Decode tensor scale chosen from the data: the smallest power of two g with
+// 2 * amax <= 6 * 448 * g, i.e. amax <= 1344 * g (amax = max |x| over the finite
+// entries, given as fp32 bits); 1 for amax = 0; exponent clamped to [-126, 127].
+// With amax = 1.m * 2^(E - 127) and 1344 = 1.3125 * 2^10: g = 2^(E - 137) when
+// 1.m <= 1.3125 (mantissa field <= 0x280000), else 2^(E - 136).
+__device__ __forceinline__ float auto_tensor_scale(uint32_t amax_bits) {
+  if (amax_bits == 0) return 1.0f;
+  const int E = (int)(amax_bits >> 23);
+  if (E == 0) return __uint_as_float(1u << 23);                  // subnormal amax: 2^-126
+  int e = ((amax_bits & 0x7FFFFFu) <= 0x280000u) ? E - 137 : E - 136;
+  e = e < -126 ? -126 : (e > 127 ? 127 : e);
+  return __uint_as_float((uint32_t)(e + 127) << 23);
+}
+
 // Tensor scale of a factor: g = pow2_ceil(max|F| / (6 * 448)), so that every block scale
 // fits E4M3 and dequantized factors stay exact in bf16.
 // Smallest power of two >= t (t >= 0 finite); 1 for t == 0.

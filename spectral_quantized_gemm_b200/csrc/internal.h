@@ -54,8 +54,14 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
 EncodeTiledFn encode_tiled();
 
 // ---- quantize.cu ----
+// Decode tensor scale chosen from the data (metis_quant_params.tensor_scale == 0):
+// launch_amax writes max |x| over the finite entries of M (bf16 or fp32, row-major) as
+// fp32 bits to *amax_bits; the quantizers then take g = auto_tensor_scale(*amax_bits).
+cudaError_t launch_amax(const void* M, bool bf16, int64_t rows, int64_t cols, int64_t ld, uint32_t* amax_bits,
+                        int sm_count, cudaStream_t st);
+// amax_bits: nullptr to use q.tensor_scale, else the word launch_amax wrote.
 cudaError_t launch_quantize_f32(const float* R, int64_t rows, int64_t cols, int64_t ld,
-                                const metis_quant_params& q, const metis_nvfp4* rowwise,
+                                const metis_quant_params& q, const uint32_t* amax_bits, const metis_nvfp4* rowwise,
                                 const metis_nvfp4* colwise, uint32_t* status, cudaStream_t st);
 cudaError_t launch_residual_f32(const void* M_bf16, int64_t rows, int64_t cols, int64_t ld, const float* U,
                                 const float* S, const float* V, int32_t k, float* out, uint32_t* status,
@@ -66,9 +72,12 @@ metis_status run_residual_quantize(metis_ctx* ctx, const metis_matrix* M, const 
                                    const metis_quant_params* q, const metis_nvfp4* row, const metis_nvfp4* col);
 
 // ---- noalloc.cu ----
-// Limits of the allocation-free residual quantizer's fixed scratch.
+// Limits of the allocation-free residual quantizer's fixed scratch: (rows + cols) x 64
+// floats of padded factors, then 64 floats of which the first word holds the amax of a
+// call that asks for a tensor scale chosen from the data.
 constexpr int64_t kNoAllocMaxRowsPlusCols = 24576;
 constexpr int kNoAllocWidth = 64;
+constexpr int64_t kNoAllocAmaxOffset = kNoAllocMaxRowsPlusCols * kNoAllocWidth;
 float* noalloc_scratch(metis_ctx* ctx, metis_status* st);
 metis_status run_residual_quantize_into(metis_ctx* ctx, const metis_matrix* M, const metis_factors* f,
                                         const metis_quant_params* q, const metis_nvfp4* row, const metis_nvfp4* col,

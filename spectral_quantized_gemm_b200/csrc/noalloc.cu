@@ -14,8 +14,9 @@
 
 #include "internal.h"
 
-// (rows + cols) * 64 floats: 6 MiB on every device that loads the library.
-static __device__ __align__(256) float g_noalloc_scratch[metis::kNoAllocMaxRowsPlusCols * metis::kNoAllocWidth];
+// (rows + cols) * 64 floats (6 MiB) and a 256-byte tail for the amax word, on every
+// device that loads the library.
+static __device__ __align__(256) float g_noalloc_scratch[metis::kNoAllocAmaxOffset + 64];
 
 namespace metis {
 namespace {

@@ -19,11 +19,12 @@ namespace {
 
 // One thread per 16-element block of the row-wise view (blocks along columns).
 __global__ void quantize_rowwise_f32_kernel(const float* __restrict__ R, int64_t rows, int64_t cols, int64_t ld,
-                                            float g, int rounding, uint64_t seed, uint32_t tag, uint32_t step,
+                                            float g_in, const uint32_t* amax_bits, int rounding, uint64_t seed, uint32_t tag, uint32_t step,
                                             uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                                             float* tensor_scale, uint32_t* status) {
   const int64_t nblk_row = cols / 16;
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const float g = amax_bits ? auto_tensor_scale(*amax_bits) : g_in;
   if (idx == 0 && tensor_scale) *tensor_scale = g;
   if (idx >= rows * nblk_row) return;
   const int64_t o = idx / nblk_row;
@@ -60,10 +61,11 @@ __global__ void quantize_rowwise_f32_kernel(const float* __restrict__ R, int64_t
 // One thread per 16-row block of one column (column-wise view, blocks along rows).
 // Consecutive threads take consecutive columns so the loads coalesce.
 __global__ void quantize_colwise_f32_kernel(const float* __restrict__ R, int64_t rows, int64_t cols, int64_t ld,
-                                            float g, int rounding, uint64_t seed, uint32_t tag, uint32_t step,
+                                            float g_in, const uint32_t* amax_bits, int rounding, uint64_t seed, uint32_t tag, uint32_t step,
                                             uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                                             float* tensor_scale, uint32_t* status) {
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const float g = amax_bits ? auto_tensor_scale(*amax_bits) : g_in;
   if (idx == 0 && tensor_scale) *tensor_scale = g;
   const int64_t nblk = rows / 16;
   if (idx >= nblk * cols) return;
@@ -134,22 +136,88 @@ __global__ void residual_f32_kernel(const __nv_bfloat16* __restrict__ M, int64_t
   }
 }
 
+// Maximum |x| over the finite entries, as fp32 bits (non-negative floats order like
+// their bit patterns), one atomicMax per warp.  A warp walks whole rows in 16-byte
+// vectors: 8 bf16 or 4 fp32 elements.
+__global__ void __launch_bounds__(256) amax_bf16_kernel(const __nv_bfloat16* __restrict__ M, int64_t rows,
+                                                        int64_t cols, int64_t ld, uint32_t* amax_bits) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int64_t cv = cols / 8;
+  uint32_t best = 0;
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    const uint4* row = reinterpret_cast<const uint4*>(M + r * ld);
+    for (int64_t c = lane; c < cv; c += 32) {
+      const uint4 v = row[c];
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t a = (w[i] >> (16 * h)) & 0x7FFFu;
+          if ((a & 0x7F80u) != 0x7F80u) best = max(best, a << 16);
+        }
+      }
+    }
+  }
+  best = __reduce_max_sync(0xffffffffu, best);
+  if (lane == 0 && best) atomicMax(amax_bits, best);
+}
+
+__global__ void __launch_bounds__(256) amax_f32_kernel(const float* __restrict__ R, int64_t rows, int64_t cols,
+                                                       int64_t ld, uint32_t* amax_bits) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int64_t cv = cols / 4;
+  uint32_t best = 0;
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    const uint4* row = reinterpret_cast<const uint4*>(R + r * ld);
+    for (int64_t c = lane; c < cv; c += 32) {
+      const uint4 v = row[c];
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t a = w[i] & 0x7FFFFFFFu;
+        if ((a & 0x7F800000u) != 0x7F800000u) best = max(best, a);
+      }
+    }
+  }
+  best = __reduce_max_sync(0xffffffffu, best);
+  if (lane == 0 && best) atomicMax(amax_bits, best);
+}
+
 }  // namespace
 
+cudaError_t launch_amax(const void* M, bool bf16, int64_t rows, int64_t cols, int64_t ld, uint32_t* amax_bits,
+                        int sm_count, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(amax_bits, 0, sizeof(uint32_t), st);
+  if (e != cudaSuccess) return e;
+  const int64_t want = (rows + 7) / 8;   // 8 warps per block, one row per warp per pass
+  const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(want, 4 * (int64_t)sm_count));
+  if (bf16)
+    amax_bf16_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(M), rows, cols, ld, amax_bits);
+  else
+    amax_f32_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float*>(M), rows, cols, ld, amax_bits);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quantize_f32(const float* R, int64_t rows, int64_t cols, int64_t ld,
-                                const metis_quant_params& q, const metis_nvfp4* rowwise,
+                                const metis_quant_params& q, const uint32_t* amax_bits, const metis_nvfp4* rowwise,
                                 const metis_nvfp4* colwise, uint32_t* status, cudaStream_t st) {
   const int threads = 256;
   if (rowwise) {
     const int64_t n = rows * (cols / 16);
     quantize_rowwise_f32_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, st>>>(
-        R, rows, cols, ld, q.tensor_scale, q.rounding, q.seed, stream_tag(q.operand_id, kPurposeSR, kSrRowwise),
+        R, rows, cols, ld, q.tensor_scale, amax_bits, q.rounding, q.seed,
+        stream_tag(q.operand_id, kPurposeSR, kSrRowwise),
         q.step, rowwise->codes, rowwise->scales, rowwise->tensor_scale, status); count_launch();
   }
   if (colwise) {
     const int64_t n = (rows / 16) * cols;
     quantize_colwise_f32_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, st>>>(
-        R, rows, cols, ld, q.tensor_scale, q.rounding, q.seed, stream_tag(q.operand_id, kPurposeSR, kSrColwise),
+        R, rows, cols, ld, q.tensor_scale, amax_bits, q.rounding, q.seed,
+        stream_tag(q.operand_id, kPurposeSR, kSrColwise),
         q.step, colwise->codes, colwise->scales, colwise->tensor_scale, status); count_launch();
   }
   return cudaGetLastError();

@@ -58,6 +58,7 @@ struct RqParams {
   uint8_t* col_scales;
   float* row_g;
   float* col_g;
+  const uint32_t* amax_bits;   // non-null: g chosen from the data (auto_tensor_scale)
   uint32_t* status;
 };
 
@@ -150,8 +151,9 @@ __global__ void __launch_bounds__(kRqThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* rcp_table = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);   // 128 entries
 
+  const float g = p.amax_bits ? auto_tensor_scale(*p.amax_bits) : p.g;
   for (int c = threadIdx.x; c < 128; c += blockDim.x)
-    rcp_table[c] = c ? __frcp_rn(__fmul_rn(e4m3_value((uint32_t)c), p.g)) : 0.0f;
+    rcp_table[c] = c ? __frcp_rn(__fmul_rn(e4m3_value((uint32_t)c), g)) : 0.0f;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -174,8 +176,8 @@ __global__ void __launch_bounds__(kRqThreads, 1)
     *abort_flag = 0;
     tc::fence_barrier_init();
     if (blockIdx.x == 0) {
-      *p.row_g = p.g;
-      *p.col_g = p.g;
+      *p.row_g = g;
+      *p.col_g = g;
     }
   }
   if (warp == 1) {
@@ -330,7 +332,7 @@ __global__ void __launch_bounds__(kRqThreads, 1)
           }
           finite &= abits < 0x7F800000u;
           uint32_t code;
-          const uint2 pk = quantize16(x, __uint_as_float(abits), p.g, rcp_table, p.rounding, p.seed, p.tag_row,
+          const uint2 pk = quantize16(x, __uint_as_float(abits), g, rcp_table, p.rounding, p.seed, p.tag_row,
                                       p.step, (uint64_t)grow * (uint64_t)p.cols + (uint64_t)(gcol + blk * 16), code);
           sc |= code << (8 * blk);
           o[2 * blk] = pk.x;
@@ -361,7 +363,7 @@ __global__ void __launch_bounds__(kRqThreads, 1)
             amax = fmaxf(amax, fabsf(x[i]));
           }
           uint32_t code;
-          const uint2 pk = quantize16(x, amax, p.g, rcp_table, p.rounding, p.seed, p.tag_col, p.step,
+          const uint2 pk = quantize16(x, amax, g, rcp_table, p.rounding, p.seed, p.tag_col, p.step,
                                       (uint64_t)gcolj * (uint64_t)p.rows + (uint64_t)(grow0 + blk * 16), code);
           sc |= code << (8 * blk);
           o[2 * blk] = pk.x;
@@ -418,7 +420,8 @@ bool map2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_
 
 template <int KK>
 metis_status launch_kk(metis_ctx* ctx, const metis_matrix* M, const float* US, const float* Vp,
-                       const metis_quant_params* q, const metis_nvfp4* row, const metis_nvfp4* col) {
+                       const metis_quant_params* q, const uint32_t* amax_bits, const metis_nvfp4* row,
+                       const metis_nvfp4* col) {
   using C = RqCfg<KK>;
   CUtensorMap mM, mU, mV;
   if (!map2d(&mM, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, M->data, M->cols, M->rows, (uint64_t)M->ld * 2, 64, 128) ||
@@ -442,6 +445,7 @@ metis_status launch_kk(metis_ctx* ctx, const metis_matrix* M, const float* US, c
   prm.col_scales = col->scales;
   prm.row_g = row->tensor_scale;
   prm.col_g = col->tensor_scale;
+  prm.amax_bits = amax_bits;
   prm.status = ctx->status;
   auto kern = resquant_kernel<KK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
@@ -457,17 +461,24 @@ metis_status run_residual_quantize(metis_ctx* ctx, const metis_matrix* M, const 
                                    const metis_quant_params* q, const metis_nvfp4* row, const metis_nvfp4* col) {
   const int k = (f && f->k > 0) ? f->k : 0;
   const int KK = k <= 32 ? 32 : 64;
-  const size_t need = (size_t)(M->rows + M->cols) * KK * 4 + 1024;
+  const size_t need = (size_t)(M->rows + M->cols) * KK * 4 + 1024 + 256;
   metis_status s = ensure_workspace(ctx, need);
   if (s != METIS_OK) return s;
   Workspace ws{ctx->ws, ctx->ws_bytes};
   float* US = static_cast<float*>(ws.take((size_t)M->rows * KK * 4));
   float* Vp = static_cast<float*>(ws.take((size_t)M->cols * KK * 4));
+  uint32_t* amax = nullptr;
+  if (q->tensor_scale == 0.0f) {
+    amax = static_cast<uint32_t*>(ws.take(256));
+    if ((s = check_cuda(ctx, launch_amax(M->data, true, M->rows, M->cols, M->ld, amax, ctx->sm_count, ctx->stream),
+                        "amax launch")) != METIS_OK)
+      return s;
+  }
   const int64_t n = (M->rows + M->cols) * KK;
   pad_factors_kernel<<<(unsigned)((n + 255) / 256), 256, 0, ctx->stream>>>(
       k ? f->U : nullptr, k ? f->S : nullptr, k ? f->V : nullptr, M->rows, M->cols, k, KK, US, Vp); count_launch();
   if ((s = check_cuda(ctx, cudaGetLastError(), "pad factors")) != METIS_OK) return s;
-  return KK == 32 ? launch_kk<32>(ctx, M, US, Vp, q, row, col) : launch_kk<64>(ctx, M, US, Vp, q, row, col);
+  return KK == 32 ? launch_kk<32>(ctx, M, US, Vp, q, amax, row, col) : launch_kk<64>(ctx, M, US, Vp, q, amax, row, col);
 }
 
 }  // namespace metis
@@ -484,12 +495,20 @@ metis_status run_residual_quantize_into(metis_ctx* ctx, const metis_matrix* M, c
   const int KK = k <= 32 ? 32 : 64;
   float* US = scratch;
   float* Vp = scratch + M->rows * KK;
+  uint32_t* amax = nullptr;
+  metis_status s;
+  if (q->tensor_scale == 0.0f) {
+    amax = reinterpret_cast<uint32_t*>(scratch + kNoAllocAmaxOffset);
+    if ((s = check_cuda(ctx, launch_amax(M->data, true, M->rows, M->cols, M->ld, amax, ctx->sm_count, ctx->stream),
+                        "amax launch")) != METIS_OK)
+      return s;
+  }
   const int64_t n = (M->rows + M->cols) * KK;
   pad_factors_kernel<<<(unsigned)((n + 255) / 256), 256, 0, ctx->stream>>>(
       k ? f->U : nullptr, k ? f->S : nullptr, k ? f->V : nullptr, M->rows, M->cols, k, KK, US, Vp); count_launch();
-  metis_status s = check_cuda(ctx, cudaGetLastError(), "pad factors");
+  s = check_cuda(ctx, cudaGetLastError(), "pad factors");
   if (s != METIS_OK) return s;
-  return KK == 32 ? launch_kk<32>(ctx, M, US, Vp, q, row, col) : launch_kk<64>(ctx, M, US, Vp, q, row, col);
+  return KK == 32 ? launch_kk<32>(ctx, M, US, Vp, q, amax, row, col) : launch_kk<64>(ctx, M, US, Vp, q, amax, row, col);
 }
 
 }  // namespace metis

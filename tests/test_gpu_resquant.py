@@ -88,3 +88,54 @@ def test_full_size_gradient_shape(ctx, metis_lib):
         wc, _ = nvfp4.quantize_blocks(R[a:a + 1], 1.0, "sr", u[None, :])
         agree.append(np.mean(codes[a] == wc[0]))
     assert np.mean(agree) > 0.99
+
+
+@pytest.mark.parametrize("scale,rounding", [(2.0 ** -24, 1), (1.0, 0), (2.0 ** 12, 1)])
+def test_tensor_scale_chosen_from_the_data(ctx, metis_lib, scale, rounding):
+    """tensor_scale = 0: g is the oracle's auto_tensor_scale of M, written to both outputs,
+    and the codes and scales are bit-exact with the oracle quantizer at that g (k = 0, so
+    the residual is M).  Scaling by a power of two keeps the bf16 values exact."""
+    cfg = synth.scaled_config("gpt2_small_mlp_up", l=1024, m=768, n=768)
+    Mt = (synth.operand_matrix(cfg, "X").float() * scale).to(torch.bfloat16)
+    M = Mt.cuda()
+    rows, cols = M.shape
+    row, col = ctx.new_nvfp4(rows, cols), ctx.new_nvfp4(cols, rows)
+    ctx.residual_quantize_nvfp4(M, None, row, col, rounding=rounding, seed=3, operand_id=2, step=5,
+                                tensor_scale=0.0)
+    torch.cuda.synchronize()
+    assert ctx.poll_device_status() == 0
+    R = Mt.float().numpy()
+    g = nvfp4.auto_tensor_scale(R)
+    mode = "sr" if rounding else "rn"
+    for t, orient in ((row, "row"), (col, "col")):
+        codes, scales, g_dev = codes_unpacked(t)
+        assert g_dev == g
+        wc, ws = nvfp4.quantize_oriented(R, orient, g=g, rounding=mode, seed=3, operand_id=2, step=5)
+        assert np.array_equal(scales, ws)
+        assert np.array_equal(codes, wc)
+
+
+def test_tensor_scale_chosen_from_the_data_single_orientation_and_f32(ctx, metis_lib):
+    """The same rule on the one-orientation path and on the fp32 quantizer surface."""
+    rng = np.random.default_rng(8)
+    R = (rng.standard_normal((256, 512)) * 3e-6).astype(np.float32)
+    g = nvfp4.auto_tensor_scale(R)
+    assert g < 2.0 ** -10
+    Rd = torch.from_numpy(R).cuda()
+    col = ctx.new_nvfp4(512, 256)
+    ctx.quantize_nvfp4_f32(Rd, None, col, rounding=0, tensor_scale=0.0)
+    Mb = torch.from_numpy(R).to(torch.bfloat16)
+    row = ctx.new_nvfp4(256, 512)
+    ctx.residual_quantize_nvfp4(Mb.cuda(), None, rowwise=row, rounding=0, tensor_scale=0.0)
+    torch.cuda.synchronize()
+    assert ctx.poll_device_status() == 0
+    codes, scales, g_dev = codes_unpacked(col)
+    assert g_dev == g
+    wc, ws = nvfp4.quantize_oriented(R, "col", g=g)
+    assert np.array_equal(scales, ws) and np.array_equal(codes, wc)
+    Rb = Mb.float().numpy()
+    gb = nvfp4.auto_tensor_scale(Rb)
+    codes, scales, g_dev = codes_unpacked(row)
+    assert g_dev == gb
+    wc, ws = nvfp4.quantize_oriented(Rb, "row", g=gb)
+    assert np.array_equal(scales, ws) and np.array_equal(codes, wc)
