@@ -179,6 +179,16 @@ metis_status metis_quantize_nvfp4_f32(metis_ctx* ctx, const float* R, int64_t ro
                                       metis_nvfp4* rowwise, metis_nvfp4* colwise);
 
 /*
+ * Decode of one NVFP4 tensor (background section: the value of an element is its E2M1
+ * code times its block's E4M3 scale, times the decode tensor scale g):
+ *   out[o * ld + i] = e2m1(code(o, i)) * e4m3(scale(o, i / 16)) * g
+ * for the outer x inner tensor t; out is caller-owned fp32 device memory (16-byte
+ * aligned, ld >= inner, ld % 4 == 0).  Exact: every product is an fp32 number.
+ * Errors: ERR_SHAPE unless inner % 64 == 0; ERR_ALIGN on the output.
+ */
+metis_status metis_dequantize_nvfp4(metis_ctx* ctx, const metis_nvfp4* t, float* out, int64_t ld);
+
+/*
  * Allocation-free residual quantization (no counterpart in the paper).
  * Same computation and results as metis_residual_quantize_nvfp4 with both
  * orientations, for callers that may not allocate device memory while they run:

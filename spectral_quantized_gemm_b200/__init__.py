@@ -41,7 +41,7 @@ EXPORTED = ["metis_create", "metis_destroy", "metis_set_stream", "metis_status_s
             "metis_poll_device_status", "metis_nvfp4_codes_bytes", "metis_nvfp4_scales_bytes",
             "metis_decompose", "metis_residual_quantize_nvfp4", "metis_quantize_nvfp4_f32", "metis_gemm_nvfp4",
             "metis_linear_fwd", "metis_linear_bwd", "metis_kernel_launches", "metis_profile_enable",
-            "metis_profile_read", "metis_residual_quantize_nvfp4_noalloc"]
+            "metis_profile_read", "metis_residual_quantize_nvfp4_noalloc", "metis_dequantize_nvfp4"]
 
 
 class Matrix(ctypes.Structure):
@@ -94,6 +94,7 @@ _resq = _sig("metis_residual_quantize_nvfp4", c_i32, c_p, ctypes.POINTER(Matrix)
 _resq_noalloc = _sig("metis_residual_quantize_nvfp4_noalloc", c_i32, c_p, ctypes.POINTER(Matrix),
                      ctypes.POINTER(FactorsStruct), ctypes.POINTER(QuantParams), ctypes.POINTER(Nvfp4Struct),
                      ctypes.POINTER(Nvfp4Struct))
+_dequant = _sig("metis_dequantize_nvfp4", c_i32, c_p, ctypes.POINTER(Nvfp4Struct), c_p, c_i64)
 _quant_f32 = _sig("metis_quantize_nvfp4_f32", c_i32, c_p, c_p, c_i64, c_i64, c_i64, ctypes.POINTER(QuantParams),
                   ctypes.POINTER(Nvfp4Struct), ctypes.POINTER(Nvfp4Struct))
 _gemm = _sig("metis_gemm_nvfp4", c_i32, c_p, ctypes.POINTER(Nvfp4Struct), ctypes.POINTER(Nvfp4Struct), c_i64, c_p,
@@ -237,6 +238,15 @@ class Context:
         self._call(_quant_f32, _ptr(R), R.shape[0], R.shape[1], R.stride(0), ctypes.byref(q),
                    None if rowwise is None else ctypes.byref(rowwise.struct),
                    None if colwise is None else ctypes.byref(colwise.struct))
+
+    def dequantize_nvfp4(self, t, out=None):
+        """Decode an Nvfp4 tensor to fp32 (outer x inner) on the device."""
+        if out is None:
+            out = torch.empty(t.outer, t.inner, dtype=torch.float32, device=self.device)
+        if out.dtype != torch.float32 or out.dim() != 2 or out.stride(1) != 1:
+            raise ValueError("expected a row-major 2-D fp32 CUDA tensor")
+        self._call(_dequant, ctypes.byref(t.struct), _ptr(out), out.stride(0))
+        return out
 
     def gemm_nvfp4(self, A, B, n_cols, C, Fa=None, Fb=None, col_scale=None):
         fold_k = 0 if Fa is None else Fa.shape[1]

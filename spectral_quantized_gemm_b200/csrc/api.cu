@@ -213,6 +213,17 @@ metis_status metis_quantize_nvfp4_f32(metis_ctx* ctx, const float* R, int64_t ro
                     "quantize launch");
 }
 
+metis_status metis_dequantize_nvfp4(metis_ctx* ctx, const metis_nvfp4* t, float* out, int64_t ld) {
+  metis_status s = enter(ctx);
+  if (s != METIS_OK) return s;
+  if (!t || !out) return fail(ctx, METIS_ERR_ARG, "null tensor or output");
+  if ((s = check_nvfp4(ctx, t, t->outer, t->inner, "tensor")) != METIS_OK) return s;
+  if (t->outer <= 0 || t->inner <= 0 || t->inner % 64) return fail(ctx, METIS_ERR_SHAPE, "inner must be a multiple of 64");
+  if (ld < t->inner || ld % 4 || !aligned16(out))
+    return fail(ctx, METIS_ERR_ALIGN, "fp32 output needs 16-byte alignment and ld % 4 == 0");
+  return check_cuda(ctx, launch_dequantize(t, out, ld, ctx->stream), "dequantize launch");
+}
+
 metis_status metis_residual_quantize_nvfp4(metis_ctx* ctx, const metis_matrix* M, const metis_factors* f,
                                            const metis_quant_params* q, metis_nvfp4* rowwise,
                                            metis_nvfp4* colwise) {

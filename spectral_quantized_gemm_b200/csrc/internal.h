@@ -59,6 +59,8 @@ EncodeTiledFn encode_tiled();
 // fp32 bits to *amax_bits; the quantizers then take g = auto_tensor_scale(*amax_bits).
 cudaError_t launch_amax(const void* M, bool bf16, int64_t rows, int64_t cols, int64_t ld, uint32_t* amax_bits,
                         int sm_count, cudaStream_t st);
+// Decode of one NVFP4 tensor into fp32 (outer x inner, leading dimension ld).
+cudaError_t launch_dequantize(const metis_nvfp4* t, float* out, int64_t ld, cudaStream_t st);
 // amax_bits: nullptr to use q.tensor_scale, else the word launch_amax wrote.
 cudaError_t launch_quantize_f32(const float* R, int64_t rows, int64_t cols, int64_t ld,
                                 const metis_quant_params& q, const uint32_t* amax_bits, const metis_nvfp4* rowwise,

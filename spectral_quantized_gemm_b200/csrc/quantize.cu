@@ -186,7 +186,49 @@ __global__ void __launch_bounds__(256) amax_f32_kernel(const float* __restrict__
   if (lane == 0 && best) atomicMax(amax_bits, best);
 }
 
+// Decode of one NVFP4 tensor: a thread per 16-element block reads 8 code bytes and its
+// scale byte (tile layout) and writes 16 fp32 values.  e2m1 x e4m3 x g is exact in fp32.
+__global__ void __launch_bounds__(256) dequantize_nvfp4_kernel(const uint8_t* __restrict__ codes,
+                                                               const uint8_t* __restrict__ scales,
+                                                               const float* __restrict__ g_ptr, int64_t outer,
+                                                               int64_t inner, float* __restrict__ out, int64_t ld) {
+  const int64_t nb = inner / 16;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= outer * nb) return;
+  const int64_t o = idx / nb;
+  const int64_t b = idx - o * nb;
+  const float g = *g_ptr;
+  const uint32_t sc =
+      scales[((o >> 7) * (inner / 64) + (b >> 2)) * 512 + (o & 31) * 16 + ((o & 127) >> 5) * 4 + (b & 3)];
+  const float s = e4m3_value(sc & 0x7Fu) * g;
+  const uint2 packed = *reinterpret_cast<const uint2*>(codes + o * (inner / 2) + b * 8);
+  const uint32_t w[2] = {packed.x, packed.y};
+  // E2M1 magnitudes of codes 0..7; bit 3 is the sign
+  const float mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+  float* dst = out + o * ld + b * 16;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t c = (w[h] >> (4 * i)) & 0xFu;
+      const float m = mag[c & 7u] * s;
+      v[i] = (c & 8u) ? -m : m;
+    }
+    reinterpret_cast<float4*>(dst + 8 * h)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(dst + 8 * h)[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_dequantize(const metis_nvfp4* t, float* out, int64_t ld, cudaStream_t st) {
+  const int64_t n = t->outer * (t->inner / 16);
+  dequantize_nvfp4_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(t->codes, t->scales, t->tensor_scale,
+                                                                       t->outer, t->inner, out, ld);
+  count_launch();
+  return cudaGetLastError();
+}
 
 cudaError_t launch_amax(const void* M, bool bf16, int64_t rows, int64_t cols, int64_t ld, uint32_t* amax_bits,
                         int sm_count, cudaStream_t st) {

@@ -128,3 +128,19 @@ def test_host_validation(ctx, metis_lib):
     assert e.value.status == 1
     with pytest.raises(metis_lib.MetisError):
         ctx.quantize_nvfp4_f32(R, ctx.new_nvfp4(256, 128), None)
+
+
+@pytest.mark.parametrize("g", [1.0, 2.0 ** -7])
+def test_dequantize_is_exact(ctx, metis_lib, g):
+    """metis_dequantize_nvfp4 gives e2m1(code) * e4m3(scale) * g exactly (oracle decode)."""
+    rng = np.random.default_rng(4)
+    R = (rng.standard_normal((256, 512)) * np.exp(rng.uniform(-3, 3, (256, 1))) * g).astype(np.float32)
+    t = ctx.new_nvfp4(256, 512)
+    ctx.quantize_nvfp4_f32(torch.from_numpy(R).cuda(), t, None, rounding=1, seed=2, tensor_scale=g)
+    out = ctx.dequantize_nvfp4(t)
+    torch.cuda.synchronize()
+    assert ctx.poll_device_status() == 0
+    codes, scales, g_dev = codes_unpacked(t)
+    assert g_dev == g
+    want = nvfp4.dequantize_blocks(codes, scales, g_dev)
+    assert np.array_equal(out.cpu().numpy().astype(np.float64), want)
