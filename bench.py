@@ -195,13 +195,26 @@ class Layer:
         return st
 
 
+def max_over_ranks(value, world, device):
+    """The largest value over all ranks (a time measured on each rank's device)."""
+    if world == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_config(cfg, rank):
+    """Weak scaling: every rank trains on its own tokens (X, D) with the shared W."""
+    return dict(cfg, seed=cfg["seed"] + 1000 * rank)
+
+
 def run_ours(args, rank, world, device):
     import spectral_quantized_gemm_b200 as lib
     cfg = synth.CONFIGS[args.config]
     l, m, n = cfg["l"], cfg["m"], cfg["n"]
     flops_per_step = 6.0 * l * m * n
-    # weak scaling: each rank its own tokens (X, D), the shared weight W
-    rcfg = dict(cfg, seed=cfg["seed"] + 1000 * rank)
+    rcfg = rank_config(cfg, rank)
     host_W = synth.operand_matrix(cfg, "W").pin_memory()
     host_batches = [(synth.batch_matrix(rcfg, "X", b).pin_memory(), synth.batch_matrix(rcfg, "D", b).pin_memory())
                     for b in range(args.batches)]
@@ -248,10 +261,7 @@ def run_ours(args, rank, world, device):
     ctx.profile_enable(False)
     clk = clocks.stop()
     ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t_ = torch.tensor([ms], device=device)
-        torch.distributed.all_reduce(t_, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t_.item())
+    ms = max_over_ranks(ms, world, device)
     ms_per_step = ms / args.steps
     value = world * flops_per_step / (ms_per_step * 1e-3) / 1e12
 
@@ -279,10 +289,7 @@ def run_ours(args, rank, world, device):
     torch.cuda.synchronize(device)
     barrier()
     e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t_ = torch.tensor([e2e_ms], device=device)
-        torch.distributed.all_reduce(t_, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t_.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, device)
     e2e_value = world * flops_per_step / (e2e_ms / e2e_steps * 1e-3) / 1e12
     status = layer.poll_device_status()
 
@@ -300,10 +307,7 @@ def run_ours(args, rank, world, device):
     torch.cuda.synchronize(device)
     barrier()
     plain_ms = p0.elapsed_time(p1) / args.steps
-    if world > 1:
-        t_ = torch.tensor([plain_ms], device=device)
-        torch.distributed.all_reduce(t_, op=torch.distributed.ReduceOp.MAX)
-        plain_ms = float(t_.item())
+    plain_ms = max_over_ranks(plain_ms, world, device)
     status |= plain.poll_device_status()
 
     peaks, kind = measured_peaks()
