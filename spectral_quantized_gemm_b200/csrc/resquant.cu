@@ -8,13 +8,15 @@
 //
 // Per 128 x 128 tile of M (persistent CTAs, contiguous row-block-major ranges):
 //   warp 0      TMA: the U*S rows of the row block (kept while the block lasts),
-//               then per tile the V rows and the two 64-column boxes of M
-//   warp 1      tensor-memory owner; one thread issues tcgen05.mma kind::tf32
-//               (U S)(V)^T -> fp32 reconstruction in a double-buffered accumulator
-//   warps 2..17 residual = M - reconstruction (fp32), row-wise quantization from
-//               registers (a warp per 32 rows x 32 columns), the tile staged in
-//               XOR-swizzled shared memory, then column-wise quantization (a thread per
-//               32 rows of a column); codes and tiled scales go straight to HBM
+//               then per tile the V rows and the two 64-column boxes of M (3 stages)
+//   warp 1      tensor-memory owner; one thread issues tcgen05.mma kind::tf32 for the
+//               reconstruction (U S) V^T and for its transpose V (U S)^T, each into a
+//               double-buffered fp32 accumulator (the same operands, swapped)
+//   warps 2..17 a warp per 32 x 32 sub-tile: row-wise quantization of M - (U S) V^T from
+//               its rows (reconstruction rows from tensor memory, M rows from shared
+//               memory), then column-wise quantization of the same sub-tile from the
+//               transposed reconstruction and M's columns; codes and tiled scales go
+//               straight to HBM.  The warps never wait for one another.
 // All mbarrier waits are bounded (METIS_DEV_TIMEOUT on expiry).
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -39,9 +41,8 @@ struct RqCfg {
   static constexpr int V_BYTES = 128 * KK * 4;
   static constexpr int M_BYTES = 128 * 128 * 2;  // two 64-column boxes of 16 KB
   static constexpr int STAGE_BYTES = V_BYTES + M_BYTES;
-  static constexpr int STAGES = 2;
-  static constexpr int R_BYTES = 128 * 128 * 4;
-  static constexpr size_t SMEM = (size_t)A_BYTES + STAGES * STAGE_BYTES + R_BYTES + 1024 + 256 + 512;
+  static constexpr int STAGES = 3;
+  static constexpr size_t SMEM = (size_t)A_BYTES + STAGES * STAGE_BYTES + 1024 + 256 + 512;
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -115,20 +116,6 @@ __device__ __forceinline__ uint2 quantize16(const float (&v)[16], float amax, fl
   return packed;
 }
 
-__device__ __forceinline__ void named_sync_epilogue() { asm volatile("bar.sync 1, %0;" ::"n"(kRqEpiThreads) : "memory"); }
-
-// OR of a predicate over the epilogue threads (a barrier: all must call it), so
-// every epilogue thread takes the same branch after a bounded wait.
-__device__ __forceinline__ bool epilogue_any(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\tbar.red.or.pred p, 1, %2, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)v), "n"(kRqEpiThreads)
-      : "memory");
-  return r != 0;
-}
-
 template <int KK>
 __global__ void __launch_bounds__(kRqThreads, 1)
     resquant_kernel(const __grid_constant__ CUtensorMap mapM, const __grid_constant__ CUtensorMap mapUS,
@@ -138,8 +125,7 @@ __global__ void __launch_bounds__(kRqThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sStage = sA + C::A_BYTES;
-  float* sR = reinterpret_cast<float*>(sStage + C::STAGES * C::STAGE_BYTES);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sR) + C::R_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + C::STAGES * C::STAGE_BYTES);
   uint64_t* a_full = bars;
   uint64_t* a_empty = bars + 1;
   uint64_t* full = bars + 2;                 // [STAGES]
@@ -180,8 +166,8 @@ __global__ void __launch_bounds__(kRqThreads, 1)
       *p.col_g = g;
     }
   }
-  if (warp == 1) {
-    tc::tmem_alloc(tmem_slot, 256);
+  if (warp == 1) {   // columns 0-255: reconstruction, 256-511: its transpose (two buffers each)
+    tc::tmem_alloc(tmem_slot, 512);
     tc::tmem_relinquish();
   }
   tc::tc_fence_before();
@@ -250,7 +236,10 @@ __global__ void __launch_bounds__(kRqThreads, 1)
           const uint64_t ad = tc::sdesc_sw128(tc::smem_addr(sA + ch * 16384));
           const uint64_t bd = tc::sdesc_sw128(tc::smem_addr(sV + ch * 16384));
 #pragma unroll
-          for (int j = 0; j < 4; ++j) mma_tf32(tmem + b * 128, ad + 2 * j, bd + 2 * j, idesc, (ch | j) ? 1u : 0u);
+          for (int j = 0; j < 4; ++j) {
+            mma_tf32(tmem + b * 128, ad + 2 * j, bd + 2 * j, idesc, (ch | j) ? 1u : 0u);          // rows of the tile
+            mma_tf32(tmem + 256 + b * 128, bd + 2 * j, ad + 2 * j, idesc, (ch | j) ? 1u : 0u);    // its columns
+          }
         }
         tc::tc_commit(&empty[stage]);
         tc::tc_commit(&acc_full[b]);
@@ -264,10 +253,16 @@ __global__ void __launch_bounds__(kRqThreads, 1)
     }
     __syncwarp();
   } else {
-    const int et = threadIdx.x - 64;   // epilogue thread 0 .. kRqEpiThreads - 1
     const int q = warp & 3;            // tensor-memory lane quarter
-    const int h = (warp - 2) >> 2;     // 32-column quarter of the tile in the row pass
+    const int h = (warp - 2) >> 2;     // 32-column quarter (row pass) = 32-row quarter (column pass)
     const int r = q * 32 + lane;       // tile row of this thread in the row pass
+    const int j = q * 32 + lane;       // tile column of this thread in the column pass
+    // M(i, j) of the column pass sits in box j >> 6 at row i, 16-byte chunk
+    // ((j & 63) >> 3) ^ (i & 7), element j & 7: the 8 chunk positions, by i & 7
+    const int jc = (j & 63) >> 3;
+    uint32_t col_off[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) col_off[t] = (uint32_t)((j >> 6) * 16384 + (((jc ^ t) << 4) | ((j & 7) << 1)));
     int stage = 0;
     uint32_t phase = 0;
     int it = 0;
@@ -277,44 +272,32 @@ __global__ void __launch_bounds__(kRqThreads, 1)
       const uint32_t use = (uint32_t)(it >> 1);
       bool ok = tc::mbar_wait(&acc_full[b], use & 1u, abort_flag);
       ok = ok && tc::mbar_wait(&full[stage], phase, abort_flag);
-      if (epilogue_any(!ok)) {
-        if (et == 0) fail_wait();
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) fail_wait();
         break;
       }
       tc::tc_fence_after();
-      // reconstruction of this thread's row, 32 columns
-      float v[32];
-      tc::tmem_load_32cols(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * 128 + h * 32), v);
-      tc::tmem_load_wait();
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&acc_empty[b]);
-      // residual = M - reconstruction (M from the 128B-swizzled 64-column box holding
-      // this quarter: chunks (h & 1) * 4 .. + 3 of box h >> 1)
-      const uint8_t* sM = sStage + stage * C::STAGE_BYTES + C::V_BYTES + (h >> 1) * 16384;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const int c = (h & 1) * 4 + cc;
-        const uint4 raw = *reinterpret_cast<const uint4*>(sM + r * 128 + ((c ^ (r & 7)) << 4));
-        const __nv_bfloat162* pr = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 f = __bfloat1622float2(pr[i]);
-          v[cc * 8 + 2 * i] = f.x - v[cc * 8 + 2 * i];
-          v[cc * 8 + 2 * i + 1] = f.y - v[cc * 8 + 2 * i + 1];
-        }
-      }
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&empty[stage]);   // this warp is done with M
-      // stage the residual row quarter in shared memory (16-byte chunks XOR-swizzled by row)
-#pragma unroll
-      for (int t4 = 0; t4 < 8; ++t4) {
-        const int cc = h * 8 + t4;
-        *reinterpret_cast<float4*>(sR + r * 128 + ((cc ^ (r & 7)) << 2)) =
-            make_float4(v[4 * t4], v[4 * t4 + 1], v[4 * t4 + 2], v[4 * t4 + 3]);
-      }
-      // row-wise quantization (blocks along columns) straight from registers
+      const uint8_t* sM = sStage + stage * C::STAGE_BYTES + C::V_BYTES;
+      // ---- row-wise quantization (blocks along columns): row r, columns h*32 .. + 31
       {
+        float v[32];
+        tc::tmem_load_32cols(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * 128 + h * 32), v);
+        tc::tmem_load_wait();
+        // residual = M - reconstruction (M from the 128B-swizzled 64-column box holding
+        // this quarter: chunks (h & 1) * 4 .. + 3 of box h >> 1)
+        const uint8_t* sMb = sM + (h >> 1) * 16384;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const int c = (h & 1) * 4 + cc;
+          const uint4 raw = *reinterpret_cast<const uint4*>(sMb + r * 128 + ((c ^ (r & 7)) << 4));
+          const __nv_bfloat162* pr = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(pr[i]);
+            v[cc * 8 + 2 * i] = f.x - v[cc * 8 + 2 * i];
+            v[cc * 8 + 2 * i + 1] = f.y - v[cc * 8 + 2 * i + 1];
+          }
+        }
         const int64_t grow = (int64_t)rb * 128 + r;
         const int64_t gcol = (int64_t)cb * 128 + h * 32;
         uint32_t sc = 0;
@@ -324,15 +307,18 @@ __global__ void __launch_bounds__(kRqThreads, 1)
 #pragma unroll
         for (int blk = 0; blk < 2; ++blk) {
           float x[16];
-          uint32_t abits = 0;   // largest |x| as a bit pattern: an integer max keeps Inf and NaN visible
+          // block maximum of |x|: fmaxf keeps an Inf but drops a NaN, which a sum of the
+          // block's magnitudes then shows (the sum is NaN exactly when an element is)
+          float amax = 0.0f, sum = 0.0f;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             x[i] = v[blk * 16 + i];
-            abits = max(abits, __float_as_uint(x[i]) & 0x7FFFFFFFu);
+            amax = fmaxf(amax, fabsf(x[i]));
+            sum += fabsf(x[i]);
           }
-          finite &= abits < 0x7F800000u;
+          finite &= (amax <= 3.402823466e38f) && (sum == sum);
           uint32_t code;
-          const uint2 pk = quantize16(x, __uint_as_float(abits), g, rcp_table, p.rounding, p.seed, p.tag_row,
+          const uint2 pk = quantize16(x, amax, g, rcp_table, p.rounding, p.seed, p.tag_row,
                                       p.step, (uint64_t)grow * (uint64_t)p.cols + (uint64_t)(gcol + blk * 16), code);
           sc |= code << (8 * blk);
           o[2 * blk] = pk.x;
@@ -342,13 +328,20 @@ __global__ void __launch_bounds__(kRqThreads, 1)
         *reinterpret_cast<uint4*>(p.row_codes + grow * (p.cols / 2) + gcol / 2) = out;
         *reinterpret_cast<uint16_t*>(p.row_scales + scale_offset(grow, gcol / 16, p.cols / 64)) = (uint16_t)sc;
       }
-      named_sync_epilogue();
-      // column-wise quantization (blocks along rows) from the staged tile: column j,
-      // rows hh * 32 .. + 31
+      // ---- column-wise quantization (blocks along rows): column j, rows h*32 .. + 31,
+      // from the transposed reconstruction (tensor-memory lane j) and M's column j
       {
-        const int j = et & 127, hh = et >> 7;
+        const uint8_t* cbase[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) cbase[t] = sM + h * 32 * 128 + col_off[t];
+        float w[32];
+        tc::tmem_load_32cols(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(256 + b * 128 + h * 32), w);
+        tc::tmem_load_wait();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&acc_empty[b]);   // both reconstructions of this tile are read
         const int64_t gcolj = (int64_t)cb * 128 + j;
-        const int64_t grow0 = (int64_t)rb * 128 + hh * 32;
+        const int64_t grow0 = (int64_t)rb * 128 + h * 32;
         uint32_t sc = 0;
         uint4 out;
         uint32_t* o = reinterpret_cast<uint32_t*>(&out);
@@ -358,8 +351,8 @@ __global__ void __launch_bounds__(kRqThreads, 1)
           float amax = 0.0f;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int rr = hh * 32 + blk * 16 + i;
-            x[i] = sR[rr * 128 + ((((j >> 2) ^ (rr & 7))) << 2) + (j & 3)];
+            const uint16_t mb = *reinterpret_cast<const uint16_t*>(cbase[i & 7] + (blk * 16 + i) * 128);  // tile row h*32+blk*16+i
+            x[i] = __uint_as_float((uint32_t)mb << 16) - w[blk * 16 + i];
             amax = fmaxf(amax, fabsf(x[i]));
           }
           uint32_t code;
@@ -369,10 +362,11 @@ __global__ void __launch_bounds__(kRqThreads, 1)
           o[2 * blk] = pk.x;
           o[2 * blk + 1] = pk.y;
         }
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&empty[stage]);   // this warp is done with M
         *reinterpret_cast<uint4*>(p.col_codes + gcolj * (p.rows / 2) + grow0 / 2) = out;
         *reinterpret_cast<uint16_t*>(p.col_scales + scale_offset(gcolj, grow0 / 16, p.rows / 64)) = (uint16_t)sc;
       }
-      named_sync_epilogue();
       if (++stage == C::STAGES) {
         stage = 0;
         phase ^= 1u;
@@ -384,7 +378,7 @@ __global__ void __launch_bounds__(kRqThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc::tc_fence_after();
-    tc::tmem_dealloc(tmem, 256);
+    tc::tmem_dealloc(tmem, 512);
   }
 }
 
