@@ -310,6 +310,10 @@ def run_ours(args, rank, world, device):
     plain_ms = max_over_ranks(plain_ms, world, device)
     status |= plain.poll_device_status()
 
+    # the achievable FP4 MMA rate on this GPU (no memory traffic), beside the roofline
+    mma_peak = ctx.nvfp4_mma_peak(iters=4096, reps=5)
+    status |= ctx.poll_device_status()
+
     peaks, kind = measured_peaks()
     peak = peaks["bf16_tflops_sustained"] * NVFP4_OVER_BF16
     achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
@@ -337,6 +341,11 @@ def run_ours(args, rank, world, device):
                                       "launch (bytes); the timed launches are the fwd, dX and dW GeMMs",
                      "launches_timed": gemm_n,
                      "peak_basis": f"{kind} bf16 sustained x {NVFP4_OVER_BF16:.0f} (nominal NVFP4/bf16 ratio)"},
+        "nvfp4_mma_peak": {
+            "value": round(mma_peak, 1), "unit": "TFLOP/s",
+            "gemm_frac": None if achieved is None else round(achieved / mma_peak, 4),
+            "what": "tcgen05 kind::mxf4nvf4 block16 MMAs (CTA pairs, M=256 N=256 K=64) on resident "
+                    "operands, no memory traffic: the rate the fused GeMM could reach"},
         "plain_nvfp4": {
             "value": round(world * flops_per_step / (plain_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
             "ms_per_step": round(plain_ms, 4),

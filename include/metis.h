@@ -260,6 +260,17 @@ metis_status metis_linear_bwd(metis_ctx* ctx, const metis_operand* X, const meti
                               float* dW, int64_t lddw);
 
 /*
+ * NVFP4 tensor-core throughput microbenchmark (no counterpart in the notes; the measured
+ * ceiling for the fused GeMM).  Launches, on the context's stream, one cluster of two
+ * CTAs per SM pair; each pair issues `iters` stages of four block-scaled MMAs
+ * (tcgen05 kind::mxf4nvf4, block16, M = 256, N = 256, K = 64) on operands resident in
+ * shared and tensor memory, with no memory traffic.  *flops receives the useful flops
+ * of the launch (2 * 256 * 256 * 256 * iters per pair); the caller times the launch.
+ * Errors: ERR_ARG for iters < 1 or more than 2^20 (keeps one launch well under a second).
+ */
+metis_status metis_nvfp4_mma_peak(metis_ctx* ctx, int64_t iters, double* flops);
+
+/*
  * Instrumentation (the notes have no counterpart; used by the benchmark).
  * metis_kernel_launches: number of kernels libmetis has launched in this process.
  * metis_profile_enable: when on, every main GeMM launch (the fused FP4 + fold

@@ -41,7 +41,8 @@ EXPORTED = ["metis_create", "metis_destroy", "metis_set_stream", "metis_status_s
             "metis_poll_device_status", "metis_nvfp4_codes_bytes", "metis_nvfp4_scales_bytes",
             "metis_decompose", "metis_residual_quantize_nvfp4", "metis_quantize_nvfp4_f32", "metis_gemm_nvfp4",
             "metis_linear_fwd", "metis_linear_bwd", "metis_kernel_launches", "metis_profile_enable",
-            "metis_profile_read", "metis_residual_quantize_nvfp4_noalloc", "metis_dequantize_nvfp4"]
+            "metis_profile_read", "metis_residual_quantize_nvfp4_noalloc", "metis_dequantize_nvfp4",
+            "metis_nvfp4_mma_peak"]
 
 
 class Matrix(ctypes.Structure):
@@ -95,6 +96,7 @@ _resq_noalloc = _sig("metis_residual_quantize_nvfp4_noalloc", c_i32, c_p, ctypes
                      ctypes.POINTER(FactorsStruct), ctypes.POINTER(QuantParams), ctypes.POINTER(Nvfp4Struct),
                      ctypes.POINTER(Nvfp4Struct))
 _dequant = _sig("metis_dequantize_nvfp4", c_i32, c_p, ctypes.POINTER(Nvfp4Struct), c_p, c_i64)
+_mma_peak = _sig("metis_nvfp4_mma_peak", c_i32, c_p, c_i64, ctypes.POINTER(ctypes.c_double))
 _quant_f32 = _sig("metis_quantize_nvfp4_f32", c_i32, c_p, c_p, c_i64, c_i64, c_i64, ctypes.POINTER(QuantParams),
                   ctypes.POINTER(Nvfp4Struct), ctypes.POINTER(Nvfp4Struct))
 _gemm = _sig("metis_gemm_nvfp4", c_i32, c_p, ctypes.POINTER(Nvfp4Struct), ctypes.POINTER(Nvfp4Struct), c_i64, c_p,
@@ -253,6 +255,23 @@ class Context:
         dtype = OUT_F32 if C.dtype == torch.float32 else OUT_BF16
         self._call(_gemm, ctypes.byref(A.struct), ctypes.byref(B.struct), n_cols, _ptr(Fa), _ptr(Fb), fold_k,
                    _ptr(col_scale), _ptr(C), C.stride(0), dtype)
+
+    def nvfp4_mma_peak(self, iters=4096, reps=5):
+        """Achievable NVFP4 MMA rate (TFLOP/s): the median of `reps` timed launches of the
+        no-memory-traffic microbenchmark (after one untimed launch)."""
+        fl = ctypes.c_double()
+        self._call(_mma_peak, iters, ctypes.byref(fl))
+        stream = torch.cuda.current_stream(self.device)
+        times = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            self._call(_mma_peak, iters, ctypes.byref(fl))
+            e1.record(stream)
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1))
+        times.sort()
+        return fl.value / (times[len(times) // 2] * 1e-3) / 1e12
 
     def profile_enable(self, on=True):
         self._call(_prof_enable, int(bool(on)))

@@ -342,6 +342,14 @@ metis_status metis_profile_enable(metis_ctx* ctx, int on) {
   return METIS_OK;
 }
 
+metis_status metis_nvfp4_mma_peak(metis_ctx* ctx, int64_t iters, double* flops) {
+  metis_status s = enter(ctx);
+  if (s != METIS_OK) return s;
+  if (!flops || iters < 1 || iters > (int64_t(1) << 20))
+    return fail(ctx, METIS_ERR_ARG, "iters must be in [1, 2^20] and flops non-null");
+  return launch_mma_peak(ctx, iters, flops);
+}
+
 metis_status metis_profile_read(metis_ctx* ctx, double* ms, int64_t* launches, double* flops) {
   if (!ctx || !ms || !launches || !flops) return METIS_ERR_ARG;
   cudaSetDevice(ctx->device);

@@ -120,3 +120,13 @@ def test_gemm_validation(ctx, metis_lib):
     B2, _ = _operand(ctx, 200 - 72, 256, rng)
     with pytest.raises(metis_lib.MetisError):
         ctx.gemm_nvfp4(A, B2, 48, C)          # thin width not in {16, 32, 64}
+
+
+def test_mma_peak_microbenchmark(ctx, metis_lib):
+    """The no-memory-traffic NVFP4 MMA loop runs cleanly and reports a rate between the
+    fused GeMM's and the nominal dense FP4 peak (about 9.5 PFLOP/s at 1.965 GHz)."""
+    rate = ctx.nvfp4_mma_peak(iters=1024, reps=3)
+    assert ctx.poll_device_status() == 0
+    assert 2000.0 < rate < 12000.0, rate
+    with pytest.raises(metis_lib.MetisError):
+        ctx.nvfp4_mma_peak(iters=0)
