@@ -260,6 +260,17 @@ metis_status metis_linear_bwd(metis_ctx* ctx, const metis_operand* X, const meti
                               float* dW, int64_t lddw);
 
 /*
+ * Self-test of failure detection (no counterpart in the notes).  Every wait of the
+ * tensor-core kernels is bounded: on expiry the kernel sets METIS_DEV_TIMEOUT in the
+ * context's status word and returns normally.  This launches one CTA that waits on a
+ * barrier nothing arrives at, with a limit of `limit_cycles` SM clock cycles
+ * (1 .. 2e8, about 0.1 s at most), so the caller can check that the timeout is reported
+ * by metis_poll_device_status and that the context stays usable.
+ * Errors: ERR_ARG for a limit outside the range.
+ */
+metis_status metis_selftest_wait_timeout(metis_ctx* ctx, int64_t limit_cycles);
+
+/*
  * NVFP4 tensor-core throughput microbenchmark (no counterpart in the notes; the measured
  * ceiling for the fused GeMM).  Launches, on the context's stream, one cluster of two
  * CTAs per SM pair; each pair issues `iters` stages of four block-scaled MMAs

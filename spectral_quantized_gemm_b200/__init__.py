@@ -42,7 +42,7 @@ EXPORTED = ["metis_create", "metis_destroy", "metis_set_stream", "metis_status_s
             "metis_decompose", "metis_residual_quantize_nvfp4", "metis_quantize_nvfp4_f32", "metis_gemm_nvfp4",
             "metis_linear_fwd", "metis_linear_bwd", "metis_kernel_launches", "metis_profile_enable",
             "metis_profile_read", "metis_residual_quantize_nvfp4_noalloc", "metis_dequantize_nvfp4",
-            "metis_nvfp4_mma_peak"]
+            "metis_nvfp4_mma_peak", "metis_selftest_wait_timeout"]
 
 
 class Matrix(ctypes.Structure):
@@ -97,6 +97,7 @@ _resq_noalloc = _sig("metis_residual_quantize_nvfp4_noalloc", c_i32, c_p, ctypes
                      ctypes.POINTER(Nvfp4Struct))
 _dequant = _sig("metis_dequantize_nvfp4", c_i32, c_p, ctypes.POINTER(Nvfp4Struct), c_p, c_i64)
 _mma_peak = _sig("metis_nvfp4_mma_peak", c_i32, c_p, c_i64, ctypes.POINTER(ctypes.c_double))
+_wait_selftest = _sig("metis_selftest_wait_timeout", c_i32, c_p, c_i64)
 _quant_f32 = _sig("metis_quantize_nvfp4_f32", c_i32, c_p, c_p, c_i64, c_i64, c_i64, ctypes.POINTER(QuantParams),
                   ctypes.POINTER(Nvfp4Struct), ctypes.POINTER(Nvfp4Struct))
 _gemm = _sig("metis_gemm_nvfp4", c_i32, c_p, ctypes.POINTER(Nvfp4Struct), ctypes.POINTER(Nvfp4Struct), c_i64, c_p,
@@ -255,6 +256,11 @@ class Context:
         dtype = OUT_F32 if C.dtype == torch.float32 else OUT_BF16
         self._call(_gemm, ctypes.byref(A.struct), ctypes.byref(B.struct), n_cols, _ptr(Fa), _ptr(Fb), fold_k,
                    _ptr(col_scale), _ptr(C), C.stride(0), dtype)
+
+    def selftest_wait_timeout(self, limit_cycles=1_000_000):
+        """Launch the bounded-wait self-test (a wait that must time out); the caller then
+        reads METIS_DEV_TIMEOUT from poll_device_status()."""
+        self._call(_wait_selftest, limit_cycles)
 
     def nvfp4_mma_peak(self, iters=4096, reps=5):
         """Achievable NVFP4 MMA rate (TFLOP/s): the median of `reps` timed launches of the

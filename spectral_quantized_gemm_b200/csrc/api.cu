@@ -342,6 +342,14 @@ metis_status metis_profile_enable(metis_ctx* ctx, int on) {
   return METIS_OK;
 }
 
+metis_status metis_selftest_wait_timeout(metis_ctx* ctx, int64_t limit_cycles) {
+  metis_status s = enter(ctx);
+  if (s != METIS_OK) return s;
+  if (limit_cycles < 1 || limit_cycles > 200000000LL)
+    return fail(ctx, METIS_ERR_ARG, "limit_cycles must be in [1, 2e8]");
+  return launch_wait_timeout_selftest(ctx, limit_cycles);
+}
+
 metis_status metis_nvfp4_mma_peak(metis_ctx* ctx, int64_t iters, double* flops) {
   metis_status s = enter(ctx);
   if (s != METIS_OK) return s;

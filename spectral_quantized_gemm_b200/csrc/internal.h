@@ -105,6 +105,8 @@ struct GemmArgs {
 // work units per SM, no empty share.
 int fp4_splits(metis_ctx* ctx, int64_t tiles, int stages);
 metis_status launch_gemm_nvfp4(metis_ctx* ctx, const GemmArgs& a);
+// ---- selftest.cu ----
+metis_status launch_wait_timeout_selftest(metis_ctx* ctx, int64_t limit_cycles);
 // ---- mma_peak.cu ----
 metis_status launch_mma_peak(metis_ctx* ctx, int64_t iters, double* flops);
 // C[s] (rows x n, fp32, split s at C + s * rows * ldc) = A (rows x K bf16, lda) * B^T

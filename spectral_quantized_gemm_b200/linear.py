@@ -120,6 +120,22 @@ class MetisLinear(torch.nn.Module):
         self.step = 0
         self._bases = [_Basis(), _Basis(), _Basis()]   # X, W, dY
 
+    # Checkpoint state beyond the weight: the step counter (it picks refresh steps and
+    # enters the random streams) and the reused bases of X, W and dY, so that training
+    # resumed from a checkpoint repeats the uninterrupted run bit for bit.
+    def get_extra_state(self):
+        return {"step": self.step,
+                "bases": [None if b.V is None else (b.V.detach().cpu().clone(), b.shape) for b in self._bases]}
+
+    def set_extra_state(self, state):
+        self.step = int(state["step"])
+        dev = self.weight.device
+        for b, saved in zip(self._bases, state["bases"]):
+            if saved is None:
+                b.V, b.shape = None, None
+            else:
+                b.V, b.shape = saved[0].to(dev).clone(), tuple(saved[1])
+
     def extra_repr(self):
         return (f"in_features={self.in_features}, out_features={self.out_features}, k={self.k}, s={self.s}, "
                 f"refresh_every={self.refresh_every}, rounding={'sr' if self.rounding else 'rn'}")
