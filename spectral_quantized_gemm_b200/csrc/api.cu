@@ -1,4 +1,5 @@
 // The C ABI of libmetis: context management, host-side validation and dispatch.
+#include <nvtx3/nvToolsExt.h>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -10,6 +11,14 @@
 #include "internal.h"
 
 namespace metis {
+
+// NVTX range over one C-ABI call (visible in profilers that record NVTX; near free otherwise).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 metis_status fail(metis_ctx* ctx, metis_status s, const std::string& msg) {
   if (ctx) ctx->last_error = msg;
@@ -191,6 +200,7 @@ int64_t metis_nvfp4_scales_bytes(int64_t outer, int64_t inner) {
 
 metis_status metis_quantize_nvfp4_f32(metis_ctx* ctx, const float* R, int64_t rows, int64_t cols, int64_t ld,
                                       const metis_quant_params* q, metis_nvfp4* rowwise, metis_nvfp4* colwise) {
+  const metis::NvtxRange nvtx_range("metis_quantize_nvfp4_f32");
   metis_status s = enter(ctx);
   if (s != METIS_OK) return s;
   if (!R) return fail(ctx, METIS_ERR_ARG, "null input");
@@ -214,6 +224,7 @@ metis_status metis_quantize_nvfp4_f32(metis_ctx* ctx, const float* R, int64_t ro
 }
 
 metis_status metis_dequantize_nvfp4(metis_ctx* ctx, const metis_nvfp4* t, float* out, int64_t ld) {
+  const metis::NvtxRange nvtx_range("metis_dequantize_nvfp4");
   metis_status s = enter(ctx);
   if (s != METIS_OK) return s;
   if (!t || !out) return fail(ctx, METIS_ERR_ARG, "null tensor or output");
@@ -227,6 +238,7 @@ metis_status metis_dequantize_nvfp4(metis_ctx* ctx, const metis_nvfp4* t, float*
 metis_status metis_residual_quantize_nvfp4(metis_ctx* ctx, const metis_matrix* M, const metis_factors* f,
                                            const metis_quant_params* q, metis_nvfp4* rowwise,
                                            metis_nvfp4* colwise) {
+  const metis::NvtxRange nvtx_range("metis_residual_quantize_nvfp4");
   metis_status s = enter(ctx);
   if (s != METIS_OK) return s;
   if (!M || !M->data) return fail(ctx, METIS_ERR_ARG, "null matrix");
@@ -266,6 +278,7 @@ metis_status metis_residual_quantize_nvfp4(metis_ctx* ctx, const metis_matrix* M
 metis_status metis_gemm_nvfp4(metis_ctx* ctx, const metis_nvfp4* A, const metis_nvfp4* B, int64_t n_cols,
                               const void* Fa, const void* Fb, int32_t fold_k, const float* col_scale, void* C,
                               int64_t ldc, int32_t c_dtype) {
+  const metis::NvtxRange nvtx_range("metis_gemm_nvfp4");
   metis_status s = enter(ctx);
   if (s != METIS_OK) return s;
   if (!A || !B || !C) return fail(ctx, METIS_ERR_ARG, "null operand");
@@ -290,6 +303,7 @@ metis_status metis_gemm_nvfp4(metis_ctx* ctx, const metis_nvfp4* A, const metis_
 
 metis_status metis_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_decomp_params* p, int refresh,
                              uint32_t step, metis_factors* f) {
+  const metis::NvtxRange nvtx_range("metis_decompose");
   metis_status s = enter(ctx);
   if (s != METIS_OK) return s;
   if (!M || !M->data || !p || !f) return fail(ctx, METIS_ERR_ARG, "null argument");
@@ -307,6 +321,7 @@ metis_status metis_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_
 
 metis_status metis_linear_fwd(metis_ctx* ctx, const metis_operand* X, const metis_operand* W, void* Y, int64_t ldy,
                               int32_t y_dtype) {
+  const metis::NvtxRange nvtx_range("metis_linear_fwd");
   metis_status s = enter(ctx);
   if (s != METIS_OK) return s;
   if (!X || !W || !Y || !X->rowwise || !W->colwise) return fail(ctx, METIS_ERR_ARG, "null operand");
@@ -315,6 +330,7 @@ metis_status metis_linear_fwd(metis_ctx* ctx, const metis_operand* X, const meti
 
 metis_status metis_linear_bwd(metis_ctx* ctx, const metis_operand* X, const metis_operand* W, const metis_operand* D,
                               void* dX, int64_t lddx, int32_t dx_dtype, float* dW, int64_t lddw) {
+  const metis::NvtxRange nvtx_range("metis_linear_bwd");
   metis_status s = enter(ctx);
   if (s != METIS_OK) return s;
   if (!X || !W || !D || !dX || !dW || !D->rowwise || !D->colwise || !W->rowwise || !X->colwise)
@@ -351,6 +367,7 @@ metis_status metis_selftest_wait_timeout(metis_ctx* ctx, int64_t limit_cycles) {
 }
 
 metis_status metis_nvfp4_mma_peak(metis_ctx* ctx, int64_t iters, double* flops) {
+  const metis::NvtxRange nvtx_range("metis_nvfp4_mma_peak");
   metis_status s = enter(ctx);
   if (s != METIS_OK) return s;
   if (!flops || iters < 1 || iters > (int64_t(1) << 20))
@@ -385,6 +402,7 @@ metis_status metis_profile_read(metis_ctx* ctx, double* ms, int64_t* launches, d
 extern "C" metis_status metis_residual_quantize_nvfp4_noalloc(metis_ctx* ctx, const metis_matrix* M,
                                                                const metis_factors* f, const metis_quant_params* q,
                                                                metis_nvfp4* rowwise, metis_nvfp4* colwise) {
+  const metis::NvtxRange nvtx_range("metis_residual_quantize_nvfp4_noalloc");
   metis_status s = enter(ctx);
   if (s != METIS_OK) return s;
   if (!M || !M->data) return fail(ctx, METIS_ERR_ARG, "null matrix");
