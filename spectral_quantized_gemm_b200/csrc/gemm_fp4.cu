@@ -82,6 +82,59 @@ struct Params {
   int k_splits;            // work units per output tile along K (split-K), >= 1
   int64_t split_stride;    // elements between the partial outputs of consecutive splits
   uint32_t* status;
+  // Grouped launch (thin GeMMs only): after the units of the problem above come the units
+  // of n_extra more problems with their own operands (maps A1/B1, A2/B2), scales, tensor
+  // scales, fp32 output and tiling; one column tile each, the same K, no fold stages.
+  int n_extra;
+  struct Extra {
+    const uint8_t* sfa;
+    const uint8_t* sfb;
+    const float* ga;
+    const float* gb;
+    float* C;
+    int64_t ldc;
+    int m_tiles, k_splits;
+    int64_t split_stride;
+  } extra[2];
+};
+
+// Where a work unit of a (possibly grouped) launch lands: problem g, output tile
+// (mb, nb), K-stage range [s0, s1), split index.
+struct Unit {
+  int g, mb, nb, s0, s1, split;
+};
+
+__device__ __forceinline__ Unit decode_unit(const Params& p, int unit, int total_stages) {
+  int g = 0, m_tiles = p.m_tiles, n_tiles = p.n_tiles, splits = p.k_splits;
+  int u = unit;
+  int units = m_tiles * n_tiles * splits;
+  for (int e = 0; e < p.n_extra && u >= units; ++e) {
+    u -= units;
+    g = e + 1;
+    m_tiles = p.extra[e].m_tiles;
+    n_tiles = 1;
+    splits = p.extra[e].k_splits;
+    units = m_tiles * splits;
+  }
+  Unit r;
+  const int num_tiles = m_tiles * n_tiles;
+  const int tile = u % num_tiles;
+  const int per = (total_stages + splits - 1) / splits;
+  r.g = g;
+  r.mb = tile % m_tiles;
+  r.nb = tile / m_tiles;
+  r.split = u / num_tiles;
+  r.s0 = r.split * per;
+  r.s1 = min(total_stages, r.s0 + per);
+  return r;
+}
+
+// Output of one problem of a launch.
+struct OutView {
+  void* C;
+  int64_t ldc;
+  int c_dtype;
+  const float* col_scale;
 };
 
 // Epilogue store of one warp's 32-row slice: lane t holds row row0 + t, columns
@@ -91,7 +144,7 @@ struct Params {
 // row directly wrote half sectors and cost a fifth of the GeMM's time.)  fp32 output
 // goes to f32_out (a split-K partial or C); bf16 output to C.
 template <int COLS>
-__device__ __forceinline__ void store_rows(const Params& p, const float (&v)[COLS], uint8_t* buf, int lane,
+__device__ __forceinline__ void store_rows(const OutView& p, const float (&v)[COLS], uint8_t* buf, int lane,
                                            int64_t row0, int64_t cbase, float alpha, float* f32_out) {
   uint4* stage_buf = reinterpret_cast<uint4*>(buf);
   const int half = lane & 1;
@@ -144,6 +197,8 @@ template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                       const __grid_constant__ CUtensorMap mapFa, const __grid_constant__ CUtensorMap mapFb,
+                      const __grid_constant__ CUtensorMap mapA1, const __grid_constant__ CUtensorMap mapB1,
+                      const __grid_constant__ CUtensorMap mapA2, const __grid_constant__ CUtensorMap mapB2,
                       const Params p) {
   using C = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -183,6 +238,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::prefetch_tensormap(&mapFa);
       tc::prefetch_tensormap(&mapFb);
     }
+    if (p.n_extra > 0) {
+      tc::prefetch_tensormap(&mapA1);
+      tc::prefetch_tensormap(&mapB1);
+    }
+    if (p.n_extra > 1) {
+      tc::prefetch_tensormap(&mapA2);
+      tc::prefetch_tensormap(&mapB2);
+    }
   }
   if (warp == 1) {
     tc::tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -193,10 +256,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int num_tiles = p.m_tiles * p.n_tiles;
   const int total_stages = p.k_stages + p.fold_stages;
-  const int num_units = num_tiles * p.k_splits;
-  const int per_split = (total_stages + p.k_splits - 1) / p.k_splits;
+  int num_units = p.m_tiles * p.n_tiles * p.k_splits;
+  for (int e = 0; e < p.n_extra; ++e) num_units += p.extra[e].m_tiles * p.extra[e].k_splits;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -204,11 +266,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       for (int unit = blockIdx.x; unit < num_units && !*abort_flag; unit += gridDim.x) {
-        const int tile = unit % num_tiles;
-        const int mb = tile % p.m_tiles;
-        const int nb = tile / p.m_tiles;
-        const int s0 = (unit / num_tiles) * per_split, s1 = min(total_stages, s0 + per_split);
-        for (int kk = s0; kk < s1; ++kk) {
+        const Unit w = decode_unit(p, unit, total_stages);
+        const int mb = w.mb, nb = w.nb;
+        const CUtensorMap* mA = w.g == 0 ? &mapA : (w.g == 1 ? &mapA1 : &mapA2);
+        const CUtensorMap* mB = w.g == 0 ? &mapB : (w.g == 1 ? &mapB1 : &mapB2);
+        const uint8_t* sfa_g = w.g == 0 ? p.sfa : p.extra[w.g - 1].sfa;
+        const uint8_t* sfb_g = w.g == 0 ? p.sfb : p.extra[w.g - 1].sfb;
+        for (int kk = w.s0; kk < w.s1; ++kk) {
           if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             *abort_flag = 1;
             raise_status(p.status, METIS_DEV_TIMEOUT);
@@ -220,13 +284,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint8_t* sSFA = sf + stage * C::SF_STAGE_BYTES;
             uint8_t* sSFB = sSFA + C::SFA_BYTES;
             tc::mbar_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES + C::SFA_BYTES + C::SFB_BYTES);
-            tc::tma_load_2d(sA, &mapA, &full[stage], kk * 128, mb * 128);
-            tc::tma_load_2d(sB, &mapB, &full[stage], kk * 128, nb * BN);
-            tc::bulk_load(sSFA, p.sfa + ((int64_t)mb * p.kb_tiles + kk * 4) * 512, C::SFA_BYTES, &full[stage]);
+            tc::tma_load_2d(sA, mA, &full[stage], kk * 128, mb * 128);
+            tc::tma_load_2d(sB, mB, &full[stage], kk * 128, nb * BN);
+            tc::bulk_load(sSFA, sfa_g + ((int64_t)mb * p.kb_tiles + kk * 4) * 512, C::SFA_BYTES, &full[stage]);
             const int64_t nb128 = (int64_t)nb * BN / 128;
 #pragma unroll
             for (int a = 0; a < C::SFB_ATOMS; ++a)
-              tc::bulk_load(sSFB + a * 2048, p.sfb + ((nb128 + a) * p.kb_tiles + kk * 4) * 512, 2048,
+              tc::bulk_load(sSFB + a * 2048, sfb_g + ((nb128 + a) * p.kb_tiles + kk * 4) * 512, 2048,
                             &full[stage]);
           } else {
             const int f = kk - p.k_stages;
@@ -252,7 +316,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t id_bf16 = tc::idesc_bf16(BN);
 
       for (int unit = blockIdx.x; unit < num_units && !*abort_flag; unit += gridDim.x, ++it) {
-        const int s0 = (unit / num_tiles) * per_split, s1 = min(total_stages, s0 + per_split);
+        const Unit w = decode_unit(p, unit, total_stages);
+        const int s0 = w.s0, s1 = w.s1;
         const int ab = it % C::ACC_BUFS;
         const uint32_t use = (uint32_t)(it / C::ACC_BUFS);
         const uint32_t t_acc = tmem + ab * BN;
@@ -312,8 +377,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       for (int unit = blockIdx.x; unit < num_units && !*abort_flag; unit += gridDim.x) {
-        const int s0 = (unit / num_tiles) * per_split, s1 = min(total_stages, s0 + per_split);
-        for (int kk = s0; kk < s1; ++kk) {
+        const Unit w = decode_unit(p, unit, total_stages);
+        for (int kk = w.s0; kk < w.s1; ++kk) {
           if (!tc::mbar_wait(&full[stage], phase, abort_flag)) {
             *abort_flag = 1;
             raise_status(p.status, METIS_DEV_TIMEOUT);
@@ -351,13 +416,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int h = (warp - 2) >> 2;          // column half
     constexpr int kColsPerWarp = BN >= 64 ? BN / 2 : BN;
     const bool active = BN >= 64 || h == 0;
-    const float alpha = (p.ga ? *p.ga : 1.0f) * (p.gb ? *p.gb : 1.0f) * p.alpha_extra;
     int it = 0;
     for (int unit = blockIdx.x; unit < num_units; unit += gridDim.x, ++it) {
-      const int tile = unit % num_tiles;
+      const Unit w = decode_unit(p, unit, total_stages);
       const int ab = it % C::ACC_BUFS;
       const uint32_t use = (uint32_t)(it / C::ACC_BUFS);
-      float* const split_out = reinterpret_cast<float*>(p.C) + (int64_t)(unit / num_tiles) * p.split_stride;
+      OutView ov{p.C, p.ldc, p.c_dtype, p.col_scale};
+      float alpha = (p.ga ? *p.ga : 1.0f) * (p.gb ? *p.gb : 1.0f) * p.alpha_extra;
+      int64_t split_stride = p.split_stride;
+      if (w.g > 0) {
+        const Params::Extra& x = p.extra[w.g - 1];
+        ov = OutView{x.C, x.ldc, METIS_OUT_F32, nullptr};
+        alpha = (x.ga ? *x.ga : 1.0f) * (x.gb ? *x.gb : 1.0f);
+        split_stride = x.split_stride;
+      }
+      float* const split_out = reinterpret_cast<float*>(ov.C) + (int64_t)w.split * split_stride;
       const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&tmem_full[ab], use & 1u, abort_flag));
       if (!ok) {
         if (lane == 0) {
@@ -367,8 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc::tc_fence_after();
-      const int mb = tile % p.m_tiles;
-      const int nb = tile / p.m_tiles;
+      const int mb = w.mb, nb = w.nb;
       float v[kColsPerWarp];
       const int col0 = active ? h * kColsPerWarp : 0;
       if (active) {
@@ -395,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&tmem_empty[ab]);
       if (active)
-        store_rows(p, v, epi_smem + (warp - 2) * 1024, lane, (int64_t)mb * 128 + q * 32, (int64_t)nb * BN + col0,
+        store_rows(ov, v, epi_smem + (warp - 2) * 1024, lane, (int64_t)mb * 128 + q * 32, (int64_t)nb * BN + col0,
                    alpha, split_out);
     }
   }
@@ -785,13 +857,20 @@ bool make_map_1d_u64(CUtensorMap* map, const void* base, uint64_t bytes) {
 
 template <int BN>
 metis_status launch_spec(metis_ctx* ctx, const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mFa,
-                         const CUtensorMap& mFb, Params prm, double flops, bool profiled) {
+                         const CUtensorMap& mFb, Params prm, double flops, bool profiled,
+                         const CUtensorMap* extra_maps = nullptr) {
   using C = Cfg<BN>;
   auto kern = gemm_nvfp4_kernel<BN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   if (e != cudaSuccess) return check_cuda(ctx, e, "cudaFuncSetAttribute(gemm)");
-  const int units = prm.m_tiles * prm.n_tiles * prm.k_splits;
+  int units = prm.m_tiles * prm.n_tiles * prm.k_splits;
+  for (int e = 0; e < prm.n_extra; ++e) units += prm.extra[e].m_tiles * prm.extra[e].k_splits;
   const int grid = std::min(units, ctx->sm_count);
+  // extra_maps: A1, B1, A2, B2 of a grouped launch (unused slots repeat the first problem's)
+  const CUtensorMap& mA1 = extra_maps ? extra_maps[0] : mA;
+  const CUtensorMap& mB1 = extra_maps ? extra_maps[1] : mB;
+  const CUtensorMap& mA2 = extra_maps ? extra_maps[2] : mA;
+  const CUtensorMap& mB2 = extra_maps ? extra_maps[3] : mB;
   const bool prof = ctx->profiling && profiled;
   cudaEvent_t ev0 = nullptr, ev1 = nullptr;
   if (prof) {
@@ -799,7 +878,7 @@ metis_status launch_spec(metis_ctx* ctx, const CUtensorMap& mA, const CUtensorMa
     cudaEventCreate(&ev1);
     cudaEventRecord(ev0, ctx->stream);
   }
-  kern<<<grid, kThreads, C::SMEM, ctx->stream>>>(mA, mB, mFa, mFb, prm); count_launch();
+  kern<<<grid, kThreads, C::SMEM, ctx->stream>>>(mA, mB, mFa, mFb, mA1, mB1, mA2, mB2, prm); count_launch();
   if (prof) {
     cudaEventRecord(ev1, ctx->stream);
     ctx->prof_events.emplace_back(ev0, ev1);
@@ -827,7 +906,7 @@ metis_status launch_bn(metis_ctx* ctx, const GemmArgs& a) {
     mFa = mA;
     mFb = mB;
   }
-  Params prm;
+  Params prm{};
   prm.sfa = a.A->scales;
   prm.sfb = a.B->scales;
   prm.kb_tiles = K / 64;
@@ -947,6 +1026,59 @@ metis_status launch_bf16_bn(metis_ctx* ctx, const void* A, int64_t lda, int64_t 
   return launch_spec<BN>(ctx, mFa, mFb, mFa, mFb, prm, 2.0 * (double)rows * BN * (double)K, false);
 }
 
+// Up to three thin NVFP4 GeMMs (the same column width BN and contraction length, fp32
+// outputs, no fold) in one persistent launch: the CTAs take the problems' work units in
+// order, so the problems share the SMs without a launch between them.
+template <int BN>
+metis_status launch_group_bn(metis_ctx* ctx, const GemmArgs* g, int n) {
+  const int64_t K = g[0].A->inner;
+  CUtensorMap maps[6];
+  for (int i = 0; i < n; ++i) {
+    if (!make_map_2d(&maps[2 * i], CU_TENSOR_MAP_DATA_TYPE_UINT8, g[i].A->codes, K / 2, g[i].A->outer, K / 2, 128,
+                     128) ||
+        !make_map_2d(&maps[2 * i + 1], CU_TENSOR_MAP_DATA_TYPE_UINT8, g[i].B->codes, K / 2, g[i].B->outer, K / 2,
+                     128, BN))
+      return fail(ctx, METIS_ERR_CUDA, "cuTensorMapEncodeTiled failed for a grouped GeMM operand");
+  }
+  for (int i = n; i < 3; ++i) maps[2 * i] = maps[0], maps[2 * i + 1] = maps[1];
+  const int stages = (int)(K / 256);
+  auto splits_of = [&](const GemmArgs& a) {
+    const int per = (stages + std::max(a.k_splits, 1) - 1) / std::max(a.k_splits, 1);
+    return (stages + per - 1) / per;
+  };
+  Params prm{};
+  prm.sfa = g[0].A->scales;
+  prm.sfb = g[0].B->scales;
+  prm.kb_tiles = K / 64;
+  prm.ga = g[0].A->tensor_scale;
+  prm.gb = g[0].B->tensor_scale;
+  prm.alpha_extra = 1.0f;
+  prm.C = g[0].C;
+  prm.ldc = g[0].ldc;
+  prm.c_dtype = METIS_OUT_F32;
+  prm.m_tiles = (int)(g[0].A->outer / 128);
+  prm.n_tiles = 1;
+  prm.k_stages = stages;
+  prm.fold_stages = 0;
+  prm.k_splits = splits_of(g[0]);
+  prm.split_stride = g[0].split_stride;
+  prm.status = ctx->status;
+  prm.n_extra = n - 1;
+  for (int i = 1; i < n; ++i) {
+    Params::Extra& x = prm.extra[i - 1];
+    x.sfa = g[i].A->scales;
+    x.sfb = g[i].B->scales;
+    x.ga = g[i].A->tensor_scale;
+    x.gb = g[i].B->tensor_scale;
+    x.C = static_cast<float*>(g[i].C);
+    x.ldc = g[i].ldc;
+    x.m_tiles = (int)(g[i].A->outer / 128);
+    x.k_splits = splits_of(g[i]);
+    x.split_stride = g[i].split_stride;
+  }
+  return launch_spec<BN>(ctx, maps[0], maps[1], maps[0], maps[1], prm, 0.0, false, maps + 2);
+}
+
 }  // namespace
 
 int fp4_splits(metis_ctx* ctx, int64_t tiles, int stages) {
@@ -976,6 +1108,22 @@ metis_status launch_gemm_bf16(metis_ctx* ctx, const void* A, int64_t lda, int64_
     case 128: return launch_bf16_bn<128>(ctx, A, lda, rows, B, ldb, K, C, ldc, splits);
     case 256: return launch_bf16_bn<256>(ctx, A, lda, rows, B, ldb, K, C, ldc, splits);
     default: return fail(ctx, METIS_ERR_SHAPE, "bf16 GeMM width must be 32, 64, 128 or 256");
+  }
+}
+
+metis_status launch_gemm_nvfp4_group(metis_ctx* ctx, const GemmArgs* g, int n) {
+  if (n < 1 || n > 3) return fail(ctx, METIS_ERR_ARG, "a grouped GeMM takes 1 to 3 problems");
+  for (int i = 0; i < n; ++i) {
+    if (g[i].q_cols != g[0].q_cols || g[i].A->inner != g[0].A->inner || g[i].fold_k != 0 ||
+        g[i].c_dtype != METIS_OUT_F32 || g[i].col_scale || g[i].B->outer != 128 || g[i].A->outer % 128 ||
+        g[i].A->inner % 256)
+      return fail(ctx, METIS_ERR_SHAPE, "grouped GeMMs need one thin width, one K, fp32 outputs and no fold");
+  }
+  switch (g[0].q_cols) {
+    case 16: return launch_group_bn<16>(ctx, g, n);
+    case 32: return launch_group_bn<32>(ctx, g, n);
+    case 64: return launch_group_bn<64>(ctx, g, n);
+    default: return fail(ctx, METIS_ERR_SHAPE, "grouped GeMM width must be 16, 32 or 64");
   }
 }
 

@@ -105,6 +105,8 @@ struct GemmArgs {
 // work units per SM, no empty share.
 int fp4_splits(metis_ctx* ctx, int64_t tiles, int stages);
 metis_status launch_gemm_nvfp4(metis_ctx* ctx, const GemmArgs& a);
+// Up to three thin GeMMs (the same width 16/32/64 and K, fp32 outputs, no fold) in one launch.
+metis_status launch_gemm_nvfp4_group(metis_ctx* ctx, const GemmArgs* g, int n);
 // ---- selftest.cu ----
 metis_status launch_wait_timeout_selftest(metis_ctx* ctx, int64_t limit_cycles);
 // ---- mma_peak.cu ----

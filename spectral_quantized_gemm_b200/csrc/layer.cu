@@ -24,16 +24,15 @@
 namespace metis {
 namespace {
 
-// Decoded value of element (row t, column i) of a k x len factor NVFP4 tensor
-// (the transposed storage of a len x k factor).
-__device__ __forceinline__ float factor_value(const uint8_t* codes, const uint8_t* scales, float g, int64_t len,
-                                              int t, int64_t i) {
-  const uint8_t byte = codes[(int64_t)t * (len / 2) + (i >> 1)];
-  const uint32_t code = (i & 1) ? (byte >> 4) : (byte & 0xF);
+// Decoded value of a k x len factor NVFP4 tensor (the transposed storage of a len x k
+// factor) at row t, column r0 + r, from a block's staged copy of columns r0 .. r0 + 31:
+// 16 code bytes and 2 block scales per row t.
+__device__ __forceinline__ float staged_factor(const uint8_t* fcodes, const uint8_t* fscales, float g, int t, int r) {
+  const uint8_t byte = fcodes[t * 16 + (r >> 1)];
+  const uint32_t code = (r & 1) ? (byte >> 4) : (byte & 0xF);
   const uint32_t mag = code & 7u;
   const float e2m1 = mag < 4 ? 0.5f * (float)mag : (mag == 4 ? 2.0f : mag == 5 ? 3.0f : mag == 6 ? 4.0f : 6.0f);
-  const float s = e4m3_value(scales[scale_offset(t, i >> 4, len / 64)]);
-  const float v = e2m1 * s * g;
+  const float v = e2m1 * e4m3_value(fscales[t * 2 + (r >> 4)]) * g;
   return (code & 8u) ? -v : v;
 }
 
@@ -50,116 +49,156 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// Operands of the correction folded into the T_A GeMM (the second term of
-// T_A^T = Q(B_R)^T Q(R_A) S_A + Q(R_B) S_B Z^T S_A, Z = Q(R_A)^T Q(L_B)):
-//   blocks [0, zblocks):  FbZ (128 x fz_k; rows a < kA) = [Z S_B / alpha_TA hi | lo | 0],
-//                         alpha_TA the T_A GeMM's tensor scales; a thread per (a, u)
-//   blocks [zblocks, ..): FaZ rows = [Q(R_B) | Q(R_B) | 0] (bf16, exact), and the same two
-//                         copies of Q(R_B) into the main fold operand Fb at [2 kpA, 2 kpA + 2 kpB)
-// Z arrives as zsplits split-K partials of 128 x kpB, summed in order.  FbZ / FaZ are null
-// when A has no factors (no correction, zblocks = 0).
-constexpr int kRowsPerBlock = 32;
-__global__ void __launch_bounds__(256) zfold_kernel(const float* __restrict__ Zp, int zsplits, int zblocks, int kA,
-                                                    int kB, int kpA, int kpB, const float* __restrict__ SB,
-                                                    const float* gBres, const float* gRA, FactorView RB, int fz_k,
-                                                    __nv_bfloat16* __restrict__ FbZ, __nv_bfloat16* __restrict__ FaZ,
-                                                    __nv_bfloat16* __restrict__ Fb, int fold_k, int64_t q) {
-  if ((int)blockIdx.x < zblocks) {
-    const int t = blockIdx.x * 256 + threadIdx.x;
-    if (t >= 128 * kpB) return;
-    const int a = t / kpB, u = t - (t / kpB) * kpB;
-    float hi = 0.0f, lo = 0.0f;
-    if (a < kA && u < kB) {
-      const float inv_alpha = 1.0f / ((*gBres) * (*gRA));   // exact: powers of two
-      float z = 0.0f;
-      for (int s = 0; s < zsplits; ++s) z += Zp[((int64_t)s * 128 + a) * kpB + u];
-      const float v = z * SB[u] * inv_alpha;
-      hi = __bfloat162float(__float2bfloat16_rn(v));
-      lo = v - hi;
+// The main GeMM's fold operands, 64 rows per block (8 warps, 8 rows each, a lane owning
+// columns j and j + 1 of a kp-wide part and writing both of its copies):
+//   Fa rows i < p:  [Q(L_A) | Q(L_A) | T_B hi | T_B lo | 0] / alpha,
+//                   T_B = (sum of the splits of Q(A_R) Q(L_B)) S_B
+//   Fb rows i < q:  [T_A^T hi | T_A^T lo | Q(R_B) | Q(R_B) | 0],
+//                   T_A^T = (sum of the splits of Q(B_R)^T Q(R_A) + Q(R_B) S_B Z^T) S_A,
+//                   Z = Q(R_A)^T Q(L_B) (sum of its splits)
+// alpha = gA * gB, the tensor scales of the main FP4 GeMM.  The correction Q(R_B) S_B Z^T
+// (k_B terms per entry) is formed here in fp32: a block of Fb rows first stages
+// S_B[u] Z[a][u] in shared memory (u-major, so the lanes read consecutive a).
+constexpr int kFoldRows = 32;
+__global__ void __launch_bounds__(256) fold_assemble_kernel(
+    const float* __restrict__ TB, int bsplits, int64_t tb_stride, const float* __restrict__ TA, int asplits,
+    int64_t ta_stride, const float* __restrict__ Zp, int zsplits, const float* __restrict__ SA,
+    const float* __restrict__ SB, int kA, int kB, int kpA, int kpB, FactorView LA, FactorView RB, int64_t p, int64_t q,
+    int fold_k, const float* ga, const float* gb, __nv_bfloat16* __restrict__ Fa, __nv_bfloat16* __restrict__ Fb) {
+  __shared__ float zs[64 * 66];   // zs[u * 66 + a] = S_B[u] Z[a][u] (row pitch 66: fewer bank conflicts)
+  __shared__ float rbs[8][64];    // per warp: Q(R_B)(i, u) of the warp's current row
+  // the block's 32 rows of the factor it decodes (Q(L_A) on Fa rows, Q(R_B) on Fb rows):
+  // 16 code bytes and 2 scale bytes per factor column t, staged with coalesced loads
+  __shared__ uint8_t fcodes[64 * 16];
+  __shared__ uint8_t fscales[64 * 2];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t nbA = (p + kFoldRows - 1) / kFoldRows;
+  const bool is_a = (int64_t)blockIdx.x < nbA;
+  const int64_t r0 = (is_a ? (int64_t)blockIdx.x : (int64_t)blockIdx.x - nbA) * kFoldRows;
+  const bool corr = !is_a && Zp != nullptr;
+  if (corr) {
+    // thread (u = tid mod 64, a = tid / 64 + 4 t): a warp reads 32 consecutive u of one row
+    // of Z; all 16 x zsplits loads of a thread are independent, so they overlap
+    const int u = threadIdx.x & 63, a0 = threadIdx.x >> 6;
+    float z[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) z[t] = 0.0f;
+    if (u < kB) {
+      for (int sp = 0; sp < zsplits; ++sp) {
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          const int a = a0 + 4 * t;
+          if (a < kA) z[t] += Zp[((int64_t)sp * 128 + a) * kpB + u];
+        }
+      }
     }
-    FbZ[a * fz_k + u] = __float2bfloat16_rn(hi);
-    FbZ[a * fz_k + kpB + u] = __float2bfloat16_rn(lo);
-    for (int c = 2 * kpB + u; c < fz_k; c += kpB) FbZ[a * fz_k + c] = __float2bfloat16_rn(0.0f);
-    return;
+    const float sb = u < kB ? SB[u] : 0.0f;
+#pragma unroll
+    for (int t = 0; t < 16; ++t) zs[u * 66 + a0 + 4 * t] = sb * z[t];
+    __syncthreads();
   }
-  const int64_t i0 = (int64_t)(blockIdx.x - zblocks) * kRowsPerBlock;
-  const float g = *RB.g;
-  for (int e = threadIdx.x; e < kRowsPerBlock * kpB; e += blockDim.x) {
-    const int r = e / kpB, u = e - (e / kpB) * kpB;
-    const int64_t i = i0 + r;
-    if (i >= q) continue;
-    const __nv_bfloat16 v = __float2bfloat16_rn(u < kB ? factor_value(RB.codes, RB.scales, g, RB.len, u, i) : 0.0f);
-    Fb[i * fold_k + 2 * kpA + u] = v;
-    Fb[i * fold_k + 2 * kpA + kpB + u] = v;
-    if (FaZ) {
-      FaZ[i * fz_k + u] = v;
-      FaZ[i * fz_k + kpB + u] = v;
-      for (int c = 2 * kpB + u; c < fz_k; c += kpB) FaZ[i * fz_k + c] = __float2bfloat16_rn(0.0f);
+  {
+    const FactorView& F = is_a ? LA : RB;
+    const int kF = is_a ? kA : kB;
+    for (int e = threadIdx.x; e < kF * 4; e += blockDim.x) {
+      const int t = e >> 2, c = e & 3;
+      *reinterpret_cast<uint32_t*>(fcodes + t * 16 + c * 4) =
+          *reinterpret_cast<const uint32_t*>(F.codes + (int64_t)t * (F.len / 2) + r0 / 2 + c * 4);
     }
+    for (int e = threadIdx.x; e < kF * 2; e += blockDim.x) {
+      const int t = e >> 1, b = e & 1;
+      fscales[t * 2 + b] = F.scales[scale_offset(t, (r0 >> 4) + b, F.len / 64)];
+    }
+    __syncthreads();
   }
-}
-
-// The main GeMM's fold operands, one warp per output row:
-//   Fa rows i < p:  [Q(L_A) | Q(L_A) | T_B hi | T_B lo | 0] / alpha,  T_B = (sum of splits) S_B
-//   Fb rows i < q:  [T_A^T hi | T_A^T lo | (Q(R_B) copies, written by zfold_kernel) | 0],
-//                   T_A^T = (sum of splits) S_A
-// alpha = gA * gB, the tensor scales of the main FP4 GeMM.  A lane owns columns j and j + 1
-// of a kp-wide part and writes both of its copies (hi and lo, or the two Q(L_A) copies).
-__global__ void __launch_bounds__(256) assemble_kernel(const float* __restrict__ TB, int bsplits, int64_t tb_stride,
-                                                       const float* __restrict__ TA, int asplits, int64_t ta_stride,
-                                                       const float* __restrict__ SA, const float* __restrict__ SB,
-                                                       int kA, int kB, int kpA, int kpB, FactorView LA, int64_t p,
-                                                       int64_t q, int fold_k, const float* ga, const float* gb,
-                                                       __nv_bfloat16* __restrict__ Fa, __nv_bfloat16* __restrict__ Fb) {
-  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= p + q) return;
-  const bool is_a = row < p;
-  const int64_t i = is_a ? row : row - p;
-  __nv_bfloat16* dst = (is_a ? Fa : Fb) + i * fold_k;
   const float inv_alpha = is_a ? 1.0f / ((*ga) * (*gb)) : 1.0f;   // exact: a power of two
-  // part 1 (columns [0, 2 kpA)): Q(L_A) copies on Fa rows, T_A^T hi / lo on Fb rows
-  for (int j = 2 * lane; j < kpA; j += 64) {
-    float v0 = 0.0f, v1 = 0.0f;
+  for (int rr = warp; rr < kFoldRows; rr += 8) {
+    const int64_t i = r0 + rr;
+    if (i >= (is_a ? p : q)) break;
+    __nv_bfloat16* dst = (is_a ? Fa : Fb) + i * fold_k;
     if (is_a) {
-      const float gl = *LA.g;
-      if (j < kA) v0 = factor_value(LA.codes, LA.scales, gl, LA.len, j, i) * inv_alpha;
-      if (j + 1 < kA) v1 = factor_value(LA.codes, LA.scales, gl, LA.len, j + 1, i) * inv_alpha;
-      const uint32_t w = pack_bf16x2(v0, v1);
-      *reinterpret_cast<uint32_t*>(dst + j) = w;
-      *reinterpret_cast<uint32_t*>(dst + kpA + j) = w;
+      // Q(L_A) copies
+      const float gl = kA ? *LA.g : 1.0f;
+      for (int j = 2 * lane; j < kpA; j += 64) {
+        const float v0 = j < kA ? staged_factor(fcodes, fscales, gl, j, rr) * inv_alpha : 0.0f;
+        const float v1 = j + 1 < kA ? staged_factor(fcodes, fscales, gl, j + 1, rr) * inv_alpha : 0.0f;
+        const uint32_t w = pack_bf16x2(v0, v1);
+        *reinterpret_cast<uint32_t*>(dst + j) = w;
+        *reinterpret_cast<uint32_t*>(dst + kpA + j) = w;
+      }
+      // T_B hi / lo
+      for (int j = 2 * lane; j < kpB; j += 64) {
+        float v0 = 0.0f, v1 = 0.0f;
+        for (int sp = 0; sp < bsplits; ++sp) {
+          const float2 t = *reinterpret_cast<const float2*>(TB + sp * tb_stride + i * kpB + j);
+          v0 += t.x;
+          v1 += t.y;
+        }
+        v0 = j < kB ? v0 * SB[j] * inv_alpha : 0.0f;
+        v1 = j + 1 < kB ? v1 * SB[j + 1] * inv_alpha : 0.0f;
+        const float h0 = __bfloat162float(__float2bfloat16_rn(v0)), h1 = __bfloat162float(__float2bfloat16_rn(v1));
+        *reinterpret_cast<uint32_t*>(dst + 2 * kpA + j) = pack_bf16x2(h0, h1);
+        *reinterpret_cast<uint32_t*>(dst + 2 * kpA + kpB + j) = pack_bf16x2(v0 - h0, v1 - h1);
+      }
     } else {
-      for (int s = 0; s < asplits; ++s) {
-        const float2 t = *reinterpret_cast<const float2*>(TA + s * ta_stride + i * kpA + j);
-        v0 += t.x;
-        v1 += t.y;
+      // Q(R_B)(i, u) for u = lane and lane + 32 (exact in bf16)
+      const float gr = kB ? *RB.g : 1.0f;
+      const float rb0 = lane < kB ? staged_factor(fcodes, fscales, gr, lane, rr) : 0.0f;
+      const float rb1 = lane + 32 < kB ? staged_factor(fcodes, fscales, gr, lane + 32, rr) : 0.0f;
+      // T_A^T hi / lo: lane owns columns j, j + 1 (kpA <= 64, so at most one pair per lane)
+      const int j = 2 * lane;
+      float c0 = 0.0f, c1 = 0.0f;
+      if (corr) {
+        rbs[warp][lane] = rb0;
+        rbs[warp][lane + 32] = rb1;
+        __syncwarp();
+        if (j < kpA) {
+          // four partial sums break the FMA dependency chain (fixed order: bit-reproducible)
+          float p0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, p1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          int u = 0;
+          for (; u + 4 <= kB; u += 4) {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              const float r = rbs[warp][u + t];
+              const float2 z = *reinterpret_cast<const float2*>(zs + (u + t) * 66 + j);
+              p0[t] = fmaf(r, z.x, p0[t]);
+              p1[t] = fmaf(r, z.y, p1[t]);
+            }
+          }
+          for (; u < kB; ++u) {
+            const float r = rbs[warp][u];
+            const float2 z = *reinterpret_cast<const float2*>(zs + u * 66 + j);
+            p0[0] = fmaf(r, z.x, p0[0]);
+            p1[0] = fmaf(r, z.y, p1[0]);
+          }
+          c0 = (p0[0] + p0[1]) + (p0[2] + p0[3]);
+          c1 = (p1[0] + p1[1]) + (p1[2] + p1[3]);
+        }
+        __syncwarp();   // the buffer is rewritten for the warp's next row
       }
-      v0 = j < kA ? v0 * SA[j] : 0.0f;
-      v1 = j + 1 < kA ? v1 * SA[j + 1] : 0.0f;
-      const float h0 = __bfloat162float(__float2bfloat16_rn(v0)), h1 = __bfloat162float(__float2bfloat16_rn(v1));
-      *reinterpret_cast<uint32_t*>(dst + j) = pack_bf16x2(h0, h1);
-      *reinterpret_cast<uint32_t*>(dst + kpA + j) = pack_bf16x2(v0 - h0, v1 - h1);
-    }
-  }
-  // part 2 (columns [2 kpA, 2 kpA + 2 kpB)): T_B hi / lo on Fa rows (zfold_kernel fills Fb's)
-  if (is_a) {
-    for (int j = 2 * lane; j < kpB; j += 64) {
-      float v0 = 0.0f, v1 = 0.0f;
-      for (int s = 0; s < bsplits; ++s) {
-        const float2 t = *reinterpret_cast<const float2*>(TB + s * tb_stride + i * kpB + j);
-        v0 += t.x;
-        v1 += t.y;
+      if (j < kpA) {
+        float v0 = c0, v1 = c1;
+        for (int sp = 0; sp < asplits; ++sp) {
+          const float2 t = *reinterpret_cast<const float2*>(TA + sp * ta_stride + i * kpA + j);
+          v0 += t.x;
+          v1 += t.y;
+        }
+        v0 = j < kA ? v0 * SA[j] : 0.0f;
+        v1 = j + 1 < kA ? v1 * SA[j + 1] : 0.0f;
+        const float h0 = __bfloat162float(__float2bfloat16_rn(v0)), h1 = __bfloat162float(__float2bfloat16_rn(v1));
+        *reinterpret_cast<uint32_t*>(dst + j) = pack_bf16x2(h0, h1);
+        *reinterpret_cast<uint32_t*>(dst + kpA + j) = pack_bf16x2(v0 - h0, v1 - h1);
       }
-      v0 = j < kB ? v0 * SB[j] * inv_alpha : 0.0f;
-      v1 = j + 1 < kB ? v1 * SB[j + 1] * inv_alpha : 0.0f;
-      const float h0 = __bfloat162float(__float2bfloat16_rn(v0)), h1 = __bfloat162float(__float2bfloat16_rn(v1));
-      *reinterpret_cast<uint32_t*>(dst + 2 * kpA + j) = pack_bf16x2(h0, h1);
-      *reinterpret_cast<uint32_t*>(dst + 2 * kpA + kpB + j) = pack_bf16x2(v0 - h0, v1 - h1);
+      // Q(R_B) copies
+      for (int u = lane; u < kpB; u += 32) {
+        const __nv_bfloat16 v = __float2bfloat16_rn(u < 32 ? rb0 : rb1);
+        dst[2 * kpA + u] = v;
+        dst[2 * kpA + kpB + u] = v;
+      }
     }
+    // padding columns
+    for (int c = 2 * kpA + 2 * kpB + 2 * lane; c < fold_k; c += 64) *reinterpret_cast<uint32_t*>(dst + c) = 0u;
   }
-  // padding columns
-  for (int c = 2 * kpA + 2 * kpB + 2 * lane; c < fold_k; c += 64)
-    *reinterpret_cast<uint32_t*>(dst + c) = 0u;
 }
 
 int pad_rank(int k) { return k == 0 ? 0 : k <= 16 ? 16 : k <= 32 ? 32 : 64; }
@@ -199,53 +238,48 @@ metis_status run_linear(metis_ctx* ctx, const metis_operand* A, const metis_nvfp
 
   const bool corr = kA && kB;   // T_A picks up the correction Q(R_B) S_B Z^T S_A
   const int stagesK = (int)(K / 256);
-  const int fz_k = corr ? ((2 * kpB + 63) / 64) * 64 : 0;
-  const int zsplits = corr ? fp4_splits(ctx, 1, stagesK) : 0;
-  const int bsplits = kB ? fp4_splits(ctx, p / 128, stagesK) : 0;
-  const int asplits = kA ? fp4_splits(ctx, q / 128, stagesK + fz_k / 64) : 0;
-  const size_t need = 256 * 12 + (size_t)bsplits * p * kpB * 4 + (size_t)asplits * q * kpA * 4 +
-                      (size_t)zsplits * 128 * kpB * 4 + (size_t)q * fz_k * 2 + (size_t)128 * fz_k * 2 +
-                      (size_t)p * fold_k * 2 + (size_t)q * fold_k * 2;
+  // one split count for the three thin GeMMs of one grouped launch (about two units per SM)
+  const int64_t thin_tiles = (corr ? 1 : 0) + (kB ? p / 128 : 0) + (kA ? q / 128 : 0);
+  const int splits = fp4_splits(ctx, thin_tiles, stagesK);
+  const int zsplits = corr ? splits : 0, bsplits = kB ? splits : 0, asplits = kA ? splits : 0;
+  const size_t need = 256 * 8 + (size_t)bsplits * p * kpB * 4 + (size_t)asplits * q * kpA * 4 +
+                      (size_t)zsplits * 128 * kpB * 4 + (size_t)p * fold_k * 2 + (size_t)q * fold_k * 2;
   if ((s = ensure_workspace(ctx, need)) != METIS_OK) return s;
   Workspace ws{ctx->ws, ctx->ws_bytes};
   float* TB32 = static_cast<float*>(ws.take((size_t)std::max(bsplits, 1) * p * std::max(kpB, 1) * 4));
   float* TA32 = static_cast<float*>(ws.take((size_t)std::max(asplits, 1) * q * std::max(kpA, 1) * 4));
   float* Zp = static_cast<float*>(ws.take((size_t)std::max(zsplits, 1) * 128 * std::max(kpB, 1) * 4));
-  __nv_bfloat16* FaZ = static_cast<__nv_bfloat16*>(ws.take((size_t)q * std::max(fz_k, 64) * 2));
-  __nv_bfloat16* FbZ = static_cast<__nv_bfloat16*>(ws.take((size_t)128 * std::max(fz_k, 64) * 2));
   __nv_bfloat16* Fa = static_cast<__nv_bfloat16*>(ws.take((size_t)p * fold_k * 2));
   __nv_bfloat16* Fb = static_cast<__nv_bfloat16*>(ws.take((size_t)q * fold_k * 2));
   if (!Fb) return fail(ctx, METIS_ERR_WORKSPACE, "fold workspace layout");
   cudaStream_t st = ctx->stream;
 
+  // the thin GeMMs: Z = Q(R_A)^T Q(L_B) (128 x kpB), T_B = Q(A_R) Q(L_B) (p x kpB) and
+  // T_A^T / S_A = Q(B_R)^T Q(R_A) (q x kpA), as split-K fp32 partials, in one launch when
+  // their widths agree
+  GemmArgs thin[3];
+  int nthin = 0;
+  if (corr) thin[nthin++] = GemmArgs{RAq, LBq, nullptr, nullptr, 0, nullptr, Zp, kpB, METIS_OUT_F32, 1.0f, kpB,
+                                     zsplits, 128 * kpB};
+  if (kB) thin[nthin++] = GemmArgs{A_res, LBq, nullptr, nullptr, 0, nullptr, TB32, kpB, METIS_OUT_F32, 1.0f, kpB,
+                                   bsplits, p * kpB};
+  if (kA) thin[nthin++] = GemmArgs{B_res, RAq, nullptr, nullptr, 0, nullptr, TA32, kpA, METIS_OUT_F32, 1.0f, kpA,
+                                   asplits, q * kpA};
+  if (kpA == kpB || !kA || !kB) {
+    if ((s = launch_gemm_nvfp4_group(ctx, thin, nthin)) != METIS_OK) return s;
+  } else {
+    for (int i = 0; i < nthin; ++i)
+      if ((s = launch_gemm_nvfp4(ctx, thin[i])) != METIS_OK) return s;
+  }
   FactorView vLA{}, vRB{};
   if (kA) vLA = {LAq->codes, LAq->scales, LAq->tensor_scale, LAq->inner, kA};
   if (kB) vRB = {RBq->codes, RBq->scales, RBq->tensor_scale, RBq->inner, kB};
-  // Z = Q(R_A)^T Q(L_B) on the tensor cores (128 x kpB, split-K over the contraction length)
-  if (corr) {
-    GemmArgs g{RAq, LBq, nullptr, nullptr, 0, nullptr, Zp, kpB, METIS_OUT_F32, 1.0f, kpB, zsplits, 128 * kpB};
-    if ((s = launch_gemm_nvfp4(ctx, g)) != METIS_OK) return s;
-  }
-  if (kB) {
-    const int zblocks = corr ? (128 * kpB + 255) / 256 : 0;
-    zfold_kernel<<<(unsigned)(zblocks + (q + kRowsPerBlock - 1) / kRowsPerBlock), 256, 0, st>>>(
-        Zp, zsplits, zblocks, kA, kB, kpA, kpB, fb->S, B_res->tensor_scale, corr ? RAq->tensor_scale : nullptr,
-        vRB, fz_k, corr ? FbZ : nullptr, corr ? FaZ : nullptr, Fb, fold_k, q); count_launch();
-    // T_B = Q(A_R) Q(L_B)  (p x kpB partials; S_B applied when assembling)
-    GemmArgs g{A_res, LBq, nullptr, nullptr, 0, nullptr, TB32, kpB, METIS_OUT_F32, 1.0f, kpB, bsplits,
-               p * kpB};
-    if ((s = launch_gemm_nvfp4(ctx, g)) != METIS_OK) return s;
-  }
-  // T_A^T / S_A = Q(B_R)^T Q(R_A) + [Q(R_B) | Q(R_B)] [Z S_B hi | lo]^T / alpha_TA  (q x kpA partials)
-  if (kA) {
-    GemmArgs g{B_res, RAq, corr ? FaZ : nullptr, corr ? FbZ : nullptr, fz_k, nullptr, TA32, kpA, METIS_OUT_F32,
-               1.0f, kpA, asplits, q * kpA};
-    if ((s = launch_gemm_nvfp4(ctx, g)) != METIS_OK) return s;
-  }
-  assemble_kernel<<<(unsigned)((p + q + 7) / 8), 256, 0, st>>>(TB32, bsplits, p * kpB, TA32, asplits, q * kpA,
-                                                               kA ? fa->S : nullptr, kB ? fb->S : nullptr, kA, kB,
-                                                               kpA, kpB, vLA, p, q, fold_k, A_res->tensor_scale,
-                                                               B_res->tensor_scale, Fa, Fb); count_launch();
+  const int64_t blocks = (p + kFoldRows - 1) / kFoldRows + (q + kFoldRows - 1) / kFoldRows;
+  fold_assemble_kernel<<<(unsigned)blocks, 256, 0, st>>>(
+      TB32, bsplits, p * kpB, TA32, asplits, q * kpA, corr ? Zp : nullptr, zsplits, kA ? fa->S : nullptr,
+      kB ? fb->S : nullptr, kA, kB, kpA, kpB, vLA, vRB, p, q, fold_k, A_res->tensor_scale, B_res->tensor_scale, Fa,
+      Fb);
+  count_launch();
   if ((s = check_cuda(ctx, cudaGetLastError(), "fold preparation")) != METIS_OK) return s;
   GemmArgs g{A_res, B_res, Fa, Fb, fold_k, nullptr, C, ldc, c_dtype, 1.0f, q, 1, 0};
   return launch_gemm_nvfp4(ctx, g);
