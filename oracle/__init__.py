@@ -23,9 +23,13 @@ Modules, in the order the method uses them:
                    residual M_R = M - U S V^T.
 * ``metis``     -- the mixed-precision product for the forward, dX and dW
                    GEMMs, and the end-to-end layer.
+* ``lora_svd``  -- the LoRA-SVD linear projection W = W_res + beta L2 L1
+                   ("Full-Stack FP4" technical summary, section 2.1): the branch
+                   product, its gradients, the Cholesky-QR constraint and the
+                   randomized-SVD realignment.
 
 Parity status of every function is listed in its module header.  Nothing in
 this package is "parity unpinned" except where a header says so explicitly.
 """
 
-from . import philox, formats, nvfp4, linalg, decompose, metis  # noqa: F401
+from . import philox, formats, nvfp4, linalg, decompose, metis, lora_svd  # noqa: F401
