@@ -260,6 +260,47 @@ metis_status metis_linear_bwd(metis_ctx* ctx, const metis_operand* X, const meti
                               float* dW, int64_t lddw);
 
 /*
+ * LoRA-SVD linear projection ("Full-Stack FP4", gist.science technical summary, section
+ * 2.1): the weight is W = W_res + beta L2 L1 with the compact principal subspace L2 L1
+ * (L2: m x k, L1: k x n, fp32 row-major masters, used in bf16 on the tensor cores) and
+ * the residual W_res in NVFP4.  k in [1, 64].
+ *
+ * metis_lora_linear: one fused FP4 GeMM with the branch in its bf16 rank fold
+ *   which = 0 (forward):        C = Q(A) Q(B)^T + beta (M bf16(L2)) bf16(L1)
+ *       A = Q(X) row-wise (l x m), B = Q(W_res) column-wise (outer n, inner m), M = X.
+ *   which = 1 (input gradient): C = Q(A) Q(B)^T + beta (M bf16(L1)^T) bf16(L2)^T
+ *       A = Q(D) row-wise (l x n), B = Q(W_res) row-wise (outer m, inner n), M = D.
+ *   Q(A) Q(B)^T is decoded with the tensor scales, as in metis_gemm_nvfp4.  T (nullable,
+ *   l x k fp32): receives M bf16(L2) (which 0) or M bf16(L1)^T (which 1), the input of
+ *   metis_lora_branch_grad.  B.outer (the columns of C) must be a multiple of 256; M is
+ *   A.outer x A.inner bf16.  C: leading dimension ldc, type c_dtype.
+ * metis_lora_branch_grad: G = beta M^T T (c x k fp32; transpose_out != 0 writes G^T,
+ *   k x c) for M (p x c bf16) and T (p x k fp32), on the bf16 tensor cores (T as a bf16
+ *   hi/lo pair).  With M = X and T from which = 1 this is dL/dL2 = beta X^T D L1^T; with
+ *   M = D, T from which = 0 and transpose_out it is dL/dL1 = beta (X L2)^T D.
+ * metis_lora_constrain: the Cholesky-QR constraint, in place: L2 = Q R (CholQR in fp64,
+ *   dependent columns dropped), L2 <- Q, L1 <- R L1; the product L2 L1 is unchanged up
+ *   to rounding and L2 has orthonormal columns.
+ * metis_lora_realign: randomized-SVD realignment, in place.  W_eff = W_res + beta L2 L1
+ *   (fp32, leading dimension ldw); bf16(W_eff) is written to W_bf16 (m x n, caller
+ *   scratch) and decomposed by metis_decompose with refresh (params p, k = p->k, the
+ *   caller's factors f of shape m x n as buffers) into U S V^T; then L2 <- U,
+ *   L1 <- diag(S / beta) V^T and W_res <- W_eff - beta L2 L1 (fp32), so W_res + beta L2 L1
+ *   equals W_eff up to fp32 rounding.  beta must be nonzero.
+ * Errors: ERR_ARG (null, bad which, non-finite beta), ERR_SHAPE, ERR_ALIGN (16-byte
+ * aligned buffers).  Device: as metis_decompose for the realignment.
+ */
+metis_status metis_lora_linear(metis_ctx* ctx, int32_t which, const metis_nvfp4* A, const metis_nvfp4* B,
+                               const metis_matrix* M, const float* L2, const float* L1, int32_t k, float beta,
+                               float* T, void* C, int64_t ldc, int32_t c_dtype);
+metis_status metis_lora_branch_grad(metis_ctx* ctx, const metis_matrix* M, const float* T, int32_t k, float beta,
+                                    int32_t transpose_out, float* G);
+metis_status metis_lora_constrain(metis_ctx* ctx, float* L2, int64_t m, float* L1, int64_t n, int32_t k);
+metis_status metis_lora_realign(metis_ctx* ctx, float* W_res, int64_t m, int64_t n, int64_t ldw, float* L2,
+                                float* L1, int32_t k, float beta, const metis_decomp_params* p, uint32_t step,
+                                metis_factors* f, void* W_bf16);
+
+/*
  * Self-test of failure detection (no counterpart in the notes).  Every wait of the
  * tensor-core kernels is bounded: on expiry the kernel sets METIS_DEV_TIMEOUT in the
  * context's status word and returns normally.  This launches one CTA that waits on a

@@ -42,7 +42,8 @@ EXPORTED = ["metis_create", "metis_destroy", "metis_set_stream", "metis_status_s
             "metis_decompose", "metis_residual_quantize_nvfp4", "metis_quantize_nvfp4_f32", "metis_gemm_nvfp4",
             "metis_linear_fwd", "metis_linear_bwd", "metis_kernel_launches", "metis_profile_enable",
             "metis_profile_read", "metis_residual_quantize_nvfp4_noalloc", "metis_dequantize_nvfp4",
-            "metis_nvfp4_mma_peak", "metis_selftest_wait_timeout"]
+            "metis_nvfp4_mma_peak", "metis_selftest_wait_timeout", "metis_lora_linear",
+            "metis_lora_branch_grad", "metis_lora_constrain", "metis_lora_realign"]
 
 
 class Matrix(ctypes.Structure):
@@ -106,7 +107,12 @@ _fwd = _sig("metis_linear_fwd", c_i32, c_p, ctypes.POINTER(OperandStruct), ctype
             c_i64, c_i32)
 _bwd = _sig("metis_linear_bwd", c_i32, c_p, ctypes.POINTER(OperandStruct), ctypes.POINTER(OperandStruct),
             ctypes.POINTER(OperandStruct), c_p, c_i64, c_i32, c_p, c_i64)
-
+_lora_linear = _sig("metis_lora_linear", c_i32, c_p, c_i32, ctypes.POINTER(Nvfp4Struct), ctypes.POINTER(Nvfp4Struct),
+                    ctypes.POINTER(Matrix), c_p, c_p, c_i32, c_f32, c_p, c_p, c_i64, c_i32)
+_lora_grad = _sig("metis_lora_branch_grad", c_i32, c_p, ctypes.POINTER(Matrix), c_p, c_i32, c_f32, c_i32, c_p)
+_lora_constrain = _sig("metis_lora_constrain", c_i32, c_p, c_p, c_i64, c_p, c_i64, c_i32)
+_lora_realign = _sig("metis_lora_realign", c_i32, c_p, c_p, c_i64, c_i64, c_i64, c_p, c_p, c_i32, c_f32,
+                     ctypes.POINTER(DecompParams), c_u32, ctypes.POINTER(FactorsStruct), c_p)
 
 _launches = _sig("metis_kernel_launches", c_u64)
 _prof_enable = _sig("metis_profile_enable", c_i32, c_p, ctypes.c_int)
@@ -297,6 +303,42 @@ class Context:
     def linear_fwd(self, X, W, Y):
         dtype = OUT_F32 if Y.dtype == torch.float32 else OUT_BF16
         self._call(_fwd, ctypes.byref(X), ctypes.byref(W), _ptr(Y), Y.stride(0), dtype)
+
+    # -- LoRA-SVD linear projection (W = W_res + beta L2 L1) --------------------
+    @staticmethod
+    def _f32(t, name):
+        if t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError(f"{name}: expected a contiguous fp32 CUDA tensor")
+        return _ptr(t)
+
+    def lora_linear(self, which, A, B, M, L2, L1, beta, C, T=None):
+        """which 0: C = Q(X) Q(W_res) + beta (X L2) L1 (A = Q(X) row-wise, B = Q(W_res) column-wise,
+        M = X); which 1: C = Q(D) Q(W_res)^T + beta (D L1^T) L2^T (A = Q(D) row-wise, B = Q(W_res)
+        row-wise, M = D).  T (rows x k fp32, optional) receives X L2 or D L1^T."""
+        dtype = OUT_F32 if C.dtype == torch.float32 else OUT_BF16
+        self._call(_lora_linear, int(which), ctypes.byref(A.struct), ctypes.byref(B.struct),
+                   ctypes.byref(_matrix(M)), self._f32(L2, "L2"), self._f32(L1, "L1"), L2.shape[1], float(beta),
+                   None if T is None else self._f32(T, "T"), _ptr(C), C.stride(0), dtype)
+
+    def lora_branch_grad(self, M, T, beta, G, transpose_out=False):
+        """G = beta M^T T (cols x k), or its transpose (k x cols) with transpose_out."""
+        self._call(_lora_grad, ctypes.byref(_matrix(M)), self._f32(T, "T"), T.shape[1], float(beta),
+                   int(bool(transpose_out)), self._f32(G, "G"))
+
+    def lora_constrain(self, L2, L1):
+        """Cholesky-QR constraint in place: L2 = Q R -> L2 = Q, L1 = R L1."""
+        self._call(_lora_constrain, self._f32(L2, "L2"), L2.shape[0], self._f32(L1, "L1"), L1.shape[1],
+                   L2.shape[1])
+
+    def lora_realign(self, W_res, L2, L1, beta, factors, W_bf16, s, l_k, seed, operand_id, step, rounding=0):
+        """Randomized-SVD realignment in place (factors: m x n rank-k buffers; W_bf16: m x n scratch)."""
+        k = L2.shape[1]
+        p = DecompParams(k, s, l_k, seed, operand_id, rounding)
+        if W_bf16.dtype != torch.bfloat16 or not W_bf16.is_contiguous():
+            raise ValueError("W_bf16: expected a contiguous bf16 CUDA tensor")
+        self._call(_lora_realign, self._f32(W_res, "W_res"), W_res.shape[0], W_res.shape[1], W_res.stride(0),
+                   self._f32(L2, "L2"), self._f32(L1, "L1"), k, float(beta), ctypes.byref(p), int(step),
+                   ctypes.byref(factors.struct), _ptr(W_bf16))
 
     def linear_bwd(self, X, W, D, dX, dW):
         dtype = OUT_F32 if dX.dtype == torch.float32 else OUT_BF16

@@ -342,6 +342,79 @@ metis_status metis_linear_bwd(metis_ctx* ctx, const metis_operand* X, const meti
   return run_linear(ctx, X, X->colwise, D, D->colwise, true, false, dW, lddw, METIS_OUT_F32);
 }
 
+metis_status metis_lora_linear(metis_ctx* ctx, int32_t which, const metis_nvfp4* A, const metis_nvfp4* B,
+                               const metis_matrix* M, const float* L2, const float* L1, int32_t k, float beta,
+                               float* T, void* C, int64_t ldc, int32_t c_dtype) {
+  const metis::NvtxRange nvtx_range("metis_lora_linear");
+  metis_status s = enter(ctx);
+  if (s != METIS_OK) return s;
+  if (which != 0 && which != 1) return fail(ctx, METIS_ERR_ARG, "which must be 0 (forward) or 1 (input gradient)");
+  if (!A || !B || !M || !M->data || !L2 || !L1 || !C) return fail(ctx, METIS_ERR_ARG, "null argument");
+  if (k < 1 || k > 64) return fail(ctx, METIS_ERR_SHAPE, "LoRA rank must be in [1, 64]");
+  if (!std::isfinite(beta)) return fail(ctx, METIS_ERR_ARG, "beta must be finite");
+  const int64_t p = A->outer, K = A->inner, q = B->outer;
+  if (B->inner != K || K <= 0 || K % 256) return fail(ctx, METIS_ERR_SHAPE, "A.inner must equal B.inner and be a multiple of 256");
+  if ((s = check_dims(ctx, p, K)) != METIS_OK) return s;
+  if (q <= 0 || q % 256) return fail(ctx, METIS_ERR_SHAPE, "B.outer (the output columns) must be a multiple of 256");
+  if ((s = check_nvfp4(ctx, A, p, K, "A")) != METIS_OK) return s;
+  if ((s = check_nvfp4(ctx, B, q, K, "B")) != METIS_OK) return s;
+  if (M->rows != p || M->cols != K) return fail(ctx, METIS_ERR_SHAPE, "M must be A.outer x A.inner");
+  if (M->ld < M->cols || M->ld % 8 || !aligned16(M->data))
+    return fail(ctx, METIS_ERR_ALIGN, "bf16 matrix needs 16-byte alignment and ld % 8 == 0");
+  if (c_dtype != METIS_OUT_F32 && c_dtype != METIS_OUT_BF16) return fail(ctx, METIS_ERR_ARG, "bad output dtype");
+  if (ldc < q || ldc % (c_dtype == METIS_OUT_F32 ? 4 : 8) || !aligned16(C))
+    return fail(ctx, METIS_ERR_ALIGN, "output needs 16-byte alignment and a 16-byte multiple leading dimension");
+  if (!aligned16(L2) || !aligned16(L1) || (T && !aligned16(T)))
+    return fail(ctx, METIS_ERR_ALIGN, "L2, L1 and T must be 16-byte aligned");
+  return run_lora_linear(ctx, which, A, B, M, L2, L1, k, beta, T, C, ldc, c_dtype);
+}
+
+metis_status metis_lora_branch_grad(metis_ctx* ctx, const metis_matrix* M, const float* T, int32_t k, float beta,
+                                    int32_t transpose_out, float* G) {
+  const metis::NvtxRange nvtx_range("metis_lora_branch_grad");
+  metis_status s = enter(ctx);
+  if (s != METIS_OK) return s;
+  if (!M || !M->data || !T || !G) return fail(ctx, METIS_ERR_ARG, "null argument");
+  if (k < 1 || k > 64) return fail(ctx, METIS_ERR_SHAPE, "LoRA rank must be in [1, 64]");
+  if (!std::isfinite(beta)) return fail(ctx, METIS_ERR_ARG, "beta must be finite");
+  if ((s = check_dims(ctx, M->rows, M->cols)) != METIS_OK) return s;
+  if (M->ld < M->cols || M->ld % 8 || !aligned16(M->data))
+    return fail(ctx, METIS_ERR_ALIGN, "bf16 matrix needs 16-byte alignment and ld % 8 == 0");
+  if (!aligned16(T) || !aligned16(G)) return fail(ctx, METIS_ERR_ALIGN, "T and G must be 16-byte aligned");
+  return run_lora_branch_grad(ctx, M, T, k, beta, transpose_out != 0, G);
+}
+
+metis_status metis_lora_constrain(metis_ctx* ctx, float* L2, int64_t m, float* L1, int64_t n, int32_t k) {
+  const metis::NvtxRange nvtx_range("metis_lora_constrain");
+  metis_status s = enter(ctx);
+  if (s != METIS_OK) return s;
+  if (!L2 || !L1) return fail(ctx, METIS_ERR_ARG, "null argument");
+  if (k < 1 || k > 64) return fail(ctx, METIS_ERR_SHAPE, "LoRA rank must be in [1, 64]");
+  if ((s = check_dims(ctx, m, n)) != METIS_OK) return s;
+  if (!aligned16(L2) || !aligned16(L1)) return fail(ctx, METIS_ERR_ALIGN, "L2 and L1 must be 16-byte aligned");
+  return run_lora_constrain(ctx, L2, m, L1, n, k);
+}
+
+metis_status metis_lora_realign(metis_ctx* ctx, float* W_res, int64_t m, int64_t n, int64_t ldw, float* L2,
+                                float* L1, int32_t k, float beta, const metis_decomp_params* p, uint32_t step,
+                                metis_factors* f, void* W_bf16) {
+  const metis::NvtxRange nvtx_range("metis_lora_realign");
+  metis_status s = enter(ctx);
+  if (s != METIS_OK) return s;
+  if (!W_res || !L2 || !L1 || !p || !f || !W_bf16) return fail(ctx, METIS_ERR_ARG, "null argument");
+  if (!(std::isfinite(beta) && beta != 0.0f)) return fail(ctx, METIS_ERR_ARG, "beta must be finite and nonzero");
+  if ((s = check_dims(ctx, m, n)) != METIS_OK) return s;
+  if (ldw < n || ldw % 4 || !aligned16(W_res) || !aligned16(W_bf16) || !aligned16(L2) || !aligned16(L1))
+    return fail(ctx, METIS_ERR_ALIGN, "W_res, W_bf16, L2, L1 need 16-byte alignment and ldw % 4 == 0");
+  if (k < 1 || k > 64 || p->k != k || f->k != k)
+    return fail(ctx, METIS_ERR_SHAPE, "LoRA rank must be in [1, 64] and equal params.k and factors.k");
+  if (p->s < 0 || p->k + p->s > 128 || p->l_k < p->k + p->s || p->l_k > m || p->k + p->s > n)
+    return fail(ctx, METIS_ERR_SHAPE, "need k + s <= 128, k + s <= l_k <= m, k + s <= n");
+  if (p->rounding != 0 && p->rounding != 1) return fail(ctx, METIS_ERR_ARG, "rounding must be 0 or 1");
+  if ((s = check_factors(ctx, f, m, n)) != METIS_OK) return s;
+  return run_lora_realign(ctx, W_res, m, n, ldw, L2, L1, k, beta, p, step, f, W_bf16);
+}
+
 }  // extern "C"
 
 namespace metis {

@@ -127,6 +127,33 @@ metis_status launch_gemm_bf16(metis_ctx* ctx, const void* A, int64_t lda, int64_
 metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_decomp_params* p, int refresh,
                            uint32_t step, metis_factors* f);
 
+// Shared with lora.cu.  Mt (c x r bf16) = M^T for M (r x c bf16, leading dimension ld),
+// r and c multiples of 64.
+cudaError_t launch_transpose_bf16(const void* M, int64_t ld, int64_t r, int64_t c, void* Mt, cudaStream_t st);
+// out (2 kp x n bf16) = [F^T hi ; F^T lo] for F (n x k fp32), rows k .. kp - 1 of each half zero.
+cudaError_t launch_split_hi_lo_t(const float* F, int64_t n, int k, int kp, void* out, cudaStream_t st);
+// CholQR factor of a tall fp32 matrix A (n x w, row-major, w <= 64): G = A^T A (fp64,
+// w x w) and T = R^+ (fp64, w rows of leading dimension 128; upper triangular, a zero
+// column for a dropped dependent column), so that A T has orthonormal columns.  G and T
+// live in `scratch` (cholqr_factor_scratch_doubles(ctx, w) doubles).
+size_t cholqr_factor_scratch_doubles(metis_ctx* ctx, int w);
+// C (n x k2 fp32) = A (n x k1 fp32) T (fp64, leading dimension 128), fp64 sums.
+cudaError_t launch_times_small(const float* A, int64_t n, int k1, const double* T, int k2, float* C,
+                               cudaStream_t st);
+metis_status launch_cholqr_factor(metis_ctx* ctx, const float* A, int64_t n, int w, double* scratch,
+                                  double** G_out, double** T_out);
+
+// ---- lora.cu ----
+metis_status run_lora_linear(metis_ctx* ctx, int which, const metis_nvfp4* A, const metis_nvfp4* B,
+                             const metis_matrix* M, const float* L2, const float* L1, int k, float beta, float* T,
+                             void* C, int64_t ldc, int32_t c_dtype);
+metis_status run_lora_branch_grad(metis_ctx* ctx, const metis_matrix* M, const float* T, int k, float beta,
+                                  bool transpose_out, float* G);
+metis_status run_lora_constrain(metis_ctx* ctx, float* L2, int64_t m, float* L1, int64_t n, int k);
+metis_status run_lora_realign(metis_ctx* ctx, float* W, int64_t m, int64_t n, int64_t ldw, float* L2, float* L1,
+                              int k, float beta, const metis_decomp_params* p, uint32_t step, metis_factors* f,
+                              void* W_bf16);
+
 // ---- layer.cu ----
 metis_status run_linear(metis_ctx* ctx, const metis_operand* A, const metis_nvfp4* A_res, const metis_operand* B,
                         const metis_nvfp4* B_res, bool a_transposed_factors, bool b_transposed_factors, void* C,
