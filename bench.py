@@ -195,6 +195,94 @@ class Layer:
         return st
 
 
+class LoraStep:
+    """One training step of the LoRA-SVD projection W = W_res + beta L2 L1 ("Full-Stack
+    FP4", section 2.1) on the same batches: X, bf16(W_res) and D quantized to plain NVFP4
+    (both orientations) on three streams; then the forward and input-gradient products
+    with the bf16 branch in the FP4 GeMM's fold, the NVFP4 residual gradient, the two
+    branch gradients on the caller's stream; the Cholesky-QR constraint on a stream of
+    its own once the input-gradient product has read L2 and L1, so that it overlaps the
+    residual gradient, the branch gradients and the next step's quantization (none of
+    which read L2 or L1); the next forward product waits for it."""
+
+    NAMES = ("X", "W", "D")
+
+    def __init__(self, lib, ctx, cfg, batches, W):
+        self.lib, self.ctx, self.cfg, self.batches = lib, ctx, cfg, batches
+        dev = W.device
+        l, m, n, k = cfg["l"], cfg["m"], cfg["n"], cfg["k"]
+        self.k, self.beta = k, 1.0
+        gen = torch.Generator(device=dev).manual_seed(cfg["seed"] + 17)
+        self.L2 = torch.linalg.qr(torch.randn(m, k, device=dev, generator=gen))[0].contiguous()
+        self.L1 = (0.05 * torch.randn(k, n, device=dev, generator=gen)).contiguous()
+        self.mats = {"X": batches[0][0], "W": W, "D": batches[0][1]}
+        self.streams = {name: torch.cuda.Stream(dev) for name in self.NAMES}
+        self.ctxs = {}
+        for name in self.NAMES:
+            with torch.cuda.stream(self.streams[name]):
+                self.ctxs[name] = lib.Context(dev.index)
+        self.cstream = torch.cuda.Stream(dev)
+        with torch.cuda.stream(self.cstream):
+            self.cctx = lib.Context(dev.index)
+        self.c_done = None
+        self.q = {name: (ctx.new_nvfp4(*M.shape), ctx.new_nvfp4(M.shape[1], M.shape[0]))
+                  for name, M in self.mats.items()}
+        self.Y = torch.empty(l, n, dtype=torch.bfloat16, device=dev)
+        self.dX = torch.empty(l, m, dtype=torch.bfloat16, device=dev)
+        self.dW = torch.empty(m, n, dtype=torch.float32, device=dev)
+        self.Tx = torch.empty(l, k, dtype=torch.float32, device=dev)
+        self.Td = torch.empty(l, k, dtype=torch.float32, device=dev)
+        self.dL2 = torch.empty(m, k, dtype=torch.float32, device=dev)
+        self.dL1 = torch.empty(k, n, dtype=torch.float32, device=dev)
+
+    def step(self, t):
+        cfg, ctx = self.cfg, self.ctx
+        self.mats["X"], self.mats["D"] = self.batches[t % len(self.batches)]
+        main = torch.cuda.current_stream(self.Y.device)
+        start = torch.cuda.Event()
+        start.record(main)
+        ready = {}
+        for i, name in enumerate(self.NAMES):
+            stream = self.streams[name]
+            stream.wait_event(start)
+            with torch.cuda.stream(stream):
+                row, col = self.q[name]
+                self.ctxs[name].residual_quantize_nvfp4(self.mats[name], None, row, col,
+                                                        rounding=1 if name == "D" else 0, seed=cfg["seed"],
+                                                        operand_id=i, step=t, tensor_scale=0.0)
+                ready[name] = torch.cuda.Event()
+                ready[name].record(stream)
+        (xr, xc), (wr, wc), (dr, dc) = self.q["X"], self.q["W"], self.q["D"]
+        X, D = self.mats["X"], self.mats["D"]
+        main.wait_event(ready["X"])
+        main.wait_event(ready["W"])
+        self.finish()
+        ctx.lora_linear(0, xr, wc, X, self.L2, self.L1, self.beta, self.Y, T=self.Tx)
+        main.wait_event(ready["D"])
+        ctx.lora_linear(1, dr, wr, D, self.L2, self.L1, self.beta, self.dX, T=self.Td)
+        read = torch.cuda.Event()
+        read.record(main)
+        ctx.gemm_nvfp4(xc, dc, cfg["n"], self.dW)
+        ctx.lora_branch_grad(X, self.Td, self.beta, self.dL2)
+        ctx.lora_branch_grad(D, self.Tx, self.beta, self.dL1, transpose_out=True)
+        self.cstream.wait_event(read)
+        with torch.cuda.stream(self.cstream):
+            self.cctx.lora_constrain(self.L2, self.L1)
+            self.c_done = torch.cuda.Event()
+            self.c_done.record(self.cstream)
+
+    def finish(self):
+        """The caller's stream waits for the last step's constraint."""
+        if self.c_done is not None:
+            torch.cuda.current_stream(self.Y.device).wait_event(self.c_done)
+
+    def poll_device_status(self):
+        st = self.ctx.poll_device_status() | self.cctx.poll_device_status()
+        for c in self.ctxs.values():
+            st |= c.poll_device_status()
+        return st
+
+
 def max_over_ranks(value, world, device):
     """The largest value over all ranks (a time measured on each rank's device)."""
     if world == 1:
@@ -310,6 +398,23 @@ def run_ours(args, rank, world, device):
     plain_ms = max_over_ranks(plain_ms, world, device)
     status |= plain.poll_device_status()
 
+    # ---- the LoRA-SVD projection's training step on the same batches, same timing
+    lora = LoraStep(lib, ctx, cfg, dev_batches, dev_W)
+    for t in range(3):
+        lora.step(t)
+    barrier()
+    torch.cuda.synchronize(device)
+    q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    q0.record(stream)
+    for t in range(3, 3 + args.steps):
+        lora.step(t)
+    lora.finish()
+    q1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    lora_ms = max_over_ranks(q0.elapsed_time(q1) / args.steps, world, device)
+    status |= lora.poll_device_status()
+
     # the achievable FP4 MMA rate on this GPU (no memory traffic), beside the roofline
     mma_peak = ctx.nvfp4_mma_peak(iters=4096, reps=5)
     status |= ctx.poll_device_status()
@@ -352,6 +457,13 @@ def run_ours(args, rank, world, device):
             "metis_over_plain": round(ms_per_step / plain_ms, 4),
             "what": "the same step with k = 0: residual = operand, plain NVFP4 in both orientations, "
                     "three FP4 GeMMs without the rank fold"},
+        "lora_svd": {
+            "value": round(world * flops_per_step / (lora_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(lora_ms, 4), "k": cfg["k"],
+            "what": "LoRA-SVD projection (W = W_res + beta L2 L1, rank-k bf16 branch, NVFP4 residual) on the "
+                    "same batches: plain NVFP4 quantization of X, bf16(W_res), D; forward and dX with the "
+                    "branch in the FP4 GeMM fold; NVFP4 dW_res; branch gradients dL2, dL1; the Cholesky-QR "
+                    "constraint (on its own stream, overlapping the gradients and the next quantization)"},
         "decomposition": {
             "refresh_every": cfg["refresh_every"],
             "refresh_steps_timed": len(refresh_ms),

@@ -1475,37 +1475,20 @@ cudaError_t launch_split_hi_lo_t(const float* F, int64_t n, int k, int kp, void*
   return cudaGetLastError();
 }
 
-cudaError_t launch_times_small(const float* A, int64_t n, int k1, const double* T, int k2, float* C,
-                               cudaStream_t st) {
-  times_small_kernel<<<blocks_for(n * k2), 256, 0, st>>>(A, n, k1, T, k2, C);
-  count_launch();
-  return cudaGetLastError();
-}
+size_t gram_scratch_doubles(metis_ctx* ctx, int w) { return (size_t)(ctx->sm_count + 1) * w * w; }
 
-size_t cholqr_factor_scratch_doubles(metis_ctx* ctx, int w) {
-  return (size_t)ctx->sm_count * w * w + (size_t)w * w + (size_t)w * kMaxW;
-}
-
-metis_status launch_cholqr_factor(metis_ctx* ctx, const float* A, int64_t n, int w, double* scratch,
-                                  double** G_out, double** T_out) {
-  if (w < 1 || w > 64) return fail(ctx, METIS_ERR_SHAPE, "CholQR width must be in [1, 64]");
+metis_status launch_gram(metis_ctx* ctx, const float* A, int64_t n, int w, double* scratch, double** G_out) {
+  if (w < 1 || w > 64) return fail(ctx, METIS_ERR_SHAPE, "Gram width must be in [1, 64]");
   cudaStream_t st = ctx->stream;
   double* gpart = scratch;
   double* G = gpart + (size_t)ctx->sm_count * w * w;
-  double* T = G + (size_t)w * w;
   const int64_t chunks = (n + kGramRows - 1) / kGramRows;
   const int64_t per_block = ((chunks + ctx->sm_count - 1) / ctx->sm_count) * kGramRows;
   const int nb = (int)((n + per_block - 1) / per_block);
   gram_partial_kernel<1><<<nb, 256, 0, st>>>(A, n, w, per_block, gpart, ctx->status); count_launch();
   gram_reduce_kernel<<<(unsigned)((w * w + 7) / 8), 256, 0, st>>>(gpart, nb, w, G); count_launch();
-  cudaError_t e = cudaFuncSetAttribute(chol_inverse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)chol_smem_bytes(kSmallMaxN));
-  if (e != cudaSuccess) return check_cuda(ctx, e, "cudaFuncSetAttribute(chol_inverse_kernel)");
-  SmallOut so{T, nullptr, nullptr, nullptr, nullptr};
-  chol_inverse_kernel<<<1, kCholThreads, chol_smem_bytes(w), st>>>(G, w, so); count_launch();
   *G_out = G;
-  *T_out = T;
-  return check_cuda(ctx, cudaGetLastError(), "CholQR factor");
+  return check_cuda(ctx, cudaGetLastError(), "Gram");
 }
 
 }  // namespace metis

@@ -132,16 +132,10 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
 cudaError_t launch_transpose_bf16(const void* M, int64_t ld, int64_t r, int64_t c, void* Mt, cudaStream_t st);
 // out (2 kp x n bf16) = [F^T hi ; F^T lo] for F (n x k fp32), rows k .. kp - 1 of each half zero.
 cudaError_t launch_split_hi_lo_t(const float* F, int64_t n, int k, int kp, void* out, cudaStream_t st);
-// CholQR factor of a tall fp32 matrix A (n x w, row-major, w <= 64): G = A^T A (fp64,
-// w x w) and T = R^+ (fp64, w rows of leading dimension 128; upper triangular, a zero
-// column for a dropped dependent column), so that A T has orthonormal columns.  G and T
-// live in `scratch` (cholqr_factor_scratch_doubles(ctx, w) doubles).
-size_t cholqr_factor_scratch_doubles(metis_ctx* ctx, int w);
-// C (n x k2 fp32) = A (n x k1 fp32) T (fp64, leading dimension 128), fp64 sums.
-cudaError_t launch_times_small(const float* A, int64_t n, int k1, const double* T, int k2, float* C,
-                               cudaStream_t st);
-metis_status launch_cholqr_factor(metis_ctx* ctx, const float* A, int64_t n, int w, double* scratch,
-                                  double** G_out, double** T_out);
+// G = A^T A (fp64, w x w, full) of a tall fp32 matrix A (n x w, row-major, w <= 64),
+// deterministic; G lives in `scratch` (gram_scratch_doubles(ctx, w) doubles).
+size_t gram_scratch_doubles(metis_ctx* ctx, int w);
+metis_status launch_gram(metis_ctx* ctx, const float* A, int64_t n, int w, double* scratch, double** G_out);
 
 // ---- lora.cu ----
 metis_status run_lora_linear(metis_ctx* ctx, int which, const metis_nvfp4* A, const metis_nvfp4* B,

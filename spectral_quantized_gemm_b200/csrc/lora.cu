@@ -146,32 +146,166 @@ __global__ void lora_grad_reduce_kernel(const float* __restrict__ partial, int s
   G[e] = beta * a;
 }
 
-// L1 (k x n fp32, in place) <- R L1 with R = T^T G (k x k, fp64), which equals the upper
-// Cholesky factor of G = L2^T L2 on the kept columns (a dropped column has a zero column
-// in T, so its row of R is zero).  A thread owns one column of L1.
-__global__ void __launch_bounds__(256) lora_left_multiply_kernel(const double* __restrict__ T,
-                                                                 const double* __restrict__ G, int k,
-                                                                 float* __restrict__ L1, int64_t n) {
-  __shared__ double R[64][65];
-  for (int e = threadIdx.x; e < k * k; e += blockDim.x) {
-    const int j = e / k, t = e - (e / k) * k;
-    double a = 0.0;
-    for (int l = 0; l <= j; ++l) a = fma(T[l * 128 + j], G[l * k + t], a);   // T upper triangular
-    R[j][t] = a;
+// R (k x k upper, fp64, leading dimension 64): the Cholesky factor of G = L2^T L2
+// (G = R^T R) with the decomposition's CholQR rule for dependent columns: a pivot
+// d_j = G_jj - sum_{i<j} R_ij^2 not above 1e-12 * max_i G_ii drops column j (row j of R
+// zero).  And Rinv (same layout): the inverse of R on the kept rows and columns, zero
+// elsewhere, so that L2 Rinv has orthonormal kept columns and zero dropped ones.
+// One CTA of 256 threads, everything in shared memory, one barrier per pivot:
+//   factorization, j ascending: every thread reads d_j from the diagonal, then every
+//     (i, t), j < i <= t, takes A_it -= A_ji A_jt / d_j at once (a thread per entry,
+//     through a table of the trailing triangle's entries); rows are scaled at the end;
+//   inverse, j descending (R X = I, X starting as the identity): every (i, t),
+//     i < j <= t, takes X_it -= R_ij X_jt / R_jj, with row j of X still unscaled; the
+//     rows of X are scaled by 1 / R_jj at the end.
+constexpr double kLoraDropTol = 1e-12;
+constexpr int kLoraCholThreads = 256;
+constexpr size_t kLoraCholSmem = (size_t)2 * 64 * 65 * sizeof(double);
+__global__ void __launch_bounds__(kLoraCholThreads) lora_chol_kernel(const double* __restrict__ G, int k,
+                                                                     double* __restrict__ Rout,
+                                                                     double* __restrict__ Rinv) {
+  extern __shared__ double lora_smem[];
+  double(*A)[65] = reinterpret_cast<double(*)[65]>(lora_smem);
+  double(*X)[65] = reinterpret_cast<double(*)[65]>(lora_smem + 64 * 65);
+  __shared__ uint16_t pairs[64 * 65 / 2];   // (i << 8) | t over i <= t, rows in descending order
+  __shared__ double dinv[64];               // 1 / d_j, 0 for a dropped pivot
+  __shared__ double rinv[64];               // 1 / R_jj, 0 for a dropped pivot
+  __shared__ double gmax_s;
+  const int tid = threadIdx.x;
+  for (int e = tid; e < k * k; e += kLoraCholThreads) {
+    const int i = e / k, t = e - (e / k) * k;
+    A[i][t] = G[e];
+    X[i][t] = i == t ? 1.0 : 0.0;
+    // rows i' > i come first in the table: they hold (k - 1 - i)(k - i) / 2 entries
+    if (i <= t) pairs[(k - 1 - i) * (k - i) / 2 + (t - i)] = (uint16_t)((i << 8) | t);
+  }
+  if (tid < 32) {
+    double g = 0.0;
+    for (int j = tid; j < k; j += 32) g = fmax(g, G[j * k + j]);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) g = fmax(g, __shfl_xor_sync(0xffffffffu, g, off));
+    if (tid == 0) gmax_s = g;
   }
   __syncthreads();
-  const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= n) return;
-  float col[64];
-#pragma unroll
-  for (int t = 0; t < 64; ++t)
-    if (t < k) col[t] = L1[(int64_t)t * n + c];
+  const double tol = kLoraDropTol * gmax_s;
   for (int j = 0; j < k; ++j) {
-    double a = 0.0;
+    const double d = A[j][j];
+    const double di = (!(d > tol) || gmax_s == 0.0) ? 0.0 : 1.0 / d;
+    if (tid == 0) dinv[j] = di;
+    // the trailing triangle i > j: the first (k - 1 - j)(k - j) / 2 table entries (at most
+    // 8 per thread); all loads are issued before any store, so they overlap
+    const int cnt = (k - 1 - j) * (k - j) / 2;
+    double v[8];
+    int at[8];
 #pragma unroll
-    for (int t = 0; t < 64; ++t)
-      if (t < k) a = fma(R[j][t], (double)col[t], a);
-    L1[(int64_t)j * n + c] = (float)a;
+    for (int u = 0; u < 8; ++u) {
+      const int e = tid + u * kLoraCholThreads;
+      at[u] = -1;
+      if (e < cnt) {
+        const int i = pairs[e] >> 8, t = pairs[e] & 0xFF;
+        at[u] = i * 65 + t;
+        v[u] = fma(-A[j][i] * di, A[j][t], A[i][t]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (at[u] >= 0) (&A[0][0])[at[u]] = v[u];
+    __syncthreads();
+  }
+  // R_jj = sqrt(d_j), R_jt = A_jt / sqrt(d_j); a dropped row is zero
+  for (int e = tid; e < k * k; e += kLoraCholThreads) {
+    const int j = e / k, t = e - (e / k) * k;
+    if (t >= j) A[j][t] = dinv[j] == 0.0 ? 0.0 : A[j][t] * sqrt(dinv[j]);
+  }
+  for (int j = tid; j < k; j += kLoraCholThreads) rinv[j] = sqrt(dinv[j]);
+  __syncthreads();
+  for (int j = k - 1; j > 0; --j) {
+    const double ri = rinv[j];
+    const int w = k - j;   // j * w <= 1024 entries: at most 4 per thread
+    double v[4];
+    int at[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = tid + u * kLoraCholThreads;
+      at[u] = -1;
+      if (e < j * w) {
+        const int i = e / w, t = j + (e - (e / w) * w);
+        at[u] = i * 65 + t;
+        v[u] = fma(-A[i][j] * ri, X[j][t], X[i][t]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (at[u] >= 0) (&X[0][0])[at[u]] = v[u];
+    __syncthreads();
+  }
+  for (int e = tid; e < k * 64; e += kLoraCholThreads) {
+    const int i = e / 64, t = e - (e / 64) * 64;
+    Rout[e] = (t < k && t >= i) ? A[i][t] : 0.0;
+    Rinv[e] = (t < k && t >= i) ? X[i][t] * rinv[i] : 0.0;
+  }
+}
+
+// In place, a block per 32 rows of L2 (m x k): L2 <- L2 Rinv (Rinv upper triangular,
+// leading dimension 64; zero below the diagonal, so full-length sums are exact), fp32
+// sums of the fp32-rounded Rinv.  Thread (row r = tid / 8, g = tid % 8) forms the
+// outputs j = g, g + 8, ... of its row with independent accumulators.
+__global__ void __launch_bounds__(256) lora_times_rinv_kernel(const double* __restrict__ Rinv, int k,
+                                                              float* __restrict__ L2, int64_t m) {
+  __shared__ float ri[64][65];
+  __shared__ float rows[32][65];
+  const int64_t r0 = (int64_t)blockIdx.x * 32;
+  for (int e = threadIdx.x; e < k * k; e += blockDim.x) {
+    const int i = e / k, j = e - (e / k) * k;
+    ri[i][j] = (float)Rinv[i * 64 + j];
+  }
+  for (int e = threadIdx.x; e < 32 * k; e += blockDim.x) {
+    const int r = e / k, j = e - (e / k) * k;
+    rows[r][j] = r0 + r < m ? L2[(r0 + r) * k + j] : 0.0f;
+  }
+  __syncthreads();
+  const int r = threadIdx.x >> 3, g = threadIdx.x & 7;
+  float acc[8] = {};
+  for (int i = 0; i < k; ++i) {
+    const float x = rows[r][i];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (g + 8 * u < k) acc[u] = fmaf(x, ri[i][g + 8 * u], acc[u]);
+  }
+  if (r0 + r < m) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (g + 8 * u < k) L2[(r0 + r) * k + g + 8 * u] = acc[u];
+  }
+}
+
+// In place, a block per 32 columns of L1 (k x n): L1 <- R L1 (R upper triangular, leading
+// dimension 64, zero below the diagonal), fp32 sums of the fp32-rounded R.  Lane = column,
+// warp w forms the rows j = w, w + 8, ... with independent accumulators.
+__global__ void __launch_bounds__(256) lora_left_multiply_kernel(const double* __restrict__ R, int k,
+                                                                 float* __restrict__ L1, int64_t n) {
+  __shared__ float rs[64][65];
+  __shared__ float cols[64][33];
+  const int64_t c0 = (int64_t)blockIdx.x * 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int e = threadIdx.x; e < k * k; e += blockDim.x) {
+    const int j = e / k, t = e - (e / k) * k;
+    rs[j][t] = (float)R[j * 64 + t];
+  }
+  const bool in = c0 + lane < n;
+  for (int t = warp; t < k; t += 8) cols[t][lane] = in ? L1[(int64_t)t * n + c0 + lane] : 0.0f;
+  __syncthreads();
+  float acc[8] = {};
+  for (int t = 0; t < k; ++t) {
+    const float x = cols[t][lane];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (warp + 8 * u < k) acc[u] = fmaf(rs[warp + 8 * u][t], x, acc[u]);
+  }
+  if (in) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (warp + 8 * u < k) L1[(int64_t)(warp + 8 * u) * n + c0 + lane] = acc[u];
   }
 }
 
@@ -300,24 +434,25 @@ metis_status run_lora_branch_grad(metis_ctx* ctx, const metis_matrix* M, const f
 }
 
 metis_status run_lora_constrain(metis_ctx* ctx, float* L2, int64_t m, float* L1, int64_t n, int k) {
-  const size_t nd = cholqr_factor_scratch_doubles(ctx, k);
-  metis_status s = ensure_workspace(ctx, nd * 8 + (size_t)m * k * 4 + 2 * 256);
+  const size_t nd = gram_scratch_doubles(ctx, k);
+  metis_status s = ensure_workspace(ctx, nd * 8 + (size_t)2 * 64 * 64 * 8 + 3 * 256);
   if (s != METIS_OK) return s;
   Workspace ws{ctx->ws, ctx->ws_bytes};
   auto* scratch = static_cast<double*>(ws.take(nd * 8));
-  auto* Q = static_cast<float*>(ws.take((size_t)m * k * 4));
-  if (!Q) return fail(ctx, METIS_ERR_WORKSPACE, "LoRA constraint workspace layout");
-  double *G = nullptr, *Tinv = nullptr;
-  if ((s = launch_cholqr_factor(ctx, L2, m, k, scratch, &G, &Tinv)) != METIS_OK) return s;
+  auto* R = static_cast<double*>(ws.take((size_t)64 * 64 * 8));
+  auto* Rinv = static_cast<double*>(ws.take((size_t)64 * 64 * 8));
+  if (!Rinv) return fail(ctx, METIS_ERR_WORKSPACE, "LoRA constraint workspace layout");
   cudaStream_t st = ctx->stream;
-  cudaError_t e = launch_times_small(L2, m, k, Tinv, k, Q, st);   // Q = L2 R^+
-  if (e == cudaSuccess) {
-    lora_left_multiply_kernel<<<blocks_of(n), 256, 0, st>>>(Tinv, G, k, L1, n);   // L1 <- R L1
-    count_launch();
-    e = cudaGetLastError();
-  }
-  if (e == cudaSuccess) e = cudaMemcpyAsync(L2, Q, (size_t)m * k * 4, cudaMemcpyDeviceToDevice, st);
-  return check_cuda(ctx, e, "LoRA constraint");
+  double* G = nullptr;
+  if ((s = launch_gram(ctx, L2, m, k, scratch, &G)) != METIS_OK) return s;
+  cudaError_t e = cudaFuncSetAttribute(lora_chol_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kLoraCholSmem);
+  if (e != cudaSuccess) return check_cuda(ctx, e, "cudaFuncSetAttribute(lora_chol_kernel)");
+  lora_chol_kernel<<<1, kLoraCholThreads, kLoraCholSmem, st>>>(G, k, R, Rinv);
+  lora_times_rinv_kernel<<<blocks_of(m, 32), 256, 0, st>>>(Rinv, k, L2, m);
+  lora_left_multiply_kernel<<<blocks_of(n, 32), 256, 0, st>>>(R, k, L1, n);
+  count_launch(3);
+  return check_cuda(ctx, cudaGetLastError(), "LoRA constraint");
 }
 
 metis_status run_lora_realign(metis_ctx* ctx, float* W, int64_t m, int64_t n, int64_t ldw, float* L2, float* L1,
