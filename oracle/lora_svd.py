@@ -55,6 +55,16 @@ def bf16_round(x):
     return r.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
+def branch_input(which, M, L2, L1):
+    """T = M bf16(L2) (which 0) or M bf16(L1)^T (which 1): the branch's first product."""
+    M = np.asarray(M, dtype=np.float64)
+    if which == 0:
+        return M @ bf16_round(L2)
+    if which == 1:
+        return M @ bf16_round(L1).T
+    raise ValueError("which must be 0 or 1")
+
+
 def lora_linear(which, A_hat, B_hat, M, L2, L1, beta):
     """One product with the branch, from the decoded NVFP4 operands.
 
@@ -64,16 +74,8 @@ def lora_linear(which, A_hat, B_hat, M, L2, L1, beta):
     Returns (C, T) with T = M bf16(L2) or M bf16(L1)^T (p x k)."""
     A_hat = np.asarray(A_hat, dtype=np.float64)
     B_hat = np.asarray(B_hat, dtype=np.float64)
-    M = np.asarray(M, dtype=np.float64)
-    L2b, L1b = bf16_round(L2), bf16_round(L1)
-    if which == 0:
-        T = M @ L2b
-        branch = T @ L1b
-    elif which == 1:
-        T = M @ L1b.T
-        branch = T @ L2b.T
-    else:
-        raise ValueError("which must be 0 or 1")
+    T = branch_input(which, M, L2, L1)
+    branch = T @ bf16_round(L1) if which == 0 else T @ bf16_round(L2).T
     return A_hat @ B_hat.T + beta * branch, T
 
 

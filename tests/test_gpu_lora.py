@@ -185,3 +185,51 @@ def test_lora_svd_layer_trains(ctx):
         losses.append(loss.item())
     assert ctx.poll_device_status() == 0
     assert losses[-1] < 0.8 * losses[0]
+
+
+def test_lora_llama_up_full_size_sampled(ctx):
+    """LLaMA-3 8B MLP-up at full size (the benchmark's LoRA-SVD launches, k = 64):
+    256 sampled rows of Y and dX against the oracle on the decoded operands, the branch
+    gradients dL2 in full and dL1 on 256 sampled columns."""
+    from tests.gpu_helpers import dequant
+    cfg = synth.CONFIGS["llama3_8b_mlp_up"]
+    l, m, n, k, beta = cfg["l"], cfg["m"], cfg["n"], 64, 1.0
+    X, W, D = (synth.operand_matrix(cfg, name) for name in ("X", "W", "D"))
+    rng = np.random.default_rng(21)
+    L2 = torch.from_numpy((rng.standard_normal((m, k)) / np.sqrt(m)).astype(np.float32))
+    L1 = torch.from_numpy((rng.standard_normal((k, n)) * 0.05).astype(np.float32))
+    Xg, Wg, Dg, L2g, L1g = (t.cuda() for t in (X, W, D, L2, L1))
+    xr, _ = _quantize_both(ctx, Xg, 0)
+    wr, wc = _quantize_both(ctx, Wg, 1)
+    dr, _ = _quantize_both(ctx, Dg, 2)
+    Y = torch.empty(l, n, dtype=torch.float32, device="cuda")
+    dX = torch.empty(l, m, dtype=torch.float32, device="cuda")
+    Tx = torch.empty(l, k, dtype=torch.float32, device="cuda")
+    Td = torch.empty(l, k, dtype=torch.float32, device="cuda")
+    ctx.lora_linear(0, xr, wc, Xg, L2g, L1g, beta, Y, T=Tx)
+    ctx.lora_linear(1, dr, wr, Dg, L2g, L1g, beta, dX, T=Td)
+    dL2 = torch.empty(m, k, dtype=torch.float32, device="cuda")
+    dL1 = torch.empty(k, n, dtype=torch.float32, device="cuda")
+    ctx.lora_branch_grad(Xg, Td, beta, dL2)
+    ctx.lora_branch_grad(Dg, Tx, beta, dL1, transpose_out=True)
+    torch.cuda.synchronize()
+    assert ctx.poll_device_status() == 0
+
+    rows = np.sort(rng.choice(l, 256, replace=False))
+    Xn, Dn = X.double().numpy(), D.double().numpy()
+    L2n, L1n = L2.numpy(), L1.numpy()
+    x_hat = dequant(xr)[rows]
+    Y_ref, Tx_rows = lora_svd.lora_linear(0, x_hat, dequant(wc), Xn[rows], L2n, L1n, beta)
+    assert rel_fro(Y[rows].double().cpu().numpy(), Y_ref) < 1e-4
+    assert rel_fro(Tx[rows].double().cpu().numpy(), Tx_rows) < 1e-5
+    d_hat = dequant(dr)[rows]
+    dX_ref, Td_rows = lora_svd.lora_linear(1, d_hat, dequant(wr), Dn[rows], L2n, L1n, beta)
+    assert rel_fro(dX[rows].double().cpu().numpy(), dX_ref) < 1e-4
+    assert rel_fro(Td[rows].double().cpu().numpy(), Td_rows) < 1e-5
+    # the gradients from the oracle's own T (all rows)
+    Td_all = lora_svd.branch_input(1, Dn, L2n, L1n)
+    assert rel_fro(dL2.double().cpu().numpy(), lora_svd.branch_grad(Xn, Td_all, beta)) < 2e-5
+    cols = np.sort(rng.choice(n, 256, replace=False))
+    Tx_all = lora_svd.branch_input(0, Xn, L2n, L1n)
+    ref_dl1 = lora_svd.branch_grad(Dn[:, cols], Tx_all, beta).T
+    assert rel_fro(dL1[:, cols].double().cpu().numpy(), ref_dl1) < 2e-5
