@@ -23,8 +23,6 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
-#include <algorithm>
-
 #include "internal.h"
 
 namespace metis {
