@@ -61,60 +61,122 @@ def measured_peaks():
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+    """SM clock and clock-event (throttle) reasons of this GPU while the timed region runs.
+
+    Reads only.  With NVML (pynvml) a thread polls every ``period`` seconds and
+    ``stop(t0, t1)`` keeps the samples taken between the host times t0 (just before the
+    timed launches are issued) and t1 (after the closing synchronize), so the record covers
+    the timed region itself even when it lasts a few tens of milliseconds.  Without NVML it
+    falls back to ``nvidia-smi -lms 200`` over the same window (fewer samples)."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "HwSlowdown"), ("hw_thermal_slowdown", "HwThermalSlowdown"),
+               ("sw_thermal_slowdown", "SwThermalSlowdown"), ("sw_power_cap", "SwPowerCap"))
 
-    def __init__(self, device):
+    def __init__(self, device, period=0.002, nvml=None):
+        self.period = period
+        self.samples = []          # (host time, sm MHz, max sm MHz, set of reason names)
+        self.proc = None
+        self.thread = None
+        self.running = False
         try:
             uuid = str(torch.cuda.get_device_properties(device).uuid)
             self.ident = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
         except Exception:
-            self.ident = str(device.index)
-        self.proc = None
-        self.lines = []
+            self.ident = str(getattr(device, "index", 0))
+        self.nvml, self.handle = None, None
+        try:
+            if nvml is None:
+                import pynvml as nvml
+            nvml.nvmlInit()
+            self.handle = nvml.nvmlDeviceGetHandleByUUID(self.ident)
+            self.nvml = nvml
+            self._sample_nvml()          # every query the poll makes works here, or NVML is not used
+            self.samples.clear()
+        except Exception:
+            self.nvml = None
+
+    def _reason_bits(self):
+        nv = self.nvml
+        out = []
+        for name, suffix in self.REASONS:
+            bit = getattr(nv, "nvmlClocksEventReason" + suffix, None)
+            if bit is None:
+                bit = getattr(nv, "nvmlClocksThrottleReason" + suffix)
+            out.append((name, bit))
+        return out
+
+    def _sample_nvml(self):
+        nv, h = self.nvml, self.handle
+        reasons_fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        t = time.perf_counter()
+        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+        smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        active = reasons_fn(h)
+        self.samples.append((t, float(sm), float(smax), {name for name, bit in self._reason_bits() if active & bit}))
+
+    def _poll_nvml(self):
+        while self.running:
+            try:
+                self._sample_nvml()
+            except Exception:
+                return
+            time.sleep(self.period)
+
+    def _read_smi(self):
+        names = [name for name, _ in self.REASONS]
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.strip().split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm, smax = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            self.samples.append((time.perf_counter(), sm, smax,
+                                 {nm for nm, val in zip(names, parts[5:9]) if val.lower() == "active"}))
 
     def start(self):
+        self.running = True
+        if self.nvml is not None:
+            self.thread = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.thread.start()
+            return
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.ident}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread = threading.Thread(target=self._read_smi, daemon=True)
             self.thread.start()
         except (OSError, FileNotFoundError):
             self.proc = None
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
-    def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.thread.join(timeout=2)
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
+    def stop(self, t0=None, t1=None):
+        self.running = False
+        if self.proc is not None:
+            self.proc.terminate()
             try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+        if self.nvml is None and self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no NVML and no nvidia-smi"], "samples": 0}
+        inside = [x for x in self.samples if (t0 is None or x[0] >= t0) and (t1 is None or x[0] <= t1)]
+        window = "timed region"
+        if not inside:                       # nothing landed inside: report the nearest samples
+            inside, window = self.samples, "around the timed region"
+        sm = [x[1] for x in inside]
+        reasons = set().union(*[x[3] for x in inside]) if inside else set()
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": inside[-1][2] if inside else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "source": ("nvml, every %.0f ms" % (1e3 * self.period)) if self.nvml else "nvidia-smi, every 200 ms",
+                "window": window}
 
 
 # ------------------------------------------------------------------ our arm
@@ -326,19 +388,21 @@ def run_ours(args, rank, world, device):
     # ---- timed region: inputs resident in HBM
     clocks = ClockSampler(device)
     clocks.start()
-    time.sleep(0.3)
+    time.sleep(0.05)
     ctx.profile_enable(True)
     launches0 = lib.kernel_launches()
     barrier()
     torch.cuda.synchronize(device)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t_region0 = time.perf_counter()
     ev0.record(stream)
     for i, t in enumerate(range(args.warmup, args.warmup + args.steps)):
         step_ev[i].record(stream)     # a step's operand work starts after the previous step's GeMMs
         layer.step(t)
     ev1.record(stream)
     torch.cuda.synchronize(device)
+    t_region1 = time.perf_counter()
     barrier()
     bounds = step_ev + [ev1]
     step_ms = [bounds[i].elapsed_time(bounds[i + 1]) for i in range(args.steps)]
@@ -347,7 +411,7 @@ def run_ours(args, rank, world, device):
     launches = lib.kernel_launches() - launches0
     gemm_ms, gemm_n, gemm_flops = ctx.profile_read()
     ctx.profile_enable(False)
-    clk = clocks.stop()
+    clk = clocks.stop(t_region0, t_region1)
     ms = ev0.elapsed_time(ev1)
     ms = max_over_ranks(ms, world, device)
     ms_per_step = ms / args.steps
