@@ -233,3 +233,41 @@ def test_lora_llama_up_full_size_sampled(ctx):
     Tx_all = lora_svd.branch_input(0, Xn, L2n, L1n)
     ref_dl1 = lora_svd.branch_grad(Dn[:, cols], Tx_all, beta).T
     assert rel_fro(dL1[:, cols].double().cpu().numpy(), ref_dl1) < 2e-5
+
+
+def test_lora_validation(ctx, metis_lib):
+    """Host-side checks of the LoRA-SVD calls return their status before any launch, and
+    the context stays usable afterwards."""
+    l, m, n, k = 256, 256, 512, 8
+    X = torch.zeros(l, m, dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros(m, n, dtype=torch.bfloat16, device="cuda")
+    xr, _ = _quantize_both(ctx, X, 0)
+    _, wc = _quantize_both(ctx, W, 1)
+    L2 = torch.zeros(m, k, device="cuda")
+    L1 = torch.zeros(k, n, device="cuda")
+    Y = torch.empty(l, n, device="cuda")
+
+    def status(fn, *args, **kw):
+        with pytest.raises(metis_lib.MetisError) as e:
+            fn(*args, **kw)
+        return e.value.status
+
+    assert status(ctx.lora_linear, 2, xr, wc, X, L2, L1, 1.0, Y) == 1                     # which
+    assert status(ctx.lora_linear, 0, xr, wc, X, torch.zeros(m, 65, device="cuda"),
+                  torch.zeros(65, n, device="cuda"), 1.0, Y) == 2                         # rank 65
+    assert status(ctx.lora_linear, 0, xr, wc, X, L2, L1, float("nan"), Y) == 1           # beta
+    w128c = ctx.new_nvfp4(128, m)     # a B operand with 128 output columns (never read)
+    assert status(ctx.lora_linear, 0, xr, w128c, X, L2, torch.zeros(k, 128, device="cuda"), 1.0,
+                  torch.empty(l, 128, device="cuda")) == 2                                # 128 output columns
+    assert status(ctx.lora_linear, 0, xr, wc, X[:, :128], L2, L1, 1.0, Y) == 2           # M is not l x m
+    assert status(ctx.lora_linear, 0, xr, wc, X, L2, L1, 1.0, torch.empty(l, n - 4, device="cuda")) == 3
+    assert status(ctx.lora_branch_grad, torch.zeros(200, m, dtype=torch.bfloat16, device="cuda"),
+                  torch.zeros(200, k, device="cuda"), 1.0, torch.zeros(m, k, device="cuda")) == 2
+    assert status(ctx.lora_constrain, torch.zeros(200, k, device="cuda"), L1) == 2
+    f = metis_lib.Factors(m, n, k)
+    Wb = torch.empty(m, n, dtype=torch.bfloat16, device="cuda")
+    assert status(ctx.lora_realign, torch.zeros(m, n, device="cuda"), L2, L1, 0.0, f, Wb, s=8, l_k=m,
+                  seed=0, operand_id=1, step=0) == 1                                      # beta = 0
+    ctx.lora_linear(0, xr, wc, X, L2, L1, 1.0, Y)
+    torch.cuda.synchronize()
+    assert ctx.poll_device_status() == 0 and torch.count_nonzero(Y).item() == 0
