@@ -1,5 +1,5 @@
 // Thin inline-PTX wrappers for the sm_100a tensor-core path: mbarriers with
-// bounded waits, TMA tile loads (no multicast), bulk copies, tensor-memory
+// bounded waits, TMA tile loads (one destination CTA each), bulk copies, tensor-memory
 // allocation, tcgen05 MMA / copy / load, and the shared-memory matrix and
 // instruction descriptors.
 #pragma once
@@ -66,7 +66,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
-// 2-D TMA tile load into shared memory, completing on `bar` (no multicast).
+// 2-D TMA tile load into this CTA's shared memory, completing on `bar`.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t x,
                                             int32_t y) {
   asm volatile(
