@@ -140,3 +140,19 @@ def test_realign_keeps_w_and_recovers_an_exact_rank_k_split():
     Wn2, L2n2, L1n2, S2 = lora_svd.realign(noise, L2, L1, beta, k, s, seed=7, operand_id=1, step=0)
     assert np.allclose(Wn2 + beta * L2n2 @ L1n2, noise + W_eff, atol=1e-12)
     assert np.allclose(S2, np.linalg.svd(noise + W_eff, compute_uv=False)[:k], rtol=1e-2)
+
+
+def test_realign_decomposes_the_bf16_copy():
+    """A constant W_eff = c (c = 1 + 2^-8 + 2^-10, not a bf16 number; bf16(c) = 1 + 2^-7):
+    the decomposition sees bf16(W_eff), a rank-1 matrix with singular value
+    bf16(c) sqrt(m n), and the new residual is exactly the rounding c - bf16(c)."""
+    m, n, beta = 64, 48, 2.0
+    c = 1.0 + 2.0 ** -8 + 2.0 ** -10
+    cb = 1.0 + 2.0 ** -7
+    assert lora_svd.bf16_round(np.float32(c)) == cb
+    W_res = np.full((m, n), c)
+    Wn, L2n, L1n, S = lora_svd.realign(W_res, np.zeros((m, 1)), np.zeros((1, n)), beta, 1, 4, seed=3,
+                                       operand_id=1, step=0)
+    assert abs(S[0] - cb * np.sqrt(m * n)) <= 1e-12 * S[0]
+    assert np.allclose(Wn, c - cb, rtol=0, atol=1e-12)
+    assert np.allclose(beta * L2n @ L1n, cb, rtol=0, atol=1e-12)
