@@ -102,3 +102,25 @@ def test_metis_preserves_small_singular_components():
     err_m = np.linalg.norm((xm - X) @ T) / np.linalg.norm(X @ T)
     err_p = np.linalg.norm((xp - X) @ T) / np.linalg.norm(X @ T)
     assert err_m < 0.75 * err_p
+
+
+def test_weight_gradient_uses_the_column_wise_residual():
+    """Reading R5: each GeMM reads the quantization with 16-blocks along its own
+    contraction dimension.  X below is exact in column-wise blocks (16 rows of a column
+    share a power-of-two scale) but lossy in row-wise blocks (columns of scale 2^6 and
+    2^-6 side by side); D is exact column-wise.  So dW = X^T D exactly, while the
+    row-wise quantization of X would lose its small columns."""
+    rng = np.random.default_rng(7)
+    l, m, n = 64, 32, 48
+    mags = formats.E2M1_MAGNITUDES
+    expo = np.where(np.arange(m) % 2 == 0, 6.0, -6.0)
+    X = mags[rng.integers(0, 8, size=(l, m))] * rng.choice([-1.0, 1.0], size=(l, m))
+    X[::16, :] = 6.0
+    X = X * 2.0 ** expo[None, :]
+    D = mags[rng.integers(0, 8, size=(l, n))] * rng.choice([-1.0, 1.0], size=(l, n))
+    D[::16, :] = 6.0
+    W = rng.standard_normal((m, n))
+    ops = [metis.prepare_operand(M, None) for M in (X, W, D)]
+    _, dW = metis.linear_bwd(*ops)
+    assert np.array_equal(dW, X.T @ D)
+    assert not np.array_equal(metis.dequant_residual(ops[0], "row"), X)   # the row-wise one is lossy
