@@ -124,3 +124,35 @@ def test_weight_gradient_uses_the_column_wise_residual():
     _, dW = metis.linear_bwd(*ops)
     assert np.array_equal(dW, X.T @ D)
     assert not np.array_equal(metis.dequant_residual(ops[0], "row"), X)   # the row-wise one is lossy
+
+
+def _exact_one_way(rows, cols, rng, exact):
+    """Grid values whose 16-blocks are exact in one orientation only: exact="row" gives
+    every row a power-of-two scale of its own (2^6 or 2^-6, alternating), so row-wise
+    blocks are exact and column-wise blocks, which mix the two, are not; exact="col"
+    does the same per column."""
+    mags = formats.E2M1_MAGNITUDES
+    v = mags[rng.integers(0, 8, size=(rows, cols))] * rng.choice([-1.0, 1.0], size=(rows, cols))
+    if exact == "row":
+        v[:, ::16] = 6.0
+        return v * np.where(np.arange(rows) % 2 == 0, 2.0 ** 6, 2.0 ** -6)[:, None]
+    v[::16, :] = 6.0
+    return v * np.where(np.arange(cols) % 2 == 0, 2.0 ** 6, 2.0 ** -6)[None, :]
+
+
+def test_forward_and_input_gradient_use_their_own_orientations():
+    """Reading R5 for the other two GeMMs: Y = X W reads X row-wise and W column-wise;
+    dX = D W^T reads D and W row-wise.  With each operand exact only in the orientation
+    its GeMM should read, both products are exact."""
+    rng = np.random.default_rng(8)
+    l, m, n = 64, 48, 32
+    X, W = _exact_one_way(l, m, rng, "row"), _exact_one_way(m, n, rng, "col")
+    ops = [metis.prepare_operand(M, None) for M in (X, W)]
+    assert np.array_equal(metis.linear_fwd(*ops), X @ W)
+    assert not np.array_equal(metis.dequant_residual(ops[0], "col"), X)
+    assert not np.array_equal(metis.dequant_residual(ops[1], "row"), W)
+    D, W2 = _exact_one_way(l, n, rng, "row"), _exact_one_way(m, n, rng, "row")
+    ops = [metis.prepare_operand(M, None) for M in (X, W2, D)]
+    dX, _ = metis.linear_bwd(*ops)
+    assert np.array_equal(dX, D @ W2.T)
+    assert not np.array_equal(metis.dequant_residual(ops[2], "col"), D)
