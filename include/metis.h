@@ -135,8 +135,12 @@ typedef struct {
  * refresh != 0: sample l_k rows (Philox), draw Omega ~ N(0,1) (Philox + Box-Muller),
  *   sketch Y = M_s Omega, CholQR(Y) = Q R, Bm = Q^T M_s, CholQR(Bm^T) = Q2 R2,
  *   one-sided Jacobi SVD of R2^T, V = Q2 W'[:, :k].
- * Every call: P = M V, CholQR(P) = Q_P R_P, Jacobi SVD R_P = U_r S_r V_r^T,
- *   U = Q_P U_r, S = S_r, V <- V V_r (sign-fixed), then Uq and Vq.
+ * Every call: P = M V, then the k x k symmetric eigenproblem of the Gram matrix
+ *   G = P^T P = V_r diag(S_r^2) V_r^T (two-sided Jacobi in fp64; an eigenvalue at or
+ *   below 1e-12 * lambda_max counts as zero and gives a zero column), U = P V_r
+ *   diag(1 / S_r), S = S_r, V <- V V_r (sign-fixed), then Uq and Vq.  This equals the
+ *   route CholQR(P) = Q_P R_P, SVD R_P = U_r S_r V_r^T, U = Q_P U_r of the method's
+ *   statement (same U, S, V up to rounding and signs).
  * `step` enters the Philox counters (row sample, Omega, stochastic rounding).
  * Errors: ERR_SHAPE for k/s/l_k outside the limits; device: METIS_DEV_NONFINITE,
  * METIS_DEV_NUMERIC.

@@ -57,18 +57,26 @@ def sample_rows(rows, l_k, seed, operand_id, step):
     return np.sort(order[:l_k]).astype(np.int64)
 
 
+def box_muller(a, b):
+    """Two N(0,1) draws (fp64) from two 32-bit words a, b (arrays of equal shape).
+
+    u1 = (a + 1) 2^-32 lies in (0, 1], so the logarithm is finite for every word
+    (a = 0xffffffff gives u1 = 1 and radius 0); u2 = b 2^-32 lies in [0, 1).
+    """
+    u1 = (np.asarray(a, dtype=np.float64) + 1.0) * 2.0 ** -32
+    u2 = np.asarray(b, dtype=np.float64) * 2.0 ** -32
+    rad = np.sqrt(-2.0 * np.log(u1))
+    return rad * np.cos(2.0 * np.pi * u2), rad * np.sin(2.0 * np.pi * u2)
+
+
 def omega(cols, width, seed, operand_id, step):
     n = cols * width
     ncalls = (n + 3) // 4
     w = philox.stream_words(seed, philox.tag(operand_id, philox.PURPOSE_OMEGA), step,
-                            np.arange(ncalls, dtype=np.uint64)).astype(np.float64)
+                            np.arange(ncalls, dtype=np.uint64))
     out = np.empty(ncalls * 4, dtype=np.float64)
     for first, second, dst in ((0, 1, 0), (2, 3, 2)):
-        u1 = (w[:, first] + 1.0) * 2.0 ** -32
-        u2 = w[:, second] * 2.0 ** -32
-        rad = np.sqrt(-2.0 * np.log(u1))
-        out[dst::4] = rad * np.cos(2.0 * np.pi * u2)
-        out[dst + 1::4] = rad * np.sin(2.0 * np.pi * u2)
+        out[dst::4], out[dst + 1::4] = box_muller(w[:, first], w[:, second])
     return out[:n].astype(np.float32).reshape(cols, width)
 
 

@@ -40,6 +40,35 @@ def test_omega_box_muller_structure_and_moments():
     assert np.allclose(r2, -2 * np.log(u1), rtol=1e-6)
 
 
+def test_box_muller_at_the_extreme_words():
+    """u1 = (a + 1) 2^-32: the largest word gives u1 = 1 (radius exactly 0) and the
+    smallest u1 = 2^-32 (radius sqrt(64 ln 2), finite).  Without the +1 the word 0
+    would give log(0) and the largest word a small nonzero radius, so both ends pin it.
+    The angle u2 = b 2^-32: b = 0 puts the whole radius on the first draw, b = 2^30
+    (a quarter turn) on the second."""
+    z0, z1 = decompose.box_muller(np.array([0xFFFFFFFF, 0xFFFFFFFF]), np.array([0, 0x40000000]))
+    assert np.all(z0 == 0.0) and np.all(z1 == 0.0)
+    z0, z1 = decompose.box_muller(np.array([0, 0]), np.array([0, 0x40000000]))
+    rad = np.sqrt(64.0 * np.log(2.0))
+    assert np.all(np.isfinite(z0)) and np.all(np.isfinite(z1))
+    assert z0[0] == rad and z1[0] == 0.0
+    assert abs(z0[1]) < 1e-15 * rad and abs(z1[1] - rad) < 1e-15 * rad
+    # the half turn b = 2^31 flips the sign of the first draw
+    z0, z1 = decompose.box_muller(np.array([0]), np.array([0x80000000]))
+    assert z0[0] == -rad and abs(z1[0]) < 1e-15 * rad
+
+
+def test_omega_takes_box_muller_of_its_counter_words_in_pairs():
+    """Element 4t, 4t+1 of Omega (row-major) come from words (w0, w1) of counter t,
+    elements 4t+2, 4t+3 from (w2, w3), each draw rounded to fp32."""
+    Om = decompose.omega(3, 8, 5, 2, 7).reshape(-1)
+    w = philox.stream_words(5, philox.tag(2, philox.PURPOSE_OMEGA), 7, np.arange(6, dtype=np.uint64))
+    for t in range(6):
+        a0, a1 = decompose.box_muller(w[t, 0], w[t, 1])
+        b0, b1 = decompose.box_muller(w[t, 2], w[t, 3])
+        assert list(Om[4 * t:4 * t + 4]) == [np.float32(a0), np.float32(a1), np.float32(b0), np.float32(b1)]
+
+
 def _planted(r, c, k, seed):
     rng = np.random.default_rng(seed)
     return rng.standard_normal((r, k)) @ (np.geomspace(100, 10, k)[:, None] * rng.standard_normal((k, c)))

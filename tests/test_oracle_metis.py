@@ -2,7 +2,7 @@
 
 import numpy as np
 
-from oracle import decompose, formats, metis, nvfp4
+from oracle import decompose, formats, metis, nvfp4, philox
 from workloads import synth
 
 
@@ -156,3 +156,52 @@ def test_forward_and_input_gradient_use_their_own_orientations():
     dX, _ = metis.linear_bwd(*ops)
     assert np.array_equal(dX, D @ W2.T)
     assert not np.array_equal(metis.dequant_residual(ops[2], "col"), D)
+
+
+def test_factor_sr_sub_streams_by_hand():
+    """Which stochastic-rounding stream each factor draws (reading R4: U from sub-stream 2,
+    V from sub-stream 3 of the operand's SR purpose), worked by hand on a 16 x 16 factor.
+
+    Every block (a column of F: blocks run along the long dimension) has maximum 6, so
+    g = 2^-8 (the smallest power of two with 6 <= 2688 g), the block scale is E4M3(256) =
+    256 and the scaled values are F itself.  All other entries sit at midpoints of the
+    E2M1 grid (p = 1/2), where the rule rounds up iff the element's 16-bit field is at
+    least 2^15: its top bit.  The expected codes follow from the fields alone."""
+    rng = np.random.default_rng(11)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    lo_idx = np.array([0, 1, 2, 3, 4, 5, 6])          # index of the grid point below each midpoint
+    pick = rng.integers(0, 7, size=(16, 16))
+    sign = rng.choice([-1.0, 1.0], size=(16, 16))
+    F = (mids[pick] * sign).astype(np.float32)
+    F[0, :] = 6.0
+    pick[0, :] = -1
+    seed, op_id, step = 21, 4, 9
+    for sub in (philox.SR_SUB_LEFT, philox.SR_SUB_RIGHT):
+        codes, scales, g = metis.quantize_factor(F, seed, op_id, sub, step, "sr")
+        assert g == 2.0 ** -8 and np.all(scales == formats.e4m3_encode_rn(np.array([256.0]))[0])
+        fields = philox.sr_fields(seed, op_id, sub, step, 256).reshape(16, 16)   # k x long view
+        want = np.empty((16, 16), dtype=np.uint8)
+        for i in range(16):              # column i of F = row i of the transposed view
+            for j in range(16):          # row j of F = element j of the block
+                if pick[j, i] < 0:
+                    want[i, j] = 7
+                else:
+                    want[i, j] = lo_idx[pick[j, i]] + (fields[i, j] >> 15)
+                want[i, j] |= np.uint8(8) if sign[j, i] < 0 and pick[j, i] >= 0 else np.uint8(0)
+        assert np.array_equal(codes, want), sub
+    left = metis.quantize_factor(F, seed, op_id, philox.SR_SUB_LEFT, step, "sr")[0]
+    right = metis.quantize_factor(F, seed, op_id, philox.SR_SUB_RIGHT, step, "sr")[0]
+    assert np.mean(left != right) > 0.3                 # the two streams are distinct draws
+
+
+def test_prepare_operand_draws_u_from_left_and_v_from_right():
+    """prepare_operand quantizes U with sub-stream 2 and V with sub-stream 3 (the
+    convention the test above works by hand), not the other way round."""
+    M = synth.operand_matrix(synth.CONFIGS["tiny_fwd"], "X", as_numpy=True)
+    V = decompose.refresh_basis(M, 4, 4, 32, 0, 0, 0)["V"]
+    op = metis.prepare_operand(M, V, seed=5, operand_id=0, step=3, rounding="sr")
+    U32, V32 = op["U"].astype(np.float32), op["V"].astype(np.float32)
+    for F, q, own, other in ((U32, op["Uq"], philox.SR_SUB_LEFT, philox.SR_SUB_RIGHT),
+                             (V32, op["Vq"], philox.SR_SUB_RIGHT, philox.SR_SUB_LEFT)):
+        assert np.array_equal(q[0], metis.quantize_factor(F, 5, 0, own, 3, "sr")[0])
+        assert not np.array_equal(q[0], metis.quantize_factor(F, 5, 0, other, 3, "sr")[0])

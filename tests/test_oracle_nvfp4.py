@@ -184,3 +184,61 @@ def test_auto_tensor_scale_keeps_small_gradients():
     g = nvfp4.auto_tensor_scale(M)
     c, s = nvfp4.quantize_blocks(M, g)
     assert np.linalg.norm(nvfp4.dequantize_blocks(c, s, g) - M) < 0.15 * np.linalg.norm(M)
+
+
+def _pair_decisions(p0, p1, pos0, pos1):
+    """Up-rounding decisions of two elements of one 4-group over every value of the
+    16 random bits they share: the word's bytes b2:b0 (positions 0, 1) or b3:b1
+    (positions 2, 3); the other two bytes are held at zero, which neither decision
+    reads.  Returns (up0, up1) boolean arrays over the 2^16 values."""
+    v = np.arange(1 << 16, dtype=np.uint64)
+    lo, hi = v & np.uint64(0xFF), v >> np.uint64(8)
+    shift = 0 if pos0 < 2 else 8
+    words = (lo << np.uint64(shift)) | (hi << np.uint64(16 + shift))
+    grid = formats.E2M1_MAGNITUDES
+    ups = []
+    for p, pos in ((p0, pos0), (p1, pos1)):
+        a = np.full(v.shape, 1.0 + 0.5 * p)       # between grid points 1 and 1.5
+        f = philox.fields_from_words(words, pos)
+        ups.append(nvfp4._sr_magnitude(a, f) == 3)
+        assert grid[2] == 1.0 and grid[3] == 1.5
+    return ups
+
+
+def test_paired_sr_decisions_are_nearly_independent():
+    """Reading R4's field layout gives positions 0 and 1 (and 2 and 3) of a group the
+    same 16 bits, one of them bit-reversed.  Each decision is unbiased on its own
+    (test_sr_up_count_over_all_fields); this bounds their dependence.  Over all 2^16
+    shared bit patterns, at probabilities with at most 8 significant bits the two
+    decisions read disjoint bits and are exactly independent; at any probabilities
+    the covariance of the two up-roundings stays below 1e-4 (the largest found by a
+    search over ~16 million probability pairs is 8.0e-5 at p = 0.646, 0.677, i.e. a
+    correlation coefficient of 3.5e-4)."""
+    exact = [0.5, 0.25, 0.75, 0.375, 0.9921875, 3 / 256]
+    for pos0, pos1 in ((0, 1), (2, 3)):
+        for p0 in exact:
+            for p1 in exact:
+                up0, up1 = _pair_decisions(p0, p1, pos0, pos1)
+                t0, t1 = np.floor(p0 * 65536) / 65536, np.floor(p1 * 65536) / 65536
+                assert up0.mean() == t0 and up1.mean() == t1
+                assert (up0 & up1).mean() == t0 * t1
+        worst = [(0.6461639404296875, 0.6769256591796875), (0.3, 0.7), (0.1234, 0.5678), (0.999, 0.001),
+                 (1 / 3, 1 / 3), (0.6471895, 0.3565648)]
+        for p0, p1 in worst:
+            up0, up1 = _pair_decisions(p0, p1, pos0, pos1)
+            cov = (up0 & up1).mean() - up0.mean() * up1.mean()
+            assert abs(cov) < 1e-4, (p0, p1, cov)
+
+
+def test_sr_positions_of_different_byte_pairs_read_disjoint_bits():
+    """Positions 0/1 read only bytes 0 and 2 of the word, positions 2/3 only bytes 1
+    and 3, so decisions across the two pairs are independent for a uniform word."""
+    rng = np.random.default_rng(4)
+    w = rng.integers(0, 1 << 32, size=4096, dtype=np.uint64)
+    m02, m13 = np.uint64(0x00FF00FF), np.uint64(0xFF00FF00)
+    w2 = (w & m02) | (rng.integers(0, 1 << 32, size=4096, dtype=np.uint64) & m13)
+    w3 = (w & m13) | (rng.integers(0, 1 << 32, size=4096, dtype=np.uint64) & m02)
+    for p in (0, 1):
+        assert np.array_equal(philox.fields_from_words(w, p), philox.fields_from_words(w2, p))
+    for p in (2, 3):
+        assert np.array_equal(philox.fields_from_words(w, p), philox.fields_from_words(w3, p))
