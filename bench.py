@@ -48,6 +48,12 @@ METRIC = "effective TFLOP/s of Metis W4A4G4 linear fwd+bwd; % of NVFP4 MMA peak"
 # kernel version (profile_case.py gemm --bf16; the summary sits under profiles/).
 # Must be retaken whenever the kernel changes.
 GEMM_FWD_DRAM_BYTES = 69.383424e6 + 192.398336e6
+# DRAM bytes (read + write) of one launch of the residual quantizer on the benchmark's D
+# (8192 x 14336, k = 64, SR), from one ncu capture of this kernel version
+# (bench.py --stage resquant; the summary sits under profiles/); None until retaken.
+RESQUANT_D_DRAM_BYTES = None
+RESQUANT_TRAFFIC_BASIS = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch on D (8192 x 14336), "
+                          "bytes; the timed launches cover X, W and D")
 
 
 def measured_peaks():
@@ -222,10 +228,34 @@ class Layer:
         self.dX = torch.empty(l, m, dtype=torch.bfloat16, device=dev)
         self.dW = torch.empty(m, n, dtype=torch.float32, device=dev)
 
-    def step(self, t):
+    def profile(self, on):
+        """CUDA events around the instrumented launches of every context (or off)."""
+        self.ctx.profile_enable(on)
+        for c in self.ctxs.values():
+            c.profile_enable(on)
+
+    def profile_read(self, kind):
+        """(ms, launches, work) of one instrumented kernel kind over all contexts."""
+        tot = [0.0, 0, 0.0]
+        for c in [self.ctx] + list(self.ctxs.values()):
+            ms, n, w = c.profile_read(kind)
+            tot[0] += ms
+            tot[1] += n
+            tot[2] += w
+        return tuple(tot)
+
+    def step(self, t, operands=None, outputs=None):
+        """One training step on batch t mod len(batches), or on explicit device operands
+        (X, W, D) and outputs (Y, dX, dW) (the end-to-end run's double buffers; W must keep
+        the shape of the layer's weight)."""
         cfg = self.cfg
         refresh = t % cfg["refresh_every"] == 0
-        self.mats["X"], self.mats["D"] = self.batches[t % len(self.batches)]
+        if operands is None:
+            self.mats["X"], self.mats["D"] = self.batches[t % len(self.batches)]
+        else:
+            self.mats["X"], self.mats["W"], self.mats["D"] = operands
+        if outputs is not None:
+            self.Y, self.dX, self.dW = outputs
         main = torch.cuda.current_stream(self.Y.device)
         start = torch.cuda.Event()
         start.record(main)               # inputs in place, previous GeMMs issued
@@ -359,20 +389,170 @@ def rank_config(cfg, rank):
     return dict(cfg, seed=cfg["seed"] + 1000 * rank)
 
 
+def gen_operands(cfg, batches, rank=0):
+    """W and `batches` token batches (X, D) of a configuration, pinned host bf16, generated
+    on host threads (the seeded recipe of workloads/synth.py)."""
+    from concurrent.futures import ThreadPoolExecutor
+    rcfg = rank_config(cfg, rank)
+    with ThreadPoolExecutor(max(1, min(8, os.cpu_count() or 1))) as ex:
+        fw = ex.submit(synth.operand_matrix, cfg, "W")
+        fb = [(ex.submit(synth.batch_matrix, rcfg, "X", b), ex.submit(synth.batch_matrix, rcfg, "D", b))
+              for b in range(batches)]
+        W = fw.result().pin_memory()
+        host_batches = [(x.result().pin_memory(), d.result().pin_memory()) for x, d in fb]
+    return W, host_batches
+
+
+def timed_steps(layer, device, first, steps, world, barrier, per_step=False):
+    """Time `steps` consecutive layer steps t = first .. (CUDA events on the caller's stream,
+    synchronize and barrier on both sides); returns (total ms, per-step ms or None)."""
+    stream = torch.cuda.current_stream(device)
+    barrier()
+    torch.cuda.synchronize(device)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps)] if per_step else None
+    ev0.record(stream)
+    for i, t in enumerate(range(first, first + steps)):
+        if per_step:
+            step_ev[i].record(stream)     # a step's operand work starts after the previous step's GeMMs
+        layer.step(t)
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    ms = ev0.elapsed_time(ev1)
+    if not per_step:
+        return ms, None
+    bounds = step_ev + [ev1]
+    return ms, [bounds[i].elapsed_time(bounds[i + 1]) for i in range(steps)]
+
+
+def refresh_share(step_ms, first, refresh_every):
+    """(refresh step ms, reuse step ms, amortised share) from per-step times."""
+    refresh = [d for i, d in enumerate(step_ms) if (first + i) % refresh_every == 0]
+    reuse = [d for i, d in enumerate(step_ms) if (first + i) % refresh_every != 0]
+    if not refresh or not reuse:
+        return (statistics.mean(refresh) if refresh else None), (statistics.median(reuse) if reuse else None), None
+    r, n = statistics.mean(refresh), statistics.median(reuse)
+    return r, n, (r - n) / (refresh_every * n)
+
+
+def kernel_roofline(ms, n, work, peak, unit, bound, kernel, basis, traffic=None, traffic_basis=None):
+    """One kernel's roofline entry from its CUDA-event-timed launches (work in flops or bytes)."""
+    if not n or ms <= 0:
+        return {"kernel": kernel, "bound": bound, "achieved": None, "peak": round(peak, 1), "unit": unit,
+                "frac": None, "traffic": traffic, "launches_timed": 0}
+    scale = 1e12 if unit == "TFLOP/s" else 1e9
+    achieved = work / (ms * 1e-3) / scale
+    return {"kernel": kernel, "bound": bound, "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": unit,
+            "frac": round(achieved / peak, 4), "traffic": traffic, "traffic_basis": traffic_basis,
+            "launches_timed": n, "us_per_launch": round(1e3 * ms / n, 2),
+            "work_per_launch": round(work / n), "peak_basis": basis}
+
+
+def run_e2e(layer, host_W, host_batches, device, first, steps, world, barrier):
+    """End to end through the public API with host buffers: every step uploads its inputs (W,
+    X, D) from pinned host memory and downloads its results (Y, dX, dW) into pinned host
+    memory.  Copies run on two copy streams against double-buffered device operands and
+    outputs, so step t+1's upload and step t's download overlap step t's compute."""
+    h2d, d2h = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    main = torch.cuda.current_stream(device)
+    dev_in = [tuple(torch.empty_like(x, device=device) for x in (host_batches[0][0], host_W, host_batches[0][1]))
+              for _ in range(2)]
+    dev_out = [tuple(torch.empty_like(y) for y in (layer.Y, layer.dX, layer.dW)) for _ in range(2)]
+    host_out = [tuple(torch.empty_like(y, device="cpu").pin_memory() for y in (layer.Y, layer.dX, layer.dW))
+                for _ in range(2)]
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
+
+    def upload(t):
+        b = t % 2
+        x, d = host_batches[t % len(host_batches)]
+        h2d.wait_event(computed[b])            # the step two back has finished reading this buffer
+        with torch.cuda.stream(h2d):
+            for dst, src in zip(dev_in[b], (x, host_W, d)):
+                dst.copy_(src, non_blocking=True)
+            in_ready[b].record(h2d)
+
+    saved = (layer.mats["X"], layer.mats["W"], layer.mats["D"], layer.Y, layer.dX, layer.dW)
+    barrier()
+    torch.cuda.synchronize(device)
+    for b in range(2):                          # nothing to wait for yet
+        computed[b].record(main)
+        out_done[b].record(main)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(main)
+    h2d.wait_event(computed[0])
+    upload(first)
+    for i, t in enumerate(range(first, first + steps)):
+        b = t % 2
+        main.wait_event(in_ready[b])
+        main.wait_event(out_done[b])            # the download two steps back has read these outputs
+        layer.step(t, operands=dev_in[b], outputs=dev_out[b])
+        computed[b].record(main)
+        if i + 1 < steps:
+            upload(t + 1)
+        d2h.wait_event(computed[b])
+        with torch.cuda.stream(d2h):
+            for dst, src in zip(host_out[b], dev_out[b]):
+                dst.copy_(src, non_blocking=True)
+            out_done[b].record(d2h)
+    main.wait_event(out_done[(first + steps - 1) % 2])
+    main.wait_event(out_done[(first + steps - 2) % 2])
+    e1.record(main)
+    torch.cuda.synchronize(device)
+    barrier()
+    layer.mats["X"], layer.mats["W"], layer.mats["D"], layer.Y, layer.dX, layer.dW = saved
+    h2d_bytes = sum(v.numel() * v.element_size() for v in (host_W,) + host_batches[0])
+    d2h_bytes = sum(v.numel() * v.element_size() for v in host_out[0])
+    return e0.elapsed_time(e1), h2d_bytes, d2h_bytes
+
+
+def config_line(lib, cfg_name, device, steps=8, warmup=3, batches=2, world=1, barrier=lambda: None):
+    """A short run of another workload: effective TFLOP/s, ms per step, the main GeMM's
+    fraction of the NVFP4 peak and the refresh share."""
+    if cfg_name == "long_token_stress_r8":     # the stress workload again, refreshed every 8th step
+        cfg = dict(synth.CONFIGS["long_token_stress"], refresh_every=8)
+    else:
+        cfg = synth.CONFIGS[cfg_name]
+    host_W, host_batches = gen_operands(cfg, batches)
+    W = host_W.to(device)
+    dev_batches = [(x.to(device), d.to(device)) for x, d in host_batches]
+    ctx = lib.Context(device.index)
+    layer = Layer(lib, ctx, cfg, dev_batches, W)
+    for t in range(warmup):
+        layer.step(t)
+    layer.profile(True)
+    ms, step_ms = timed_steps(layer, device, warmup, steps, world, barrier, per_step=True)
+    gemm = layer.profile_read(lib.PROF_GEMM)
+    layer.profile(False)
+    status = layer.poll_device_status()
+    l, m, n = cfg["l"], cfg["m"], cfg["n"]
+    flops = (2.0 if cfg["fwd_only"] else 6.0) * l * m * n
+    r_ms, n_ms, share = refresh_share(step_ms, warmup, cfg["refresh_every"])
+    out = {"workload": f"{cfg_name}: X {l}x{m}, W {m}x{n}, D {l}x{n}, k={cfg['k']}, s={cfg['s']}, "
+                       f"l_k={cfg['l_k']}, refresh every {cfg['refresh_every']}",
+           "value": round(flops / (ms / steps * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+           "ms_per_step": round(ms / steps, 4), "steps": steps, "warmup": warmup, "batches": batches,
+           "gemm_tflops": round(gemm[2] / (gemm[0] * 1e-3) / 1e12, 1) if gemm[1] else None,
+           "refresh_step_ms": None if r_ms is None else round(r_ms, 4),
+           "reuse_step_ms": None if n_ms is None else round(n_ms, 4),
+           "amortised_share": None if share is None else round(share, 4), "device_status": status}
+    del layer, dev_batches, W
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, rank, world, device):
     import spectral_quantized_gemm_b200 as lib
     cfg = synth.CONFIGS[args.config]
     l, m, n = cfg["l"], cfg["m"], cfg["n"]
     flops_per_step = 6.0 * l * m * n
-    rcfg = rank_config(cfg, rank)
-    host_W = synth.operand_matrix(cfg, "W").pin_memory()
-    host_batches = [(synth.batch_matrix(rcfg, "X", b).pin_memory(), synth.batch_matrix(rcfg, "D", b).pin_memory())
-                    for b in range(args.batches)]
+    host_W, host_batches = gen_operands(cfg, args.batches, rank)
     dev_W = host_W.to(device)
     dev_batches = [(x.to(device), d.to(device)) for x, d in host_batches]
     ctx = lib.Context(device.index)
     layer = Layer(lib, ctx, cfg, dev_batches, dev_W)
-    stream = torch.cuda.current_stream(device)
 
     def barrier():
         if world > 1:
@@ -389,58 +569,24 @@ def run_ours(args, rank, world, device):
     clocks = ClockSampler(device)
     clocks.start()
     time.sleep(0.05)
-    ctx.profile_enable(True)
+    layer.profile(True)
     launches0 = lib.kernel_launches()
-    barrier()
-    torch.cuda.synchronize(device)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     t_region0 = time.perf_counter()
-    ev0.record(stream)
-    for i, t in enumerate(range(args.warmup, args.warmup + args.steps)):
-        step_ev[i].record(stream)     # a step's operand work starts after the previous step's GeMMs
-        layer.step(t)
-    ev1.record(stream)
-    torch.cuda.synchronize(device)
+    ms, step_ms = timed_steps(layer, device, args.warmup, args.steps, world, barrier, per_step=True)
     t_region1 = time.perf_counter()
-    barrier()
-    bounds = step_ev + [ev1]
-    step_ms = [bounds[i].elapsed_time(bounds[i + 1]) for i in range(args.steps)]
-    refresh_ms = [d for i, d in enumerate(step_ms) if (args.warmup + i) % cfg["refresh_every"] == 0]
-    normal_ms = [d for i, d in enumerate(step_ms) if (args.warmup + i) % cfg["refresh_every"] != 0]
     launches = lib.kernel_launches() - launches0
-    gemm_ms, gemm_n, gemm_flops = ctx.profile_read()
-    ctx.profile_enable(False)
+    prof = {kind: layer.profile_read(kind) for kind in (lib.PROF_GEMM, lib.PROF_RESQUANT, lib.PROF_PROJECTION)}
+    layer.profile(False)
     clk = clocks.stop(t_region0, t_region1)
-    ms = ev0.elapsed_time(ev1)
     ms = max_over_ranks(ms, world, device)
     ms_per_step = ms / args.steps
     value = world * flops_per_step / (ms_per_step * 1e-3) / 1e12
+    r_ms, n_ms, share = refresh_share(step_ms, args.warmup, cfg["refresh_every"])
 
-    # ---- end to end through the public API: host inputs in, host results out
-    out_host = {"Y": torch.empty_like(layer.Y, device="cpu").pin_memory(),
-                "dX": torch.empty_like(layer.dX, device="cpu").pin_memory(),
-                "dW": torch.empty_like(layer.dW, device="cpu").pin_memory()}
-    h2d = sum(v.numel() * v.element_size() for v in (host_W,) + host_batches[0])
-    d2h = sum(v.numel() * v.element_size() for v in out_host.values())
-    e2e_steps = max(2, min(args.steps, 6))
-    barrier()
-    torch.cuda.synchronize(device)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for t in range(args.warmup + args.steps, args.warmup + args.steps + e2e_steps):
-        b = t % len(dev_batches)
-        dev_W.copy_(host_W, non_blocking=True)
-        dev_batches[b][0].copy_(host_batches[b][0], non_blocking=True)
-        dev_batches[b][1].copy_(host_batches[b][1], non_blocking=True)
-        layer.step(t)
-        out_host["Y"].copy_(layer.Y, non_blocking=True)
-        out_host["dX"].copy_(layer.dX, non_blocking=True)
-        out_host["dW"].copy_(layer.dW, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize(device)
-    barrier()
-    e2e_ms = e0.elapsed_time(e1)
+    # ---- end to end through the public API: host inputs in, host results out, copies overlapped
+    e2e_steps = max(4, min(args.steps, 8))
+    first = args.warmup + args.steps
+    e2e_ms, h2d, d2h = run_e2e(layer, host_W, host_batches, device, first, e2e_steps, world, barrier)
     e2e_ms = max_over_ranks(e2e_ms, world, device)
     e2e_value = world * flops_per_step / (e2e_ms / e2e_steps * 1e-3) / 1e12
     status = layer.poll_device_status()
@@ -449,17 +595,8 @@ def run_ours(args, rank, world, device):
     plain = Layer(lib, ctx, cfg, dev_batches, dev_W, plain=True)
     for t in range(3):
         plain.step(t)
-    barrier()
-    torch.cuda.synchronize(device)
-    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    p0.record(stream)
-    for t in range(3, 3 + args.steps):
-        plain.step(t)
-    p1.record(stream)
-    torch.cuda.synchronize(device)
-    barrier()
-    plain_ms = p0.elapsed_time(p1) / args.steps
-    plain_ms = max_over_ranks(plain_ms, world, device)
+    plain_ms, _ = timed_steps(plain, device, 3, args.steps, world, barrier)
+    plain_ms = max_over_ranks(plain_ms / args.steps, world, device)
     status |= plain.poll_device_status()
 
     # ---- the LoRA-SVD projection's training step on the same batches, same timing
@@ -468,6 +605,7 @@ def run_ours(args, rank, world, device):
         lora.step(t)
     barrier()
     torch.cuda.synchronize(device)
+    stream = torch.cuda.current_stream(device)
     q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     q0.record(stream)
     for t in range(3, 3 + args.steps):
@@ -478,14 +616,34 @@ def run_ours(args, rank, world, device):
     barrier()
     lora_ms = max_over_ranks(q0.elapsed_time(q1) / args.steps, world, device)
     status |= lora.poll_device_status()
+    del lora, plain
 
     # the achievable FP4 MMA rate on this GPU (no memory traffic), beside the roofline
     mma_peak = ctx.nvfp4_mma_peak(iters=4096, reps=5)
     status |= ctx.poll_device_status()
 
     peaks, kind = measured_peaks()
-    peak = peaks["bf16_tflops_sustained"] * NVFP4_OVER_BF16
-    achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
+    # the timed region lasts tens of milliseconds at full clock: the burst peaks apply
+    nvfp4_peak = peaks["bf16_tflops"] * NVFP4_OVER_BF16
+    nvfp4_sustained = peaks["bf16_tflops_sustained"] * NVFP4_OVER_BF16
+    hbm = peaks["hbm_gbs"]
+    gemm = kernel_roofline(*prof[lib.PROF_GEMM], nvfp4_peak, "TFLOP/s", "tensor",
+                           "gemm_nvfp4_pair_kernel (fused FP4 GeMM + rank fold, CTA pairs; fwd, dX, dW)",
+                           f"{kind} bf16 burst x {NVFP4_OVER_BF16:.0f} (nominal NVFP4/bf16 ratio)",
+                           traffic=round(GEMM_FWD_DRAM_BYTES),
+                           traffic_basis="ncu dram__bytes_read.sum + dram__bytes_write.sum of one forward-shape "
+                                         "launch (bytes)")
+    if gemm["achieved"] is not None:
+        gemm["frac_of_sustained_peak"] = round(gemm["achieved"] / nvfp4_sustained, 4)
+        gemm["frac_of_mma_microbenchmark"] = round(gemm["achieved"] / mma_peak, 4)
+        gemm["frac_of_datasheet_9pf"] = round(gemm["achieved"] / 9000.0, 4)
+    resq = kernel_roofline(*prof[lib.PROF_RESQUANT], hbm, "GB/s", "hbm",
+                           "resquant_kernel (residual + NVFP4, both orientations; X, W, D)",
+                           f"{kind} HBM copy bandwidth", traffic=RESQUANT_D_DRAM_BYTES,
+                           traffic_basis=RESQUANT_TRAFFIC_BASIS)
+    proj = kernel_roofline(*prof[lib.PROF_PROJECTION], hbm, "GB/s", "hbm",
+                           "per-step projection P = M V (bf16 hi/lo tensor-core GeMM with its split and "
+                           "reduction launches; X, W, D)", f"{kind} HBM copy bandwidth")
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
@@ -499,20 +657,13 @@ def run_ours(args, rank, world, device):
                    "batches": args.batches,
                    "streams": "X, W and D decomposed and quantized on three streams; the GeMMs on one",
                    "outputs": "Y and dX bf16, dW fp32 (fp32 accumulation)",
-                   "pct_of_nvfp4_peak": round(100 * value / (world * peak), 2),
-                   "nvfp4_peak_tflops": round(peak, 1),
-                   "nvfp4_peak_basis": f"bf16_tflops_sustained x {NVFP4_OVER_BF16:.0f} ({kind})"},
-        "roofline": {"bound": "tensor", "kernel": "gemm_nvfp4_pair_kernel (fused FP4 GeMM + fold, CTA pairs)",
-                     "achieved": None if achieved is None else round(achieved, 1), "peak": round(peak, 1),
-                     "unit": "TFLOP/s", "frac": None if achieved is None else round(achieved / peak, 4),
-                     "traffic": round(GEMM_FWD_DRAM_BYTES),
-                     "traffic_basis": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one forward-shape "
-                                      "launch (bytes); the timed launches are the fwd, dX and dW GeMMs",
-                     "launches_timed": gemm_n,
-                     "peak_basis": f"{kind} bf16 sustained x {NVFP4_OVER_BF16:.0f} (nominal NVFP4/bf16 ratio)"},
+                   "pct_of_nvfp4_peak": round(100 * value / (world * nvfp4_peak), 2),
+                   "nvfp4_peak_tflops": round(nvfp4_peak, 1),
+                   "nvfp4_peak_basis": f"bf16_tflops (burst) x {NVFP4_OVER_BF16:.0f} ({kind})"},
+        "roofline": gemm,
+        "rooflines": {"resquant": resq, "projection": proj},
         "nvfp4_mma_peak": {
             "value": round(mma_peak, 1), "unit": "TFLOP/s",
-            "gemm_frac": None if achieved is None else round(achieved / mma_peak, 4),
             "what": "tcgen05 kind::mxf4nvf4 block16 MMAs (CTA pairs, M=256 N=256 K=64) on resident "
                     "operands, no memory traffic: the rate the fused GeMM could reach"},
         "plain_nvfp4": {
@@ -530,19 +681,25 @@ def run_ours(args, rank, world, device):
                     "constraint (on its own stream, overlapping the gradients and the next quantization)"},
         "decomposition": {
             "refresh_every": cfg["refresh_every"],
-            "refresh_steps_timed": len(refresh_ms),
-            "refresh_step_ms": round(statistics.mean(refresh_ms), 4) if refresh_ms else None,
-            "reuse_step_ms": round(statistics.median(normal_ms), 4) if normal_ms else None,
-            "amortised_share": (round((statistics.mean(refresh_ms) - statistics.median(normal_ms))
-                                      / (cfg["refresh_every"] * statistics.median(normal_ms)), 4)
-                                if refresh_ms and normal_ms else None),
+            "refresh_steps_timed": sum(1 for i in range(args.steps) if (args.warmup + i) % cfg["refresh_every"] == 0),
+            "refresh_step_ms": None if r_ms is None else round(r_ms, 4),
+            "reuse_step_ms": None if n_ms is None else round(n_ms, 4),
+            "amortised_share": None if share is None else round(share, 4),
             "basis": "(refresh step - reuse step) / (refresh_every x reuse step), CUDA events per step"},
         "clocks": clk,
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps, "ms_per_step": round(e2e_ms / e2e_steps, 4),
+                "copies": "pinned host memory; uploads and downloads on two copy streams, double-buffered "
+                          "operands and outputs, overlapping the step's compute"},
         "gpu_launches": launches,
         "device_status": status,
     }
+    del layer
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_configs:
+        result["configs"] = {}
+        for name in ("gpt2_small_mlp_up", "llama3_8b_down_reuse", "long_token_stress", "long_token_stress_r8"):
+            result["configs"][name] = config_line(lib, name, device)
     return result
 
 
@@ -625,6 +782,46 @@ def run_reference(args, rank, world):
                                         "d2h_bytes_per_step": 0}}
 
 
+def run_stage(args, device):
+    """Profiling mode (``--stage``): issue one stage of the benchmark step ``--reps`` times on
+    the benchmark workload's own operands and exit, for a profiler to capture by kernel
+    name.  Prints no benchmark line and times nothing.
+
+    resquant   the residual quantization of D (both orientations, rank-k factors)
+    decompose  the per-step factor update of X (projection, eigensolve, factors)
+    gemm       the forward fused GeMM of the layer (FP4 + rank fold, bf16 out)
+    step       whole layer steps"""
+    import spectral_quantized_gemm_b200 as lib
+    cfg = synth.CONFIGS[args.config]
+    W = synth.operand_matrix(cfg, "W").to(device)
+    batches = [(synth.batch_matrix(cfg, "X", 0).to(device), synth.batch_matrix(cfg, "D", 0).to(device))]
+    ctx = lib.Context(device.index)
+    layer = Layer(lib, ctx, cfg, batches, W)
+    layer.step(0)                         # refresh: the bases every stage starts from
+    torch.cuda.synchronize(device)
+    rnd = layer.rounding
+    for t in range(1, args.reps + 1):
+        if args.stage == "step":
+            layer.step(t)
+            continue
+        name = {"resquant": "D", "decompose": "X", "gemm": "X"}[args.stage]
+        f, row, col, _ = layer.ops[name]
+        M = layer.mats[name]
+        i = layer.NAMES.index(name)
+        if args.stage == "resquant":
+            ctx.residual_quantize_nvfp4(M, f, row, col, rounding=rnd, seed=cfg["seed"], operand_id=i, step=t)
+        elif args.stage == "decompose":
+            l_k = layer.l_k[name]
+            ctx.decompose(M, k=cfg["k"], s=cfg["s"], l_k=l_k, seed=cfg["seed"], operand_id=i, refresh=False, step=t,
+                          factors=f, rounding=rnd)
+        else:
+            ctx.linear_fwd(layer.ops["X"][3], layer.ops["W"][3], layer.Y)
+    torch.cuda.synchronize(device)
+    status = layer.poll_device_status()
+    print(f"stage {args.stage}: {args.config}, {args.reps} repetitions, device status {status}", flush=True)
+    return status
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -633,10 +830,18 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(synth.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the short runs of the other workloads")
     ap.add_argument("--batches", type=int, default=4, help="distinct token batches (X, D) cycled over the steps")
     ap.add_argument("--ref-rows", type=int, default=256, help="token rows of the oracle's bounded sample")
     ap.add_argument("--ref-cols", type=int, default=1024, help="output columns of the oracle's bounded sample")
+    ap.add_argument("--stage", choices=["resquant", "decompose", "gemm", "step"],
+                    help="profiling mode: run one stage --reps times for a profiler; no benchmark line")
+    ap.add_argument("--reps", type=int, default=3, help="repetitions of --stage")
     args = ap.parse_args()
+    if args.stage:
+        device = torch.device("cuda", 0)
+        torch.cuda.set_device(device)
+        raise SystemExit(1 if run_stage(args, device) else 0)
     if args.warmup < 3:
         raise SystemExit("need at least 3 warm-up steps")
 

@@ -174,6 +174,23 @@ metis_status metis_residual_quantize_nvfp4(metis_ctx* ctx, const metis_matrix* M
                                            metis_nvfp4* rowwise, metis_nvfp4* colwise);
 
 /*
+ * Parity surface of the residual quantization (key design 1): the same pass as
+ * metis_residual_quantize_nvfp4 with both orientations, which also writes the fp32
+ * residual that its quantizer rounded to `residual` (rows x cols, leading dimension ldr,
+ * caller-owned device memory, 16-byte aligned, ldr % 4 == 0).  With k > 0 the pass
+ * rebuilds U diag(S) V^T on the tensor cores from fp16 hi/lo splits of power-of-two
+ * scaled 128-row blocks of U diag(S) and V (hi*hi + hi*lo + lo*hi, fp32 accumulation),
+ * so this residual differs from M - U diag(S) V^T by about 2^-21 of the largest
+ * reconstruction term; its NVFP4 codes and scales are exactly the block rule applied to
+ * it.  Errors as metis_residual_quantize_nvfp4; ERR_ARG without both outputs and the
+ * residual; ERR_ALIGN on the residual buffer.
+ */
+metis_status metis_residual_quantize_nvfp4_dump(metis_ctx* ctx, const metis_matrix* M,
+                                                const metis_factors* f, const metis_quant_params* q,
+                                                metis_nvfp4* rowwise, metis_nvfp4* colwise,
+                                                float* residual, int64_t ldr);
+
+/*
  * NVFP4 quantization of an fp32 device matrix R (rows x cols, leading dimension ld):
  * the quantizer alone, bit-exact with the block rule (background section; training
  * strategy for stochastic rounding).  Same outputs as above.
@@ -199,9 +216,9 @@ metis_status metis_dequantize_nvfp4(metis_ctx* ctx, const metis_nvfp4* t, float*
  * a step being captured into a CUDA graph cannot call cudaMalloc, and a
  * framework that manages device memory through its own caching allocator must
  * not have a library allocate behind it.  This call allocates nothing: its
- * scratch (rank-padded copies of U diag(S) and V) is a fixed 6 MiB device array
- * inside libmetis, present on every GPU that loads the library until the process
- * exits.  The caller still provides every input and output.
+ * scratch (the fp16 hi/lo tiles of U diag(S) and V that the tensor cores read, and
+ * their block factors) is a fixed 6 MiB device array inside libmetis, present on every
+ * GPU that loads the library until the process exits.  The caller still provides every input and output.
  *   - rows + cols must not exceed 24576 (k <= 64); larger shapes return
  *     METIS_ERR_SHAPE with a message.  rowwise and colwise are both required.
  *   - The first call on a device looks up the array's device address (once per
@@ -329,16 +346,25 @@ metis_status metis_nvfp4_mma_peak(metis_ctx* ctx, int64_t iters, double* flops);
 /*
  * Instrumentation (the notes have no counterpart; used by the benchmark).
  * metis_kernel_launches: number of kernels libmetis has launched in this process.
- * metis_profile_enable: when on, every main GeMM launch (the fused FP4 + fold
- *   kernel of the layer calls and metis_gemm_nvfp4 with n_cols >= 256) is
- *   bracketed by CUDA events on the context's stream.
- * metis_profile_read: synchronizes the stream and returns the summed event time
- *   (ms), the number of timed launches and their algorithmic flops 2*p*q*K, then
- *   resets the record.
+ * metis_profile_enable: when on, the launches of three kernels are bracketed by CUDA
+ *   events on the context's stream: every main GeMM (the fused FP4 + fold kernel of
+ *   the layer calls and metis_gemm_nvfp4 with n_cols >= 256; METIS_PROF_GEMM), every
+ *   two-orientation residual quantization pass (METIS_PROF_RESQUANT) and every per-step
+ *   projection P = M V of metis_decompose (METIS_PROF_PROJECTION).
+ * metis_profile_read_kind: synchronizes the stream and returns, for one kind, the summed
+ *   event time (ms), the number of timed launches and their algorithmic work -- flops
+ *   2*p*q*K for the GeMM, bytes for the two HBM-bound kernels (3.125 per element of M
+ *   for the quantizer: 2 read, 2 x (1/2 + 1/16) written; 2 per element of M read for the
+ *   projection) -- then resets that kind's record.  metis_profile_read is the GeMM kind.
  */
+#define METIS_PROF_GEMM       0
+#define METIS_PROF_RESQUANT   1
+#define METIS_PROF_PROJECTION 2
 uint64_t metis_kernel_launches(void);
 metis_status metis_profile_enable(metis_ctx* ctx, int on);
 metis_status metis_profile_read(metis_ctx* ctx, double* ms, int64_t* launches, double* flops);
+metis_status metis_profile_read_kind(metis_ctx* ctx, int32_t kind, double* ms, int64_t* launches,
+                                     double* work);
 
 #ifdef __cplusplus
 }

@@ -43,7 +43,10 @@ EXPORTED = ["metis_create", "metis_destroy", "metis_set_stream", "metis_status_s
             "metis_linear_fwd", "metis_linear_bwd", "metis_kernel_launches", "metis_profile_enable",
             "metis_profile_read", "metis_residual_quantize_nvfp4_noalloc", "metis_dequantize_nvfp4",
             "metis_nvfp4_mma_peak", "metis_selftest_wait_timeout", "metis_lora_linear",
-            "metis_lora_branch_grad", "metis_lora_constrain", "metis_lora_realign"]
+            "metis_lora_branch_grad", "metis_lora_constrain", "metis_lora_realign",
+            "metis_residual_quantize_nvfp4_dump", "metis_profile_read_kind"]
+
+PROF_GEMM, PROF_RESQUANT, PROF_PROJECTION = 0, 1, 2
 
 
 class Matrix(ctypes.Structure):
@@ -96,6 +99,9 @@ _resq = _sig("metis_residual_quantize_nvfp4", c_i32, c_p, ctypes.POINTER(Matrix)
 _resq_noalloc = _sig("metis_residual_quantize_nvfp4_noalloc", c_i32, c_p, ctypes.POINTER(Matrix),
                      ctypes.POINTER(FactorsStruct), ctypes.POINTER(QuantParams), ctypes.POINTER(Nvfp4Struct),
                      ctypes.POINTER(Nvfp4Struct))
+_resq_dump = _sig("metis_residual_quantize_nvfp4_dump", c_i32, c_p, ctypes.POINTER(Matrix),
+                  ctypes.POINTER(FactorsStruct), ctypes.POINTER(QuantParams), ctypes.POINTER(Nvfp4Struct),
+                  ctypes.POINTER(Nvfp4Struct), c_p, c_i64)
 _dequant = _sig("metis_dequantize_nvfp4", c_i32, c_p, ctypes.POINTER(Nvfp4Struct), c_p, c_i64)
 _mma_peak = _sig("metis_nvfp4_mma_peak", c_i32, c_p, c_i64, ctypes.POINTER(ctypes.c_double))
 _wait_selftest = _sig("metis_selftest_wait_timeout", c_i32, c_p, c_i64)
@@ -118,6 +124,8 @@ _launches = _sig("metis_kernel_launches", c_u64)
 _prof_enable = _sig("metis_profile_enable", c_i32, c_p, ctypes.c_int)
 _prof_read = _sig("metis_profile_read", c_i32, c_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(c_i64),
                   ctypes.POINTER(ctypes.c_double))
+_prof_read_kind = _sig("metis_profile_read_kind", c_i32, c_p, c_i32, ctypes.POINTER(ctypes.c_double),
+                       ctypes.POINTER(c_i64), ctypes.POINTER(ctypes.c_double))
 
 
 def kernel_launches():
@@ -231,6 +239,16 @@ class Context:
                    ctypes.byref(q), None if rowwise is None else ctypes.byref(rowwise.struct),
                    None if colwise is None else ctypes.byref(colwise.struct))
 
+    def residual_quantize_nvfp4_dump(self, M, factors, rowwise, colwise, residual, rounding=0, seed=0, operand_id=0,
+                                     step=0, tensor_scale=1.0):
+        """Both orientations, plus the fp32 residual the quantizer rounded (parity surface)."""
+        if residual.dtype != torch.float32 or residual.dim() != 2 or residual.stride(1) != 1:
+            raise ValueError("residual: expected a row-major 2-D fp32 CUDA tensor")
+        q = QuantParams(rounding, seed, operand_id, step, tensor_scale)
+        self._call(_resq_dump, ctypes.byref(_matrix(M)), None if factors is None else ctypes.byref(factors.struct),
+                   ctypes.byref(q), ctypes.byref(rowwise.struct), ctypes.byref(colwise.struct), _ptr(residual),
+                   residual.stride(0))
+
     def residual_quantize_nvfp4_noalloc(self, M, factors, rowwise, colwise, rounding=0, seed=0, operand_id=0,
                                         step=0, tensor_scale=1.0):
         """Allocation-free residual quantization: libmetis calls no cudaMalloc here
@@ -288,11 +306,13 @@ class Context:
     def profile_enable(self, on=True):
         self._call(_prof_enable, int(bool(on)))
 
-    def profile_read(self):
-        """(milliseconds, launches, flops) of the main GeMM launches since the last read."""
-        ms, n, fl = ctypes.c_double(), c_i64(), ctypes.c_double()
-        self._call(_prof_read, ctypes.byref(ms), ctypes.byref(n), ctypes.byref(fl))
-        return ms.value, n.value, fl.value
+    def profile_read(self, kind=PROF_GEMM):
+        """(milliseconds, launches, work) of the instrumented launches of one kind since the
+        last read: flops for the main GeMM, algorithmic bytes for the residual quantizer
+        and the projection."""
+        ms, n, w = ctypes.c_double(), c_i64(), ctypes.c_double()
+        self._call(_prof_read_kind, int(kind), ctypes.byref(ms), ctypes.byref(n), ctypes.byref(w))
+        return ms.value, n.value, w.value
 
     @staticmethod
     def operand(rowwise=None, colwise=None, factors=None):

@@ -156,6 +156,11 @@ void metis_destroy(metis_ctx* ctx) {
   cudaStreamSynchronize(ctx->stream);
   if (ctx->ws) cudaFree(ctx->ws);
   if (ctx->status) cudaFree(ctx->status);
+  for (auto& evs : ctx->prof_events)
+    for (auto& ev : evs) {
+      cudaEventDestroy(ev.first);
+      cudaEventDestroy(ev.second);
+    }
   delete ctx;
 }
 
@@ -273,6 +278,26 @@ metis_status metis_residual_quantize_nvfp4(metis_ctx* ctx, const metis_matrix* M
                     launch_quantize_f32(R, M->rows, M->cols, M->cols, *q, amax, rowwise, colwise, ctx->status,
                                         ctx->stream),
                     "quantize launch");
+}
+
+metis_status metis_residual_quantize_nvfp4_dump(metis_ctx* ctx, const metis_matrix* M, const metis_factors* f,
+                                                const metis_quant_params* q, metis_nvfp4* rowwise,
+                                                metis_nvfp4* colwise, float* residual, int64_t ldr) {
+  const metis::NvtxRange nvtx_range("metis_residual_quantize_nvfp4_dump");
+  metis_status s = enter(ctx);
+  if (s != METIS_OK) return s;
+  if (!M || !M->data) return fail(ctx, METIS_ERR_ARG, "null matrix");
+  if ((s = check_dims(ctx, M->rows, M->cols)) != METIS_OK) return s;
+  if (M->ld < M->cols || M->ld % 8 || !aligned16(M->data))
+    return fail(ctx, METIS_ERR_ALIGN, "bf16 matrix needs 16-byte alignment and ld % 8 == 0");
+  if ((s = check_quant(ctx, q)) != METIS_OK) return s;
+  if ((s = check_factors(ctx, f, M->rows, M->cols)) != METIS_OK) return s;
+  if (!rowwise || !colwise || !residual) return fail(ctx, METIS_ERR_ARG, "both orientations and the residual are required");
+  if ((s = check_nvfp4(ctx, rowwise, M->rows, M->cols, "rowwise")) != METIS_OK) return s;
+  if ((s = check_nvfp4(ctx, colwise, M->cols, M->rows, "colwise")) != METIS_OK) return s;
+  if (ldr < M->cols || ldr % 4 || !aligned16(residual))
+    return fail(ctx, METIS_ERR_ALIGN, "fp32 residual needs 16-byte alignment and ld % 4 == 0");
+  return run_residual_quantize(ctx, M, f, q, rowwise, colwise, residual, ldr);
 }
 
 metis_status metis_gemm_nvfp4(metis_ctx* ctx, const metis_nvfp4* A, const metis_nvfp4* B, int64_t n_cols,
@@ -419,6 +444,11 @@ metis_status metis_lora_realign(metis_ctx* ctx, float* W_res, int64_t m, int64_t
 
 namespace metis {
 std::atomic<uint64_t> g_launches{0};
+
+void profile_record(metis_ctx* ctx, int kind, cudaEvent_t ev0, cudaEvent_t ev1, double work) {
+  ctx->prof_events[kind].emplace_back(ev0, ev1);
+  ctx->prof_work[kind].push_back(work);
+}
 }  // namespace metis
 
 extern "C" {
@@ -448,26 +478,32 @@ metis_status metis_nvfp4_mma_peak(metis_ctx* ctx, int64_t iters, double* flops) 
   return launch_mma_peak(ctx, iters, flops);
 }
 
-metis_status metis_profile_read(metis_ctx* ctx, double* ms, int64_t* launches, double* flops) {
-  if (!ctx || !ms || !launches || !flops) return METIS_ERR_ARG;
+metis_status metis_profile_read_kind(metis_ctx* ctx, int32_t kind, double* ms, int64_t* launches, double* work) {
+  if (!ctx || !ms || !launches || !work || kind < 0 || kind >= metis::kProfKinds) return METIS_ERR_ARG;
   cudaSetDevice(ctx->device);
   metis_status s = metis::check_cuda(ctx, cudaStreamSynchronize(ctx->stream), "cudaStreamSynchronize");
   if (s != METIS_OK) return s;
-  double total = 0.0, fl = 0.0;
-  for (size_t i = 0; i < ctx->prof_events.size(); ++i) {
+  auto& evs = ctx->prof_events[kind];
+  auto& wk = ctx->prof_work[kind];
+  double total = 0.0, w = 0.0;
+  for (size_t i = 0; i < evs.size(); ++i) {
     float t = 0.0f;
-    cudaEventElapsedTime(&t, ctx->prof_events[i].first, ctx->prof_events[i].second);
+    cudaEventElapsedTime(&t, evs[i].first, evs[i].second);
     total += t;
-    fl += ctx->prof_flops[i];
-    cudaEventDestroy(ctx->prof_events[i].first);
-    cudaEventDestroy(ctx->prof_events[i].second);
+    w += wk[i];
+    cudaEventDestroy(evs[i].first);
+    cudaEventDestroy(evs[i].second);
   }
   *ms = total;
-  *launches = (int64_t)ctx->prof_events.size();
-  *flops = fl;
-  ctx->prof_events.clear();
-  ctx->prof_flops.clear();
+  *launches = (int64_t)evs.size();
+  *work = w;
+  evs.clear();
+  wk.clear();
   return METIS_OK;
+}
+
+metis_status metis_profile_read(metis_ctx* ctx, double* ms, int64_t* launches, double* flops) {
+  return metis_profile_read_kind(ctx, METIS_PROF_GEMM, ms, launches, flops);
 }
 
 }  // extern "C"
@@ -491,7 +527,10 @@ extern "C" metis_status metis_residual_quantize_nvfp4_noalloc(metis_ctx* ctx, co
   if (!rowwise || !colwise) return fail(ctx, METIS_ERR_ARG, "the allocation-free path writes both orientations");
   if ((s = check_nvfp4(ctx, rowwise, M->rows, M->cols, "rowwise")) != METIS_OK) return s;
   if ((s = check_nvfp4(ctx, colwise, M->cols, M->rows, "colwise")) != METIS_OK) return s;
-  float* scratch = noalloc_scratch(ctx, &s);
+  char* scratch = noalloc_scratch(ctx, &s);
   if (!scratch) return s;
-  return run_residual_quantize_into(ctx, M, f, q, rowwise, colwise, scratch);
+  if (residual_quantize_scratch_bytes(M->rows, M->cols) > kNoAllocAmaxOffset)
+    return fail(ctx, METIS_ERR_SHAPE, "shape needs more than the allocation-free scratch");
+  return run_residual_quantize_into(ctx, M, f, q, rowwise, colwise, scratch,
+                                    reinterpret_cast<uint32_t*>(scratch + kNoAllocAmaxOffset), nullptr, 0);
 }

@@ -1440,7 +1440,17 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
     times_small_kernel<<<blocks_for(c * k), 256, 0, st>>>(Bt, c, w, T, k, f->V); count_launch();
   }
   // per step: P = M V ; R = chol(P^T P) ; SVD(R) ; U = P R^+ U_r ; V <- V V_r
+  cudaEvent_t pev0 = nullptr, pev1 = nullptr;
+  if (ctx->profiling) {
+    cudaEventCreate(&pev0);
+    cudaEventCreate(&pev1);
+    cudaEventRecord(pev0, st);
+  }
   if ((s = project(f->V, k, Y)) != METIS_OK) return s;
+  if (ctx->profiling) {   // algorithmic bytes: one bf16 read of M
+    cudaEventRecord(pev1, st);
+    profile_record(ctx, kProfProjection, pev0, pev1, 2.0 * (double)r * (double)c);
+  }
   gram(Y, r, k);
   so.S = f->S;
   solve(k, 2);

@@ -881,8 +881,7 @@ metis_status launch_spec(metis_ctx* ctx, const CUtensorMap& mA, const CUtensorMa
   kern<<<grid, kThreads, C::SMEM, ctx->stream>>>(mA, mB, mFa, mFb, mA1, mB1, mA2, mB2, prm); count_launch();
   if (prof) {
     cudaEventRecord(ev1, ctx->stream);
-    ctx->prof_events.emplace_back(ev0, ev1);
-    ctx->prof_flops.push_back(flops);
+    profile_record(ctx, kProfGemm, ev0, ev1, flops);
   }
   return check_cuda(ctx, cudaGetLastError(), "gemm launch");
 }
@@ -997,8 +996,7 @@ metis_status launch_pair(metis_ctx* ctx, const GemmArgs& a) {
   count_launch();
   if (prof) {
     cudaEventRecord(ev1, ctx->stream);
-    ctx->prof_events.emplace_back(ev0, ev1);
-    ctx->prof_flops.push_back(2.0 * (double)p_rows * (double)q_cols * (double)K);
+    profile_record(ctx, kProfGemm, ev0, ev1, 2.0 * (double)p_rows * (double)q_cols * (double)K);
   }
   return check_cuda(ctx, cudaGetLastError(), "gemm pair launch");
 }

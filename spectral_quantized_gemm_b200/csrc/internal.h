@@ -20,8 +20,10 @@ struct metis_ctx {
   size_t ws_bytes = 0;
   std::string last_error;
   bool profiling = false;
-  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> prof_events;
-  std::vector<double> prof_flops;
+  // per instrumented kernel kind (metis::kProf*): event pairs around each launch and the
+  // launch's algorithmic work (flops or bytes)
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> prof_events[3];
+  std::vector<double> prof_work[3];
 };
 
 namespace metis {
@@ -29,6 +31,11 @@ namespace metis {
 // Process-wide count of kernels launched by libmetis.
 extern std::atomic<uint64_t> g_launches;
 inline void count_launch(uint64_t n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// Kernels bracketed by CUDA events while profiling is on (metis_profile_read_kind).
+enum : int { kProfGemm = 0, kProfResquant = 1, kProfProjection = 2, kProfKinds = 3 };
+// Records one launch of `kind` between events ev0 and ev1 (already recorded on ctx->stream).
+void profile_record(metis_ctx* ctx, int kind, cudaEvent_t ev0, cudaEvent_t ev1, double work);
 
 // Sub-allocator over the context workspace: hands out 256-byte aligned slices.
 struct Workspace {
@@ -70,20 +77,29 @@ cudaError_t launch_residual_f32(const void* M_bf16, int64_t rows, int64_t cols, 
                                 cudaStream_t st);
 
 // ---- resquant.cu ----
+// Both orientations in one pass over M; `residual` (nullable, fp32, leading dimension ld_res)
+// receives the residual the quantizer rounded.  Scratch in the context workspace.
 metis_status run_residual_quantize(metis_ctx* ctx, const metis_matrix* M, const metis_factors* f,
-                                   const metis_quant_params* q, const metis_nvfp4* row, const metis_nvfp4* col);
-
-// ---- noalloc.cu ----
-// Limits of the allocation-free residual quantizer's fixed scratch: (rows + cols) x 64
-// floats of padded factors, then 64 floats of which the first word holds the amax of a
-// call that asks for a tensor scale chosen from the data.
-constexpr int64_t kNoAllocMaxRowsPlusCols = 24576;
-constexpr int kNoAllocWidth = 64;
-constexpr int64_t kNoAllocAmaxOffset = kNoAllocMaxRowsPlusCols * kNoAllocWidth;
-float* noalloc_scratch(metis_ctx* ctx, metis_status* st);
+                                   const metis_quant_params* q, const metis_nvfp4* row, const metis_nvfp4* col,
+                                   float* residual = nullptr, int64_t ld_res = 0);
+// Device scratch the pass needs besides the amax word: the fp16 hi/lo factor tiles and
+// their per-block power-of-two factors.
+size_t residual_quantize_scratch_bytes(int64_t rows, int64_t cols);
+// The same pass with caller-provided scratch (residual_quantize_scratch_bytes(rows, cols)
+// bytes, 256-byte aligned) and amax word (used when q->tensor_scale == 0).
 metis_status run_residual_quantize_into(metis_ctx* ctx, const metis_matrix* M, const metis_factors* f,
                                         const metis_quant_params* q, const metis_nvfp4* row, const metis_nvfp4* col,
-                                        float* scratch);
+                                        void* scratch, uint32_t* amax_word, float* residual, int64_t ld_res);
+
+// ---- noalloc.cu ----
+// Limits of the allocation-free residual quantizer's fixed scratch: the factor tiles and
+// block factors of residual_quantize_scratch_bytes for rows + cols <= 24576 (256 bytes
+// per row or column, at most 1 KiB of block factors), then 256 bytes whose first word
+// holds the amax of a call that asks for a tensor scale chosen from the data.
+constexpr int64_t kNoAllocMaxRowsPlusCols = 24576;
+constexpr size_t kNoAllocAmaxOffset = (size_t)kNoAllocMaxRowsPlusCols * 256 + 1024;   // bytes
+constexpr size_t kNoAllocBytes = kNoAllocAmaxOffset + 256;
+char* noalloc_scratch(metis_ctx* ctx, metis_status* st);
 
 // ---- gemm_fp4.cu ----
 struct GemmArgs {

@@ -6,20 +6,31 @@
 // strategy: stochastic rounding).  Every residual is quantized twice, with
 // blocks along each GeMM contraction dimension that reads it.
 //
+// Reconstruction precision.  The notes write the split as exact, so the rank-k part
+// U S V^T is rebuilt on the tensor cores to about 21 bits: every 128-row block of
+// U diag(S) and of V is scaled by a power of two (largest entry in [2^14, 2^15)) and
+// split into fp16 hi + lo, and the MMA accumulates hi*hi + hi*lo + lo*hi in fp32
+// (the dropped lo*lo term and the two splits are each below 2^-22 of a product).  The
+// residual is then one fp32 fused multiply-add, M + acc * (-2^-(a+b)), exact apart
+// from its own rounding.
+//
 // Per 128 x 128 tile of M (persistent CTAs, contiguous row-block-major ranges):
-//   warp 0      TMA: the U*S rows of the row block (kept while the block lasts),
-//               then per tile the V rows and the two 64-column boxes of M (3 stages)
-//   warp 1      tensor-memory owner; one thread issues tcgen05.mma kind::tf32 for the
-//               reconstruction (U S) V^T and for its transpose V (U S)^T, each into a
-//               double-buffered fp32 accumulator (the same operands, swapped)
-//   warps 2..17 a warp per 32 x 32 sub-tile: row-wise quantization of M - (U S) V^T from
-//               its rows (reconstruction rows from tensor memory, M rows from shared
-//               memory), then column-wise quantization of the same sub-tile from the
-//               transposed reconstruction and M's columns; codes and tiled scales go
-//               straight to HBM.  The warps never wait for one another.
-// All mbarrier waits are bounded (METIS_DEV_TIMEOUT on expiry).
+//   warp 0      TMA: the scaled U S hi/lo rows of the row block (kept while the block
+//               lasts), per tile the V hi/lo rows (2 stages) and the two 64-column
+//               boxes of M (3 stages; 5 without factors)
+//   warp 1      tensor-memory owner; one thread issues the twelve tcgen05.mma kind::f16
+//               (M = N = 128, K = 16) of a tile into one of two fp32 accumulators
+//   warps 2..17 a warp per 32 x 32 sub-tile (rows: its tensor-memory lane quarter):
+//               residual of its rows from the accumulator and M, row-wise NVFP4 of
+//               both 16-blocks of each row; the residual passes through a 2 KB
+//               per-warp shared-memory transpose (two halves of 16 columns) and each
+//               lane quantizes one 16-row block of a column per half.  Codes and
+//               tiled scales go straight to HBM.  The warps never wait for one another.
+// All mbarrier waits are bounded (METIS_DEV_TIMEOUT on expiry); on an abort the
+// producer waits (bounded) for the tile loads it issued before the CTA exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -34,17 +45,30 @@ namespace {
 constexpr int kRqEpiWarps = 16;                 // 4 per tensor-memory lane quarter
 constexpr int kRqEpiThreads = kRqEpiWarps * 32;
 constexpr int kRqThreads = 64 + kRqEpiThreads;
+constexpr int kSplitWidth = 64;                 // factor columns (k <= 64), zero-padded
+constexpr long long kDrainLimitCycles = 20000000LL;   // ~10 ms: in-flight loads after an abort
 
-template <int KK>
+template <bool kRecon>
 struct RqCfg {
-  static constexpr int A_BYTES = 128 * KK * 4;   // KK/32 swizzle atoms of 128 rows x 128 B
-  static constexpr int V_BYTES = 128 * KK * 4;
-  static constexpr int M_BYTES = 128 * 128 * 2;  // two 64-column boxes of 16 KB
-  static constexpr int STAGE_BYTES = V_BYTES + M_BYTES;
-  static constexpr int STAGES = 3;
-  static constexpr size_t SMEM = (size_t)A_BYTES + STAGES * STAGE_BYTES + 1024 + 256 + 512;
+  static constexpr int A_BYTES = kRecon ? 32768 : 0;   // U S hi | lo: 2 boxes of 128 rows x 128 B
+  static constexpr int V_BYTES = 32768;                // V hi | lo of the tile's 128 columns
+  static constexpr int V_STAGES = kRecon ? 2 : 0;
+  static constexpr int M_BYTES = 32768;                // two 64-column boxes of 16 KB
+  static constexpr int M_STAGES = kRecon ? 4 : 6;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int RCP_BYTES = 512;
+  static constexpr size_t SMEM =
+      1024 + (size_t)A_BYTES + V_STAGES * V_BYTES + M_STAGES * M_BYTES + BAR_BYTES + RCP_BYTES;
   static_assert(SMEM <= 232448, "shared memory budget");
 };
+
+// Output staging inside a consumed M stage (byte offsets): the tile's row-wise codes
+// (128 rows x 64 B) and column-wise codes (128 columns x 64 B), both in the 64-byte
+// swizzle of their TMA store boxes, then its two 1 KB runs of tiled scales.
+constexpr int kStRowCodes = 0;
+constexpr int kStColCodes = 8192;
+constexpr int kStRowScales = 16384;
+constexpr int kStColScales = 17408;
 
 struct RqParams {
   int64_t rows, cols;
@@ -60,20 +84,77 @@ struct RqParams {
   float* row_g;
   float* col_g;
   const uint32_t* amax_bits;   // non-null: g chosen from the data (auto_tensor_scale)
+  const float* fac_a;          // 2^-a per 128-row block of U S (rows / 128)
+  const float* fac_b;          // 2^-b per 128-row block of V (cols / 128)
+  float* residual;             // non-null (parity surface): the fp32 residual, leading dimension ld_res
+  int64_t ld_res;
   uint32_t* status;
 };
 
-__host__ __device__ __forceinline__ uint32_t idesc_tf32(uint32_t n) {
-  return (1u << 4) | (2u << 7) | (2u << 10) | ((n >> 3) << 17) | ((128u >> 4) << 24);
+// fp16 x fp16 -> fp32, both operands K-major, M = N = 128.
+constexpr uint32_t kIdescF16 = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %3, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %4, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(accumulate), "r"(kIdescF16)
+      : "memory");
 }
 
-__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
+// ---- shared-memory accesses by 32-bit shared address ------------------------
+__device__ __forceinline__ void sts_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ float4 lds_f32x4(uint32_t addr) {
+  float4 r;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w) : "r"(addr)
+               : "memory");
+  return r;
+}
+__device__ __forceinline__ uint4 lds_u32x4(uint32_t addr) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(addr)
+               : "memory");
+  return r;
+}
+
+// ---- packed fp32 pairs (sm_100a) and the block maximum ----------------------
+// d = a * s + c per lane, each an IEEE fused multiply-add rounded to nearest.
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float s, float c0, float c1) {
+  asm("{\n\t.reg .b64 ra, rs, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rs, {%4, %4};\n\tmov.b64 rc, {%5, %6};\n\t"
+      "fma.rn.f32x2 rd, ra, rs, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(s), "f"(c0), "f"(c1));
+}
+// d = a * s per lane, rounded to nearest.
+__device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1, float s) {
+  asm("{\n\t.reg .b64 ra, rs, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rs, {%4, %4};\n\t"
+      "mul.rn.f32x2 rd, ra, rs;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(s));
+}
+// Largest of three magnitudes; NaN if any input is NaN.
+__device__ __forceinline__ float max3_abs(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(fabsf(a)), "f"(fabsf(b)), "f"(fabsf(c)));
+  return d;
+}
+__device__ __forceinline__ float max3_nan(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// max |x_i| over a 16-block (NaN if an element is NaN, Inf if one is infinite).
+__device__ __forceinline__ float block_amax(const float* x) {
+  const float m0 = max3_abs(x[0], x[1], x[2]);
+  const float m1 = max3_abs(x[3], x[4], x[5]);
+  const float m2 = max3_abs(x[6], x[7], x[8]);
+  const float m3 = max3_abs(x[9], x[10], x[11]);
+  const float m4 = max3_abs(x[12], x[13], x[14]);
+  return max3_nan(max3_nan(m0, m1, m2), max3_nan(m3, m4, fabsf(x[15])), 0.0f);
 }
 
 // The block rule of block_scale() with two exact shortcuts for this kernel:
@@ -100,42 +181,47 @@ __device__ __forceinline__ BlockScale block_scale_fast(float amax, float g, cons
   return bs;
 }
 
-// One 16-element block: scale code and packed codes (RN or SR with the Philox
-// stream of element index e0 .. e0 + 15 in the orientation's blocked order).  amax is
-// the block's largest |v| (computed by the caller).
-__device__ __forceinline__ uint2 quantize16(const float (&v)[16], float amax, float g, const float* rcp_table,
+// One 16-element block with its maximum: scale code and packed codes (RN, or SR with
+// the Philox call of element index e0 .. e0 + 15 in the orientation's blocked order).
+__device__ __forceinline__ uint2 quantize16(const float* v, float amax, float g, const float* rcp_table,
                                             int rounding, uint64_t seed, uint32_t tag, uint32_t step, uint64_t e0,
                                             uint32_t& scale_code) {
   const BlockScale bs = block_scale_fast(amax, g, rcp_table);
   float x[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) x[i] = __fmul_rn(v[i], bs.rcp);
+  for (int i = 0; i < 16; i += 2) mul2(x[i], x[i + 1], v[i], v[i + 1], bs.rcp);
   uint2 packed = encode_block16(x, rounding, seed, tag, step, e0);
   if (bs.code == 0) packed = make_uint2(0, 0);
   scale_code = bs.code;
   return packed;
 }
 
-template <int KK>
+template <bool kRecon, bool kDump>
 __global__ void __launch_bounds__(kRqThreads, 1)
-    resquant_kernel(const __grid_constant__ CUtensorMap mapM, const __grid_constant__ CUtensorMap mapUS,
-                    const __grid_constant__ CUtensorMap mapV, const RqParams p) {
-  using C = RqCfg<KK>;
+    resquant_kernel(const __grid_constant__ CUtensorMap mapM, const __grid_constant__ CUtensorMap mapA,
+                    const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapRowCodes,
+                    const __grid_constant__ CUtensorMap mapColCodes, const RqParams p) {
+  using C = RqCfg<kRecon>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sStage = sA + C::A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + C::STAGES * C::STAGE_BYTES);
+  uint8_t* sV = sA + C::A_BYTES;
+  uint8_t* sM = sV + C::V_STAGES * C::V_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sM + C::M_STAGES * C::M_BYTES);
   uint64_t* a_full = bars;
   uint64_t* a_empty = bars + 1;
-  uint64_t* full = bars + 2;                 // [STAGES]
-  uint64_t* empty = full + C::STAGES;        // [STAGES]
-  uint64_t* acc_full = empty + C::STAGES;    // [2]
-  uint64_t* acc_empty = acc_full + 2;        // [2]
+  uint64_t* v_full = bars + 2;                    // [2]
+  uint64_t* v_empty = v_full + 2;                 // [2]
+  uint64_t* m_full = v_empty + 2;                 // [M_STAGES <= 6]
+  uint64_t* m_empty = m_full + 6;                 // [6]
+  uint64_t* acc_full = m_empty + 6;               // [2]
+  uint64_t* acc_empty = acc_full + 2;             // [2]
   uint64_t* drain = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* ep_done = drain + 1;                  // every epilogue warp is done with the tile's M stage
+  uint64_t* ep_staged = ep_done + 1;              // every epilogue warp has staged the tile's outputs
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ep_staged + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* rcp_table = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);   // 128 entries
+  float* rcp_table = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + C::BAR_BYTES);   // 128 entries
 
   const float g = p.amax_bits ? auto_tensor_scale(*p.amax_bits) : p.g;
   for (int c = threadIdx.x; c < 128; c += blockDim.x)
@@ -143,22 +229,25 @@ __global__ void __launch_bounds__(kRqThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int per = (p.n_units + gridDim.x - 1) / gridDim.x;
-  const int u_begin = blockIdx.x * per;
-  const int u_end = min(p.n_units, u_begin + per);
+  const int u_begin = (int)(((int64_t)blockIdx.x * p.n_units) / gridDim.x);
+  const int u_end = (int)(((int64_t)(blockIdx.x + 1) * p.n_units) / gridDim.x);
 
   if (threadIdx.x == 0) {
     tc::mbar_init(a_full, 1);
     tc::mbar_init(a_empty, 1);
-    for (int s = 0; s < C::STAGES; ++s) {
-      tc::mbar_init(&full[s], 1);
-      tc::mbar_init(&empty[s], 1 + kRqEpiThreads / 32);
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&v_full[s], 1);
+      tc::mbar_init(&v_empty[s], 1);
+      tc::mbar_init(&acc_full[s], 1);
+      tc::mbar_init(&acc_empty[s], kRqEpiWarps);
     }
-    for (int b = 0; b < 2; ++b) {
-      tc::mbar_init(&acc_full[b], 1);
-      tc::mbar_init(&acc_empty[b], kRqEpiThreads / 32);
+    for (int s = 0; s < C::M_STAGES; ++s) {
+      tc::mbar_init(&m_full[s], 1);
+      tc::mbar_init(&m_empty[s], 1);   // released by the thread that stores the staged outputs
     }
     tc::mbar_init(drain, 1);
+    tc::mbar_init(ep_done, kRqEpiWarps);
+    tc::mbar_init(ep_staged, kRqEpiWarps);
     *abort_flag = 0;
     tc::fence_barrier_init();
     if (blockIdx.x == 0) {
@@ -166,14 +255,14 @@ __global__ void __launch_bounds__(kRqThreads, 1)
       *p.col_g = g;
     }
   }
-  if (warp == 1) {   // columns 0-255: reconstruction, 256-511: its transpose (two buffers each)
-    tc::tmem_alloc(tmem_slot, 512);
+  if (kRecon && warp == 1) {   // two 128-column fp32 accumulators
+    tc::tmem_alloc(tmem_slot, 256);
     tc::tmem_relinquish();
   }
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = kRecon ? *tmem_slot : 0u;
 
   auto fail_wait = [&]() {
     *abort_flag = 1;
@@ -182,246 +271,435 @@ __global__ void __launch_bounds__(kRqThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0, a_phase = 0;
+      // parity of the last load issued into each slot (bit s), and which slots were used
+      uint32_t m_par = 0, m_used = 0, v_par = 0, v_used = 0, a_par = 0, a_used = 0;
+      int ms = 0, vs = 0;
+      uint32_t mph = 0, vph = 0, aph = 0;
       int cur_rb = -1;
       for (int u = u_begin; u < u_end && !*abort_flag; ++u) {
         const int rb = u / p.n_cb, cb = u % p.n_cb;
-        if (rb != cur_rb) {
-          if (!tc::mbar_wait(a_empty, a_phase ^ 1u, abort_flag)) { fail_wait(); break; }
-          tc::mbar_expect_tx(a_full, C::A_BYTES);
-#pragma unroll
-          for (int ch = 0; ch < KK / 32; ++ch) tc::tma_load_2d(sA + ch * 16384, &mapUS, a_full, ch * 32, rb * 128);
-          a_phase ^= 1u;
-          cur_rb = rb;
+        if (kRecon) {
+          if (rb != cur_rb) {
+            if (!tc::mbar_wait(a_empty, aph ^ 1u, abort_flag)) { fail_wait(); break; }
+            tc::mbar_expect_tx(a_full, C::A_BYTES);
+            tc::tma_load_2d(sA, &mapA, a_full, 0, rb * 128);
+            tc::tma_load_2d(sA + 16384, &mapA, a_full, 64, rb * 128);
+            a_par = aph;
+            a_used = 1;
+            aph ^= 1u;
+            cur_rb = rb;
+          }
+          if (!tc::mbar_wait(&v_empty[vs], vph ^ 1u, abort_flag)) { fail_wait(); break; }
+          uint8_t* dv = sV + vs * C::V_BYTES;
+          tc::mbar_expect_tx(&v_full[vs], C::V_BYTES);
+          tc::tma_load_2d(dv, &mapV, &v_full[vs], 0, cb * 128);
+          tc::tma_load_2d(dv + 16384, &mapV, &v_full[vs], 64, cb * 128);
+          v_par = (v_par & ~(1u << vs)) | (vph << vs);
+          v_used |= 1u << vs;
+          if (++vs == 2) {
+            vs = 0;
+            vph ^= 1u;
+          }
         }
-        if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { fail_wait(); break; }
-        uint8_t* sV = sStage + stage * C::STAGE_BYTES;
-        uint8_t* sM = sV + C::V_BYTES;
-        tc::mbar_expect_tx(&full[stage], C::STAGE_BYTES);
-#pragma unroll
-        for (int ch = 0; ch < KK / 32; ++ch) tc::tma_load_2d(sV + ch * 16384, &mapV, &full[stage], ch * 32, cb * 128);
-        tc::tma_load_2d(sM, &mapM, &full[stage], cb * 128, rb * 128);
-        tc::tma_load_2d(sM + 16384, &mapM, &full[stage], cb * 128 + 64, rb * 128);
-        if (++stage == C::STAGES) {
-          stage = 0;
-          phase ^= 1u;
+        if (!tc::mbar_wait(&m_empty[ms], mph ^ 1u, abort_flag)) { fail_wait(); break; }
+        uint8_t* dm = sM + ms * C::M_BYTES;
+        tc::mbar_expect_tx(&m_full[ms], C::M_BYTES);
+        tc::tma_load_2d(dm, &mapM, &m_full[ms], cb * 128, rb * 128);
+        tc::tma_load_2d(dm + 16384, &mapM, &m_full[ms], cb * 128 + 64, rb * 128);
+        m_par = (m_par & ~(1u << ms)) | (mph << ms);
+        m_used |= 1u << ms;
+        if (++ms == C::M_STAGES) {
+          ms = 0;
+          mph ^= 1u;
         }
       }
+      // No copy into this CTA's shared memory may still be in flight when it exits:
+      // wait for the last phase issued on every slot (already complete unless aborted).
+      for (int s = 0; s < C::M_STAGES; ++s)
+        if (m_used >> s & 1u) tc::mbar_wait(&m_full[s], m_par >> s & 1u, nullptr, kDrainLimitCycles);
+      for (int s = 0; s < 2; ++s)
+        if (v_used >> s & 1u) tc::mbar_wait(&v_full[s], v_par >> s & 1u, nullptr, kDrainLimitCycles);
+      if (a_used) tc::mbar_wait(a_full, a_par, nullptr, kDrainLimitCycles);
     }
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0, a_phase = 0;
+    if (kRecon && lane == 0) {
+      int vs = 0;
+      uint32_t vph = 0, aph = 0;
       int cur_rb = -1;
       int it = 0;
-      const uint32_t idesc = idesc_tf32(128);
       for (int u = u_begin; u < u_end && !*abort_flag; ++u, ++it) {
         const int rb = u / p.n_cb;
         if (rb != cur_rb) {
-          if (cur_rb >= 0) tc::tc_commit(a_empty);  // the old U*S rows are no longer read
-          if (!tc::mbar_wait(a_full, a_phase, abort_flag)) { fail_wait(); break; }
-          a_phase ^= 1u;
+          if (cur_rb >= 0) tc::tc_commit(a_empty);  // the old U S rows are no longer read
+          if (!tc::mbar_wait(a_full, aph, abort_flag)) { fail_wait(); break; }
+          aph ^= 1u;
           cur_rb = rb;
         }
         const int b = it & 1;
         const uint32_t use = (uint32_t)(it >> 1);
-        if (!tc::mbar_wait(&full[stage], phase, abort_flag)) { fail_wait(); break; }
+        if (!tc::mbar_wait(&v_full[vs], vph, abort_flag)) { fail_wait(); break; }
         if (!tc::mbar_wait(&acc_empty[b], (use & 1u) ^ 1u, abort_flag)) { fail_wait(); break; }
         tc::tc_fence_after();
-        const uint8_t* sV = sStage + stage * C::STAGE_BYTES;
+        const uint8_t* v = sV + vs * C::V_BYTES;
+        const uint64_t a_hi = tc::sdesc_sw128(tc::smem_addr(sA));
+        const uint64_t a_lo = tc::sdesc_sw128(tc::smem_addr(sA + 16384));
+        const uint64_t b_hi = tc::sdesc_sw128(tc::smem_addr(v));
+        const uint64_t b_lo = tc::sdesc_sw128(tc::smem_addr(v + 16384));
+        const uint32_t d = tmem + (uint32_t)(b * 128);
+        // K = 64 in four steps of 16 halfs (32 bytes of the 128-byte swizzled rows)
 #pragma unroll
-        for (int ch = 0; ch < KK / 32; ++ch) {
-          const uint64_t ad = tc::sdesc_sw128(tc::smem_addr(sA + ch * 16384));
-          const uint64_t bd = tc::sdesc_sw128(tc::smem_addr(sV + ch * 16384));
+        for (int j = 0; j < 4; ++j) mma_f16(d, a_hi + 2 * j, b_hi + 2 * j, j ? 1u : 0u);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            mma_tf32(tmem + b * 128, ad + 2 * j, bd + 2 * j, idesc, (ch | j) ? 1u : 0u);          // rows of the tile
-            mma_tf32(tmem + 256 + b * 128, bd + 2 * j, ad + 2 * j, idesc, (ch | j) ? 1u : 0u);    // its columns
-          }
-        }
-        tc::tc_commit(&empty[stage]);
+        for (int j = 0; j < 4; ++j) mma_f16(d, a_hi + 2 * j, b_lo + 2 * j, 1u);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mma_f16(d, a_lo + 2 * j, b_hi + 2 * j, 1u);
+        tc::tc_commit(&v_empty[vs]);
         tc::tc_commit(&acc_full[b]);
-        if (++stage == C::STAGES) {
-          stage = 0;
-          phase ^= 1u;
+        if (++vs == 2) {
+          vs = 0;
+          vph ^= 1u;
         }
       }
       tc::tc_commit(drain);
-      tc::mbar_wait(drain, 0, nullptr);
+      tc::mbar_wait(drain, 0, nullptr, kDrainLimitCycles);
     }
     __syncwarp();
   } else {
-    const int q = warp & 3;            // tensor-memory lane quarter
-    const int h = (warp - 2) >> 2;     // 32-column quarter (row pass) = 32-row quarter (column pass)
-    const int r = q * 32 + lane;       // tile row of this thread in the row pass
-    const int j = q * 32 + lane;       // tile column of this thread in the column pass
-    // M(i, j) of the column pass sits in box j >> 6 at row i, 16-byte chunk
-    // ((j & 63) >> 3) ^ (i & 7), element j & 7: the 8 chunk positions, by i & 7
-    const int jc = (j & 63) >> 3;
-    uint32_t col_off[8];
-#pragma unroll
-    for (int t = 0; t < 8; ++t) col_off[t] = (uint32_t)((j >> 6) * 16384 + (((jc ^ t) << 4) | ((j & 7) << 1)));
-    int stage = 0;
-    uint32_t phase = 0;
+    const int e = warp - 2;
+    const int q = warp & 3;            // tensor-memory lane quarter: tile rows q*32 .. + 31
+    const int h = e >> 2;              // tile columns h*32 .. + 31
+    const int r = q * 32 + lane;       // tile row of this lane in the row pass
+    const int jc = lane & 15;          // column (within a half) of this lane in the column pass
+    const int hh = lane >> 4;          // 16-row half of the sub-tile in the column pass
+    const bool issuer = (e == 0 && lane == 0);
+    // The warp's own bytes of an M stage (rows q*32 .. + 31 of box h >> 1, its four 16-byte
+    // chunks of each row) double as its transpose buffer once it has read them: element
+    // (row l, column c) of a 32 x 16 half sits in row rho = q*32 + 8*(c & 3) + ((l >> 2) ^ (c & 7)),
+    // chunk (h & 1)*4 + (c >> 2) (swizzled like M), word l & 3 -- conflict-free for the
+    // 32 row-wise stores of a column and for the 128-bit loads of 16-row column blocks.
+    const uint32_t box_off = (uint32_t)(h >> 1) * 16384;
+    // Address parts of those accesses that depend on the lane only.  With S the (1024-byte
+    // aligned) shared address of the stage's box, the fields below bit 10 combine by XOR:
+    //   M row read, chunk j of the half:   (S + m_part) ^ (16 j)
+    //   transpose store of column c:       ((S + t_part) ^ x(c)) + 1024 (c & 3)
+    //   transpose load of chunk m4:         (S + l_part) ^ (144 m4)
+    const uint32_t Kh = (uint32_t)(h & 1) * 4;
+    const uint32_t L = (uint32_t)lane >> 2;
+    const uint32_t m_part = (uint32_t)r * 128 + 16 * (Kh ^ ((uint32_t)r & 7));
+    const uint32_t t_part = (uint32_t)q * 4096 + 128 * L + 16 * (Kh ^ L) + 4 * ((uint32_t)lane & 3);
+    const uint32_t j7 = (uint32_t)jc & 7, k0 = 4 * (uint32_t)hh;
+    const uint32_t l_part = (uint32_t)q * 4096 + 1024 * ((uint32_t)jc & 3) + 128 * (k0 ^ j7) +
+                            16 * (Kh ^ ((uint32_t)jc >> 2) ^ k0 ^ j7);
+    int ms = 0;
+    uint32_t mph = 0;
+    int pending = -1;                  // stage whose staged outputs are still being stored
     int it = 0;
     for (int u = u_begin; u < u_end; ++u, ++it) {
       const int rb = u / p.n_cb, cb = u % p.n_cb;
       const int b = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
-      bool ok = tc::mbar_wait(&acc_full[b], use & 1u, abort_flag);
-      ok = ok && tc::mbar_wait(&full[stage], phase, abort_flag);
+      bool ok = true;
+      if (kRecon) ok = tc::mbar_wait(&acc_full[b], use & 1u, abort_flag);
+      ok = ok && tc::mbar_wait(&m_full[ms], mph, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) fail_wait();
         break;
       }
-      tc::tc_fence_after();
-      const uint8_t* sM = sStage + stage * C::STAGE_BYTES + C::V_BYTES;
-      // ---- row-wise quantization (blocks along columns): row r, columns h*32 .. + 31
-      {
-        float v[32];
-        tc::tmem_load_32cols(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * 128 + h * 32), v);
-        tc::tmem_load_wait();
-        // residual = M - reconstruction (M from the 128B-swizzled 64-column box holding
-        // this quarter: chunks (h & 1) * 4 .. + 3 of box h >> 1)
-        const uint8_t* sMb = sM + (h >> 1) * 16384;
+      uint8_t* stage = sM + ms * C::M_BYTES;
+      const uint32_t S = tc::smem_addr(stage) + box_off;
+      const int64_t grow = (int64_t)rb * 128 + r;
+      const int64_t gcol = (int64_t)cb * 128 + h * 32;
+      const int64_t grow_t = (int64_t)rb * 128 + q * 32 + hh * 16;   // first row of this lane's column blocks
+      float nf = 0.0f;
+      if (kRecon) nf = -__fmul_rn(__ldg(p.fac_a + rb), __ldg(p.fac_b + cb));   // -2^-(a + b), exact
+      uint4 row_out;
+      uint32_t row_sc = 0;
+      uint2 col_out[2];
+      uint32_t col_sc[2];
+      bool finite = true;
+      // M row r, columns h*32 .. + 31: box h >> 1, chunks (h & 1)*4 .. + 3, all read before the
+      // first transpose store reuses the region
+      uint32_t mrow[16];
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int c = (h & 1) * 4 + cc;
-          const uint4 raw = *reinterpret_cast<const uint4*>(sMb + r * 128 + ((c ^ (r & 7)) << 4));
-          const __nv_bfloat162* pr = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 f = __bfloat1622float2(pr[i]);
-            v[cc * 8 + 2 * i] = f.x - v[cc * 8 + 2 * i];
-            v[cc * 8 + 2 * i + 1] = f.y - v[cc * 8 + 2 * i + 1];
-          }
-        }
-        const int64_t grow = (int64_t)rb * 128 + r;
-        const int64_t gcol = (int64_t)cb * 128 + h * 32;
-        uint32_t sc = 0;
-        uint4 out;
-        uint32_t* o = reinterpret_cast<uint32_t*>(&out);
-        bool finite = true;
-#pragma unroll
-        for (int blk = 0; blk < 2; ++blk) {
-          float x[16];
-          // block maximum of |x|: fmaxf keeps an Inf but drops a NaN, which a sum of the
-          // block's magnitudes then shows (the sum is NaN exactly when an element is)
-          float amax = 0.0f, sum = 0.0f;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            x[i] = v[blk * 16 + i];
-            amax = fmaxf(amax, fabsf(x[i]));
-            sum += fabsf(x[i]);
-          }
-          finite &= (amax <= 3.402823466e38f) && (sum == sum);
-          uint32_t code;
-          const uint2 pk = quantize16(x, amax, g, rcp_table, p.rounding, p.seed, p.tag_row,
-                                      p.step, (uint64_t)grow * (uint64_t)p.cols + (uint64_t)(gcol + blk * 16), code);
-          sc |= code << (8 * blk);
-          o[2 * blk] = pk.x;
-          o[2 * blk + 1] = pk.y;
-        }
-        if (!finite) raise_status(p.status, METIS_DEV_NONFINITE);
-        *reinterpret_cast<uint4*>(p.row_codes + grow * (p.cols / 2) + gcol / 2) = out;
-        *reinterpret_cast<uint16_t*>(p.row_scales + scale_offset(grow, gcol / 16, p.cols / 64)) = (uint16_t)sc;
+      for (int cc = 0; cc < 4; ++cc) {
+        const uint4 raw = lds_u32x4((S + m_part) ^ (uint32_t)(16 * cc));
+        mrow[4 * cc] = raw.x;
+        mrow[4 * cc + 1] = raw.y;
+        mrow[4 * cc + 2] = raw.z;
+        mrow[4 * cc + 3] = raw.w;
       }
-      // ---- column-wise quantization (blocks along rows): column j, rows h*32 .. + 31,
-      // from the transposed reconstruction (tensor-memory lane j) and M's column j
-      {
-        const uint8_t* cbase[8];
+      __syncwarp();   // every lane has read its M row before the region is reused
+      // the sub-tile in two halves of 16 columns: residual, row-wise block, transpose, column-wise block
 #pragma unroll
-        for (int t = 0; t < 8; ++t) cbase[t] = sM + h * 32 * 128 + col_off[t];
-        float w[32];
-        tc::tmem_load_32cols(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(256 + b * 128 + h * 32), w);
-        tc::tmem_load_wait();
-        tc::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&acc_empty[b]);   // both reconstructions of this tile are read
-        const int64_t gcolj = (int64_t)cb * 128 + j;
-        const int64_t grow0 = (int64_t)rb * 128 + h * 32;
-        uint32_t sc = 0;
-        uint4 out;
-        uint32_t* o = reinterpret_cast<uint32_t*>(&out);
-#pragma unroll
-        for (int blk = 0; blk < 2; ++blk) {
-          float x[16];
-          float amax = 0.0f;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const uint16_t mb = *reinterpret_cast<const uint16_t*>(cbase[i & 7] + (blk * 16 + i) * 128);  // tile row h*32+blk*16+i
-            x[i] = __uint_as_float((uint32_t)mb << 16) - w[blk * 16 + i];
-            amax = fmaxf(amax, fabsf(x[i]));
+      for (int half = 0; half < 2; ++half) {
+        const uint32_t* mw = mrow + 8 * half;
+        float v[16];
+        if (kRecon) {
+          float acc[16];
+          if (half == 0) tc::tc_fence_after();
+          tc::tmem_load_16cols(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * 128 + h * 32 + half * 16), acc);
+          tc::tmem_load_wait();
+          if (half == 1) {
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&acc_empty[b]);   // both halves of the accumulator are read
           }
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            fma2(v[2 * i], v[2 * i + 1], acc[2 * i], acc[2 * i + 1], nf, __uint_as_float(mw[i] << 16),
+                 __uint_as_float(mw[i] & 0xFFFF0000u));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            v[2 * i] = __uint_as_float(mw[i] << 16);
+            v[2 * i + 1] = __uint_as_float(mw[i] & 0xFFFF0000u);
+          }
+        }
+        if (kDump) {
+          float4* dst = reinterpret_cast<float4*>(p.residual + grow * p.ld_res + gcol + 16 * half);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+        // transpose this half into the warp's region of the stage
+        {
+          const uint32_t T = S + t_part;
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const uint32_t x = 128u * (uint32_t)(c & 7) + 16u * ((uint32_t)(c >> 2) ^ (uint32_t)(c & 7));
+            sts_f32((T ^ x) + 1024u * (uint32_t)(c & 3), v[c]);
+          }
+        }
+        // row-wise block `half` of row r
+        {
+          const float amax = block_amax(v);
+          finite &= amax <= 3.402823466e38f;   // false for NaN and Inf
           uint32_t code;
-          const uint2 pk = quantize16(x, amax, g, rcp_table, p.rounding, p.seed, p.tag_col, p.step,
-                                      (uint64_t)gcolj * (uint64_t)p.rows + (uint64_t)(grow0 + blk * 16), code);
-          sc |= code << (8 * blk);
-          o[2 * blk] = pk.x;
-          o[2 * blk + 1] = pk.y;
+          const uint2 pk = quantize16(v, amax, g, rcp_table, p.rounding, p.seed, p.tag_row, p.step,
+                                      (uint64_t)grow * (uint64_t)p.cols + (uint64_t)(gcol + 16 * half), code);
+          row_sc |= code << (8 * half);
+          if (half == 0) {
+            row_out.x = pk.x;
+            row_out.y = pk.y;
+          } else {
+            row_out.z = pk.x;
+            row_out.w = pk.y;
+          }
         }
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&empty[stage]);   // this warp is done with M
-        *reinterpret_cast<uint4*>(p.col_codes + gcolj * (p.rows / 2) + grow0 / 2) = out;
-        *reinterpret_cast<uint16_t*>(p.col_scales + scale_offset(gcolj, grow0 / 16, p.rows / 64)) = (uint16_t)sc;
+        // column-wise block: column half*16 + jc of the sub-tile, rows hh*16 .. + 15
+        {
+          float w[16];
+#pragma unroll
+          for (int m4 = 0; m4 < 4; ++m4) {
+            const float4 t4 = lds_f32x4((S + l_part) ^ (144u * (uint32_t)m4));
+            w[4 * m4] = t4.x;
+            w[4 * m4 + 1] = t4.y;
+            w[4 * m4 + 2] = t4.z;
+            w[4 * m4 + 3] = t4.w;
+          }
+          const float amax = block_amax(w);
+          const int64_t gc = gcol + 16 * half + jc;
+          col_out[half] = quantize16(w, amax, g, rcp_table, p.rounding, p.seed, p.tag_col, p.step,
+                                     (uint64_t)gc * (uint64_t)p.rows + (uint64_t)grow_t, col_sc[half]);
+        }
+        __syncwarp();
+        if (half == 0 && issuer && pending >= 0) {   // the previous tile's stores have long read their stage
+          tc::bulk_wait_read_all();
+          tc::mbar_arrive(&m_empty[pending]);
+          pending = -1;
+        }
       }
-      if (++stage == C::STAGES) {
-        stage = 0;
-        phase ^= 1u;
+      if (!finite) raise_status(p.status, METIS_DEV_NONFINITE);
+      // ---- every warp is done with this M stage: stage the tile's outputs in it
+      if (lane == 0) tc::mbar_arrive(ep_done);
+      ok = tc::mbar_wait(ep_done, (uint32_t)it & 1u, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) fail_wait();
+        break;
+      }
+      {
+        // row codes: row r, bytes h*16 .. + 15 of its 64 (chunk h, 64B swizzle)
+        *reinterpret_cast<uint4*>(stage + kStRowCodes + r * 64 + ((h ^ ((r >> 1) & 3)) << 4)) = row_out;
+        // row scales: tile (h >> 1) of the two, entry (r % 32, r / 32, blocks 2(h & 1), +1)
+        *reinterpret_cast<uint16_t*>(stage + kStRowScales + (h >> 1) * 512 + lane * 16 + q * 4 + 2 * (h & 1)) =
+            (uint16_t)row_sc;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int cl = h * 32 + half * 16 + jc;   // tile column
+          // column codes: column cl, rows q*32 + hh*16 .. + 15 = bytes q*16 + hh*8 .. + 7 (chunk q)
+          *reinterpret_cast<uint2*>(stage + kStColCodes + cl * 64 + ((q ^ ((cl >> 1) & 3)) << 4) + hh * 8) =
+              col_out[half];
+          // column scales: tile (q >> 1), entry (cl % 32, cl / 32, block (2q + hh) & 3)
+          stage[kStColScales + (q >> 1) * 512 + (cl & 31) * 16 + h * 4 + ((2 * q + hh) & 3)] = (uint8_t)col_sc[half];
+        }
+      }
+      tc::fence_proxy_async();   // the staged bytes are read by the bulk-copy (async) proxy
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(ep_staged);
+      ok = tc::mbar_wait(ep_staged, (uint32_t)it & 1u, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) fail_wait();
+        break;
+      }
+      if (issuer) {
+        tc::tma_store_2d(&mapRowCodes, stage + kStRowCodes, cb * 64, rb * 128);
+        tc::tma_store_2d(&mapColCodes, stage + kStColCodes, rb * 64, cb * 128);
+        tc::bulk_store(p.row_scales + ((int64_t)rb * (p.cols / 64) + (int64_t)cb * 2) * 512, stage + kStRowScales,
+                       1024);
+        tc::bulk_store(p.col_scales + ((int64_t)cb * (p.rows / 64) + (int64_t)rb * 2) * 512, stage + kStColScales,
+                       1024);
+        tc::bulk_commit_group();
+        pending = ms;
+      }
+      if (++ms == C::M_STAGES) {
+        ms = 0;
+        mph ^= 1u;
       }
     }
+    if (issuer) tc::bulk_wait_all();   // no store may still read this CTA's shared memory at exit
   }
 
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (kRecon && warp == 1) {
     tc::tc_fence_after();
-    tc::tmem_dealloc(tmem, 512);
+    tc::tmem_dealloc(tmem, 256);
   }
 }
 
-// US (rows x KK) = U diag(S) and Vp (cols x KK) = V, zero-padded to KK columns.
-__global__ void pad_factors_kernel(const float* __restrict__ U, const float* __restrict__ S,
-                                   const float* __restrict__ V, int64_t rows, int64_t cols, int k, int KK,
-                                   float* __restrict__ US, float* __restrict__ Vp) {
-  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t nu = rows * KK;
-  if (e < nu) {
-    const int64_t i = e / KK;
-    const int j = (int)(e - i * KK);
-    US[e] = (j < k) ? U[i * k + j] * S[j] : 0.0f;
-  } else if (e < nu + cols * KK) {
-    const int64_t f = e - nu;
-    const int64_t i = f / KK;
-    const int j = (int)(f - i * KK);
-    Vp[f] = (j < k) ? V[i * k + j] : 0.0f;
+// One CTA per 128-row block of U diag(S) (the first rows / 128 CTAs) or of V (the rest):
+// the block's largest |entry| m sets the power of two 2^e with m 2^e in [2^14, 2^15)
+// (e kept in [-63, 63]; 0 for an all-zero block), and every entry x (k columns, padded
+// with zeros to 64) is written as the fp16 pair hi = RN16(x 2^e), lo = RN16(x 2^e - hi):
+// row i of the output holds the 64 hi values, then the 64 lo values.  fac[block] = 2^-e.
+__global__ void __launch_bounds__(256) split_factors_kernel(const float* __restrict__ U, const float* __restrict__ S,
+                                                            const float* __restrict__ V, int64_t rows, int k,
+                                                            __half* __restrict__ A16, __half* __restrict__ B16,
+                                                            float* __restrict__ fac_a, float* __restrict__ fac_b) {
+  __shared__ float red[8];
+  const int64_t nb_a = rows / 128;
+  const bool is_a = (int64_t)blockIdx.x < nb_a;
+  const int64_t blk = is_a ? (int64_t)blockIdx.x : (int64_t)blockIdx.x - nb_a;
+  const float* F = (is_a ? U : V) + blk * 128 * k;
+  __half* out = (is_a ? A16 : B16) + blk * 128 * 128;
+  float m = 0.0f;
+  for (int t = threadIdx.x; t < 128 * k; t += blockDim.x) {
+    float x = F[t];
+    if (is_a) x = __fmul_rn(x, S[t % k]);
+    m = fmaxf(m, fabsf(x));
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = red[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w]);
+  int ex = 0;
+  if (m > 0.0f && m <= 3.402823466e38f) {
+    const int fl = (int)((__float_as_uint(m) >> 23) & 0xFFu) - 127;   // floor(log2 m); -127 for subnormal m
+    ex = min(63, max(-63, 14 - fl));
+  }
+  const float up = __uint_as_float((uint32_t)(ex + 127) << 23);
+  if (threadIdx.x == 0) (is_a ? fac_a : fac_b)[blk] = __uint_as_float((uint32_t)(127 - ex) << 23);
+  for (int t = threadIdx.x; t < 128 * kSplitWidth; t += blockDim.x) {
+    const int i = t >> 6, j = t & 63;
+    float x = 0.0f;
+    if (j < k) {
+      x = F[i * k + j];
+      if (is_a) x = __fmul_rn(x, S[j]);
+    }
+    x = __fmul_rn(x, up);
+    const __half hi = __float2half_rn(x);
+    const __half lo = __float2half_rn(__fsub_rn(x, __half2float(hi)));
+    out[i * 128 + j] = hi;
+    out[i * 128 + 64 + j] = lo;
   }
 }
 
 bool map2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t inner, uint64_t outer,
-           uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+           uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+           CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {row_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
   EncodeTiledFn enc = encode_tiled();
   return enc && enc(map, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+                    swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int KK>
-metis_status launch_kk(metis_ctx* ctx, const metis_matrix* M, const float* US, const float* Vp,
-                       const metis_quant_params* q, const uint32_t* amax_bits, const metis_nvfp4* row,
-                       const metis_nvfp4* col) {
-  using C = RqCfg<KK>;
-  CUtensorMap mM, mU, mV;
+template <bool kRecon, bool kDump>
+metis_status launch_rq(metis_ctx* ctx, const metis_matrix* M, const CUtensorMap& mA, const CUtensorMap& mV,
+                       RqParams prm) {
+  using C = RqCfg<kRecon>;
+  CUtensorMap mM, mRow, mCol;
   if (!map2d(&mM, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, M->data, M->cols, M->rows, (uint64_t)M->ld * 2, 64, 128) ||
-      !map2d(&mU, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, US, KK, M->rows, (uint64_t)KK * 4, 32, 128) ||
-      !map2d(&mV, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Vp, KK, M->cols, (uint64_t)KK * 4, 32, 128))
+      !map2d(&mRow, CU_TENSOR_MAP_DATA_TYPE_UINT8, prm.row_codes, M->cols / 2, M->rows, M->cols / 2, 64, 128,
+             CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !map2d(&mCol, CU_TENSOR_MAP_DATA_TYPE_UINT8, prm.col_codes, M->rows / 2, M->cols, M->rows / 2, 64, 128,
+             CU_TENSOR_MAP_SWIZZLE_64B))
     return fail(ctx, METIS_ERR_CUDA, "cuTensorMapEncodeTiled failed (residual quantization)");
+  auto kern = resquant_kernel<kRecon, kDump>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  if (e != cudaSuccess) return check_cuda(ctx, e, "cudaFuncSetAttribute(resquant)");
+  const int grid = std::min(prm.n_units, ctx->sm_count);
+  const bool prof = ctx->profiling && !kDump;
+  cudaEvent_t ev0 = nullptr, ev1 = nullptr;
+  if (prof) {
+    cudaEventCreate(&ev0);
+    cudaEventCreate(&ev1);
+    cudaEventRecord(ev0, ctx->stream);
+  }
+  kern<<<grid, kRqThreads, C::SMEM, ctx->stream>>>(mM, mA, mV, mRow, mCol, prm); count_launch();
+  if (prof) {
+    cudaEventRecord(ev1, ctx->stream);
+    // algorithmic bytes: 2 B read and 2 x (1/2 + 1/16) B written per element
+    profile_record(ctx, kProfResquant, ev0, ev1, 3.125 * (double)M->rows * (double)M->cols);
+  }
+  return check_cuda(ctx, cudaGetLastError(), "resquant launch");
+}
+
+}  // namespace
+
+// Scratch layout (bytes from `scratch`, 256-byte aligned pieces):
+//   A16 rows x 128 fp16, B16 cols x 128 fp16, fac_a rows / 128 floats, fac_b cols / 128 floats.
+size_t residual_quantize_scratch_bytes(int64_t rows, int64_t cols) {
+  const auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  return up((size_t)rows * 256) + up((size_t)cols * 256) + up((size_t)rows / 128 * 4) + up((size_t)cols / 128 * 4);
+}
+
+metis_status run_residual_quantize_into(metis_ctx* ctx, const metis_matrix* M, const metis_factors* f,
+                                        const metis_quant_params* q, const metis_nvfp4* row, const metis_nvfp4* col,
+                                        void* scratch, uint32_t* amax_word, float* residual, int64_t ld_res) {
+  const int k = (f && f->k > 0) ? f->k : 0;
+  const bool recon = k > 0;
+  metis_status s;
+  Workspace ws{static_cast<char*>(scratch), residual_quantize_scratch_bytes(M->rows, M->cols)};
+  __half* A16 = static_cast<__half*>(ws.take((size_t)M->rows * 256));
+  __half* B16 = static_cast<__half*>(ws.take((size_t)M->cols * 256));
+  float* fac_a = static_cast<float*>(ws.take((size_t)M->rows / 128 * 4));
+  float* fac_b = static_cast<float*>(ws.take((size_t)M->cols / 128 * 4));
+  uint32_t* amax = nullptr;
+  if (q->tensor_scale == 0.0f) {
+    amax = amax_word;
+    if ((s = check_cuda(ctx, launch_amax(M->data, true, M->rows, M->cols, M->ld, amax, ctx->sm_count, ctx->stream),
+                        "amax launch")) != METIS_OK)
+      return s;
+  }
+  CUtensorMap mA, mV;
+  if (recon) {
+    const unsigned nblk = (unsigned)(M->rows / 128 + M->cols / 128);
+    split_factors_kernel<<<nblk, 256, 0, ctx->stream>>>(f->U, f->S, f->V, M->rows, k, A16, B16, fac_a, fac_b);
+    count_launch();
+    if ((s = check_cuda(ctx, cudaGetLastError(), "split factors")) != METIS_OK) return s;
+    if (!map2d(&mA, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, A16, 128, M->rows, 256, 64, 128) ||
+        !map2d(&mV, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, B16, 128, M->cols, 256, 64, 128))
+      return fail(ctx, METIS_ERR_CUDA, "cuTensorMapEncodeTiled failed (factor tiles)");
+  } else {
+    mA = mV = CUtensorMap{};
+  }
   RqParams prm;
   prm.rows = M->rows;
   prm.cols = M->cols;
@@ -439,70 +717,25 @@ metis_status launch_kk(metis_ctx* ctx, const metis_matrix* M, const float* US, c
   prm.col_scales = col->scales;
   prm.row_g = row->tensor_scale;
   prm.col_g = col->tensor_scale;
-  prm.amax_bits = amax_bits;
+  prm.amax_bits = amax;
+  prm.fac_a = fac_a;
+  prm.fac_b = fac_b;
+  prm.residual = residual;
+  prm.ld_res = ld_res;
   prm.status = ctx->status;
-  auto kern = resquant_kernel<KK>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-  if (e != cudaSuccess) return check_cuda(ctx, e, "cudaFuncSetAttribute(resquant)");
-  const int grid = std::min(prm.n_units, ctx->sm_count);
-  kern<<<grid, kRqThreads, C::SMEM, ctx->stream>>>(mM, mU, mV, prm); count_launch();
-  return check_cuda(ctx, cudaGetLastError(), "resquant launch");
+  if (residual)
+    return recon ? launch_rq<true, true>(ctx, M, mA, mV, prm) : launch_rq<false, true>(ctx, M, mA, mV, prm);
+  return recon ? launch_rq<true, false>(ctx, M, mA, mV, prm) : launch_rq<false, false>(ctx, M, mA, mV, prm);
 }
-
-}  // namespace
 
 metis_status run_residual_quantize(metis_ctx* ctx, const metis_matrix* M, const metis_factors* f,
-                                   const metis_quant_params* q, const metis_nvfp4* row, const metis_nvfp4* col) {
-  const int k = (f && f->k > 0) ? f->k : 0;
-  const int KK = k <= 32 ? 32 : 64;
-  const size_t need = (size_t)(M->rows + M->cols) * KK * 4 + 1024 + 256;
-  metis_status s = ensure_workspace(ctx, need);
+                                   const metis_quant_params* q, const metis_nvfp4* row, const metis_nvfp4* col,
+                                   float* residual, int64_t ld_res) {
+  const size_t bytes = residual_quantize_scratch_bytes(M->rows, M->cols);
+  metis_status s = ensure_workspace(ctx, bytes + 256);
   if (s != METIS_OK) return s;
-  Workspace ws{ctx->ws, ctx->ws_bytes};
-  float* US = static_cast<float*>(ws.take((size_t)M->rows * KK * 4));
-  float* Vp = static_cast<float*>(ws.take((size_t)M->cols * KK * 4));
-  uint32_t* amax = nullptr;
-  if (q->tensor_scale == 0.0f) {
-    amax = static_cast<uint32_t*>(ws.take(256));
-    if ((s = check_cuda(ctx, launch_amax(M->data, true, M->rows, M->cols, M->ld, amax, ctx->sm_count, ctx->stream),
-                        "amax launch")) != METIS_OK)
-      return s;
-  }
-  const int64_t n = (M->rows + M->cols) * KK;
-  pad_factors_kernel<<<(unsigned)((n + 255) / 256), 256, 0, ctx->stream>>>(
-      k ? f->U : nullptr, k ? f->S : nullptr, k ? f->V : nullptr, M->rows, M->cols, k, KK, US, Vp); count_launch();
-  if ((s = check_cuda(ctx, cudaGetLastError(), "pad factors")) != METIS_OK) return s;
-  return KK == 32 ? launch_kk<32>(ctx, M, US, Vp, q, amax, row, col) : launch_kk<64>(ctx, M, US, Vp, q, amax, row, col);
-}
-
-}  // namespace metis
-
-namespace metis {
-
-// Same work as run_residual_quantize, with the padded factor copies written to
-// caller-provided device scratch of (rows + cols) * 64 floats instead of the
-// context workspace.
-metis_status run_residual_quantize_into(metis_ctx* ctx, const metis_matrix* M, const metis_factors* f,
-                                        const metis_quant_params* q, const metis_nvfp4* row, const metis_nvfp4* col,
-                                        float* scratch) {
-  const int k = (f && f->k > 0) ? f->k : 0;
-  const int KK = k <= 32 ? 32 : 64;
-  float* US = scratch;
-  float* Vp = scratch + M->rows * KK;
-  uint32_t* amax = nullptr;
-  metis_status s;
-  if (q->tensor_scale == 0.0f) {
-    amax = reinterpret_cast<uint32_t*>(scratch + kNoAllocAmaxOffset);
-    if ((s = check_cuda(ctx, launch_amax(M->data, true, M->rows, M->cols, M->ld, amax, ctx->sm_count, ctx->stream),
-                        "amax launch")) != METIS_OK)
-      return s;
-  }
-  const int64_t n = (M->rows + M->cols) * KK;
-  pad_factors_kernel<<<(unsigned)((n + 255) / 256), 256, 0, ctx->stream>>>(
-      k ? f->U : nullptr, k ? f->S : nullptr, k ? f->V : nullptr, M->rows, M->cols, k, KK, US, Vp); count_launch();
-  s = check_cuda(ctx, cudaGetLastError(), "pad factors");
-  if (s != METIS_OK) return s;
-  return KK == 32 ? launch_kk<32>(ctx, M, US, Vp, q, amax, row, col) : launch_kk<64>(ctx, M, US, Vp, q, amax, row, col);
+  return run_residual_quantize_into(ctx, M, f, q, row, col, ctx->ws, reinterpret_cast<uint32_t*>(ctx->ws + bytes),
+                                    residual, ld_res);
 }
 
 }  // namespace metis
