@@ -167,7 +167,8 @@ typedef struct {
  *   rowwise (nullable): outer = rows, inner = cols  (blocks along columns)
  *   colwise (nullable): outer = cols, inner = rows  (blocks along rows; M_R^T)
  * Stochastic rounding uses the Philox SR stream (operand_id, sub 0 row-wise / 1
- * column-wise, step).  Device: METIS_DEV_NONFINITE on NaN/Inf input.
+ * column-wise, step).  With both orientations the pass runs fused (one read of M) and
+ * needs rows * cols <= 2^36, else ERR_SHAPE.  Device: METIS_DEV_NONFINITE on NaN/Inf input.
  */
 metis_status metis_residual_quantize_nvfp4(metis_ctx* ctx, const metis_matrix* M,
                                            const metis_factors* f, const metis_quant_params* q,

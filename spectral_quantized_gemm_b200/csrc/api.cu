@@ -95,6 +95,14 @@ metis_status check_dims(metis_ctx* ctx, int64_t rows, int64_t cols) {
   return METIS_OK;
 }
 
+// The fused residual pass numbers its stochastic-rounding counters (element index / 16) in
+// 32 bits: rows * cols <= 2^36 (a 128 GiB bf16 matrix).
+metis_status check_fused_size(metis_ctx* ctx, int64_t rows, int64_t cols) {
+  if ((double)rows * (double)cols > 68719476736.0)
+    return fail(ctx, METIS_ERR_SHAPE, "rows * cols must not exceed 2^36 for the fused residual pass");
+  return METIS_OK;
+}
+
 metis_status check_quant(metis_ctx* ctx, const metis_quant_params* q) {
   if (!q) return fail(ctx, METIS_ERR_ARG, "null quant params");
   if (q->rounding != 0 && q->rounding != 1) return fail(ctx, METIS_ERR_ARG, "rounding must be 0 (RN) or 1 (SR)");
@@ -255,7 +263,10 @@ metis_status metis_residual_quantize_nvfp4(metis_ctx* ctx, const metis_matrix* M
   if (!rowwise && !colwise) return fail(ctx, METIS_ERR_ARG, "no output orientation requested");
   if ((s = check_nvfp4(ctx, rowwise, M->rows, M->cols, "rowwise")) != METIS_OK) return s;
   if ((s = check_nvfp4(ctx, colwise, M->cols, M->rows, "colwise")) != METIS_OK) return s;
-  if (rowwise && colwise) return run_residual_quantize(ctx, M, f, q, rowwise, colwise);
+  if (rowwise && colwise) {
+    if ((s = check_fused_size(ctx, M->rows, M->cols)) != METIS_OK) return s;
+    return run_residual_quantize(ctx, M, f, q, rowwise, colwise);
+  }
   // one orientation only: fp32 residual in the workspace, then the quantizer
   const size_t bytes = (size_t)M->rows * M->cols * sizeof(float);
   if ((s = ensure_workspace(ctx, bytes + 512)) != METIS_OK) return s;
@@ -297,6 +308,7 @@ metis_status metis_residual_quantize_nvfp4_dump(metis_ctx* ctx, const metis_matr
   if ((s = check_nvfp4(ctx, colwise, M->cols, M->rows, "colwise")) != METIS_OK) return s;
   if (ldr < M->cols || ldr % 4 || !aligned16(residual))
     return fail(ctx, METIS_ERR_ALIGN, "fp32 residual needs 16-byte alignment and ld % 4 == 0");
+  if ((s = check_fused_size(ctx, M->rows, M->cols)) != METIS_OK) return s;
   return run_residual_quantize(ctx, M, f, q, rowwise, colwise, residual, ldr);
 }
 

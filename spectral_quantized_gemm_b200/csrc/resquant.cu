@@ -22,10 +22,12 @@
 //               (M = N = 128, K = 16) of a tile into one of two fp32 accumulators
 //   warps 2..17 a warp per 32 x 32 sub-tile (rows: its tensor-memory lane quarter):
 //               residual of its rows from the accumulator and M, row-wise NVFP4 of
-//               both 16-blocks of each row; the residual passes through a 2 KB
-//               per-warp shared-memory transpose (two halves of 16 columns) and each
-//               lane quantizes one 16-row block of a column per half.  Codes and
-//               tiled scales go straight to HBM.  The warps never wait for one another.
+//               both 16-blocks of each row; the residual passes through the warp's own,
+//               already read, 2 KB of the M stage as a transpose (two halves of 16
+//               columns) and each lane quantizes one 16-row block of a column per half.
+//               The warp stages its codes (1 KB) and writes them with two TMA stores;
+//               its scales go straight to their 512-byte tiles.  The warps never wait
+//               for one another.
 // All mbarrier waits are bounded (METIS_DEV_TIMEOUT on expiry); on an abort the
 // producer waits (bounded) for the tile loads it issued before the CTA exits.
 #include <cuda.h>
@@ -54,21 +56,14 @@ struct RqCfg {
   static constexpr int V_BYTES = 32768;                // V hi | lo of the tile's 128 columns
   static constexpr int V_STAGES = kRecon ? 2 : 0;
   static constexpr int M_BYTES = 32768;                // two 64-column boxes of 16 KB
-  static constexpr int M_STAGES = kRecon ? 4 : 6;
+  static constexpr int M_STAGES = kRecon ? 3 : 5;
+  static constexpr int OUT_BYTES = kRqEpiWarps * 1024;  // per warp: its row-wise then column-wise codes
   static constexpr int BAR_BYTES = 256;
   static constexpr int RCP_BYTES = 512;
-  static constexpr size_t SMEM =
-      1024 + (size_t)A_BYTES + V_STAGES * V_BYTES + M_STAGES * M_BYTES + BAR_BYTES + RCP_BYTES;
+  static constexpr size_t SMEM = 1024 + (size_t)A_BYTES + V_STAGES * V_BYTES + M_STAGES * M_BYTES + OUT_BYTES +
+                                 BAR_BYTES + RCP_BYTES;
   static_assert(SMEM <= 232448, "shared memory budget");
 };
-
-// Output staging inside a consumed M stage (byte offsets): the tile's row-wise codes
-// (128 rows x 64 B) and column-wise codes (128 columns x 64 B), both in the 64-byte
-// swizzle of their TMA store boxes, then its two 1 KB runs of tiled scales.
-constexpr int kStRowCodes = 0;
-constexpr int kStColCodes = 8192;
-constexpr int kStRowScales = 16384;
-constexpr int kStColScales = 17408;
 
 struct RqParams {
   int64_t rows, cols;
@@ -89,6 +84,9 @@ struct RqParams {
   float* residual;             // non-null (parity surface): the fp32 residual, leading dimension ld_res
   int64_t ld_res;
   uint32_t* status;
+  // Philox4x32-10 round keys of the SR stream (key = seed bumped by the Weyl constants),
+  // read by the rounds straight from the parameter bank
+  uint32_t rk0[10], rk1[10];
 };
 
 // fp16 x fp16 -> fp32, both operands K-major, M = N = 128.
@@ -181,16 +179,44 @@ __device__ __forceinline__ BlockScale block_scale_fast(float amax, float g, cons
   return bs;
 }
 
-// One 16-element block with its maximum: scale code and packed codes (RN, or SR with
-// the Philox call of element index e0 .. e0 + 15 in the orientation's blocked order).
-__device__ __forceinline__ uint2 quantize16(const float* v, float amax, float g, const float* rcp_table,
-                                            int rounding, uint64_t seed, uint32_t tag, uint32_t step, uint64_t e0,
+// The four words of the SR stream's Philox4x32-10 call for counter (q, tag, step): the same
+// generator as philox10() with the round keys taken from the kernel parameters and each
+// 32 x 32 -> 64-bit product formed by one wide multiply.
+__device__ __forceinline__ uint4 sr_words(const RqParams& p, uint32_t q, uint32_t tag) {
+  uint32_t c0 = q, c1 = 0u, c2 = tag, c3 = p.step;   // counters below 2^32: rows * cols <= 2^36
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    uint64_t p0, p1;
+    asm("mul.wide.u32 %0, %1, %2;" : "=l"(p0) : "r"(0xD2511F53u), "r"(c0));
+    asm("mul.wide.u32 %0, %1, %2;" : "=l"(p1) : "r"(0xCD9E8D57u), "r"(c2));
+    const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ p.rk0[r];
+    const uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ p.rk1[r];
+    c0 = n0;
+    c1 = (uint32_t)p1;
+    c2 = n2;
+    c3 = (uint32_t)p0;
+  }
+  return make_uint4(c0, c1, c2, c3);
+}
+
+// One 16-element block with its maximum: scale code and packed codes (RN, or SR with the
+// Philox call of counter qc = e0 / 16, e0 the index of the block's first element in the
+// orientation's blocked order).
+__device__ __forceinline__ uint2 quantize16(const RqParams& p, const float* v, float amax, float g,
+                                            const float* rcp_table, uint32_t tag, uint32_t qc,
                                             uint32_t& scale_code) {
   const BlockScale bs = block_scale_fast(amax, g, rcp_table);
   float x[16];
 #pragma unroll
   for (int i = 0; i < 16; i += 2) mul2(x[i], x[i + 1], v[i], v[i + 1], bs.rcp);
-  uint2 packed = encode_block16(x, rounding, seed, tag, step, e0);
+  uint2 packed;
+  if (p.rounding) {
+    const uint4 w = sr_words(p, qc, tag);
+    packed.x = e2m1x4_sr(x[0], x[1], x[2], x[3], w.x) | (e2m1x4_sr(x[4], x[5], x[6], x[7], w.y) << 16);
+    packed.y = e2m1x4_sr(x[8], x[9], x[10], x[11], w.z) | (e2m1x4_sr(x[12], x[13], x[14], x[15], w.w) << 16);
+  } else {
+    packed = encode_block16(x, 0, 0, 0, 0, 0);
+  }
   if (bs.code == 0) packed = make_uint2(0, 0);
   scale_code = bs.code;
   return packed;
@@ -207,7 +233,8 @@ __global__ void __launch_bounds__(kRqThreads, 1)
   uint8_t* sA = smem;
   uint8_t* sV = sA + C::A_BYTES;
   uint8_t* sM = sV + C::V_STAGES * C::V_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sM + C::M_STAGES * C::M_BYTES);
+  uint8_t* sOut = sM + C::M_STAGES * C::M_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + C::OUT_BYTES);
   uint64_t* a_full = bars;
   uint64_t* a_empty = bars + 1;
   uint64_t* v_full = bars + 2;                    // [2]
@@ -217,9 +244,7 @@ __global__ void __launch_bounds__(kRqThreads, 1)
   uint64_t* acc_full = m_empty + 6;               // [2]
   uint64_t* acc_empty = acc_full + 2;             // [2]
   uint64_t* drain = acc_empty + 2;
-  uint64_t* ep_done = drain + 1;                  // every epilogue warp is done with the tile's M stage
-  uint64_t* ep_staged = ep_done + 1;              // every epilogue warp has staged the tile's outputs
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ep_staged + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* rcp_table = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + C::BAR_BYTES);   // 128 entries
 
@@ -243,11 +268,9 @@ __global__ void __launch_bounds__(kRqThreads, 1)
     }
     for (int s = 0; s < C::M_STAGES; ++s) {
       tc::mbar_init(&m_full[s], 1);
-      tc::mbar_init(&m_empty[s], 1);   // released by the thread that stores the staged outputs
+      tc::mbar_init(&m_empty[s], kRqEpiWarps);
     }
     tc::mbar_init(drain, 1);
-    tc::mbar_init(ep_done, kRqEpiWarps);
-    tc::mbar_init(ep_staged, kRqEpiWarps);
     *abort_flag = 0;
     tc::fence_barrier_init();
     if (blockIdx.x == 0) {
@@ -372,7 +395,6 @@ __global__ void __launch_bounds__(kRqThreads, 1)
     const int r = q * 32 + lane;       // tile row of this lane in the row pass
     const int jc = lane & 15;          // column (within a half) of this lane in the column pass
     const int hh = lane >> 4;          // 16-row half of the sub-tile in the column pass
-    const bool issuer = (e == 0 && lane == 0);
     // The warp's own bytes of an M stage (rows q*32 .. + 31 of box h >> 1, its four 16-byte
     // chunks of each row) double as its transpose buffer once it has read them: element
     // (row l, column c) of a 32 x 16 half sits in row rho = q*32 + 8*(c & 3) + ((l >> 2) ^ (c & 7)),
@@ -393,7 +415,8 @@ __global__ void __launch_bounds__(kRqThreads, 1)
                             16 * (Kh ^ ((uint32_t)jc >> 2) ^ k0 ^ j7);
     int ms = 0;
     uint32_t mph = 0;
-    int pending = -1;                  // stage whose staged outputs are still being stored
+    uint8_t* wout = sOut + e * 1024;   // this warp's staged codes: 32 rows x 16 B, then 32 columns x 16 B
+    bool stored = false;               // a TMA store of this warp may still be reading wout
     int it = 0;
     for (int u = u_begin; u < u_end; ++u, ++it) {
       const int rb = u / p.n_cb, cb = u % p.n_cb;
@@ -411,6 +434,10 @@ __global__ void __launch_bounds__(kRqThreads, 1)
       const int64_t grow = (int64_t)rb * 128 + r;
       const int64_t gcol = (int64_t)cb * 128 + h * 32;
       const int64_t grow_t = (int64_t)rb * 128 + q * 32 + hh * 16;   // first row of this lane's column blocks
+      // Philox counters (element index / 16) of the row-wise blocks of row r and of the
+      // column-wise block of column gcol + jc; the second half adds 1 and rows respectively
+      const uint32_t q_row = (uint32_t)grow * (uint32_t)(p.cols >> 4) + (uint32_t)(gcol >> 4);
+      const uint32_t q_col = (uint32_t)(gcol + jc) * (uint32_t)(p.rows >> 4) + (uint32_t)(grow_t >> 4);
       float nf = 0.0f;
       if (kRecon) nf = -__fmul_rn(__ldg(p.fac_a + rb), __ldg(p.fac_b + cb));   // -2^-(a + b), exact
       uint4 row_out;
@@ -475,8 +502,7 @@ __global__ void __launch_bounds__(kRqThreads, 1)
           const float amax = block_amax(v);
           finite &= amax <= 3.402823466e38f;   // false for NaN and Inf
           uint32_t code;
-          const uint2 pk = quantize16(v, amax, g, rcp_table, p.rounding, p.seed, p.tag_row, p.step,
-                                      (uint64_t)grow * (uint64_t)p.cols + (uint64_t)(gcol + 16 * half), code);
+          const uint2 pk = quantize16(p, v, amax, g, rcp_table, p.tag_row, q_row + (uint32_t)half, code);
           row_sc |= code << (8 * half);
           if (half == 0) {
             row_out.x = pk.x;
@@ -499,65 +525,41 @@ __global__ void __launch_bounds__(kRqThreads, 1)
             w[4 * m4 + 3] = t4.w;
           }
           const float amax = block_amax(w);
-          const int64_t gc = gcol + 16 * half + jc;
-          col_out[half] = quantize16(w, amax, g, rcp_table, p.rounding, p.seed, p.tag_col, p.step,
-                                     (uint64_t)gc * (uint64_t)p.rows + (uint64_t)grow_t, col_sc[half]);
+          col_out[half] = quantize16(p, w, amax, g, rcp_table, p.tag_col, q_col + (uint32_t)half * (uint32_t)p.rows,
+                                     col_sc[half]);
         }
         __syncwarp();
-        if (half == 0 && issuer && pending >= 0) {   // the previous tile's stores have long read their stage
-          tc::bulk_wait_read_all();
-          tc::mbar_arrive(&m_empty[pending]);
-          pending = -1;
-        }
       }
+      if (lane == 0) tc::mbar_arrive(&m_empty[ms]);   // this warp is done with the M stage
       if (!finite) raise_status(p.status, METIS_DEV_NONFINITE);
-      // ---- every warp is done with this M stage: stage the tile's outputs in it
-      if (lane == 0) tc::mbar_arrive(ep_done);
-      ok = tc::mbar_wait(ep_done, (uint32_t)it & 1u, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) {
-        if (lane == 0) fail_wait();
-        break;
+      // ---- codes: staged per warp and written by two TMA stores (32 rows x 16 B each);
+      // scales: straight to their 512-byte tiles (a warp's stores land in one tile)
+      if (stored) {
+        if (lane == 0) tc::bulk_wait_read_all();   // the previous tile's stores have read wout
+        __syncwarp();
       }
-      {
-        // row codes: row r, bytes h*16 .. + 15 of its 64 (chunk h, 64B swizzle)
-        *reinterpret_cast<uint4*>(stage + kStRowCodes + r * 64 + ((h ^ ((r >> 1) & 3)) << 4)) = row_out;
-        // row scales: tile (h >> 1) of the two, entry (r % 32, r / 32, blocks 2(h & 1), +1)
-        *reinterpret_cast<uint16_t*>(stage + kStRowScales + (h >> 1) * 512 + lane * 16 + q * 4 + 2 * (h & 1)) =
-            (uint16_t)row_sc;
+      *reinterpret_cast<uint4*>(wout + lane * 16) = row_out;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int cl = h * 32 + half * 16 + jc;   // tile column
-          // column codes: column cl, rows q*32 + hh*16 .. + 15 = bytes q*16 + hh*8 .. + 7 (chunk q)
-          *reinterpret_cast<uint2*>(stage + kStColCodes + cl * 64 + ((q ^ ((cl >> 1) & 3)) << 4) + hh * 8) =
-              col_out[half];
-          // column scales: tile (q >> 1), entry (cl % 32, cl / 32, block (2q + hh) & 3)
-          stage[kStColScales + (q >> 1) * 512 + (cl & 31) * 16 + h * 4 + ((2 * q + hh) & 3)] = (uint8_t)col_sc[half];
-        }
-      }
+      for (int half = 0; half < 2; ++half)
+        *reinterpret_cast<uint2*>(wout + 512 + (half * 16 + jc) * 16 + hh * 8) = col_out[half];
       tc::fence_proxy_async();   // the staged bytes are read by the bulk-copy (async) proxy
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(ep_staged);
-      ok = tc::mbar_wait(ep_staged, (uint32_t)it & 1u, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) {
-        if (lane == 0) fail_wait();
-        break;
-      }
-      if (issuer) {
-        tc::tma_store_2d(&mapRowCodes, stage + kStRowCodes, cb * 64, rb * 128);
-        tc::tma_store_2d(&mapColCodes, stage + kStColCodes, rb * 64, cb * 128);
-        tc::bulk_store(p.row_scales + ((int64_t)rb * (p.cols / 64) + (int64_t)cb * 2) * 512, stage + kStRowScales,
-                       1024);
-        tc::bulk_store(p.col_scales + ((int64_t)cb * (p.rows / 64) + (int64_t)rb * 2) * 512, stage + kStColScales,
-                       1024);
+      if (lane == 0) {
+        tc::tma_store_2d(&mapRowCodes, wout, cb * 64 + h * 16, rb * 128 + q * 32);
+        tc::tma_store_2d(&mapColCodes, wout + 512, rb * 64 + q * 16, cb * 128 + h * 32);
         tc::bulk_commit_group();
-        pending = ms;
       }
+      stored = true;
+      *reinterpret_cast<uint16_t*>(p.row_scales + scale_offset(grow, gcol / 16, p.cols / 64)) = (uint16_t)row_sc;
+#pragma unroll
+      for (int half = 0; half < 2; ++half)
+        p.col_scales[scale_offset(gcol + half * 16 + jc, grow_t / 16, p.rows / 64)] = (uint8_t)col_sc[half];
       if (++ms == C::M_STAGES) {
         ms = 0;
         mph ^= 1u;
       }
     }
-    if (issuer) tc::bulk_wait_all();   // no store may still read this CTA's shared memory at exit
+    if (lane == 0) tc::bulk_wait_all();   // no store may still read this CTA's shared memory at exit
   }
 
   tc::tc_fence_before();
@@ -636,10 +638,10 @@ metis_status launch_rq(metis_ctx* ctx, const metis_matrix* M, const CUtensorMap&
   using C = RqCfg<kRecon>;
   CUtensorMap mM, mRow, mCol;
   if (!map2d(&mM, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, M->data, M->cols, M->rows, (uint64_t)M->ld * 2, 64, 128) ||
-      !map2d(&mRow, CU_TENSOR_MAP_DATA_TYPE_UINT8, prm.row_codes, M->cols / 2, M->rows, M->cols / 2, 64, 128,
-             CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !map2d(&mCol, CU_TENSOR_MAP_DATA_TYPE_UINT8, prm.col_codes, M->rows / 2, M->cols, M->rows / 2, 64, 128,
-             CU_TENSOR_MAP_SWIZZLE_64B))
+      !map2d(&mRow, CU_TENSOR_MAP_DATA_TYPE_UINT8, prm.row_codes, M->cols / 2, M->rows, M->cols / 2, 16, 32,
+             CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !map2d(&mCol, CU_TENSOR_MAP_DATA_TYPE_UINT8, prm.col_codes, M->rows / 2, M->cols, M->rows / 2, 16, 32,
+             CU_TENSOR_MAP_SWIZZLE_NONE))
     return fail(ctx, METIS_ERR_CUDA, "cuTensorMapEncodeTiled failed (residual quantization)");
   auto kern = resquant_kernel<kRecon, kDump>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
@@ -723,6 +725,10 @@ metis_status run_residual_quantize_into(metis_ctx* ctx, const metis_matrix* M, c
   prm.residual = residual;
   prm.ld_res = ld_res;
   prm.status = ctx->status;
+  for (int r = 0; r < 10; ++r) {   // Weyl-sequence round keys of Philox4x32-10
+    prm.rk0[r] = (uint32_t)q->seed + (uint32_t)r * 0x9E3779B9u;
+    prm.rk1[r] = (uint32_t)(q->seed >> 32) + (uint32_t)r * 0xBB67AE85u;
+  }
   if (residual)
     return recon ? launch_rq<true, true>(ctx, M, mA, mV, prm) : launch_rq<false, true>(ctx, M, mA, mV, prm);
   return recon ? launch_rq<true, false>(ctx, M, mA, mV, prm) : launch_rq<false, false>(ctx, M, mA, mV, prm);

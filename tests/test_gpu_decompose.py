@@ -139,3 +139,63 @@ def test_decompose_validation(ctx, metis_lib):
         ctx.decompose(M, k=4, s=200, l_k=32, seed=0, operand_id=0, refresh=True, step=0, factors=f)
     with pytest.raises(metis_lib.MetisError):
         ctx.decompose(M, k=4, s=4, l_k=4, seed=0, operand_id=0, refresh=True, step=0, factors=f)
+
+
+# ---- edge cases of the decomposition (each against the oracle)
+
+def test_rank_one(ctx, metis_lib):
+    """k = 1: one direction, the top singular pair of the sampled sketch."""
+    cfg = synth.scaled_config("gpt2_small_mlp_up", l=1024, m=768, n=768)
+    _compare(ctx, cfg, "X", 1, 8, 82, 0, 1)
+
+
+def test_sketch_as_wide_as_the_sample(ctx, metis_lib):
+    """k + s = l_k: the sketch Y is square (20 x 20) before CholQR."""
+    cfg = synth.scaled_config("gpt2_small_mlp_up", l=1024, m=768, n=768)
+    _compare(ctx, cfg, "X", 12, 8, 20, 0, 1)
+
+
+def test_smallest_operand(ctx, metis_lib):
+    """A 128 x 128 operand, sampled (l_k = 32) and unsampled (l_k = 128)."""
+    cfg = synth.scaled_config("tiny_fwd", l=128, m=128, n=128)
+    _compare(ctx, cfg, "X", 4, 4, 32, 0, 0)
+    _compare(ctx, cfg, "X", 4, 4, 128, 0, 0)
+
+
+def _duplicated_columns(rank, rows=256, cols=128, seed=3):
+    """A bf16 matrix whose columns repeat `rank` random base columns (exact rank `rank`)."""
+    rng = np.random.default_rng(seed)
+    base = rng.standard_normal((rows, rank)) * np.geomspace(50.0, 1.0, rank)
+    pick = rng.integers(0, rank, size=cols)
+    pick[:rank] = np.arange(rank)
+    return torch.from_numpy(np.ascontiguousarray(base[:, pick])).to(torch.bfloat16).contiguous()
+
+
+@pytest.mark.parametrize("k", [4, 6])
+def test_rank_deficient_sketch_drops_directions(ctx, metis_lib, k):
+    """Duplicated columns give M exact rank 5, so the sketch of width k + 4 (8 or 10) is
+    rank-deficient: reading R9's drop rule runs on the device (CholQR pivots and
+    eigenvalues at or below 1e-12 of the largest count as zero).  The recovered directions
+    match the oracle's; with k = 6 > rank the sixth singular value is exactly 0 and its
+    left factor column is zero, as in the oracle, and no numeric failure is raised."""
+    Mt = _duplicated_columns(5)
+    M = Mt.double().numpy()
+    rows, cols = M.shape
+    f = _gpu_decompose(ctx, Mt.cuda(), k, 4, 32, 1, 0)
+    assert ctx.poll_device_status() == 0
+    ref = decompose.refresh_basis(M, k, 4, 32, 1, 0, 0)
+    U, S, V = decompose.step_factors(M, ref["V"])
+    Y = M[ref["rows"]] @ ref["omega"].astype(np.float64)
+    _, _, dropped = linalg.cholqr(Y)
+    assert int(np.sum(dropped)) == k + 4 - 5   # the oracle drops the dependent sketch columns
+    gV, gU, gS = f.V.cpu().double().numpy(), f.U.cpu().double().numpy(), f.S.cpu().double().numpy()[:k]
+    r = min(k, 5)
+    assert linalg.principal_cosines(gV[:, :r], V[:, :r]).min() >= COS
+    assert linalg.principal_cosines(gU[:, :r], U[:, :r]).min() >= COS
+    assert np.max(np.abs(gS[:r] - S[:r]) / S[0]) < 1e-3
+    if k > 5:
+        assert np.all(S[5:] == 0.0) and np.all(gS[5:] == 0.0)
+        assert np.all(U[:, 5:] == 0.0) and np.all(gU[:, 5:] == 0.0)
+    low = (gU * gS) @ gV.T
+    if k >= 5:                                # rank 5 is captured whole
+        assert np.linalg.norm(low - M) / np.linalg.norm(M) < 1e-3

@@ -12,7 +12,7 @@ import pytest
 import torch
 
 from oracle import decompose, metis
-from tests.gpu_helpers import codes_unpacked, rel_fro
+from tests.gpu_helpers import bf16_round, codes_unpacked, rel_fro
 from workloads import synth
 
 pytestmark = pytest.mark.gpu
@@ -98,11 +98,30 @@ def test_plain_nvfp4_when_k_is_zero(ctx, metis_lib):
 
 
 def test_bf16_outputs(ctx, metis_lib):
+    """Y and dX stored in bf16 (the types the benchmark trains with).  Element by element
+    each bf16 output is the layer's fp32 result rounded once to nearest (the same launch
+    with an fp32 output, bit-exact), and against the oracle rounded to bf16 the relative
+    Frobenius error is within the 2e-3 contract, so the bf16 store adds no error beyond its
+    own rounding."""
     cfg = synth.scaled_config("gpt2_small_mlp_up", l=1024, m=768, n=768)
     res = _layer(ctx, cfg, out=torch.bfloat16)
-    y = metis.linear_fwd(res["X"].oracle(), res["W"].oracle())
-    # bf16 storage alone costs ~1.7e-3 relative; everything else must be far below
-    assert rel_fro(res["Y"].double().cpu().numpy(), y) <= 2.2e-3
+    X, W, D = res["X"], res["W"], res["D"]
+    Y32 = torch.empty(cfg["l"], cfg["n"], dtype=torch.float32, device="cuda")
+    dX32 = torch.empty(cfg["l"], cfg["m"], dtype=torch.float32, device="cuda")
+    dW32 = torch.empty(cfg["m"], cfg["n"], dtype=torch.float32, device="cuda")
+    ctx.linear_fwd(X.struct, W.struct, Y32)
+    ctx.linear_bwd(X.struct, W.struct, D.struct, dX32, dW32)
+    torch.cuda.synchronize()
+    assert ctx.poll_device_status() == 0
+    assert torch.equal(res["Y"], Y32.to(torch.bfloat16))
+    assert torch.equal(res["dX"], dX32.to(torch.bfloat16))
+    ox, ow, od = X.oracle(), W.oracle(), D.oracle()
+    y = metis.linear_fwd(ox, ow)
+    dx, _ = metis.linear_bwd(ox, ow, od)
+    for got, want in ((res["Y"], y), (res["dX"], dx)):
+        g = got.double().cpu().numpy()
+        assert rel_fro(g, bf16_round(want)) <= TOL
+        assert np.mean(g == bf16_round(want)) > 0.99
 
 
 def test_end_to_end_statistics_match_the_oracle(ctx, metis_lib):

@@ -77,6 +77,59 @@ def test_wrapper_is_the_c_abi_sequence(ctx, metis_lib):
     assert layer.step == 3
 
 
+def _oracle_operand(o):
+    """The oracle's view of one of MetisLinear's own operands: its decoded residual codes
+    and scales in both orientations, its quantized factors and singular values."""
+    from tests.gpu_helpers import codes_unpacked
+    k = o.factors.k
+    cu, su, gu = codes_unpacked(o.factors.Uq)
+    cv, sv, gv = codes_unpacked(o.factors.Vq)
+    return {"row": codes_unpacked(o.row), "col": codes_unpacked(o.col), "U": True,
+            "Uq": (cu[:k], su[:k], gu), "Vq": (cv[:k], sv[:k], gv), "S": o.factors.S.cpu().double().numpy()[:k]}
+
+
+def test_wrapper_matches_the_oracle(ctx, metis_lib):
+    """MetisLinear's Y, dX and dW against the oracle's product (oracle/metis.py) fed the
+    layer's own codes, scales and factors, over a refresh and a reuse step: dW (fp32) within
+    the 2e-3 contract, Y and dX (bf16) within it against the oracle rounded to bf16.  Every
+    operand's decode tensor scale is the one reading R1b chooses from the data
+    (oracle/nvfp4.py::auto_tensor_scale of the bf16 operand)."""
+    from oracle import metis, nvfp4
+    from tests.gpu_helpers import bf16_round, rel_fro
+    from spectral_quantized_gemm_b200.linear import MetisLinear
+    torch.manual_seed(1)
+    layer = MetisLinear(768, 1024, k=12, seed=5, device="cuda")
+    recorded = []
+    prepare = layer._prepare
+
+    def record(lib, M, op_id, step, sampled):
+        o = prepare(lib, M, op_id, step, sampled)
+        recorded.append((op_id, M.detach().clone(), o))
+        return o
+
+    layer._prepare = record
+    for step in range(2):
+        recorded.clear()
+        x = _tokens(1024, 768, 300 + step).to(torch.bfloat16).requires_grad_(True)
+        dy = (_tokens(1024, 1024, 400 + step) * 1e-4).to(torch.bfloat16)
+        layer.weight.grad = None
+        y = layer(x)
+        y.backward(dy)
+        torch.cuda.synchronize()
+        assert ctx.poll_device_status() == 0
+        ops = {op_id: (M, o) for op_id, M, o in recorded}
+        assert sorted(ops) == [0, 1, 2]
+        for op_id, (M, o) in ops.items():
+            g = nvfp4.auto_tensor_scale(M.float().cpu().numpy())
+            assert float(o.row.tensor_scale[0]) == g and float(o.col.tensor_scale[0]) == g, (step, op_id)
+        ox, ow, od = (_oracle_operand(ops[i][1]) for i in range(3))
+        Y = metis.linear_fwd(ox, ow)
+        dX, dW = metis.linear_bwd(ox, ow, od)
+        assert rel_fro(layer.weight.grad.double().cpu().numpy(), dW) <= 2e-3, step
+        for got, want in ((y, Y), (x.grad, dX)):
+            assert rel_fro(got.detach().double().cpu().numpy(), bf16_round(want)) <= 2e-3, step
+
+
 def test_refresh_schedule_and_basis_reuse(ctx, metis_lib):
     from spectral_quantized_gemm_b200.linear import MetisLinear
     layer = MetisLinear(512, 768, k=16, refresh_every=2, seed=3, device="cuda")
