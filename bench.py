@@ -50,8 +50,8 @@ METRIC = "effective TFLOP/s of Metis W4A4G4 linear fwd+bwd; % of NVFP4 MMA peak"
 GEMM_FWD_DRAM_BYTES = 69.383424e6 + 192.398336e6
 # DRAM bytes (read + write) of one launch of the residual quantizer on the benchmark's D
 # (8192 x 14336, k = 64, SR), from one ncu capture of this kernel version
-# (bench.py --stage resquant; the summary sits under profiles/); None until retaken.
-RESQUANT_D_DRAM_BYTES = None
+# (bench.py --stage resquant; the summary sits under profiles/). Must be retaken whenever the kernel changes.
+RESQUANT_D_DRAM_BYTES = 246.442752e6 + 105.63712e6
 RESQUANT_TRAFFIC_BASIS = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch on D (8192 x 14336), "
                           "bytes; the timed launches cover X, W and D")
 
@@ -208,7 +208,9 @@ class Layer:
         X, D = batches[0]
         self.mats = {"X": X, "W": W, "D": D}
         dev = W.device
-        self.streams = {name: torch.cuda.Stream(dev) for name in self.NAMES}
+        # X and W gate the forward GeMM, D only the backward: their streams get the higher
+        # priority, so their kernels take free SMs first when the three chains overlap
+        self.streams = {name: torch.cuda.Stream(dev, priority=-1 if name != "D" else 0) for name in self.NAMES}
         self.ctxs = {}
         for name in self.NAMES:
             with torch.cuda.stream(self.streams[name]):
