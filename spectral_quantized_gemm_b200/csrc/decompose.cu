@@ -1076,23 +1076,45 @@ __global__ void __launch_bounds__(32 * kJacRowsPerCta) jacobi_replay_kernel(cons
 // ------------------------------------------- tensor-core projection helpers
 // out (2kp x n, bf16 row-major): row j < k = hi(F[:, j]), row kp + j = lo(F[:, j]) with
 // hi = bf16(F), lo = bf16(F - hi); other rows zero.  F is n x k fp32 row-major.
-__global__ void split_hi_lo_t_kernel(const float* __restrict__ F, int64_t n, int k, int kp,
-                                     __nv_bfloat16* __restrict__ out) {
-  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= (int64_t)2 * kp * n) return;
-  const int j = (int)(e / n);
-  const int64_t i = e - (int64_t)j * n;
-  const int jj = j < kp ? j : j - kp;
-  float v = 0.0f;
-  if (jj < k) {
-    const float f = F[i * k + jj];
-    const __nv_bfloat16 hi = __float2bfloat16_rn(f);
-    v = j < kp ? __bfloat162float(hi) : f - __bfloat162float(hi);
+// A block transposes 64 rows of F (k <= kp <= 128) through shared memory: the rows are read
+// whole and each output row j gets 64 consecutive entries, so reads and writes coalesce.
+// Every load of a thread is issued before the first shared-memory store (one memory
+// round trip per block, not one per element).
+constexpr int kSplitRows = 64;
+constexpr int kSplitThreads = 512;
+__global__ void __launch_bounds__(kSplitThreads) split_hi_lo_t_kernel(const float* __restrict__ F, int64_t n, int k,
+                                                                      int kp, __nv_bfloat16* __restrict__ out) {
+  __shared__ float t[kSplitRows][129];
+  const int64_t i0 = (int64_t)blockIdx.x * kSplitRows;
+  const int lkp = __ffs(kp) - 1;   // kp is a power of two
+  float v[kSplitRows * 128 / kSplitThreads];
+#pragma unroll
+  for (int it = 0; it < kSplitRows * 128 / kSplitThreads; ++it) {
+    const int e = threadIdx.x + it * kSplitThreads;
+    const int r = e >> lkp, c = e & (kp - 1);
+    v[it] = (r < kSplitRows && c < k && i0 + r < n) ? F[(i0 + r) * k + c] : 0.0f;
   }
-  out[e] = __float2bfloat16_rn(v);
+#pragma unroll
+  for (int it = 0; it < kSplitRows * 128 / kSplitThreads; ++it) {
+    const int e = threadIdx.x + it * kSplitThreads;
+    if ((e >> lkp) < kSplitRows) t[e >> lkp][e & (kp - 1)] = v[it];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int it = 0; it < kSplitRows * 128 / kSplitThreads; ++it) {
+    const int e = threadIdx.x + it * kSplitThreads;
+    const int j = e / kSplitRows, r = e % kSplitRows;
+    if (j >= kp || i0 + r >= n) continue;
+    const float f = t[r][j];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(f);
+    out[(int64_t)j * n + i0 + r] = hi;
+    out[(int64_t)(kp + j) * n + i0 + r] = __float2bfloat16_rn(f - __bfloat162float(hi));
+  }
 }
 
-// out[i][j] = sum over splits (in order) of partial[s][i][j] + partial[s][i][kp + j],  j < k.
+// out (rows x k) = sum over the splits of (hi part + lo part), in split order; the loads
+// of four splits go out together
+constexpr int kMaxProjSplits = 16;
 __global__ void reduce_hi_lo_kernel(const float* __restrict__ partial, int splits, int64_t rows, int kp, int k,
                                     float* __restrict__ out) {
   const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -1100,10 +1122,18 @@ __global__ void reduce_hi_lo_kernel(const float* __restrict__ partial, int split
   const int64_t i = e / k;
   const int j = (int)(e - i * k);
   const int64_t stride = rows * 2 * kp;
+  const float* row = partial + i * 2 * kp + j;
   float a = 0.0f;
-  for (int sp = 0; sp < splits; ++sp) {
-    const float* row = partial + sp * stride + i * 2 * kp;
-    a += row[j] + row[kp + j];
+  for (int s0 = 0; s0 < splits; s0 += 4) {
+    float h[4], l[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      h[u] = s0 + u < splits ? row[(s0 + u) * stride] : 0.0f;
+      l[u] = s0 + u < splits ? row[(s0 + u) * stride + kp] : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (s0 + u < splits) a += h[u] + l[u];
   }
   out[e] = a;
 }
@@ -1142,13 +1172,24 @@ __global__ void __launch_bounds__(256) factor_products_kernel(const float* __res
   const float* src = is_u ? P : V;
   const double* M = is_u ? T : Vr;
   float* dst = is_u ? Uraw : Vn;
-  for (int e = threadIdx.x; e < 64 * 64; e += 256) {
-    const int u = e >> 6, j = e & 63;
-    sm[e] = (u < k && j < k) ? M[u * kMaxW + j] : 0.0;
-  }
-  for (int e = threadIdx.x; e < kFpRows * 64; e += 256) {
-    const int rr = e >> 6, j = e & 63;
-    sr[e] = (i0 + rr < n && j < k) ? src[(i0 + rr) * k + j] : 0.0f;
+  {
+    // all 32 loads of a thread in flight at once, then the shared-memory stores
+    double mv[64 * 64 / 256];
+    float rv[kFpRows * 64 / 256];
+#pragma unroll
+    for (int it = 0; it < 64 * 64 / 256; ++it) {
+      const int e = threadIdx.x + it * 256, u = e >> 6, j = e & 63;
+      mv[it] = (u < k && j < k) ? M[u * kMaxW + j] : 0.0;
+    }
+#pragma unroll
+    for (int it = 0; it < kFpRows * 64 / 256; ++it) {
+      const int e = threadIdx.x + it * 256, rr = e >> 6, j = e & 63;
+      rv[it] = (i0 + rr < n && j < k) ? src[(i0 + rr) * k + j] : 0.0f;
+    }
+#pragma unroll
+    for (int it = 0; it < 64 * 64 / 256; ++it) sm[threadIdx.x + it * 256] = mv[it];
+#pragma unroll
+    for (int it = 0; it < kFpRows * 64 / 256; ++it) sr[threadIdx.x + it * 256] = rv[it];
   }
   __syncthreads();
   const int rg = threadIdx.x >> 4, cg = threadIdx.x & 15;   // rows 4 rg .. +3, columns 4 cg .. +3
@@ -1186,21 +1227,31 @@ __global__ void __launch_bounds__(256) factor_products_kernel(const float* __res
     }
   }
   if (!finite) raise_status(status, METIS_DEV_NONFINITE);
+  // one atomic per block (a warp's maximum, then the block's)
+  __shared__ float wmax[8];
 #pragma unroll
   for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  if ((threadIdx.x & 31) == 0) atomicMax(&fs.amax[is_u ? 0 : 1], (unsigned long long)__float_as_uint(amax));
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = wmax[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) m = fmaxf(m, wmax[w]);
+    atomicMax(&fs.amax[is_u ? 0 : 1], (unsigned long long)__float_as_uint(m));
+  }
   if (!is_u) {
-    __syncthreads();
-    for (int j = threadIdx.x; j < k; j += 256) {
+    // the key of each column's largest-|.| entry: four threads per column, 16 rows each
+    const int j = threadIdx.x & 63, part = threadIdx.x >> 6;
+    if (j < k) {
       unsigned long long best = 0;
-      for (int q = 0; q < kFpRows && i0 + q < n; ++q) {
+      for (int q = part * (kFpRows / 4); q < (part + 1) * (kFpRows / 4) && i0 + q < n; ++q) {
         const float a = fabsf(so[q * 64 + j]);
         if (!(a <= 3.402823466e38f)) continue;   // not finite
         const unsigned long long key =
             ((unsigned long long)__float_as_uint(a) << 32) | (0xFFFFFFFFu - (uint32_t)(i0 + q));
         best = key > best ? key : best;
       }
-      atomicMax(&fs.key[j], best);
+      if (best) atomicMax(&fs.key[j], best);
     }
   }
 }
@@ -1385,8 +1436,11 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
   auto project_on = [&](const __nv_bfloat16* A, int64_t lda, int64_t rows, int64_t K, const float* B, int width,
                         float* out) -> metis_status {
     const int kp = pad_width(width);
-    split_hi_lo_t_kernel<<<blocks_for((int64_t)2 * kp * K), 256, 0, st>>>(B, K, width, kp, bt2); count_launch();
+    split_hi_lo_t_kernel<<<(unsigned)((K + kSplitRows - 1) / kSplitRows), kSplitThreads, 0, st>>>(B, K, width, kp,
+                                                                                              bt2);
+    count_launch();
     const int splits = normalize_splits(K, bf16_splits(ctx, rows, K));
+    if (splits > kMaxProjSplits) return fail(ctx, METIS_ERR_ARG, "projection split count above the reduction's limit");
     if ((size_t)splits * rows * 2 * kp * 4 > tc_partial_bytes)
       return fail(ctx, METIS_ERR_WORKSPACE, "projection partials exceed workspace");
     metis_status st2 = launch_gemm_bf16(ctx, A, lda, rows, bt2, K, 2 * kp, K, tc_partial, 2 * kp, splits);
@@ -1482,8 +1536,8 @@ cudaError_t launch_transpose_bf16(const void* M, int64_t ld, int64_t r, int64_t 
 }
 
 cudaError_t launch_split_hi_lo_t(const float* F, int64_t n, int k, int kp, void* out, cudaStream_t st) {
-  split_hi_lo_t_kernel<<<blocks_for((int64_t)2 * kp * n), 256, 0, st>>>(F, n, k, kp,
-                                                                      static_cast<__nv_bfloat16*>(out));
+  split_hi_lo_t_kernel<<<(unsigned)((n + kSplitRows - 1) / kSplitRows), kSplitThreads, 0, st>>>(
+      F, n, k, kp, static_cast<__nv_bfloat16*>(out));
   count_launch();
   return cudaGetLastError();
 }

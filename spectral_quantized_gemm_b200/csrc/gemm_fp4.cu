@@ -1079,19 +1079,33 @@ metis_status launch_group_bn(metis_ctx* ctx, const GemmArgs* g, int n) {
 
 }  // namespace
 
-int fp4_splits(metis_ctx* ctx, int64_t tiles, int stages) {
-  const int64_t want = (2 * (int64_t)ctx->sm_count + tiles - 1) / tiles;
-  const int s = (int)std::max<int64_t>(1, std::min<int64_t>(want, stages));
-  const int per = (stages + s - 1) / s;
-  return (stages + per - 1) / per;
+namespace {
+// Split-K count for `tiles` output tiles of `stages` K stages each on a persistent grid of
+// sm_count CTAs: the one that minimizes rounds x (stages per unit + 3), rounds =
+// ceil(tiles x splits / sm_count) -- the last round of equal units otherwise leaves SMs
+// idle (64 tiles in 5 splits: 320 units, 3 rounds, 72% busy) -- and 3 stage-times stand
+// for a unit's pipeline fill and its partial-tile store.  At most 16 splits.
+int wave_splits(metis_ctx* ctx, int64_t tiles, int stages) {
+  const int64_t sms = std::max(1, ctx->sm_count);
+  int best = 1;
+  int64_t best_cost = -1;
+  for (int s = 1; s <= std::min(16, stages); ++s) {
+    const int per = (stages + s - 1) / s;
+    const int eff = (stages + per - 1) / per;
+    const int64_t rounds = (tiles * eff + sms - 1) / sms;
+    const int64_t cost = rounds * (per + 3);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = eff;
+    }
+  }
+  return best;
 }
+}  // namespace
 
-int bf16_splits(metis_ctx* ctx, int64_t rows, int64_t K) {
-  const int tiles = (int)(rows / 128);
-  const int stages = (int)(K / 64);
-  const int want = (2 * ctx->sm_count + tiles - 1) / tiles;
-  return std::max(1, std::min(want, stages / 4));
-}
+// NVFP4 GeMMs: K / 256 stages per 128-row tile; bf16 GeMMs: K / 64 stages per 128-row tile
+int fp4_splits(metis_ctx* ctx, int64_t tiles, int stages) { return wave_splits(ctx, tiles, stages); }
+int bf16_splits(metis_ctx* ctx, int64_t rows, int64_t K) { return wave_splits(ctx, rows / 128, (int)(K / 64)); }
 
 metis_status launch_gemm_bf16(metis_ctx* ctx, const void* A, int64_t lda, int64_t rows, const void* B, int64_t ldb,
                               int n, int64_t K, float* C, int64_t ldc, int splits) {

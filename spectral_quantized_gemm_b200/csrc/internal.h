@@ -117,8 +117,8 @@ struct GemmArgs {
   int32_t k_splits;       // > 1: split-K over the FP4 + fold stages, partial s at C + s * split_stride (fp32)
   int64_t split_stride;   // elements between consecutive partial outputs
 };
-// Split count for an FP4 GeMM of `tiles` output tiles and `stages` K stages: about two
-// work units per SM, no empty share.
+// Split count for an FP4 GeMM of `tiles` output tiles and `stages` K stages (no empty
+// share): the one whose units fill the persistent grid's rounds best.
 int fp4_splits(metis_ctx* ctx, int64_t tiles, int stages);
 metis_status launch_gemm_nvfp4(metis_ctx* ctx, const GemmArgs& a);
 // Up to three thin GeMMs (the same width 16/32/64 and K, fp32 outputs, no fold) in one launch.
@@ -127,8 +127,7 @@ metis_status launch_gemm_nvfp4_group(metis_ctx* ctx, const GemmArgs* g, int n);
 metis_status launch_wait_timeout_selftest(metis_ctx* ctx, int64_t limit_cycles);
 // ---- mma_peak.cu ----
 metis_status launch_mma_peak(metis_ctx* ctx, int64_t iters, double* flops);
-// C[s] (rows x n, fp32, split s at C + s * rows * ldc) = A (rows x K bf16, lda) * B^T
-// (B: n x K bf16, ldb) over the s-th share of K.  splits < 1 picks a split count;
+// Split count for a bf16 GeMM of rows / 128 tiles and K / 64 stages, chosen the same way.
 int bf16_splits(metis_ctx* ctx, int64_t rows, int64_t K);
 // Split count with no empty share of the K / 64 stages (what the launch uses).
 inline int normalize_splits(int64_t K, int splits) {
@@ -136,6 +135,8 @@ inline int normalize_splits(int64_t K, int splits) {
   const int per = (stages + splits - 1) / splits;
   return (stages + per - 1) / per;
 }
+// C[s] (rows x n, fp32, split s at C + s * rows * ldc) = A (rows x K bf16, lda) * B^T
+// (B: n x K bf16, ldb) over the s-th share of K.  splits < 1 picks a split count.
 metis_status launch_gemm_bf16(metis_ctx* ctx, const void* A, int64_t lda, int64_t rows, const void* B, int64_t ldb,
                               int n, int64_t K, float* C, int64_t ldc, int splits);
 

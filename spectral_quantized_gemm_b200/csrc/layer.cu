@@ -49,8 +49,27 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// The main GeMM's fold operands, 64 rows per block (8 warps, 8 rows each, a lane owning
-// columns j and j + 1 of a kp-wide part and writing both of its copies):
+// a + the sum over sp < n of the float pairs at base + sp * stride, taken in split order;
+// the loads go out four at a time
+__device__ __forceinline__ float2 add_splits(float2 a, const float* base, int64_t stride, int n) {
+  for (int s0 = 0; s0 < n; s0 += 4) {
+    float2 t[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      t[u] = s0 + u < n ? *reinterpret_cast<const float2*>(base + (s0 + u) * stride) : make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (s0 + u < n) {
+        a.x += t[u].x;
+        a.y += t[u].y;
+      }
+  }
+  return a;
+}
+
+// The main GeMM's fold operands, 32 rows per block (8 warps, 4 consecutive rows each,
+// formed together; a lane owns columns j and j + 1 of a kp-wide part and writes both of
+// its copies):
 //   Fa rows i < p:  [Q(L_A) | Q(L_A) | T_B hi | T_B lo | 0] / alpha,
 //                   T_B = (sum of the splits of Q(A_R) Q(L_B)) S_B
 //   Fb rows i < q:  [T_A^T hi | T_A^T lo | Q(R_B) | Q(R_B) | 0],
@@ -66,7 +85,7 @@ __global__ void __launch_bounds__(256) fold_assemble_kernel(
     const float* __restrict__ SB, int kA, int kB, int kpA, int kpB, FactorView LA, FactorView RB, int64_t p, int64_t q,
     int fold_k, const float* ga, const float* gb, __nv_bfloat16* __restrict__ Fa, __nv_bfloat16* __restrict__ Fb) {
   __shared__ float zs[64 * 66];   // zs[u * 66 + a] = S_B[u] Z[a][u] (row pitch 66: fewer bank conflicts)
-  __shared__ float rbs[8][64];    // per warp: Q(R_B)(i, u) of the warp's current row
+  __shared__ __align__(16) float rbs[8][64 * 4];   // per warp: Q(R_B)(i, u) of the warp's 4 rows, u-major
   // the block's 32 rows of the factor it decodes (Q(L_A) on Fa rows, Q(R_B) on Fb rows):
   // 16 code bytes and 2 scale bytes per factor column t, staged with coalesced loads
   __shared__ uint8_t fcodes[64 * 16];
@@ -112,92 +131,131 @@ __global__ void __launch_bounds__(256) fold_assemble_kernel(
     __syncthreads();
   }
   const float inv_alpha = is_a ? 1.0f / ((*ga) * (*gb)) : 1.0f;   // exact: a power of two
-  for (int rr = warp; rr < kFoldRows; rr += 8) {
-    const int64_t i = r0 + rr;
-    if (i >= (is_a ? p : q)) break;
-    __nv_bfloat16* dst = (is_a ? Fa : Fb) + i * fold_k;
-    if (is_a) {
-      // Q(L_A) copies
-      const float gl = kA ? *LA.g : 1.0f;
-      for (int j = 2 * lane; j < kpA; j += 64) {
-        const float v0 = j < kA ? staged_factor(fcodes, fscales, gl, j, rr) * inv_alpha : 0.0f;
-        const float v1 = j + 1 < kA ? staged_factor(fcodes, fscales, gl, j + 1, rr) * inv_alpha : 0.0f;
-        const uint32_t w = pack_bf16x2(v0, v1);
-        *reinterpret_cast<uint32_t*>(dst + j) = w;
-        *reinterpret_cast<uint32_t*>(dst + kpA + j) = w;
-      }
-      // T_B hi / lo
-      for (int j = 2 * lane; j < kpB; j += 64) {
-        float v0 = 0.0f, v1 = 0.0f;
-        for (int sp = 0; sp < bsplits; ++sp) {
-          const float2 t = *reinterpret_cast<const float2*>(TB + sp * tb_stride + i * kpB + j);
-          v0 += t.x;
-          v1 += t.y;
-        }
-        v0 = j < kB ? v0 * SB[j] * inv_alpha : 0.0f;
-        v1 = j + 1 < kB ? v1 * SB[j + 1] * inv_alpha : 0.0f;
-        const float h0 = __bfloat162float(__float2bfloat16_rn(v0)), h1 = __bfloat162float(__float2bfloat16_rn(v1));
-        *reinterpret_cast<uint32_t*>(dst + 2 * kpA + j) = pack_bf16x2(h0, h1);
-        *reinterpret_cast<uint32_t*>(dst + 2 * kpA + kpB + j) = pack_bf16x2(v0 - h0, v1 - h1);
-      }
-    } else {
-      // Q(R_B)(i, u) for u = lane and lane + 32 (exact in bf16)
-      const float gr = kB ? *RB.g : 1.0f;
-      const float rb0 = lane < kB ? staged_factor(fcodes, fscales, gr, lane, rr) : 0.0f;
-      const float rb1 = lane + 32 < kB ? staged_factor(fcodes, fscales, gr, lane + 32, rr) : 0.0f;
-      // T_A^T hi / lo: lane owns columns j, j + 1 (kpA <= 64, so at most one pair per lane)
-      const int j = 2 * lane;
-      float c0 = 0.0f, c1 = 0.0f;
-      if (corr) {
-        rbs[warp][lane] = rb0;
-        rbs[warp][lane + 32] = rb1;
-        __syncwarp();
-        if (j < kpA) {
-          // four partial sums break the FMA dependency chain (fixed order: bit-reproducible)
-          float p0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, p1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-          int u = 0;
-          for (; u + 4 <= kB; u += 4) {
+  // a warp owns 4 consecutive rows and forms them together, so that the split partials of
+  // its rows are loaded together and every shared-memory value feeds four rows
+  constexpr int kRowsPerWarp = kFoldRows / 8;
+  const int rr0 = warp * kRowsPerWarp;
+  const int64_t nrows = is_a ? p : q;
+  bool live[kRowsPerWarp];
+  __nv_bfloat16* dst[kRowsPerWarp];
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              const float r = rbs[warp][u + t];
-              const float2 z = *reinterpret_cast<const float2*>(zs + (u + t) * 66 + j);
-              p0[t] = fmaf(r, z.x, p0[t]);
-              p1[t] = fmaf(r, z.y, p1[t]);
-            }
-          }
-          for (; u < kB; ++u) {
-            const float r = rbs[warp][u];
-            const float2 z = *reinterpret_cast<const float2*>(zs + u * 66 + j);
-            p0[0] = fmaf(r, z.x, p0[0]);
-            p1[0] = fmaf(r, z.y, p1[0]);
-          }
-          c0 = (p0[0] + p0[1]) + (p0[2] + p0[3]);
-          c1 = (p1[0] + p1[1]) + (p1[2] + p1[3]);
-        }
-        __syncwarp();   // the buffer is rewritten for the warp's next row
-      }
-      if (j < kpA) {
-        float v0 = c0, v1 = c1;
-        for (int sp = 0; sp < asplits; ++sp) {
-          const float2 t = *reinterpret_cast<const float2*>(TA + sp * ta_stride + i * kpA + j);
-          v0 += t.x;
-          v1 += t.y;
-        }
-        v0 = j < kA ? v0 * SA[j] : 0.0f;
-        v1 = j + 1 < kA ? v1 * SA[j + 1] : 0.0f;
-        const float h0 = __bfloat162float(__float2bfloat16_rn(v0)), h1 = __bfloat162float(__float2bfloat16_rn(v1));
-        *reinterpret_cast<uint32_t*>(dst + j) = pack_bf16x2(h0, h1);
-        *reinterpret_cast<uint32_t*>(dst + kpA + j) = pack_bf16x2(v0 - h0, v1 - h1);
-      }
-      // Q(R_B) copies
-      for (int u = lane; u < kpB; u += 32) {
-        const __nv_bfloat16 v = __float2bfloat16_rn(u < 32 ? rb0 : rb1);
-        dst[2 * kpA + u] = v;
-        dst[2 * kpA + kpB + u] = v;
+  for (int x = 0; x < kRowsPerWarp; ++x) {
+    live[x] = r0 + rr0 + x < nrows;
+    dst[x] = (is_a ? Fa : Fb) + (r0 + rr0 + x) * fold_k;
+  }
+  if (is_a) {
+    // Q(L_A) copies
+    const float gl = kA ? *LA.g : 1.0f;
+#pragma unroll
+    for (int x = 0; x < kRowsPerWarp; ++x) {
+      if (!live[x]) continue;
+      for (int j = 2 * lane; j < kpA; j += 64) {
+        const float v0 = j < kA ? staged_factor(fcodes, fscales, gl, j, rr0 + x) * inv_alpha : 0.0f;
+        const float v1 = j + 1 < kA ? staged_factor(fcodes, fscales, gl, j + 1, rr0 + x) * inv_alpha : 0.0f;
+        const uint32_t w = pack_bf16x2(v0, v1);
+        *reinterpret_cast<uint32_t*>(dst[x] + j) = w;
+        *reinterpret_cast<uint32_t*>(dst[x] + kpA + j) = w;
       }
     }
-    // padding columns
-    for (int c = 2 * kpA + 2 * kpB + 2 * lane; c < fold_k; c += 64) *reinterpret_cast<uint32_t*>(dst + c) = 0u;
+    // T_B hi / lo
+    for (int j = 2 * lane; j < kpB; j += 64) {
+      float2 a[kRowsPerWarp];
+#pragma unroll
+      for (int x = 0; x < kRowsPerWarp; ++x) a[x] = make_float2(0.0f, 0.0f);
+      for (int sp = 0; sp < bsplits; ++sp) {
+        float2 t[kRowsPerWarp];
+#pragma unroll
+        for (int x = 0; x < kRowsPerWarp; ++x)
+          t[x] = live[x] ? *reinterpret_cast<const float2*>(TB + sp * tb_stride + (r0 + rr0 + x) * kpB + j)
+                         : make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int x = 0; x < kRowsPerWarp; ++x) {
+          a[x].x += t[x].x;
+          a[x].y += t[x].y;
+        }
+      }
+#pragma unroll
+      for (int x = 0; x < kRowsPerWarp; ++x) {
+        if (!live[x]) continue;
+        const float v0 = j < kB ? a[x].x * SB[j] * inv_alpha : 0.0f;
+        const float v1 = j + 1 < kB ? a[x].y * SB[j + 1] * inv_alpha : 0.0f;
+        const float h0 = __bfloat162float(__float2bfloat16_rn(v0)), h1 = __bfloat162float(__float2bfloat16_rn(v1));
+        *reinterpret_cast<uint32_t*>(dst[x] + 2 * kpA + j) = pack_bf16x2(h0, h1);
+        *reinterpret_cast<uint32_t*>(dst[x] + 2 * kpA + kpB + j) = pack_bf16x2(v0 - h0, v1 - h1);
+      }
+    }
+  } else {
+    // Q(R_B)(i, u) for u = lane and lane + 32 (exact in bf16), staged u-major for the
+    // correction: rbs[warp][u][x]
+    const float gr = kB ? *RB.g : 1.0f;
+    float rb[kRowsPerWarp][2];
+#pragma unroll
+    for (int x = 0; x < kRowsPerWarp; ++x) {
+      rb[x][0] = lane < kB ? staged_factor(fcodes, fscales, gr, lane, rr0 + x) : 0.0f;
+      rb[x][1] = lane + 32 < kB ? staged_factor(fcodes, fscales, gr, lane + 32, rr0 + x) : 0.0f;
+    }
+    // T_A^T hi / lo: lane owns columns j, j + 1 (kpA <= 64, so at most one pair per lane)
+    const int j = 2 * lane;
+    float2 c[kRowsPerWarp];
+#pragma unroll
+    for (int x = 0; x < kRowsPerWarp; ++x) c[x] = make_float2(0.0f, 0.0f);
+    if (corr) {
+      *reinterpret_cast<float4*>(&rbs[warp][lane * 4]) = make_float4(rb[0][0], rb[1][0], rb[2][0], rb[3][0]);
+      *reinterpret_cast<float4*>(&rbs[warp][(lane + 32) * 4]) = make_float4(rb[0][1], rb[1][1], rb[2][1], rb[3][1]);
+      __syncwarp();
+      if (j < kpA) {
+        // eight independent sums (4 rows x 2 columns) per lane, each over u in order
+        for (int u = 0; u < kB; ++u) {
+          const float4 r = *reinterpret_cast<const float4*>(&rbs[warp][u * 4]);
+          const float2 z = *reinterpret_cast<const float2*>(zs + u * 66 + j);
+          const float rv[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+          for (int x = 0; x < kRowsPerWarp; ++x) {
+            c[x].x = fmaf(rv[x], z.x, c[x].x);
+            c[x].y = fmaf(rv[x], z.y, c[x].y);
+          }
+        }
+      }
+    }
+    if (j < kpA) {
+      for (int sp = 0; sp < asplits; ++sp) {
+        float2 t[kRowsPerWarp];
+#pragma unroll
+        for (int x = 0; x < kRowsPerWarp; ++x)
+          t[x] = live[x] ? *reinterpret_cast<const float2*>(TA + sp * ta_stride + (r0 + rr0 + x) * kpA + j)
+                         : make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int x = 0; x < kRowsPerWarp; ++x) {
+          c[x].x += t[x].x;
+          c[x].y += t[x].y;
+        }
+      }
+#pragma unroll
+      for (int x = 0; x < kRowsPerWarp; ++x) {
+        if (!live[x]) continue;
+        const float v0 = j < kA ? c[x].x * SA[j] : 0.0f;
+        const float v1 = j + 1 < kA ? c[x].y * SA[j + 1] : 0.0f;
+        const float h0 = __bfloat162float(__float2bfloat16_rn(v0)), h1 = __bfloat162float(__float2bfloat16_rn(v1));
+        *reinterpret_cast<uint32_t*>(dst[x] + j) = pack_bf16x2(h0, h1);
+        *reinterpret_cast<uint32_t*>(dst[x] + kpA + j) = pack_bf16x2(v0 - h0, v1 - h1);
+      }
+    }
+    // Q(R_B) copies
+#pragma unroll
+    for (int x = 0; x < kRowsPerWarp; ++x) {
+      if (!live[x]) continue;
+      for (int u = lane; u < kpB; u += 32) {
+        const __nv_bfloat16 v = __float2bfloat16_rn(u < 32 ? rb[x][0] : rb[x][1]);
+        dst[x][2 * kpA + u] = v;
+        dst[x][2 * kpA + kpB + u] = v;
+      }
+    }
+  }
+  // padding columns
+#pragma unroll
+  for (int x = 0; x < kRowsPerWarp; ++x) {
+    if (!live[x]) continue;
+    for (int cc = 2 * kpA + 2 * kpB + 2 * lane; cc < fold_k; cc += 64) *reinterpret_cast<uint32_t*>(dst[x] + cc) = 0u;
   }
 }
 

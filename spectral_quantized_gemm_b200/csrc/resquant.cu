@@ -575,21 +575,47 @@ __global__ void __launch_bounds__(kRqThreads, 1)
 // (e kept in [-63, 63]; 0 for an all-zero block), and every entry x (k columns, padded
 // with zeros to 64) is written as the fp16 pair hi = RN16(x 2^e), lo = RN16(x 2^e - hi):
 // row i of the output holds the 64 hi values, then the 64 lo values.  fac[block] = 2^-e.
-__global__ void __launch_bounds__(256) split_factors_kernel(const float* __restrict__ U, const float* __restrict__ S,
-                                                            const float* __restrict__ V, int64_t rows, int k,
-                                                            __half* __restrict__ A16, __half* __restrict__ B16,
-                                                            float* __restrict__ fac_a, float* __restrict__ fac_b) {
-  __shared__ float red[8];
+// A block of 512 threads holds its 128 x 64 tile in registers -- four runs of four
+// consecutive columns a thread, loaded as float4 when k = 64 and the factors are 16-byte
+// aligned -- reduces the maximum, then writes each run's four hi and four lo values as
+// one 8-byte store each.
+constexpr int kSplitFacThreads = 512;
+constexpr int kSplitFacRuns = 128 * kSplitWidth / 4 / kSplitFacThreads;
+__global__ void __launch_bounds__(kSplitFacThreads) split_factors_kernel(
+    const float* __restrict__ U, const float* __restrict__ S, const float* __restrict__ V, int64_t rows, int k,
+    bool vec, __half* __restrict__ A16, __half* __restrict__ B16, float* __restrict__ fac_a,
+    float* __restrict__ fac_b) {
+  __shared__ float red[kSplitFacThreads / 32];
   const int64_t nb_a = rows / 128;
   const bool is_a = (int64_t)blockIdx.x < nb_a;
   const int64_t blk = is_a ? (int64_t)blockIdx.x : (int64_t)blockIdx.x - nb_a;
   const float* F = (is_a ? U : V) + blk * 128 * k;
   __half* out = (is_a ? A16 : B16) + blk * 128 * 128;
+  float v[kSplitFacRuns][4];
+#pragma unroll
+  for (int it = 0; it < kSplitFacRuns; ++it) {
+    const int t = threadIdx.x + it * kSplitFacThreads;
+    const int i = t >> 4, j0 = (t & 15) * 4;
+    if (vec) {
+      const float4 x = *reinterpret_cast<const float4*>(F + i * kSplitWidth + j0);
+      v[it][0] = x.x;
+      v[it][1] = x.y;
+      v[it][2] = x.z;
+      v[it][3] = x.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[it][e] = j0 + e < k ? F[i * k + j0 + e] : 0.0f;
+    }
+  }
   float m = 0.0f;
-  for (int t = threadIdx.x; t < 128 * k; t += blockDim.x) {
-    float x = F[t];
-    if (is_a) x = __fmul_rn(x, S[t % k]);
-    m = fmaxf(m, fabsf(x));
+#pragma unroll
+  for (int it = 0; it < kSplitFacRuns; ++it) {
+    const int j0 = ((threadIdx.x + it * kSplitFacThreads) & 15) * 4;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (is_a) v[it][e] = j0 + e < k ? __fmul_rn(v[it][e], S[j0 + e]) : 0.0f;
+      m = fmaxf(m, fabsf(v[it][e]));
+    }
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -597,7 +623,7 @@ __global__ void __launch_bounds__(256) split_factors_kernel(const float* __restr
   __syncthreads();
   m = red[0];
 #pragma unroll
-  for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w]);
+  for (int w = 1; w < kSplitFacThreads / 32; ++w) m = fmaxf(m, red[w]);
   int ex = 0;
   if (m > 0.0f && m <= 3.402823466e38f) {
     const int fl = (int)((__float_as_uint(m) >> 23) & 0xFFu) - 127;   // floor(log2 m); -127 for subnormal m
@@ -605,18 +631,19 @@ __global__ void __launch_bounds__(256) split_factors_kernel(const float* __restr
   }
   const float up = __uint_as_float((uint32_t)(ex + 127) << 23);
   if (threadIdx.x == 0) (is_a ? fac_a : fac_b)[blk] = __uint_as_float((uint32_t)(127 - ex) << 23);
-  for (int t = threadIdx.x; t < 128 * kSplitWidth; t += blockDim.x) {
-    const int i = t >> 6, j = t & 63;
-    float x = 0.0f;
-    if (j < k) {
-      x = F[i * k + j];
-      if (is_a) x = __fmul_rn(x, S[j]);
+#pragma unroll
+  for (int it = 0; it < kSplitFacRuns; ++it) {
+    const int t = threadIdx.x + it * kSplitFacThreads;
+    const int i = t >> 4, j0 = (t & 15) * 4;
+    __half hi[4], lo[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float x = __fmul_rn(v[it][e], up);
+      hi[e] = __float2half_rn(x);
+      lo[e] = __float2half_rn(__fsub_rn(x, __half2float(hi[e])));
     }
-    x = __fmul_rn(x, up);
-    const __half hi = __float2half_rn(x);
-    const __half lo = __float2half_rn(__fsub_rn(x, __half2float(hi)));
-    out[i * 128 + j] = hi;
-    out[i * 128 + 64 + j] = lo;
+    *reinterpret_cast<uint2*>(out + i * 128 + j0) = *reinterpret_cast<const uint2*>(hi);
+    *reinterpret_cast<uint2*>(out + i * 128 + 64 + j0) = *reinterpret_cast<const uint2*>(lo);
   }
 }
 
@@ -693,7 +720,10 @@ metis_status run_residual_quantize_into(metis_ctx* ctx, const metis_matrix* M, c
   CUtensorMap mA, mV;
   if (recon) {
     const unsigned nblk = (unsigned)(M->rows / 128 + M->cols / 128);
-    split_factors_kernel<<<nblk, 256, 0, ctx->stream>>>(f->U, f->S, f->V, M->rows, k, A16, B16, fac_a, fac_b);
+    const bool vec = k == kSplitWidth && reinterpret_cast<uintptr_t>(f->U) % 16 == 0 &&
+                     reinterpret_cast<uintptr_t>(f->V) % 16 == 0;
+    split_factors_kernel<<<nblk, kSplitFacThreads, 0, ctx->stream>>>(f->U, f->S, f->V, M->rows, k, vec, A16, B16,
+                                                                     fac_a, fac_b);
     count_launch();
     if ((s = check_cuda(ctx, cudaGetLastError(), "split factors")) != METIS_OK) return s;
     if (!map2d(&mA, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, A16, 128, M->rows, 256, 64, 128) ||
