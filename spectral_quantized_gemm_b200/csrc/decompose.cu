@@ -32,6 +32,12 @@ constexpr double kDropTol = 1e-12;
 // eigenvectors to the Gram's own accuracy, and an operand whose basis already diagonalizes
 // its Gram (an unchanged matrix) needs no sweep.
 constexpr double kJacobiTol = 1e-5;
+// The two-kernel solver also leaves alone an off-diagonal entry below this, in units of
+// the largest diagonal entry (it works on the matrix scaled to make that entry 1..2):
+// entries at rounding level of a rank-deficient Gram would otherwise keep its
+// near-zero eigenvalues rotating among themselves for good, and no eigenvalue above the
+// drop threshold (kDropTol) moves by more than (1e-13)^2 / gap.
+constexpr double kJacobiFloor = 1e-13;
 constexpr int kJacobiMaxSweeps = 40;
 constexpr int kMaxW = 128;
 constexpr int kSmallMaxN = 96;                 // sketch width limit of the one-CTA solver
@@ -750,7 +756,8 @@ __global__ void __launch_bounds__(kEigThreads) eig_solver_kernel(const double* _
 //   the slot grid.  The rotation of the NEXT round's pair a' is computed in the same step
 //   by the owner of the block that holds that pair's off-diagonal element; the two new
 //   diagonal entries it needs are recomputed from the old diagonal blocks with the same
-//   correctly rounded arithmetic the diagonal owners use.  One barrier per round.  Each
+//   correctly rounded arithmetic the diagonal owners use.  One barrier per round.  The
+//   matrix is held scaled by a power of two; entries below kJacobiFloor of it are left.  Each
 //   round's rotations (c, s) go to global memory; after a whole number of sweeps every
 //   element is back in its own slot, so the diagonal is the spectrum in index order.
 // jacobi_replay_kernel (a warp per row of Z): applies the recorded rotations and slot
@@ -784,11 +791,17 @@ __device__ __forceinline__ int jac_src(int s, int m) {
   return a == m - 1 ? 2 * m - 2 : 2 * a + 3;
 }
 
+// Whether the two-kernel solver still rotates an entry g between diagonal entries a and b
+// (of the scaled matrix).
+__device__ __forceinline__ bool jac_needs(double g, double a, double b, double tol2) {
+  return g != 0.0 && g * g > tol2 * (a * b) && g * g > kJacobiFloor * kJacobiFloor;
+}
+
 // rotation (c, s) that annihilates ga in [[al, ga], [ga, be]] (x_p' = c x_p - s x_q,
-// x_q' = s x_p + c x_q), or the identity when |ga| is below tol * sqrt(al be)
+// x_q' = s x_p + c x_q), or the identity when jac_needs says no
 __device__ __forceinline__ double2 jac_rotation(double al, double be, double ga, double tol2) {
   double c = 1.0, s = 0.0;
-  if (ga != 0.0 && ga * ga > tol2 * (al * be)) {
+  if (jac_needs(ga, al, be, tol2)) {
     const double dd = be - al;
     const double g2 = 2.0 * ga;
     const double x = fma(dd, dd, g2 * g2);
@@ -830,12 +843,29 @@ __global__ void __launch_bounds__(kJacThreads, 1) jacobi_rounds_kernel(const dou
   double* dof = reinterpret_cast<double*>(dgn + 2 * m);               // [2][m] off-diagonal ga of pair p
   __shared__ double lam[kJacMaxNE];
   __shared__ int order[kJacMaxNE];
+  __shared__ double scale_s[2];
   const int tid = threadIdx.x;
   const double tol2 = kJacobiTol * kJacobiTol;
 
+  // The matrix is held scaled by 2^-E (exact), E = floor(log2) of its largest diagonal
+  // entry, so that kJacobiFloor is relative to it; the eigenvalues are scaled back.
+  if (tid < 32) {
+    double g = 0.0;
+    for (int j = tid; j < n; j += 32) g = fmax(g, fabs(G[j * n + j]));
+#pragma unroll
+    for (int off = 16; off; off >>= 1) g = fmax(g, __shfl_xor_sync(0xffffffffu, g, off));
+    if (tid == 0) {
+      const bool ok = g > 0.0 && g <= 1.7976931348623157e308;
+      const int e = ok ? max(-1000, min(1000, ilogb(g))) : 0;
+      scale_s[0] = ldexp(1.0, -e);
+      scale_s[1] = ldexp(1.0, e);
+    }
+  }
+  __syncthreads();
+  const double down = scale_s[0];
   for (int e = tid; e < ne * ne; e += kJacThreads) {
     const int i = e / ne, j = e - (e / ne) * ne;
-    Hbuf0[e] = (i < n && j < n && i <= j) ? G[i * n + j] : 0.0;
+    Hbuf0[e] = (i < n && j < n && i <= j) ? G[i * n + j] * down : 0.0;
   }
   // Roles, warp-aligned so that each warp runs one instruction stream.  The pair warps
   // (ceil(m / 32) of them, warps 0, 4, ...) own pair p: its 2 x 2 diagonal block, kept in
@@ -905,11 +935,11 @@ __global__ void __launch_bounds__(kJacThreads, 1) jacobi_rounds_kernel(const dou
       const double2 da = Dc[a], db = Dc[b];
       const double h00 = Hr[2 * a * ne + 2 * b], h01 = Hr[2 * a * ne + 2 * b + 1];
       const double h10 = Hr[(2 * a + 1) * ne + 2 * b], h11 = Hr[(2 * a + 1) * ne + 2 * b + 1];
-      need = (h00 != 0.0 && h00 * h00 > tol2 * (da.x * db.x)) || (h01 != 0.0 && h01 * h01 > tol2 * (da.x * db.y)) ||
-             (h10 != 0.0 && h10 * h10 > tol2 * (da.y * db.x)) || (h11 != 0.0 && h11 * h11 > tol2 * (da.y * db.y));
+      need = jac_needs(h00, da.x, db.x, tol2) || jac_needs(h01, da.x, db.y, tol2) ||
+             jac_needs(h10, da.y, db.x, tol2) || jac_needs(h11, da.y, db.y, tol2);
     } else if (is_pair) {
       const double2 d = Dc[p];
-      need = own_ga != 0.0 && own_ga * own_ga > tol2 * (d.x * d.y);
+      need = jac_needs(own_ga, d.x, d.y, tol2);
     }
     if (!__syncthreads_or(need)) break;
     if (sweep == kJacobiMaxSweeps) {
@@ -962,9 +992,10 @@ __global__ void __launch_bounds__(kJacThreads, 1) jacobi_rounds_kernel(const dou
     }
   }
   // after whole sweeps every element is in its own slot: the diagonal is the spectrum
+  const double up = scale_s[1];
   const double2* Dc = dgn + (round & 1) * m;
   for (int j = tid; j < ne; j += kJacThreads) {
-    const double l = (j & 1) ? Dc[j >> 1].y : Dc[j >> 1].x;
+    const double l = ((j & 1) ? Dc[j >> 1].y : Dc[j >> 1].x) * up;
     lam[j] = (l == l) ? l : -HUGE_VAL;
   }
   __syncthreads();

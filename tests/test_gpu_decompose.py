@@ -199,3 +199,25 @@ def test_rank_deficient_sketch_drops_directions(ctx, metis_lib, k):
     low = (gU * gS) @ gV.T
     if k >= 5:                                # rank 5 is captured whole
         assert np.linalg.norm(low - M) / np.linalg.norm(M) < 1e-3
+
+
+def test_rank_deficient_step_gram_converges(ctx, metis_lib):
+    """M of exact rank 20 and a per-step basis of k = 32: the Gram of P = M V has 12
+    eigenvalues at rounding level, whose mutual entries the eigensolver leaves alone once
+    they fall below 1e-13 of the largest diagonal entry (without that floor they rotate
+    among themselves until the sweep limit).  No numeric failure; the 20 captured singular
+    values and directions match the oracle's."""
+    Mt = _duplicated_columns(20, rows=512, cols=256, seed=5)
+    M = Mt.double().numpy()
+    f = _gpu_decompose(ctx, Mt.cuda(), 32, 8, 512, 3, 0)           # refresh (unsampled sketch)
+    assert ctx.poll_device_status() == 0
+    V0 = f.V.cpu().double().numpy()
+    _gpu_decompose(ctx, Mt.cuda(), 32, 8, 512, 3, 0, refresh=False, step=1, factors=f)
+    assert ctx.poll_device_status() == 0
+    U, S, V = decompose.step_factors(M, V0)
+    gS = f.S.cpu().double().numpy()[:32]
+    assert np.max(np.abs(gS[:20] - S[:20]) / S[0]) < 1e-3
+    assert np.all(gS[20:] <= 1e-3 * gS[0])
+    gV, gU = f.V.cpu().double().numpy(), f.U.cpu().double().numpy()
+    assert linalg.principal_cosines(gV[:, :20], V[:, :20]).min() >= COS
+    assert linalg.principal_cosines(gU[:, :20], U[:, :20]).min() >= COS
