@@ -45,9 +45,9 @@ DEFAULT_CONFIG = "llama3_8b_mlp_up"
 METRIC = "effective TFLOP/s of Metis W4A4G4 linear fwd+bwd; % of NVFP4 MMA peak"
 # DRAM bytes (read + write) of one launch of the fused GeMM (CTA-pair kernel) at the
 # forward shape (8192 x 14336 x 4096, fold 256, bf16 out), from one ncu capture of this
-# kernel version (profile_case.py gemm --bf16; the summary sits under profiles/).
+# kernel version (bench.py --stage gemm; the summary sits under profiles/).
 # Must be retaken whenever the kernel changes.
-GEMM_FWD_DRAM_BYTES = 69.383424e6 + 192.398336e6
+GEMM_FWD_DRAM_BYTES = 69.213184e6 + 193.452544e6
 # DRAM bytes (read + write) of one launch of the residual quantizer on the benchmark's D
 # (8192 x 14336, k = 64, SR), from one ncu capture of this kernel version
 # (bench.py --stage resquant; the summary sits under profiles/). Must be retaken whenever the kernel changes.
