@@ -73,16 +73,37 @@ __global__ void __launch_bounds__(1024) sample_select_kernel(const uint64_t* key
       if ((key & mk) == pf) atomicAdd(&hist[(key >> shift) & 255u], 1u);
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int64_t cum = 0;
-      int b = 0;
-      for (; b < 256; ++b) {
-        if (cum + hist[b] >= need) break;
-        cum += hist[b];
+    if (threadIdx.x < 32) {
+      // warp 0 finds the bin where the running count reaches `need`: lane l holds bins
+      // 8 l .. 8 l + 7; an inclusive shuffle scan of the lane sums gives each lane the count
+      // below its bins, and the lane whose bins cross `need` walks them
+      const int l = threadIdx.x;
+      unsigned int h[8], sum = 0;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        h[t] = hist[8 * l + t];
+        sum += h[t];
       }
-      need -= cum;
-      prefix |= (uint64_t)b << shift;
-      mask |= (uint64_t)255u << shift;
+      unsigned int incl = sum;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const unsigned int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (l >= off) incl += v;
+      }
+      const int64_t nd = need;
+      const int64_t below = (int64_t)(incl - sum);
+      const bool mine = below < nd && (int64_t)incl >= nd;
+      if (mine) {
+        int64_t cum = below;
+        int b = 8 * l;
+        for (int t = 0; t < 8; ++t, ++b) {
+          if (cum + h[t] >= nd) break;
+          cum += h[t];
+        }
+        need = nd - cum;
+        prefix |= (uint64_t)b << shift;
+        mask |= (uint64_t)255u << shift;
+      }
     }
     __syncthreads();
   }
@@ -91,18 +112,32 @@ __global__ void __launch_bounds__(1024) sample_select_kernel(const uint64_t* key
   const int64_t lo = threadIdx.x * chunk, hi = min(rows, lo + chunk);
   int64_t cnt = 0;
   for (int64_t i = lo; i < hi; ++i) cnt += keys[i] <= thr;
-  scan[threadIdx.x] = cnt;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int64_t acc = 0;
-    for (int t = 0; t < (int)blockDim.x; ++t) {
-      const int64_t c = scan[t];
-      scan[t] = acc;
-      acc += c;
+  // exclusive block scan of the counts: shuffle scans within warps, then of the warp totals
+  {
+    const int l = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int64_t incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int64_t v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (l >= off) incl += v;
     }
+    if (l == 31) scan[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+      const int64_t tot = l < (int)(blockDim.x >> 5) ? scan[l] : 0;
+      int64_t wi = tot;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int64_t v = __shfl_up_sync(0xffffffffu, wi, off);
+        if (l >= off) wi += v;
+      }
+      scan[32 + l] = wi - tot;   // exclusive prefix of the warp totals
+    }
+    __syncthreads();
+    cnt = scan[32 + wid] + incl - cnt;
   }
   __syncthreads();
-  int64_t pos = scan[threadIdx.x];
+  int64_t pos = cnt;
   for (int64_t i = lo; i < hi; ++i)
     if (keys[i] <= thr) out_idx[pos++] = (int32_t)i;
 }
@@ -159,20 +194,35 @@ __global__ void __launch_bounds__(256) rows_times_matrix_kernel(
   for (int i = 0; i < kPerThread; ++i) acc[i] = 0.0f;
   bool finite = true;
   for (int64_t c0 = c_begin; c0 < c_end; c0 += kColChunk) {
-    for (int e = threadIdx.x; e < kRowsPerBlock * kColChunk; e += blockDim.x) {
-      const int rr = e / kColChunk, c = e % kColChunk;
+    // every load of the chunk in flight before the first shared-memory store
+    constexpr int kML = kRowsPerBlock * kColChunk / 256, kBL = kColChunk * kMaxW / 256;
+    float mv[kML], bv[kBL];
+#pragma unroll
+    for (int it = 0; it < kML; ++it) {
+      const int e = threadIdx.x + it * 256, rr = e / kColChunk, c = e % kColChunk;
       const int64_t row = r0 + rr;
       float v = 0.0f;
       if (row < nr && c0 + c < c_end) {
         const int64_t src = rowmap ? rowmap[row] : row;
         v = __bfloat162float(M[src * ld + c0 + c]);
-        finite &= isfinite(v);
       }
-      sm[rr][c] = v;
+      mv[it] = v;
     }
-    for (int e = threadIdx.x; e < kColChunk * kMaxW; e += blockDim.x) {
-      const int c = e / kMaxW, j = e % kMaxW;
-      sb[c][j] = (c0 + c < c_end && j < w) ? B[(c0 + c) * w + j] : 0.0f;
+#pragma unroll
+    for (int it = 0; it < kBL; ++it) {
+      const int e = threadIdx.x + it * 256, c = e / kMaxW, j = e % kMaxW;
+      bv[it] = (c0 + c < c_end && j < w) ? B[(c0 + c) * w + j] : 0.0f;
+    }
+#pragma unroll
+    for (int it = 0; it < kML; ++it) {
+      const int e = threadIdx.x + it * 256;
+      finite &= isfinite(mv[it]);
+      sm[e / kColChunk][e % kColChunk] = mv[it];
+    }
+#pragma unroll
+    for (int it = 0; it < kBL; ++it) {
+      const int e = threadIdx.x + it * 256;
+      sb[e / kMaxW][e % kMaxW] = bv[it];
     }
     __syncthreads();
 #pragma unroll 4
@@ -214,18 +264,32 @@ __global__ void __launch_bounds__(256) cols_times_matrix_kernel(
 #pragma unroll
   for (int i = 0; i < kPerThread; ++i) acc[i] = 0.0f;
   for (int64_t r0 = 0; r0 < nr; r0 += 16) {
-    for (int e = threadIdx.x; e < 16 * 64; e += blockDim.x) {
-      const int rr = e / 64, cc = e % 64;
+    // every load of the chunk in flight before the first shared-memory store
+    float mv[16 * 64 / 256], qv[16 * kMaxW / 256];
+#pragma unroll
+    for (int it = 0; it < 16 * 64 / 256; ++it) {
+      const int e = threadIdx.x + it * 256, rr = e / 64, cc = e % 64;
       float v = 0.0f;
       if (r0 + rr < nr && c0 + cc < ncols) {
         const int64_t src = rowmap ? rowmap[r0 + rr] : r0 + rr;
         v = __bfloat162float(M[src * ld + c0 + cc]);
       }
-      sm[rr][cc] = v;
+      mv[it] = v;
     }
-    for (int e = threadIdx.x; e < 16 * kMaxW; e += blockDim.x) {
-      const int rr = e / kMaxW, j = e % kMaxW;
-      sq[rr][j] = (r0 + rr < nr && j < w) ? Q[(r0 + rr) * w + j] : 0.0f;
+#pragma unroll
+    for (int it = 0; it < 16 * kMaxW / 256; ++it) {
+      const int e = threadIdx.x + it * 256, rr = e / kMaxW, j = e % kMaxW;
+      qv[it] = (r0 + rr < nr && j < w) ? Q[(r0 + rr) * w + j] : 0.0f;
+    }
+#pragma unroll
+    for (int it = 0; it < 16 * 64 / 256; ++it) {
+      const int e = threadIdx.x + it * 256;
+      sm[e / 64][e % 64] = mv[it];
+    }
+#pragma unroll
+    for (int it = 0; it < 16 * kMaxW / 256; ++it) {
+      const int e = threadIdx.x + it * 256;
+      sq[e / kMaxW][e % kMaxW] = qv[it];
     }
     __syncthreads();
 #pragma unroll 4
