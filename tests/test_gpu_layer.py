@@ -223,3 +223,40 @@ def test_long_token_stress(ctx, metis_lib):
     res = _layer(ctx, cfg)
     errs = _sampled_parity(res, cfg["l"], cfg["m"], 128, 1)
     assert max(errs) <= TOL, errs
+
+
+@pytest.mark.parametrize("name,shape", [("tiny_fwd", None), ("gpt2_small_mlp_up", (1024, 768, 768)),
+                                        ("llama3_8b_mlp_up", (512, 1024, 1024))])
+def test_error_against_exact_metis_and_plain(ctx, metis_lib, name, shape):
+    """The comparison behind the pages' main results, on the GPU path with stochastic
+    rounding: for Y, dX and dW, the Metis and the plain NVFP4 (k = 0) errors against the
+    exact product from the same raw bf16 inputs.  Each agrees with the oracle's error for
+    the same inputs and seeds within 10% relative (codes differ at rounding boundaries
+    where the two decompositions round differently), and where the oracle separates the
+    two by more than 10%, the smaller one is the same on both sides."""
+    base = synth.CONFIGS[name] if shape is None else synth.scaled_config(name, l=shape[0], m=shape[1], n=shape[2])
+    cfg = dict(base, rounding="sr")
+    met, pla = _layer(ctx, cfg), _layer(ctx, cfg, k=0)
+    Xn, Wn, Dn = (met["mats"][n].double().cpu().numpy() for n in ("X", "W", "D"))
+    exact = {"Y": Xn @ Wn, "dX": Dn @ Wn.T, "dW": Xn.T @ Dn}
+    k, s, seed = cfg["k"], cfg["s"], cfg["seed"]
+    bases = [decompose.refresh_basis(M, k, s, l_k, seed, i, 0)["V"]
+             for i, (M, l_k) in enumerate(((Xn, cfg["l_k"]), (Wn, cfg["m"]), (Dn, cfg["l_k"])))]
+    oracle = {}
+    for label, vs in (("metis", bases), ("plain", (None, None, None))):
+        ox, ow, od = (metis.prepare_operand(M, V, seed=seed, operand_id=i, rounding="sr")
+                      for i, (M, V) in enumerate(zip((Xn, Wn, Dn), vs)))
+        dx, dw = metis.linear_bwd(ox, ow, od)
+        oracle[label] = {"Y": metis.linear_fwd(ox, ow), "dX": dx, "dW": dw}
+    report = {}
+    for out in ("Y", "dX", "dW"):
+        e = {}
+        for label, res in (("metis", met), ("plain", pla)):
+            e[label] = (rel_fro(res[out].double().cpu().numpy(), exact[out]), rel_fro(oracle[label][out], exact[out]))
+            gpu, orc = e[label]
+            assert abs(gpu - orc) <= 0.10 * orc, (name, out, label, gpu, orc)
+        om, op = e["metis"][1], e["plain"][1]
+        if abs(om - op) > 0.10 * max(om, op):      # the oracle separates the two clearly
+            assert (e["metis"][0] < e["plain"][0]) == (om < op), (name, out, e)
+        report[out] = e
+    print(name, {o: {l: round(v[0], 4) for l, v in r.items()} for o, r in report.items()})
