@@ -417,9 +417,14 @@ __global__ void __launch_bounds__(kRqThreads, 1)
     uint32_t mph = 0;
     uint8_t* wout = sOut + e * 1024;   // this warp's staged codes: 32 rows x 16 B, then 32 columns x 16 B
     bool stored = false;               // a TMA store of this warp may still be reading wout
-    int it = 0;
-    for (int u = u_begin; u < u_end; ++u, ++it) {
-      const int rb = u / p.n_cb, cb = u % p.n_cb;
+    // this lane's byte offsets in the scale tiles, less the tile's (row block, column block)
+    // terms: the row-wise scale of (row r, block h) and the column-wise scales of (column
+    // half * 16 + jc of this warp's 32, row block hh of its 32 rows)
+    // (a 128-row block of the row-wise tiles spans cols / 64 tiles of 512 bytes: cols * 8)
+    const int row_sc_lane = (h >> 1) * 512 + lane * 16 + q * 4 + 2 * (h & 1);
+    const int col_sc_lane = (q >> 1) * 512 + jc * 16 + h * 4 + 2 * (q & 1) + hh;
+    int rb = u_begin / p.n_cb, cb = u_begin % p.n_cb;   // the unit's 128-row and 128-column blocks
+    for (int it = 0; it < u_end - u_begin; ++it, cb = cb + 1 == p.n_cb ? 0 : cb + 1, rb += cb == 0 ? 1 : 0) {
       const int b = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
       bool ok = true;
@@ -550,10 +555,11 @@ __global__ void __launch_bounds__(kRqThreads, 1)
         tc::bulk_commit_group();
       }
       stored = true;
-      *reinterpret_cast<uint16_t*>(p.row_scales + scale_offset(grow, gcol / 16, p.cols / 64)) = (uint16_t)row_sc;
+      *reinterpret_cast<uint16_t*>(p.row_scales + (int64_t)rb * p.cols * 8 + (cb * 1024 + row_sc_lane)) =
+          (uint16_t)row_sc;
 #pragma unroll
       for (int half = 0; half < 2; ++half)
-        p.col_scales[scale_offset(gcol + half * 16 + jc, grow_t / 16, p.rows / 64)] = (uint8_t)col_sc[half];
+        p.col_scales[(int64_t)cb * p.rows * 8 + (rb * 1024 + col_sc_lane + half * 256)] = (uint8_t)col_sc[half];
       if (++ms == C::M_STAGES) {
         ms = 0;
         mph ^= 1u;
