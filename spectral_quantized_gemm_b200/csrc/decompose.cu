@@ -1459,8 +1459,12 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
   const int kpw = pad_width(std::max(w, k));
   const bool unsampled = lk >= r;   // the refresh's Bm^T = M^T Q then runs on M^T (tensor cores)
   need += (size_t)2 * kpw * std::max(r, c) * 2 + 256;             // hi/lo transposed operand
-  const int splits_est = std::max(normalize_splits(c, bf16_splits(ctx, r, c)),
-                                  unsampled ? normalize_splits(r, bf16_splits(ctx, c, r)) : 1);
+  // the largest split count of the projections below: M Omega and M V (widths w and k), and
+  // M^T Q for the unsampled operand
+  const int splits_est =
+      std::max({normalize_splits(c, bf16_splits(ctx, r, c, 2 * pad_width(w))),
+                normalize_splits(c, bf16_splits(ctx, r, c, 2 * pad_width(k))),
+                unsampled ? normalize_splits(r, bf16_splits(ctx, c, r, 2 * pad_width(w))) : 1});
   const size_t tc_partial_bytes = (size_t)splits_est * std::max(r, c) * 2 * kpw * 4;
   need += tc_partial_bytes + 256;                                 // split partials
   if (unsampled) need += (size_t)r * c * 2 + 256;                 // M^T
@@ -1534,7 +1538,7 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
     split_hi_lo_t_kernel<<<(unsigned)((K + kSplitRows - 1) / kSplitRows), kSplitThreads, 0, st>>>(B, K, width, kp,
                                                                                               bt2);
     count_launch();
-    const int splits = normalize_splits(K, bf16_splits(ctx, rows, K));
+    const int splits = normalize_splits(K, bf16_splits(ctx, rows, K, 2 * kp));
     if (splits > kMaxProjSplits) return fail(ctx, METIS_ERR_ARG, "projection split count above the reduction's limit");
     if ((size_t)splits * rows * 2 * kp * 4 > tc_partial_bytes)
       return fail(ctx, METIS_ERR_WORKSPACE, "projection partials exceed workspace");

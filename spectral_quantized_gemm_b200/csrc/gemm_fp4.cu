@@ -1081,19 +1081,20 @@ metis_status launch_group_bn(metis_ctx* ctx, const GemmArgs* g, int n) {
 
 namespace {
 // Split-K count for `tiles` output tiles of `stages` K stages each on a persistent grid of
-// sm_count CTAs: the one that minimizes rounds x (stages per unit + 3), rounds =
-// ceil(tiles x splits / sm_count) -- the last round of equal units otherwise leaves SMs
-// idle (64 tiles in 5 splits: 320 units, 3 rounds, 72% busy) -- and 3 stage-times stand
-// for a unit's pipeline fill and its partial-tile store.  At most 16 splits.
-int wave_splits(metis_ctx* ctx, int64_t tiles, int stages) {
+// sm_count CTAs: the one that minimizes rounds x (stages per unit + 3) + splits x
+// split_cost, rounds = ceil(tiles x splits / sm_count) -- the last round of equal units
+// otherwise leaves SMs idle (64 tiles in 5 splits: 320 units, 3 rounds, 72% busy) -- 3
+// stage-times stand for a unit's pipeline fill and its partial-tile store, and split_cost
+// (in stage-times) for writing and summing one more set of fp32 partials.  At most 16.
+int wave_splits(metis_ctx* ctx, int64_t tiles, int stages, double split_cost = 0.0) {
   const int64_t sms = std::max(1, ctx->sm_count);
   int best = 1;
-  int64_t best_cost = -1;
+  double best_cost = -1;
   for (int s = 1; s <= std::min(16, stages); ++s) {
     const int per = (stages + s - 1) / s;
     const int eff = (stages + per - 1) / per;
     const int64_t rounds = (tiles * eff + sms - 1) / sms;
-    const int64_t cost = rounds * (per + 3);
+    const double cost = (double)(rounds * (per + 3)) + split_cost * eff;
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       best = eff;
@@ -1103,15 +1104,21 @@ int wave_splits(metis_ctx* ctx, int64_t tiles, int stages) {
 }
 }  // namespace
 
-// NVFP4 GeMMs: K / 256 stages per 128-row tile; bf16 GeMMs: K / 64 stages per 128-row tile
+// NVFP4 GeMMs: K / 256 stages per 128-row tile.  bf16 GeMMs of width n: K / 64 stages per
+// 128-row tile; a split's partials (rows x n fp32, written and read once) cost
+// 8 rows n / (sm_count x the stage's 128 x 64 + n x 64 bf16 bytes) stage-times.
 int fp4_splits(metis_ctx* ctx, int64_t tiles, int stages) { return wave_splits(ctx, tiles, stages); }
-int bf16_splits(metis_ctx* ctx, int64_t rows, int64_t K) { return wave_splits(ctx, rows / 128, (int)(K / 64)); }
+int bf16_splits(metis_ctx* ctx, int64_t rows, int64_t K, int n) {
+  const double stage_bytes = 128.0 * 64 * 2 + (double)n * 64 * 2;
+  const double split_cost = 8.0 * (double)rows * n / ((double)std::max(1, ctx->sm_count) * stage_bytes);
+  return wave_splits(ctx, rows / 128, (int)(K / 64), split_cost);
+}
 
 metis_status launch_gemm_bf16(metis_ctx* ctx, const void* A, int64_t lda, int64_t rows, const void* B, int64_t ldb,
                               int n, int64_t K, float* C, int64_t ldc, int splits) {
   if (rows % 128 || K % 64 || lda % 8 || ldb % 8)
     return fail(ctx, METIS_ERR_SHAPE, "bf16 GeMM needs rows % 128, K % 64 and 16-byte row strides");
-  if (splits < 1) splits = bf16_splits(ctx, rows, K);
+  if (splits < 1) splits = bf16_splits(ctx, rows, K, n);
   if (splits > 1 && (int64_t)splits * rows * ldc > (int64_t(1) << 40))
     return fail(ctx, METIS_ERR_SHAPE, "split output too large");
   switch (n) {

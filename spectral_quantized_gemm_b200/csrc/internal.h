@@ -127,8 +127,9 @@ metis_status launch_gemm_nvfp4_group(metis_ctx* ctx, const GemmArgs* g, int n);
 metis_status launch_wait_timeout_selftest(metis_ctx* ctx, int64_t limit_cycles);
 // ---- mma_peak.cu ----
 metis_status launch_mma_peak(metis_ctx* ctx, int64_t iters, double* flops);
-// Split count for a bf16 GeMM of rows / 128 tiles and K / 64 stages, chosen the same way.
-int bf16_splits(metis_ctx* ctx, int64_t rows, int64_t K);
+// Split count for a bf16 GeMM of rows / 128 tiles, K / 64 stages and output width n,
+// chosen the same way, with the cost of each split's partials counted.
+int bf16_splits(metis_ctx* ctx, int64_t rows, int64_t K, int n);
 // Split count with no empty share of the K / 64 stages (what the launch uses).
 inline int normalize_splits(int64_t K, int splits) {
   const int stages = (int)(K / 64);

@@ -382,7 +382,7 @@ metis_status run_lora_linear(metis_ctx* ctx, int which, const metis_nvfp4* A, co
   // Lout(c, j) = L2[c][j]
   const float* Lin = which == 0 ? L2 : L1;
   const float* Lout = which == 0 ? L1 : L2;
-  const int splits = normalize_splits(K, bf16_splits(ctx, p, K));
+  const int splits = normalize_splits(K, bf16_splits(ctx, p, K, kp));
   const size_t need = (size_t)kp * K * 2 + (size_t)splits * p * kp * 4 + (size_t)p * fold_k * 2 +
                       (size_t)q * fold_k * 2 + 4 * 256;
   metis_status s = ensure_workspace(ctx, need);
@@ -411,7 +411,7 @@ metis_status run_lora_branch_grad(metis_ctx* ctx, const metis_matrix* M, const f
                                   bool transpose_out, float* G) {
   const int64_t p = M->rows, c = M->cols;
   const int kp = lora_pad(k);
-  const int splits = normalize_splits(p, bf16_splits(ctx, c, p));
+  const int splits = normalize_splits(p, bf16_splits(ctx, c, p, 2 * kp));
   const size_t need = (size_t)c * p * 2 + (size_t)2 * kp * p * 2 + (size_t)splits * c * 2 * kp * 4 + 4 * 256;
   metis_status s = ensure_workspace(ctx, need);
   if (s != METIS_OK) return s;
