@@ -208,9 +208,11 @@ class Layer:
         X, D = batches[0]
         self.mats = {"X": X, "W": W, "D": D}
         dev = W.device
-        # X and W gate the forward GeMM, D only the backward: their streams get the higher
-        # priority, so their kernels take free SMs first when the three chains overlap
-        self.streams = {name: torch.cuda.Stream(dev, priority=-1 if name != "D" else 0) for name in self.NAMES}
+        # X and W gate the forward GeMM, D only the backward; X's chain finishes last of the
+        # two.  Stream priorities X > W > D > the GeMM stream, so when the three chains
+        # overlap, free SMs go first to the chain that gates the forward GeMM longest.
+        prio = {"X": -3, "W": -2, "D": -1}
+        self.streams = {name: torch.cuda.Stream(dev, priority=prio[name]) for name in self.NAMES}
         self.ctxs = {}
         for name in self.NAMES:
             with torch.cuda.stream(self.streams[name]):
