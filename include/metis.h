@@ -61,6 +61,16 @@ metis_status metis_create(int device, void* stream, metis_ctx** out);
 /* Frees the context's workspace and status word (synchronizes its stream). */
 void metis_destroy(metis_ctx* ctx);
 metis_status metis_set_stream(metis_ctx* ctx, void* stream);
+/* Sizes this context's later launches for n SMs instead of the device's count: the
+ * persistent kernels (fused GeMM, residual quantizer, thin and projection GeMMs) launch
+ * at most n CTAs (pairs: n / 2) and the split-K counts are chosen for n, so work the
+ * caller runs on other streams at the same time keeps the remaining SMs (the counterpart
+ * of a library's SM-count target). n = 0 restores the device's count; otherwise
+ * 2 <= n <= the device's SM count, else METIS_ERR_ARG. Outputs of the quantizers and of
+ * the fused GeMM do not depend on n; the fp32 sums of split-K products (projection,
+ * Gram, fold preparation) may differ in their last bits, as their split count follows n.
+ * Applies to calls issued after it; not thread-safe against calls in flight on ctx. */
+metis_status metis_set_sm_count_target(metis_ctx* ctx, int n);
 const char* metis_status_str(metis_status s);
 /* Message of the last failed call on this context; owned by the context. */
 const char* metis_last_error(const metis_ctx* ctx);

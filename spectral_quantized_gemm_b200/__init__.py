@@ -44,7 +44,7 @@ EXPORTED = ["metis_create", "metis_destroy", "metis_set_stream", "metis_status_s
             "metis_profile_read", "metis_residual_quantize_nvfp4_noalloc", "metis_dequantize_nvfp4",
             "metis_nvfp4_mma_peak", "metis_selftest_wait_timeout", "metis_lora_linear",
             "metis_lora_branch_grad", "metis_lora_constrain", "metis_lora_realign",
-            "metis_residual_quantize_nvfp4_dump", "metis_profile_read_kind"]
+            "metis_residual_quantize_nvfp4_dump", "metis_profile_read_kind", "metis_set_sm_count_target"]
 
 PROF_GEMM, PROF_RESQUANT, PROF_PROJECTION = 0, 1, 2
 
@@ -87,6 +87,7 @@ def _sig(name, restype, *args):
 _create = _sig("metis_create", c_i32, ctypes.c_int, c_p, ctypes.POINTER(c_p))
 _destroy = _sig("metis_destroy", None, c_p)
 _set_stream = _sig("metis_set_stream", c_i32, c_p, c_p)
+_set_sm_target = _sig("metis_set_sm_count_target", c_i32, c_p, ctypes.c_int)
 _status_str = _sig("metis_status_str", ctypes.c_char_p, c_i32)
 _last_error = _sig("metis_last_error", ctypes.c_char_p, c_p)
 _poll = _sig("metis_poll_device_status", c_i32, c_p, ctypes.POINTER(c_u32), ctypes.c_int)
@@ -222,6 +223,12 @@ class Context:
         return Factors(rows, cols, k, s, l_k, self.device, keep_sketch)
 
     # -- the C ABI ---------------------------------------------------------
+    def set_sm_count_target(self, n):
+        """Size this context's later launches for n SMs (0: the device's count)."""
+        st = _set_sm_target(self._h, int(n))
+        if st != METIS_OK:
+            raise MetisError(st, _last_error(self._h).decode())
+
     def poll_device_status(self, clear=True):
         bits = c_u32(0)
         self._call(_poll, ctypes.byref(bits), int(clear))

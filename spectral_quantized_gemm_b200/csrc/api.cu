@@ -145,6 +145,7 @@ metis_status metis_create(int device, void* stream, metis_ctx** out) {
   ctx->device = device;
   ctx->stream = static_cast<cudaStream_t>(stream);
   ctx->sm_count = prop.multiProcessorCount;
+  ctx->sm_count_device = prop.multiProcessorCount;
   if (cudaMalloc(&ctx->status, sizeof(uint32_t)) != cudaSuccess || cudaMemset(ctx->status, 0, sizeof(uint32_t)) != cudaSuccess) {
     delete ctx;
     return METIS_ERR_CUDA;
@@ -175,6 +176,14 @@ void metis_destroy(metis_ctx* ctx) {
 metis_status metis_set_stream(metis_ctx* ctx, void* stream) {
   if (!ctx) return METIS_ERR_ARG;
   ctx->stream = static_cast<cudaStream_t>(stream);
+  return METIS_OK;
+}
+
+metis_status metis_set_sm_count_target(metis_ctx* ctx, int n) {
+  if (!ctx) return METIS_ERR_ARG;
+  if (n < 0 || n > ctx->sm_count_device || (n > 0 && n < 2))
+    return fail(ctx, METIS_ERR_ARG, "SM count target must be 0 or between 2 and the device's SM count");
+  ctx->sm_count = n == 0 ? ctx->sm_count_device : n;
   return METIS_OK;
 }
 

@@ -14,7 +14,8 @@
 struct metis_ctx {
   int device = 0;
   cudaStream_t stream = nullptr;
-  int sm_count = 0;
+  int sm_count = 0;            // SMs the persistent grids and split counts are sized for
+  int sm_count_device = 0;     // the device's SM count
   uint32_t* status = nullptr;  // device status word (METIS_DEV_* bits)
   char* ws = nullptr;          // device workspace, grown on demand
   size_t ws_bytes = 0;
