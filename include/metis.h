@@ -233,7 +233,7 @@ metis_status metis_dequantize_nvfp4(metis_ctx* ctx, const metis_nvfp4* t, float*
  *   - rows + cols must not exceed 24576 (k <= 64); larger shapes return
  *     METIS_ERR_SHAPE with a message.  rowwise and colwise are both required.
  *   - The first call on a device looks up the array's device address (once per
- *     device); make that first call before any stream capture begins.
+ *     device, cached for the process).
  *   - All calls share the one array and it keeps the last call's contents (every
  *     call overwrites the part it reads first).  Calls whose GPU work overlaps --
  *     e.g. issued on two streams without ordering -- race on it.
