@@ -344,6 +344,17 @@ metis_status metis_lora_realign(metis_ctx* ctx, float* W_res, int64_t m, int64_t
 metis_status metis_selftest_wait_timeout(metis_ctx* ctx, int64_t limit_cycles);
 
 /*
+ * Self-test of the numeric-failure latch (no counterpart in the notes).  The small
+ * eigensolver latches METIS_DEV_NUMERIC when a solve reaches its sweep limit unconverged.
+ * This runs it, on the context's stream, on a fixed 8 x 8 symmetric matrix (2 on the
+ * diagonal, 1 elsewhere) with the limit set to zero sweeps, so the solve stops at once,
+ * raises the bit and returns normally; the caller checks metis_poll_device_status and
+ * that the context stays usable.  Uses the context's workspace (grown if needed).
+ * Errors: ERR_WORKSPACE if the workspace cannot grow.
+ */
+metis_status metis_selftest_numeric(metis_ctx* ctx);
+
+/*
  * NVFP4 tensor-core throughput microbenchmark (no counterpart in the notes; the measured
  * ceiling for the fused GeMM).  Launches, on the context's stream, one cluster of two
  * CTAs per SM pair; each pair issues `iters` stages of four block-scaled MMAs

@@ -44,7 +44,8 @@ EXPORTED = ["metis_create", "metis_destroy", "metis_set_stream", "metis_status_s
             "metis_profile_read", "metis_residual_quantize_nvfp4_noalloc", "metis_dequantize_nvfp4",
             "metis_nvfp4_mma_peak", "metis_selftest_wait_timeout", "metis_lora_linear",
             "metis_lora_branch_grad", "metis_lora_constrain", "metis_lora_realign",
-            "metis_residual_quantize_nvfp4_dump", "metis_profile_read_kind", "metis_set_sm_count_target"]
+            "metis_residual_quantize_nvfp4_dump", "metis_profile_read_kind", "metis_set_sm_count_target",
+            "metis_selftest_numeric"]
 
 PROF_GEMM, PROF_RESQUANT, PROF_PROJECTION = 0, 1, 2
 
@@ -106,6 +107,7 @@ _resq_dump = _sig("metis_residual_quantize_nvfp4_dump", c_i32, c_p, ctypes.POINT
 _dequant = _sig("metis_dequantize_nvfp4", c_i32, c_p, ctypes.POINTER(Nvfp4Struct), c_p, c_i64)
 _mma_peak = _sig("metis_nvfp4_mma_peak", c_i32, c_p, c_i64, ctypes.POINTER(ctypes.c_double))
 _wait_selftest = _sig("metis_selftest_wait_timeout", c_i32, c_p, c_i64)
+_numeric_selftest = _sig("metis_selftest_numeric", c_i32, c_p)
 _quant_f32 = _sig("metis_quantize_nvfp4_f32", c_i32, c_p, c_p, c_i64, c_i64, c_i64, ctypes.POINTER(QuantParams),
                   ctypes.POINTER(Nvfp4Struct), ctypes.POINTER(Nvfp4Struct))
 _gemm = _sig("metis_gemm_nvfp4", c_i32, c_p, ctypes.POINTER(Nvfp4Struct), ctypes.POINTER(Nvfp4Struct), c_i64, c_p,
@@ -292,6 +294,11 @@ class Context:
         """Launch the bounded-wait self-test (a wait that must time out); the caller then
         reads METIS_DEV_TIMEOUT from poll_device_status()."""
         self._call(_wait_selftest, limit_cycles)
+
+    def selftest_numeric(self):
+        """Launch the numeric-latch self-test (an eigensolve allowed no sweep); the caller
+        then reads METIS_DEV_NUMERIC from poll_device_status()."""
+        self._call(_numeric_selftest)
 
     def nvfp4_mma_peak(self, iters=4096, reps=5):
         """Achievable NVFP4 MMA rate (TFLOP/s): the median of `reps` timed launches of the

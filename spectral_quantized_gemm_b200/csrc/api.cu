@@ -490,6 +490,12 @@ metis_status metis_selftest_wait_timeout(metis_ctx* ctx, int64_t limit_cycles) {
   return launch_wait_timeout_selftest(ctx, limit_cycles);
 }
 
+metis_status metis_selftest_numeric(metis_ctx* ctx) {
+  metis_status s = enter(ctx);
+  if (s != METIS_OK) return s;
+  return launch_numeric_selftest(ctx);
+}
+
 metis_status metis_nvfp4_mma_peak(metis_ctx* ctx, int64_t iters, double* flops) {
   const metis::NvtxRange nvtx_range("metis_nvfp4_mma_peak");
   metis_status s = enter(ctx);

@@ -897,7 +897,7 @@ struct JacOut {
 
 __global__ void __launch_bounds__(kJacThreads, 1) jacobi_rounds_kernel(const double* __restrict__ G, int n, int k,
                                                                        int mode, JacOut jo, SmallOut out,
-                                                                       uint32_t* status) {
+                                                                       uint32_t* status, int max_sweeps) {
   extern __shared__ double smem_d[];
   const int ne = jac_ne(n), m = ne / 2;
   double* Hbuf0 = smem_d;                       // off-diagonal blocks of the slot grid, upper triangle
@@ -1006,7 +1006,7 @@ __global__ void __launch_bounds__(kJacThreads, 1) jacobi_rounds_kernel(const dou
       need = jac_needs(own_ga, d.x, d.y, tol2);
     }
     if (!__syncthreads_or(need)) break;
-    if (sweep == kJacobiMaxSweeps) {
+    if (sweep == max_sweeps) {
       if (tid == 0) {
         raise_status(status, METIS_DEV_NUMERIC);
         out.flags[0] = 1;
@@ -1510,7 +1510,8 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
       if (n <= kSmallMaxN) chol_inverse_kernel<<<1, kCholThreads, chol_smem_bytes(n), st>>>(G, n, so);
       else cholqr_solver_kernel<<<1, kSolverThreads, 0, st>>>(G, n, so);
     } else if (jac_ne(n) <= kJacMaxNE) {
-      jacobi_rounds_kernel<<<1, kJacThreads, jac_smem_bytes(jac_ne(n)), st>>>(G, n, k, mode, jo, so, ctx->status);
+      jacobi_rounds_kernel<<<1, kJacThreads, jac_smem_bytes(jac_ne(n)), st>>>(G, n, k, mode, jo, so, ctx->status,
+                                                                          kJacobiMaxSweeps);
       count_launch();
       jacobi_replay_kernel<<<(n + kJacRowsPerCta - 1) / kJacRowsPerCta, 32 * kJacRowsPerCta, 0, st>>>(
           jrot, jinfo, n, k, mode, jorder, jinv, so);
@@ -1623,6 +1624,47 @@ metis_status run_decompose(metis_ctx* ctx, const metis_matrix* M, const metis_de
       Q, r, Bt, c, k, fs, p->rounding, p->seed, stream_tag(p->operand_id, kPurposeSR, kSrLeft),
       stream_tag(p->operand_id, kPurposeSR, kSrRight), step, f->U, f->V, f->Uq, f->Vq); count_launch();
   return check_cuda(ctx, cudaGetLastError(), "decompose");
+}
+
+// ---- self-test of the numeric-failure latch ----
+namespace {
+// G = the n x n matrix with 2 on the diagonal and 1 elsewhere (symmetric positive
+// definite, far from diagonal)
+__global__ void numeric_selftest_fill_kernel(double* G, int n) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e < n * n) G[e] = (e / n == e % n) ? 2.0 : 1.0;
+}
+}  // namespace
+
+metis_status launch_numeric_selftest(metis_ctx* ctx) {
+  constexpr int n = 8;
+  const size_t need = (size_t)n * n * 8 + jac_rot_entries(n) * sizeof(double2) + (size_t)2 * n * kMaxW * 8 +
+                      (size_t)kMaxW * (4 + 4 + 8 + 4) + 8 * 256;
+  metis_status s = ensure_workspace(ctx, need);
+  if (s != METIS_OK) return s;
+  Workspace ws{ctx->ws, ctx->ws_bytes};
+  double* G = static_cast<double*>(ws.take((size_t)n * n * 8));
+  double2* rot = static_cast<double2*>(ws.take(jac_rot_entries(n) * sizeof(double2)));
+  double* T = static_cast<double*>(ws.take((size_t)n * kMaxW * 8));
+  double* Vr = static_cast<double*>(ws.take((size_t)n * kMaxW * 8));
+  float* S = static_cast<float*>(ws.take((size_t)kMaxW * 4));
+  int* flags = static_cast<int*>(ws.take((size_t)kMaxW * 4));
+  int* order = static_cast<int*>(ws.take((size_t)kMaxW * 4));
+  double* inv = static_cast<double*>(ws.take((size_t)kMaxW * 8));
+  int* info = static_cast<int*>(ws.take(64));
+  if (!info) return fail(ctx, METIS_ERR_WORKSPACE, "numeric self-test workspace layout");
+  cudaStream_t st = ctx->stream;
+  numeric_selftest_fill_kernel<<<1, 64, 0, st>>>(G, n);
+  count_launch();
+  cudaError_t e = cudaFuncSetAttribute(jacobi_rounds_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)jac_smem_bytes(kJacMaxNE));
+  if (e != cudaSuccess) return check_cuda(ctx, e, "cudaFuncSetAttribute(numeric self-test)");
+  SmallOut so{T, Vr, S, flags, nullptr};
+  JacOut jo{rot, info, order, inv};
+  // a sweep limit of zero: the solve stops before its first sweep, unconverged
+  jacobi_rounds_kernel<<<1, kJacThreads, jac_smem_bytes(jac_ne(n)), st>>>(G, n, n, 2, jo, so, ctx->status, 0);
+  count_launch();
+  return check_cuda(ctx, cudaGetLastError(), "numeric self-test launch");
 }
 
 // ---- launchers shared with the LoRA-SVD calls (lora.cu) ----

@@ -126,6 +126,8 @@ metis_status launch_gemm_nvfp4(metis_ctx* ctx, const GemmArgs& a);
 metis_status launch_gemm_nvfp4_group(metis_ctx* ctx, const GemmArgs* g, int n);
 // ---- selftest.cu ----
 metis_status launch_wait_timeout_selftest(metis_ctx* ctx, int64_t limit_cycles);
+// (decompose.cu) the eigensolver on a fixed 8 x 8 matrix with a sweep limit of zero
+metis_status launch_numeric_selftest(metis_ctx* ctx);
 // ---- mma_peak.cu ----
 metis_status launch_mma_peak(metis_ctx* ctx, int64_t iters, double* flops);
 // Split count for a bf16 GeMM of rows / 128 tiles, K / 64 stages and output width n,

@@ -2,6 +2,8 @@
 
 * A bounded wait that runs out is reported as METIS_DEV_TIMEOUT and leaves the context
   usable (the self-test waits on a barrier nothing arrives at; nothing faults or hangs).
+* An eigensolve that stops unconverged is reported as METIS_DEV_NUMERIC (the self-test
+  allows it no sweep) and leaves the context usable.
 * NaN canaries around output buffers: the fused GeMM (CTA-pair and single-CTA paths, bf16
   and fp32) and the residual quantizer write every element they own and nothing beyond.
 * MetisLinear resumed from a checkpoint after 4 steps gives the same step-8 results, bit
@@ -36,6 +38,31 @@ def test_wait_timeout_is_reported_and_the_context_survives(ctx, metis_lib):
     assert np.array_equal(codes, wc) and np.array_equal(scales, ws)
     with pytest.raises(metis_lib.MetisError):
         ctx.selftest_wait_timeout(0)
+
+
+def test_numeric_failure_is_reported_and_the_context_survives(ctx, metis_lib):
+    """An eigensolve that reaches its sweep limit unconverged latches METIS_DEV_NUMERIC
+    (the self-test allows it no sweep); the bit clears on read and a decomposition right
+    after is clean and agrees with the oracle's singular values."""
+    from oracle import decompose
+    from workloads import synth
+    assert ctx.poll_device_status() == 0
+    ctx.selftest_numeric()
+    st = ctx.poll_device_status()
+    assert st & metis_lib.DEV_NUMERIC
+    assert not st & (metis_lib.DEV_TIMEOUT | metis_lib.DEV_NONFINITE)
+    assert ctx.poll_device_status() == 0          # cleared by the read
+    cfg = synth.CONFIGS["tiny_fwd"]
+    Mt = synth.operand_matrix(cfg, "X")
+    f = ctx.new_factors(256, 256, 4, 4, 32)
+    ctx.decompose(Mt.cuda(), k=4, s=4, l_k=32, seed=0, operand_id=0, refresh=True, step=0, factors=f)
+    torch.cuda.synchronize()
+    assert ctx.poll_device_status() == 0
+    M = Mt.double().numpy()
+    ref = decompose.refresh_basis(M, 4, 4, 32, 0, 0, 0)
+    _, S, _ = decompose.step_factors(M, ref["V"])
+    gS = f.S.cpu().double().numpy()[:4]
+    assert np.max(np.abs(gS - S) / S[0]) < 1e-3
 
 
 def _operand(ctx, outer, inner, seed):
